@@ -1,0 +1,318 @@
+"""CPU oracle for the integer-only ViT encoder block (test infrastructure).
+
+TEST INFRASTRUCTURE ONLY.  Only the test suite, ``__graft_entry__.smoke()`` and
+the CPU-baseline leg of ``bench.py`` may import this package.  The product
+library (``integer_only_quantized_int8_b200``) never imports it and shares no
+code with it; the two meet only in the seeded input generator (``synthetic``),
+which holds none of the method's arithmetic.
+
+The arithmetic lives in ``ivit_oracle.c`` (plain single-threaded C, built with
+gcc).  This module builds it on first use and exposes numpy-friendly wrappers,
+plus the oracle's own derivation of integer parameters from real scales
+(dyadic numbers, I_0 values) following "I-ViT: Integer-only Quantization for
+Efficient Vision Transformer Inference", sections 3.2-3.5.
+"""
+from __future__ import annotations
+
+import ctypes as C
+import os
+import subprocess
+import threading
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "ivit_oracle.c")
+_LIB = os.path.join(_HERE, "libivit_oracle.so")
+_lock = threading.Lock()
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile ivit_oracle.c into a shared library next to it."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        tmp = _LIB + f".tmp{os.getpid()}"
+        subprocess.check_call(["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-o", tmp, _SRC, "-lm"])
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+def _i8p(a):
+    return a.ctypes.data_as(C.POINTER(C.c_int8))
+
+
+def _i32p(a):
+    return a.ctypes.data_as(C.POINTER(C.c_int32))
+
+
+def _opt_i32p(a):
+    return None if a is None else _i32p(a)
+
+
+class BlockParamsC(C.Structure):
+    _fields_ = [(n, t) for n, t in [
+        ("D", C.c_int32), ("H", C.c_int32), ("Dm", C.c_int32),
+        ("ln1_gamma", C.c_void_p), ("ln1_beta", C.c_void_p), ("ln1_b", C.c_int32), ("ln1_c", C.c_int32),
+        ("w_qkv", C.c_void_p), ("bias_qkv", C.c_void_p), ("b_qkv", C.c_void_p), ("c_qkv", C.c_void_p),
+        ("logit_b", C.c_int32), ("logit_c", C.c_int32), ("k_s", C.c_int32), ("attn_I0", C.c_int32),
+        ("attn_M", C.c_int32), ("attn_k_out", C.c_int32), ("attn_out_b", C.c_int32), ("attn_out_c", C.c_int32),
+        ("w_o", C.c_void_p), ("bias_o", C.c_void_p), ("b_o", C.c_void_p), ("c_o", C.c_void_p),
+        ("res1_b_skip", C.c_int32), ("res1_b_branch", C.c_int32), ("res1_c", C.c_int32),
+        ("ln2_gamma", C.c_void_p), ("ln2_beta", C.c_void_p), ("ln2_b", C.c_int32), ("ln2_c", C.c_int32),
+        ("w1", C.c_void_p), ("bias1", C.c_void_p), ("b1", C.c_void_p), ("c1", C.c_void_p),
+        ("gelu_I0", C.c_int32), ("gelu_M", C.c_int32), ("gelu_k_out", C.c_int32), ("gelu_b", C.c_int32),
+        ("gelu_c", C.c_int32),
+        ("w2", C.c_void_p), ("bias2", C.c_void_p), ("b2", C.c_void_p), ("c2", C.c_void_p),
+        ("res2_b_skip", C.c_int32), ("res2_b_branch", C.c_int32), ("res2_c", C.c_int32),
+        ("ln_F", C.c_int32), ("ln_M", C.c_int32),
+    ]]
+
+
+def lib():
+    global _lib
+    with _lock:
+        if _lib is None:
+            L = C.CDLL(build())
+            L.orc_quantize.restype = C.c_int32
+            L.orc_quantize.argtypes = [C.c_double, C.c_double, C.c_int]
+            L.orc_dyadic.restype = C.c_int
+            L.orc_dyadic.argtypes = [C.c_double, C.POINTER(C.c_int32), C.POINTER(C.c_int32)]
+            L.orc_dyadic_pair.restype = C.c_int
+            L.orc_dyadic_pair.argtypes = [C.c_double, C.c_double, C.POINTER(C.c_int32),
+                                          C.POINTER(C.c_int32), C.POINTER(C.c_int32)]
+            L.orc_recip_i0.restype = C.c_int32
+            L.orc_recip_i0.argtypes = [C.c_double]
+            L.orc_requant.restype = C.c_int64
+            L.orc_requant.argtypes = [C.c_int64, C.c_int32, C.c_int32, C.c_int]
+            L.orc_linear_requant.restype = None
+            L.orc_linear_requant.argtypes = [C.c_void_p, C.c_int64, C.c_int32, C.c_void_p, C.c_int32,
+                                             C.c_void_p, C.c_void_p, C.c_void_p, C.c_int,
+                                             C.c_void_p, C.c_int32, C.c_int32, C.c_int32, C.c_void_p]
+            L.orc_shift_exp.restype = C.c_int64
+            L.orc_shift_exp.argtypes = [C.c_int64, C.c_int64]
+            L.orc_int_div.restype = C.c_int64
+            L.orc_int_div.argtypes = [C.c_int64, C.c_int64, C.c_int, C.c_int]
+            L.orc_shiftmax_row.restype = None
+            L.orc_shiftmax_row.argtypes = [C.c_void_p, C.c_int, C.c_int32, C.c_int, C.c_int, C.c_void_p]
+            L.orc_attention.restype = None
+            L.orc_attention.argtypes = [C.c_void_p, C.c_int32, C.c_int32, C.c_int32,
+                                        C.c_int32, C.c_int32, C.c_int32, C.c_int32,
+                                        C.c_int32, C.c_int32, C.c_int32, C.c_int32, C.c_void_p]
+            L.orc_shift_sigmoid.restype = C.c_int64
+            L.orc_shift_sigmoid.argtypes = [C.c_int64, C.c_int64, C.c_int32, C.c_int32]
+            L.orc_shiftgelu_one.restype = C.c_int32
+            L.orc_shiftgelu_one.argtypes = [C.c_int32, C.c_int32, C.c_int32, C.c_int32, C.c_int32,
+                                            C.c_int32, C.POINTER(C.c_int32)]
+            L.orc_shiftgelu.restype = None
+            L.orc_shiftgelu.argtypes = [C.c_void_p, C.c_int64, C.c_int32, C.c_int32, C.c_int32,
+                                        C.c_int32, C.c_int32, C.c_void_p]
+            L.orc_isqrt_newton.restype = C.c_int64
+            L.orc_isqrt_newton.argtypes = [C.c_int64]
+            L.orc_layernorm.restype = None
+            L.orc_layernorm.argtypes = [C.c_void_p, C.c_int64, C.c_int32, C.c_void_p, C.c_void_p,
+                                        C.c_int32, C.c_int32, C.c_int32, C.c_int32, C.c_void_p]
+            L.orc_block_forward.restype = C.c_int
+            L.orc_block_forward.argtypes = [C.POINTER(BlockParamsC), C.c_void_p, C.c_void_p,
+                                            C.c_int32, C.c_int32]
+            _lib = L
+    return _lib
+
+
+# ---------------------------------------------------------------------------
+# scalar helpers
+# ---------------------------------------------------------------------------
+
+def quantize(R: float, m: float, k: int = 8) -> int:
+    return int(lib().orc_quantize(float(R), float(m), int(k)))
+
+
+def dyadic(s: float):
+    """DN(s) -> (b, c) with b / 2^c ~ s (I-ViT section 3.2)."""
+    b, c = C.c_int32(), C.c_int32()
+    if lib().orc_dyadic(float(s), C.byref(b), C.byref(c)) != 0:
+        raise ValueError(f"no dyadic number for {s!r}")
+    return int(b.value), int(c.value)
+
+
+def dyadic_pair(s1: float, s2: float):
+    b1, b2, c = C.c_int32(), C.c_int32(), C.c_int32()
+    if lib().orc_dyadic_pair(float(s1), float(s2), C.byref(b1), C.byref(b2), C.byref(c)) != 0:
+        raise ValueError(f"no dyadic pair for {s1!r}, {s2!r}")
+    return int(b1.value), int(b2.value), int(c.value)
+
+
+def recip_i0(S: float) -> int:
+    return int(lib().orc_recip_i0(float(S)))
+
+
+def requant(acc: int, b: int, c: int, bits: int = 8) -> int:
+    return int(lib().orc_requant(int(acc), int(b), int(c), int(bits)))
+
+
+def shift_exp(I_delta: int, I0: int) -> int:
+    return int(lib().orc_shift_exp(int(I_delta), int(I0)))
+
+
+def int_div(e: int, total: int, M: int = 30, k_out: int = 8) -> int:
+    return int(lib().orc_int_div(int(e), int(total), int(M), int(k_out)))
+
+
+def isqrt_newton(V: int) -> int:
+    return int(lib().orc_isqrt_newton(int(V)))
+
+
+def shift_sigmoid(I_p: int, I0: int, M: int = 30, k_out: int = 8) -> int:
+    """Integer sigmoid of S*I_p (S = 1/I0), scale 2^-(k_out-1) (I-ViT section 3.4)."""
+    return int(lib().orc_shift_sigmoid(int(I_p), int(I0), int(M), int(k_out)))
+
+
+def shiftgelu_one(I: int, I0: int, M: int = 30, k_out: int = 8, b_g: int = 1, c_g: int = 0):
+    """Returns (g, sigma_int) for one int8 input."""
+    s = C.c_int32()
+    g = lib().orc_shiftgelu_one(int(I), int(I0), int(M), int(k_out), int(b_g), int(c_g), C.byref(s))
+    return int(g), int(s.value)
+
+
+# ---------------------------------------------------------------------------
+# tensor ops (numpy in, numpy out)
+# ---------------------------------------------------------------------------
+
+def shiftmax_row(L, I0: int, M: int = 30, k_out: int = 8):
+    L = np.ascontiguousarray(L, dtype=np.int32)
+    P = np.zeros_like(L)
+    lib().orc_shiftmax_row(L.ctypes.data, int(L.size), int(I0), int(M), int(k_out), P.ctypes.data)
+    return P
+
+
+def linear_requant(X, W, bias, b, c, out_bits: int = 8, skip=None, res=(0, 0, 0)):
+    """X [M x K] int8, W [N x K] int8, bias/b/c [N] -> Y [M x N] int8."""
+    X = np.ascontiguousarray(X, dtype=np.int8)
+    W = np.ascontiguousarray(W, dtype=np.int8)
+    M, K = X.shape
+    N = W.shape[0]
+    assert W.shape[1] == K
+    bias = None if bias is None else np.ascontiguousarray(bias, dtype=np.int32)
+    b = np.ascontiguousarray(b, dtype=np.int32)
+    c = np.ascontiguousarray(c, dtype=np.int32)
+    Y = np.zeros((M, N), dtype=np.int8)
+    sk = None
+    if skip is not None:
+        sk = np.ascontiguousarray(skip, dtype=np.int8)
+        assert sk.shape == (M, N)
+    lib().orc_linear_requant(X.ctypes.data, M, K, W.ctypes.data, N,
+                             None if bias is None else bias.ctypes.data, b.ctypes.data, c.ctypes.data,
+                             int(out_bits), None if sk is None else sk.ctypes.data,
+                             int(res[0]), int(res[1]), int(res[2]), Y.ctypes.data)
+    return Y
+
+
+def attention(qkv, B: int, N: int, H: int, logit, k_s: int, I0: int, M: int, k_out: int, out):
+    """qkv [B*N x 3*H*64] int8 -> ctx [B*N x H*64] int8."""
+    qkv = np.ascontiguousarray(qkv, dtype=np.int8)
+    assert qkv.shape == (B * N, 3 * H * 64)
+    ctx = np.zeros((B * N, H * 64), dtype=np.int8)
+    lib().orc_attention(qkv.ctypes.data, B, N, H, int(logit[0]), int(logit[1]), int(k_s), int(I0),
+                        int(M), int(k_out), int(out[0]), int(out[1]), ctx.ctypes.data)
+    return ctx
+
+
+def shiftgelu(x, I0: int, M: int, k_out: int, out):
+    x = np.ascontiguousarray(x, dtype=np.int8)
+    y = np.zeros_like(x)
+    lib().orc_shiftgelu(x.ctypes.data, x.size, int(I0), int(M), int(k_out), int(out[0]), int(out[1]),
+                        y.ctypes.data)
+    return y
+
+
+def layernorm(x, gamma, beta, F: int, M_ln: int, out):
+    x = np.ascontiguousarray(x, dtype=np.int8)
+    rows, cols = x.shape
+    gamma = np.ascontiguousarray(gamma, dtype=np.int8)
+    beta = np.ascontiguousarray(beta, dtype=np.int32)
+    y = np.zeros_like(x)
+    lib().orc_layernorm(x.ctypes.data, rows, cols, gamma.ctypes.data, beta.ctypes.data,
+                        int(F), int(M_ln), int(out[0]), int(out[1]), y.ctypes.data)
+    return y
+
+
+# ---------------------------------------------------------------------------
+# integer parameters of a block, derived from the real scales
+# ---------------------------------------------------------------------------
+
+def block_params(q, attn_M: int = 30, attn_k_out: int = 8, k_s: int = 8,
+                 gelu_M: int = 30, gelu_k_out: int = 8, ln_F: int = 7, ln_M: int = 23):
+    """Integer parameters of one block from a ``synthetic.QuantBlock``.
+
+    Every multiplier is the oracle's own DN of a ratio of real scales
+    (I-ViT section 3.2); I_0 values are the oracle's own reciprocal rounding
+    (section 3.3).  Returns a dict of numpy arrays / ints.
+    """
+    S = q.scales
+    D, H, Dm = q.D, q.H, q.Dm
+
+    def per_channel(s_in, s_w, s_out):
+        bc = [dyadic(s_in * float(sw) / float(so)) for sw, so in zip(s_w, s_out)]
+        return (np.array([x[0] for x in bc], dtype=np.int32), np.array([x[1] for x in bc], dtype=np.int32))
+
+    qkv_out = np.concatenate([np.full(D, S["q"]), np.full(D, S["k"]), np.full(D, S["v"])])
+    p = dict(D=D, H=H, Dm=Dm, ln_F=ln_F, ln_M=ln_M, k_s=k_s,
+             attn_M=attn_M, attn_k_out=attn_k_out, gelu_M=gelu_M, gelu_k_out=gelu_k_out)
+    p["ln1_gamma"], p["ln1_beta"] = q.ln1_gamma, q.ln1_beta
+    p["ln1_out"] = dyadic(S["gamma1"] * 2.0 ** -ln_F / S["ln1"])
+    p["w_qkv"], p["bias_qkv"] = q.w_qkv, q.bias_qkv
+    p["b_qkv"], p["c_qkv"] = per_channel(S["ln1"], q.s_w_qkv, qkv_out)
+    p["logit"] = dyadic(S["q"] * S["k"] / (8.0 * S["logit"]))
+    p["attn_I0"] = recip_i0(S["logit"])
+    p["attn_out"] = dyadic(S["v"] * 2.0 ** -(attn_k_out - 1) / S["ctx"])
+    p["w_o"], p["bias_o"] = q.w_o, q.bias_o
+    p["b_o"], p["c_o"] = per_channel(S["ctx"], q.s_w_o, np.full(D, S["o"]))
+    p["res1"] = dyadic_pair(S["x"] / S["xh"], S["o"] / S["xh"])
+    p["ln2_gamma"], p["ln2_beta"] = q.ln2_gamma, q.ln2_beta
+    p["ln2_out"] = dyadic(S["gamma2"] * 2.0 ** -ln_F / S["ln2"])
+    p["w1"], p["bias1"] = q.w1, q.bias1
+    p["b1"], p["c1"] = per_channel(S["ln2"], q.s_w1, np.full(Dm, S["h"]))
+    p["gelu_I0"] = recip_i0(S["h"])
+    p["gelu_out"] = dyadic(S["h"] * 2.0 ** -(gelu_k_out - 1) / S["g"])
+    p["w2"], p["bias2"] = q.w2, q.bias2
+    p["b2"], p["c2"] = per_channel(S["g"], q.s_w2, np.full(D, S["f"]))
+    p["res2"] = dyadic_pair(S["xh"] / S["y"], S["f"] / S["y"])
+    return p
+
+
+def block_forward(p, x, B: int, N: int):
+    """x [B*N x D] int8 -> y [B*N x D] int8 through one block."""
+    x = np.ascontiguousarray(x, dtype=np.int8)
+    keep = []
+
+    def arr(a, dt):
+        a = np.ascontiguousarray(a, dtype=dt)
+        keep.append(a)
+        return a.ctypes.data
+
+    s = BlockParamsC()
+    s.D, s.H, s.Dm = p["D"], p["H"], p["Dm"]
+    s.ln1_gamma, s.ln1_beta = arr(p["ln1_gamma"], np.int8), arr(p["ln1_beta"], np.int32)
+    s.ln1_b, s.ln1_c = p["ln1_out"]
+    s.w_qkv, s.bias_qkv = arr(p["w_qkv"], np.int8), arr(p["bias_qkv"], np.int32)
+    s.b_qkv, s.c_qkv = arr(p["b_qkv"], np.int32), arr(p["c_qkv"], np.int32)
+    s.logit_b, s.logit_c = p["logit"]
+    s.k_s, s.attn_I0, s.attn_M, s.attn_k_out = p["k_s"], p["attn_I0"], p["attn_M"], p["attn_k_out"]
+    s.attn_out_b, s.attn_out_c = p["attn_out"]
+    s.w_o, s.bias_o = arr(p["w_o"], np.int8), arr(p["bias_o"], np.int32)
+    s.b_o, s.c_o = arr(p["b_o"], np.int32), arr(p["c_o"], np.int32)
+    s.res1_b_skip, s.res1_b_branch, s.res1_c = p["res1"]
+    s.ln2_gamma, s.ln2_beta = arr(p["ln2_gamma"], np.int8), arr(p["ln2_beta"], np.int32)
+    s.ln2_b, s.ln2_c = p["ln2_out"]
+    s.w1, s.bias1 = arr(p["w1"], np.int8), arr(p["bias1"], np.int32)
+    s.b1, s.c1 = arr(p["b1"], np.int32), arr(p["c1"], np.int32)
+    s.gelu_I0, s.gelu_M, s.gelu_k_out = p["gelu_I0"], p["gelu_M"], p["gelu_k_out"]
+    s.gelu_b, s.gelu_c = p["gelu_out"]
+    s.w2, s.bias2 = arr(p["w2"], np.int8), arr(p["bias2"], np.int32)
+    s.b2, s.c2 = arr(p["b2"], np.int32), arr(p["c2"], np.int32)
+    s.res2_b_skip, s.res2_b_branch, s.res2_c = p["res2"]
+    s.ln_F, s.ln_M = p["ln_F"], p["ln_M"]
+    y = np.zeros_like(x)
+    rc = lib().orc_block_forward(C.byref(s), x.ctypes.data, y.ctypes.data, int(B), int(N))
+    if rc != 0:
+        raise MemoryError("oracle block forward could not allocate scratch")
+    return y

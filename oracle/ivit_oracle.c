@@ -1,0 +1,484 @@
+/*
+ * ivit_oracle.c -- CPU oracle for the integer-only ViT encoder block.
+ *
+ * TEST INFRASTRUCTURE ONLY.  This file is the plain, slow, single-threaded
+ * statement of what the integer-only block computes.  Only the test suite,
+ * the smoke check and the benchmark's CPU-baseline leg may load it; the
+ * product library never does, and this file shares no code, header, table or
+ * helper with the CUDA path.
+ *
+ * Sources (cited by page title and section / equation):
+ *   [IVIT]  "I-ViT: Integer-only Quantization for Efficient Vision Transformer
+ *           Inference" (mer.run notes), sections 3.1-3.5.
+ *   [TRIO]  "Trio-ViT" article (cloud.tencent.com), eqs. (1)-(3) (standard ViT
+ *           block, 1/sqrt(d) attention scaling) and eq. (12) (dyadic requant).
+ *
+ * Conventions used everywhere below:
+ *   - ">> s" on a signed value is floor division by 2^s.  It is written out as
+ *     floor division (shr_floor) so that the meaning does not depend on the C
+ *     compiler's treatment of negative shifts.
+ *   - sat_k(v) clamps v to [-2^(k-1), 2^(k-1) - 1].
+ *   - All arithmetic on the hot path is on int64; no floating point is used
+ *     except in the host-side helpers that turn a real scale into integers
+ *     (quantiser, dyadic number, reciprocal), which the pages also place
+ *     off-line.
+ *
+ * Readings of the pages where they leave a step open are marked READING and
+ * listed, with reasons, in the design notes of the repository.
+ *
+ * Parity status: every function here is pinned by tests against closed forms,
+ * invariants, hand-derived examples or textbook routines, except the block
+ * composition's floating-point accuracy, which has no pin (no trained model
+ * or dataset exists to compare against): "parity unpinned" for that aspect
+ * only; the integer composition itself is pinned by the residual identity
+ * special case.
+ */
+#include <stdint.h>
+#include <stddef.h>
+#include <stdlib.h>
+#include <string.h>
+#include <math.h>
+
+/* ------------------------------------------------------------------------ */
+/* integer helpers                                                          */
+/* ------------------------------------------------------------------------ */
+
+/* floor(a / b) for b > 0 (C division truncates toward zero). */
+static int64_t floor_div(int64_t a, int64_t b)
+{
+    int64_t q = a / b;
+    if ((a % b) != 0 && a < 0)
+        q -= 1;
+    return q;
+}
+
+/* a >> s as floor division by 2^s, 0 <= s <= 62. */
+static int64_t shr_floor(int64_t a, int s)
+{
+    return floor_div(a, (int64_t)1 << s);
+}
+
+/* sat_k: clamp to the signed k-bit range. */
+static int64_t sat_bits(int64_t v, int bits)
+{
+    int64_t lo = -((int64_t)1 << (bits - 1));
+    int64_t hi = ((int64_t)1 << (bits - 1)) - 1;
+    if (v < lo) return lo;
+    if (v > hi) return hi;
+    return v;
+}
+
+/* number of significant bits of v >= 0 (bit(0) = 0). */
+static int bit_length(int64_t v)
+{
+    int n = 0;
+    while (v > 0) { n += 1; v >>= 1; }
+    return n;
+}
+
+/* ------------------------------------------------------------------------ */
+/* host-side scale helpers ([IVIT] 3.1 quantiser, 3.2 dyadic numbers)       */
+/* ------------------------------------------------------------------------ */
+
+/*
+ * Uniform symmetric quantiser, [IVIT] 3.1: I = round(clip(R, -m, m) / S) with
+ * S = 2m / (2^k - 1).  READING: round half away from zero, and the result is
+ * kept in the narrow symmetric range +-(2^(k-1) - 1), because R = m lands on
+ * 2^(k-1) - 1/2 which would otherwise round out of range.
+ */
+int32_t orc_quantize(double R, double m, int k)
+{
+    double S = 2.0 * m / (double)((1 << k) - 1);
+    double r = R;
+    if (r > m) r = m;
+    if (r < -m) r = -m;
+    double v = round(r / S);
+    double lim = (double)((1 << (k - 1)) - 1);
+    if (v > lim) v = lim;
+    if (v < -lim) v = -lim;
+    return (int32_t)v;
+}
+
+/*
+ * Dyadic number DN(s) = b / 2^c, [IVIT] 3.2 and [TRIO] eq. (12).  READING (the
+ * pages give no algorithm): c is the largest integer in [0, 31] for which
+ * b = round(s * 2^c) stays below 2^31; then |b / 2^c - s| <= 2^-(c+1).
+ * Returns 0 on success, -1 if s is negative, not finite or too large.
+ */
+int orc_dyadic(double s, int32_t *b, int32_t *c)
+{
+    if (!(s >= 0.0) || !(s < 2147483647.5))
+        return -1;
+    for (int cc = 31; cc >= 0; --cc) {
+        double v = round(ldexp(s, cc));
+        if (v < 2147483648.0) {
+            *b = (int32_t)v;
+            *c = cc;
+            return 0;
+        }
+    }
+    return -1;
+}
+
+/*
+ * Two dyadic numbers that share one shift, for the residual additions of
+ * [IVIT] 3.1 (X^ = MSA(LN(X)) + X, Y = MLP(LN(X^)) + X^).  READING: the pages
+ * do not say how two tensors of different scales are added; both are
+ * rescaled to the output scale with multipliers b1, b2 over a common 2^c,
+ * c = min of the two individual shifts.
+ */
+int orc_dyadic_pair(double s1, double s2, int32_t *b1, int32_t *b2, int32_t *c)
+{
+    int32_t bb1, cc1, bb2, cc2;
+    if (orc_dyadic(s1, &bb1, &cc1) != 0 || orc_dyadic(s2, &bb2, &cc2) != 0)
+        return -1;
+    int32_t cc = cc1 < cc2 ? cc1 : cc2;
+    *b1 = (int32_t)round(ldexp(s1, cc));
+    *b2 = (int32_t)round(ldexp(s2, cc));
+    *c = cc;
+    return 0;
+}
+
+/*
+ * I_0 of the shift-exponential, [IVIT] 3.3.  READING: the page's identity
+ * S_delta * [((-r) >> 1) + I_0] = S_delta * (-r) / 2 + 1 forces I_0 = 1 / S_delta;
+ * as an integer, round half away from zero, at least 1.
+ */
+int32_t orc_recip_i0(double S)
+{
+    double v = round(1.0 / S);
+    if (v < 1.0) v = 1.0;
+    if (v > 2147483647.0) v = 2147483647.0;
+    return (int32_t)v;
+}
+
+/* ------------------------------------------------------------------------ */
+/* dyadic requantisation, [IVIT] 3.2 / [TRIO] eq. (12)                      */
+/* ------------------------------------------------------------------------ */
+
+/*
+ * I_out = sat_bits((b * acc) >> c).  READING: the integer operation is the
+ * plain floor shift the page writes (not round-to-nearest), followed by
+ * saturation to the output width (the quantiser's clip).
+ */
+int64_t orc_requant(int64_t acc, int32_t b, int32_t c, int bits)
+{
+    return sat_bits(shr_floor((int64_t)b * acc, c), bits);
+}
+
+/* ------------------------------------------------------------------------ */
+/* INT8 linear layer with dyadic epilogue, [IVIT] 3.1-3.2, [TRIO] eq. (1)   */
+/* ------------------------------------------------------------------------ */
+
+/*
+ * Y[i, j] = sat_out((b_j * (sum_k X[i, k] * W[j, k] + bias_j)) >> c_j)
+ * X is [M x K] row-major, W is [N x K] row-major (one output channel per row),
+ * bias may be NULL.  If skip is non-NULL the residual addition follows:
+ *   Y[i, j] = sat_8((b_skip * skip[i, j] + b_branch * o_ij) >> c_res)
+ * where o_ij is the requantised linear output above.
+ */
+void orc_linear_requant(const int8_t *X, int64_t M, int32_t K,
+                        const int8_t *W, int32_t N,
+                        const int32_t *bias, const int32_t *b, const int32_t *c,
+                        int out_bits,
+                        const int8_t *skip, int32_t b_skip, int32_t b_branch,
+                        int32_t c_res, int8_t *Y)
+{
+    for (int64_t i = 0; i < M; ++i) {
+        for (int32_t j = 0; j < N; ++j) {
+            int64_t acc = 0;
+            for (int32_t k = 0; k < K; ++k)
+                acc += (int64_t)X[i * K + k] * (int64_t)W[(int64_t)j * K + k];
+            if (bias)
+                acc += bias[j];
+            int64_t o = orc_requant(acc, b[j], c[j], out_bits);
+            if (skip) {
+                int64_t s = skip[i * N + j];
+                o = sat_bits(shr_floor((int64_t)b_skip * s + (int64_t)b_branch * o,
+                                       c_res), 8);
+            }
+            Y[i * N + j] = (int8_t)o;
+        }
+    }
+}
+
+/* ------------------------------------------------------------------------ */
+/* Shiftmax, [IVIT] 3.3                                                     */
+/* ------------------------------------------------------------------------ */
+
+/*
+ * Shift-exponential of I_delta <= 0 with I_0 = 1/S_delta.
+ *   e^(S*I_delta) = 2^(S * I_delta * log2 e), and log2 e ~ 1.0111b, so
+ *   I_p = I_delta + (I_delta >> 1) - (I_delta >> 4).
+ *   S*I_p = -q + S*(-r): READING (the page garbles this step) q and r come
+ *   from floor division of -I_p by I_0, so q >= 0 and 0 <= r < I_0.
+ *   2^(S*(-r)) ~ 1 + S*(-r)/2 = S * (I_0 + ((-r) >> 1)), and 2^-q is a right
+ *   shift by q.  The result has scale S_delta.
+ */
+int64_t orc_shift_exp(int64_t I_delta, int64_t I0)
+{
+    int64_t I_p = I_delta + shr_floor(I_delta, 1) - shr_floor(I_delta, 4);
+    int64_t q = floor_div(-I_p, I0);
+    int64_t r = -I_p - q * I0;
+    int64_t t = I0 + shr_floor(-r, 1);
+    if (q > 62)
+        return 0;                 /* t < 2^62, so floor(t / 2^q) = 0 */
+    return shr_floor(t, (int)q);
+}
+
+/*
+ * IntDiv of [IVIT] 3.3: (floor(2^M / sum) * e) >> (M - (k_out - 1)); the
+ * result has scale 2^-(k_out - 1).
+ */
+int64_t orc_int_div(int64_t e, int64_t sum, int M, int k_out)
+{
+    int64_t Dv = floor_div((int64_t)1 << M, sum);
+    return shr_floor(Dv * e, M - (k_out - 1));
+}
+
+/*
+ * Shiftmax over one row of n integer logits L (scale S, I_0 = round(1/S)):
+ * subtract the row maximum, shift-exponential, row sum, IntDiv.
+ * P[j] in [0, 2^(k_out-1)], scale 2^-(k_out-1).
+ */
+void orc_shiftmax_row(const int32_t *L, int n, int32_t I0, int M, int k_out,
+                      int32_t *P)
+{
+    int32_t mx = L[0];
+    for (int j = 1; j < n; ++j)
+        if (L[j] > mx) mx = L[j];
+    int64_t sum = 0;
+    for (int j = 0; j < n; ++j)
+        sum += orc_shift_exp((int64_t)L[j] - mx, I0);
+    for (int j = 0; j < n; ++j)
+        P[j] = (int32_t)orc_int_div(orc_shift_exp((int64_t)L[j] - mx, I0), sum,
+                                    M, k_out);
+}
+
+/* ------------------------------------------------------------------------ */
+/* attention, [IVIT] 3.1-3.3 and [TRIO] eqs. (1)-(3)                        */
+/* ------------------------------------------------------------------------ */
+
+/*
+ * Multi-head self-attention core on a fused QKV tensor.
+ * QKV is [B*N x 3*H*64] row-major: columns [0, D) hold Q (head h at h*64),
+ * [D, 2D) hold K, [2D, 3D) hold V, D = H*64.  For every image, head and query:
+ *   S_ij  = sum_d Q_id K_jd                                (int32 product)
+ *   L_ij  = sat_{k_s}((b_s * S_ij) >> c_s)   b_s/2^c_s ~ S_q S_k / (sqrt(64) S_L)
+ *   P_i.  = Shiftmax(L_i., I_0, M, k_out)
+ *   ctx_id = sat_8((b_o * sum_j P_ij V_jd) >> c_o)  b_o/2^c_o ~ S_v 2^-(k_out-1) / S_ctx
+ * ctx is [B*N x D], heads concatenated in column order ([TRIO] eq. (3)).
+ */
+void orc_attention(const int8_t *QKV, int32_t B, int32_t N, int32_t H,
+                   int32_t b_s, int32_t c_s, int32_t k_s, int32_t I0,
+                   int32_t M, int32_t k_out, int32_t b_o, int32_t c_o,
+                   int8_t *ctx)
+{
+    const int64_t D = (int64_t)H * 64;
+    const int64_t ld = 3 * D;
+    int32_t *L = (int32_t *)malloc(sizeof(int32_t) * (size_t)N);
+    int32_t *P = (int32_t *)malloc(sizeof(int32_t) * (size_t)N);
+    for (int32_t bi = 0; bi < B; ++bi) {
+        const int8_t *base = QKV + (int64_t)bi * N * ld;
+        for (int32_t h = 0; h < H; ++h) {
+            for (int32_t i = 0; i < N; ++i) {
+                const int8_t *q = base + (int64_t)i * ld + h * 64;
+                for (int32_t j = 0; j < N; ++j) {
+                    const int8_t *k = base + (int64_t)j * ld + D + h * 64;
+                    int64_t s = 0;
+                    for (int d = 0; d < 64; ++d)
+                        s += (int64_t)q[d] * (int64_t)k[d];
+                    L[j] = (int32_t)orc_requant(s, b_s, c_s, k_s);
+                }
+                orc_shiftmax_row(L, N, I0, M, k_out, P);
+                int8_t *out = ctx + ((int64_t)bi * N + i) * D + h * 64;
+                for (int d = 0; d < 64; ++d) {
+                    int64_t acc = 0;
+                    for (int32_t j = 0; j < N; ++j)
+                        acc += (int64_t)P[j] *
+                               (int64_t)base[(int64_t)j * ld + 2 * D + h * 64 + d];
+                    out[d] = (int8_t)orc_requant(acc, b_o, c_o, 8);
+                }
+            }
+        }
+    }
+    free(L);
+    free(P);
+}
+
+/* ------------------------------------------------------------------------ */
+/* ShiftGELU, [IVIT] 3.4                                                    */
+/* ------------------------------------------------------------------------ */
+
+/*
+ * GELU(x) ~ x * sigmoid(1.702 x), 1.702 ~ 1.1011b:
+ *   I_p = I + (I >> 1) + (I >> 3) + (I >> 4).
+ * sigmoid(S I_p) = e^(S(I_p - I_max)) / (e^(S(I_p - I_max)) + e^(S(-I_max))),
+ * each exponential by the Shiftmax shift-exponential (with its log2 e step)
+ * and the quotient by IntDiv.  READING (the page stops mid-derivation and never
+ * defines I_max): I_max is the larger of the two exponents, max(I_p, 0), per
+ * element.  The product I * sigma_int has scale S * 2^-(k_out-1) and is
+ * requantised to 8 bits with (b_g, c_g).
+ */
+int64_t orc_shift_sigmoid(int64_t I_p, int64_t I0, int32_t M, int32_t k_out)
+{
+    int64_t I_max = I_p > 0 ? I_p : 0;
+    int64_t e1 = orc_shift_exp(I_p - I_max, I0);
+    int64_t e2 = orc_shift_exp(-I_max, I0);
+    return orc_int_div(e1, e1 + e2, M, k_out);
+}
+
+int32_t orc_shiftgelu_one(int32_t I, int32_t I0, int32_t M, int32_t k_out,
+                          int32_t b_g, int32_t c_g, int32_t *sigma_out)
+{
+    int64_t x = I;
+    int64_t I_p = x + shr_floor(x, 1) + shr_floor(x, 3) + shr_floor(x, 4);
+    int64_t sigma = orc_shift_sigmoid(I_p, I0, M, k_out);
+    if (sigma_out)
+        *sigma_out = (int32_t)sigma;
+    return (int32_t)orc_requant(x * sigma, b_g, c_g, 8);
+}
+
+void orc_shiftgelu(const int8_t *x, int64_t n, int32_t I0, int32_t M,
+                   int32_t k_out, int32_t b_g, int32_t c_g, int8_t *y)
+{
+    for (int64_t i = 0; i < n; ++i)
+        y[i] = (int8_t)orc_shiftgelu_one(x[i], I0, M, k_out, b_g, c_g, NULL);
+}
+
+/* ------------------------------------------------------------------------ */
+/* I-LayerNorm, [IVIT] 3.5                                                  */
+/* ------------------------------------------------------------------------ */
+
+/*
+ * Integer square root by Newton's iteration
+ *   I_{i+1} = (I_i + floor(V / I_i)) >> 1,  I_0 = 2^floor(bit(V) / 2),
+ * run for exactly 10 iterations (the page replaced the stopping rule by a
+ * fixed count).  READING: V = 0 would divide by zero at the second step; it
+ * returns 0 without iterating.
+ */
+int64_t orc_isqrt_newton(int64_t V)
+{
+    if (V <= 0)
+        return 0;
+    int64_t I = (int64_t)1 << (bit_length(V) / 2);
+    for (int it = 0; it < 10; ++it)
+        I = shr_floor(I + floor_div(V, I), 1);
+    return I;
+}
+
+/*
+ * One row of n int8 values:
+ *   mu = floor(sum x / n);  d_i = x_i - mu;  V = floor(sum d_i^2 / n)
+ *   sigma = max(isqrt(V), 1)         READING: no epsilon on the page
+ *   f = floor(2^M_ln / sigma);  n_i = (d_i * f) >> (M_ln - F)   (scale 2^-F)
+ *   acc_i = n_i * gamma_i + beta_i   (gamma int8 at S_gamma, beta int32 at S_gamma 2^-F)
+ *   y_i = sat_8((b * acc_i) >> c)
+ * READING: the page writes x - Mean over Var; the square root it then
+ * computes is what divides.  Mean/variance use floor division; F and M_ln are
+ * parameters.
+ */
+void orc_layernorm(const int8_t *x, int64_t rows, int32_t cols,
+                   const int8_t *gamma, const int32_t *beta,
+                   int32_t F, int32_t M_ln, int32_t b, int32_t c, int8_t *y)
+{
+    for (int64_t r = 0; r < rows; ++r) {
+        const int8_t *xr = x + r * cols;
+        int64_t sx = 0;
+        for (int32_t i = 0; i < cols; ++i)
+            sx += xr[i];
+        int64_t mu = floor_div(sx, cols);
+        int64_t sd2 = 0;
+        for (int32_t i = 0; i < cols; ++i) {
+            int64_t d = xr[i] - mu;
+            sd2 += d * d;
+        }
+        int64_t V = floor_div(sd2, cols);
+        int64_t sigma = orc_isqrt_newton(V);
+        if (sigma < 1)
+            sigma = 1;
+        int64_t f = floor_div((int64_t)1 << M_ln, sigma);
+        for (int32_t i = 0; i < cols; ++i) {
+            int64_t d = xr[i] - mu;
+            int64_t nv = shr_floor(d * f, M_ln - F);
+            int64_t acc = nv * gamma[i] + beta[i];
+            y[r * cols + i] = (int8_t)orc_requant(acc, b, c, 8);
+        }
+    }
+}
+
+/* ------------------------------------------------------------------------ */
+/* the encoder block, [IVIT] 3.1 (pre-LN, two residuals), [TRIO] eqs (1)-(3)*/
+/* ------------------------------------------------------------------------ */
+
+/* Integer parameters of one block.  All arrays are host memory. */
+typedef struct {
+    int32_t D, H, Dm;
+    /* I-LayerNorm 1 */
+    const int8_t *ln1_gamma; const int32_t *ln1_beta; int32_t ln1_b, ln1_c;
+    /* QKV linear: W [3D x D], per-output-channel (b, c) */
+    const int8_t *w_qkv; const int32_t *bias_qkv; const int32_t *b_qkv; const int32_t *c_qkv;
+    /* attention */
+    int32_t logit_b, logit_c, k_s, attn_I0, attn_M, attn_k_out, attn_out_b, attn_out_c;
+    /* output projection W^O [D x D] + residual 1 */
+    const int8_t *w_o; const int32_t *bias_o; const int32_t *b_o; const int32_t *c_o;
+    int32_t res1_b_skip, res1_b_branch, res1_c;
+    /* I-LayerNorm 2 */
+    const int8_t *ln2_gamma; const int32_t *ln2_beta; int32_t ln2_b, ln2_c;
+    /* fc1 [Dm x D] */
+    const int8_t *w1; const int32_t *bias1; const int32_t *b1; const int32_t *c1;
+    /* ShiftGELU */
+    int32_t gelu_I0, gelu_M, gelu_k_out, gelu_b, gelu_c;
+    /* fc2 [D x Dm] + residual 2 */
+    const int8_t *w2; const int32_t *bias2; const int32_t *b2; const int32_t *c2;
+    int32_t res2_b_skip, res2_b_branch, res2_c;
+    /* I-LayerNorm constants */
+    int32_t ln_F, ln_M;
+} orc_block_params;
+
+/*
+ * X^ = MSA(LN1(X)) + X;  Y = MLP(LN2(X^)) + X^   ([IVIT] 3.1)
+ * x, y: [B*N x D] int8.  Returns 0, or -1 if scratch allocation failed.
+ */
+int orc_block_forward(const orc_block_params *p, const int8_t *x, int8_t *y,
+                      int32_t B, int32_t N)
+{
+    const int64_t T = (int64_t)B * N;
+    const int32_t D = p->D, Dm = p->Dm;
+    int8_t *ln = (int8_t *)malloc((size_t)(T * D));
+    int8_t *qkv = (int8_t *)malloc((size_t)(T * 3 * D));
+    int8_t *ctx = (int8_t *)malloc((size_t)(T * D));
+    int8_t *xh = (int8_t *)malloc((size_t)(T * D));
+    int8_t *h = (int8_t *)malloc((size_t)(T * Dm));
+    int8_t *g = (int8_t *)malloc((size_t)(T * Dm));
+    if (!ln || !qkv || !ctx || !xh || !h || !g) {
+        free(ln); free(qkv); free(ctx); free(xh); free(h); free(g);
+        return -1;
+    }
+    /* a1: LN1 */
+    orc_layernorm(x, T, D, p->ln1_gamma, p->ln1_beta, p->ln_F, p->ln_M,
+                  p->ln1_b, p->ln1_c, ln);
+    /* a2: QKV */
+    orc_linear_requant(ln, T, D, p->w_qkv, 3 * D, p->bias_qkv, p->b_qkv, p->c_qkv,
+                       8, NULL, 0, 0, 0, qkv);
+    /* a3-a5: logits, Shiftmax, A.V */
+    orc_attention(qkv, B, N, p->H, p->logit_b, p->logit_c, p->k_s, p->attn_I0,
+                  p->attn_M, p->attn_k_out, p->attn_out_b, p->attn_out_c, ctx);
+    /* a6: W^O + residual 1 */
+    orc_linear_requant(ctx, T, D, p->w_o, D, p->bias_o, p->b_o, p->c_o, 8,
+                       x, p->res1_b_skip, p->res1_b_branch, p->res1_c, xh);
+    /* a7: LN2 */
+    orc_layernorm(xh, T, D, p->ln2_gamma, p->ln2_beta, p->ln_F, p->ln_M,
+                  p->ln2_b, p->ln2_c, ln);
+    /* a8: fc1 */
+    orc_linear_requant(ln, T, D, p->w1, Dm, p->bias1, p->b1, p->c1, 8,
+                       NULL, 0, 0, 0, h);
+    /* a9: ShiftGELU */
+    orc_shiftgelu(h, T * Dm, p->gelu_I0, p->gelu_M, p->gelu_k_out, p->gelu_b,
+                  p->gelu_c, g);
+    /* a10: fc2 + residual 2 */
+    orc_linear_requant(g, T, Dm, p->w2, D, p->bias2, p->b2, p->c2, 8,
+                       xh, p->res2_b_skip, p->res2_b_branch, p->res2_c, y);
+    free(ln); free(qkv); free(ctx); free(xh); free(h); free(g);
+    return 0;
+}

@@ -1,0 +1,459 @@
+"""Pins of the CPU oracle against what the pages and mathematics fix.
+
+Each test checks the oracle against something other than itself: a worked
+example derived by hand from the formulas (tests/golden), a closed-form bound,
+an invariant, or a special case that reduces to a textbook routine (numpy
+integer matmul, math.isqrt, argmax, floor division).  Sources: "I-ViT:
+Integer-only Quantization for Efficient Vision Transformer Inference",
+sections 3.1-3.5, and the Trio-ViT article, eqs. (1)-(3) and (12).
+"""
+import math
+import os
+
+import numpy as np
+import pytest
+
+import oracle
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _kv(name):
+    out = {}
+    with open(os.path.join(GOLDEN, name)) as f:
+        for line in f:
+            line = line.strip()
+            if not line or line.startswith("#"):
+                continue
+            k, *v = line.split()
+            out[k] = [int(t) for t in v]
+    return out
+
+
+# --------------------------------------------------------------------------
+# quantiser (section 3.1)
+# --------------------------------------------------------------------------
+
+def test_quantizer_endpoints_and_grid():
+    m = 3.0
+    S = 2 * m / 255
+    assert oracle.quantize(m, m) == 127            # 127.5 -> narrow range
+    assert oracle.quantize(-m, m) == -127
+    assert oracle.quantize(10 * m, m) == 127       # clip
+    assert oracle.quantize(0.0, m) == 0
+    for k in (-100, -3, 1, 77, 126):
+        assert oracle.quantize(k * S, m) == k      # exact grid points
+    assert oracle.quantize(2.5 * S, m) == 3        # half away from zero
+    assert oracle.quantize(-2.5 * S, m) == -3
+
+
+# --------------------------------------------------------------------------
+# dyadic numbers (section 3.2, Trio-ViT eq. 12)
+# --------------------------------------------------------------------------
+
+def test_dyadic_closed_form_bound():
+    r = np.random.default_rng(1)
+    for s in np.exp(r.uniform(math.log(2.0 ** -20), math.log(2.0 ** 8), size=20000)):
+        b, c = oracle.dyadic(s)
+        assert 0 <= c <= 31 and 0 <= b < 2 ** 31
+        assert abs(b / 2.0 ** c - s) <= 2.0 ** -(c + 1) * (1 + 1e-12)
+        # c is maximal: one more bit of shift would overflow int32
+        if c < 31:
+            assert round(s * 2.0 ** (c + 1)) >= 2 ** 31
+
+
+def test_dyadic_exact_values():
+    assert oracle.dyadic(0.5) == (2 ** 30, 31)
+    assert oracle.dyadic(1.0) == (2 ** 30, 30)
+    assert oracle.dyadic(0.0) == (0, 31)
+    assert oracle.dyadic(3.0) == (3 * 2 ** 29, 29)
+    with pytest.raises(ValueError):
+        oracle.dyadic(-1.0)
+    with pytest.raises(ValueError):
+        oracle.dyadic(2.0 ** 32)
+
+
+def test_dyadic_pair_common_shift():
+    r = np.random.default_rng(2)
+    for _ in range(2000):
+        s1, s2 = np.exp(r.uniform(-6, 3, size=2))
+        b1, b2, c = oracle.dyadic_pair(s1, s2)
+        assert c == min(oracle.dyadic(s1)[1], oracle.dyadic(s2)[1])
+        assert 0 <= b1 < 2 ** 31 and 0 <= b2 < 2 ** 31
+        assert abs(b1 / 2.0 ** c - s1) <= 2.0 ** -(c + 1) * (1 + 1e-12)
+        assert abs(b2 / 2.0 ** c - s2) <= 2.0 ** -(c + 1) * (1 + 1e-12)
+
+
+def test_recip_i0():
+    assert oracle.recip_i0(8 / 127) == 16
+    assert oracle.recip_i0(0.05) == 20
+    assert oracle.recip_i0(10.0) == 1            # at least 1
+    assert oracle.recip_i0(1 / 2.5) == 3         # half away from zero
+
+
+# --------------------------------------------------------------------------
+# requantisation (section 3.2)
+# --------------------------------------------------------------------------
+
+def test_requant_floor_and_saturation():
+    assert oracle.requant(-1, 1, 1) == -1         # floor(-0.5) = -1, not 0
+    assert oracle.requant(1, 1, 1) == 0
+    assert oracle.requant(-3, 1, 1) == -2
+    assert oracle.requant(1000, 1, 0) == 127
+    assert oracle.requant(-1000, 1, 0) == -128
+    assert oracle.requant(300, 3, 3) == 112       # floor(900 / 8)
+    for c in range(0, 31, 5):
+        for v in (-128, -77, -1, 0, 5, 127):
+            assert oracle.requant(v, 2 ** c, c) == v     # b = 2^c: identity on int8
+
+
+def test_linear_requant_reduces_to_integer_matmul():
+    r = np.random.default_rng(3)
+    M, K, N = 37, 80, 48                          # non-square: a transposed W fails
+    X = r.integers(-128, 128, size=(M, K), dtype=np.int8)
+    W = r.integers(-128, 128, size=(N, K), dtype=np.int8)
+    bias = r.integers(-5000, 5000, size=N).astype(np.int32)
+    acc = X.astype(np.int64) @ W.astype(np.int64).T + bias
+    # b = 1, c = j % 5: floor division of the exact integer matmul by 2^c_j
+    b = np.ones(N, np.int32)
+    c = (np.arange(N) % 5).astype(np.int32)
+    want = np.clip(np.floor_divide(acc, (2 ** c)[None, :]), -128, 127)
+    got = oracle.linear_requant(X, W, bias, b, c)
+    np.testing.assert_array_equal(got, want)
+    # narrower output width saturates to it
+    got4 = oracle.linear_requant(X, W, bias, b, c, out_bits=4)
+    np.testing.assert_array_equal(got4, np.clip(np.floor_divide(acc, (2 ** c)[None, :]), -8, 7))
+    # residual with unit multipliers is a saturated int8 add
+    skip = r.integers(-128, 128, size=(M, N), dtype=np.int8)
+    got_r = oracle.linear_requant(X, W, bias, b, c, skip=skip, res=(1, 1, 0))
+    np.testing.assert_array_equal(got_r, np.clip(skip.astype(np.int64) + want, -128, 127))
+
+
+def test_linear_requant_no_bias():
+    r = np.random.default_rng(4)
+    X = r.integers(-128, 128, size=(5, 16), dtype=np.int8)
+    W = r.integers(-128, 128, size=(7, 16), dtype=np.int8)
+    acc = X.astype(np.int64) @ W.astype(np.int64).T
+    got = oracle.linear_requant(X, W, None, np.full(7, 1, np.int32), np.full(7, 10, np.int32))
+    np.testing.assert_array_equal(got, np.clip(np.floor_divide(acc, 1024), -128, 127))
+
+
+# --------------------------------------------------------------------------
+# shift-exponential and Shiftmax (section 3.3)
+# --------------------------------------------------------------------------
+
+def test_shift_exp_zero_and_monotone():
+    for I0 in (1, 2, 5, 13, 16, 20, 64, 1000, 40000):
+        assert oracle.shift_exp(0, I0) == I0     # 2^0 = 1 at scale 1/I0
+        prev = None
+        for d in range(-min(16 * I0, 6000), 1):
+            e = oracle.shift_exp(d, I0)
+            assert e >= 0
+            if prev is not None:
+                assert e >= prev                  # non-decreasing in I_delta
+            prev = e
+
+
+def test_shift_exp_error_bound():
+    """|I_exp/I0 - e^x| within the bound that the approximation steps imply.
+
+    x = I_delta / I0.  log2 e ~ 1.4375 over-estimates e^x by 2^(0.005195 |x|);
+    the two floors in I_p move the exponent by < 1 LSB either way (2^(+-1/I0));
+    the linear 2^-f ~ 1 - f/2 is high by at most 6.16 %; the final floors lose
+    at most 1.5 LSB.
+    """
+    for I0 in (16, 20, 50, 128, 1000):
+        for d in range(-8 * I0, 1):
+            x = d / I0
+            e = oracle.shift_exp(d, I0) / I0
+            hi = math.exp(x) * 2 ** (0.005195 * abs(x) + 1 / I0) * 1.0616
+            lo = math.exp(x) * 2 ** (-1 / I0) - 1.5 / I0
+            assert lo <= e <= hi, (I0, d, e, math.exp(x))
+
+
+def test_shiftmax_worked_example():
+    g = _kv("shiftmax_worked_example.txt")
+    I0, M, k_out = g["I0"][0], g["M"][0], g["k_out"][0]
+    for L, ie in zip(g["L"], g["I_exp"]):
+        assert oracle.shift_exp(L - max(g["L"]), I0) == ie
+    assert sum(g["I_exp"]) == g["sum"][0]
+    P = oracle.shiftmax_row(g["L"], I0, M, k_out)
+    assert list(P) == g["P"]
+    for e, p in zip(g["I_exp"], g["P"]):
+        assert oracle.int_div(e, g["sum"][0], M, k_out) == p
+
+
+def test_shiftmax_bounds_and_special_cases():
+    r = np.random.default_rng(5)
+    for _ in range(3000):
+        n = int(r.integers(1, 200))
+        I0 = int(r.integers(1, 300))
+        L = r.integers(-128, 128, size=n)
+        P = oracle.shiftmax_row(L, I0)
+        assert P.min() >= 0 and P.max() <= 128
+        assert P.sum() <= 128                     # floor(2^M / sum) * sum <= 2^M
+        # shift invariance: only differences to the row max matter
+        c = int(r.integers(-50, 50))
+        np.testing.assert_array_equal(oracle.shiftmax_row(L + c, I0), P)
+    # one key: P = floor(floor(2^30 / I0) * I0 / 2^23), i.e. 128 only when I0
+    # divides 2^30; floor(2^30 / 9) * 9 = 2^30 - 1 gives 127
+    assert list(oracle.shiftmax_row([17], 16)) == [128]
+    assert list(oracle.shiftmax_row([17], 9)) == [127]
+    # two equal keys: 64 for I0 = 32; floor(2^30 / 40) * 20 = 2^29 - 12 gives 63
+    assert list(oracle.shiftmax_row([-3, -3], 32)) == [64, 64]
+    assert list(oracle.shiftmax_row([-3, -3], 20)) == [63, 63]
+    assert list(oracle.shiftmax_row([0] * 4, 8)) == [32] * 4
+    assert list(oracle.shiftmax_row([0] * 4, 7)) == [31] * 4
+
+
+def test_shiftmax_hardmax_special_case():
+    """I_0 = 1: every non-maximal key gets I_exp = 0, so Shiftmax is a hard max
+    that splits 2^(k_out-1) evenly (floor) among the arg-max keys."""
+    r = np.random.default_rng(6)
+    for _ in range(500):
+        L = r.integers(-10, 10, size=int(r.integers(1, 50)))
+        P = oracle.shiftmax_row(L, 1)
+        cnt = int(np.sum(L == L.max()))
+        want = np.where(L == L.max(), 128 // cnt, 0)
+        np.testing.assert_array_equal(P, want)
+
+
+def test_shiftmax_fp_error(capsys):
+    """FP check of Shiftmax against softmax of the dequantised logits.
+
+    Fine resolution (I_0 = 4096, 16-bit logits): every shift-exponential term
+    is within [-1/I_0 exponent LSB, +6.16 % linear step + 3 % log2 e error at
+    |x| <= 8] of e^x, and loses at most 1.5 LSB to floors, so
+    |P - softmax| <= (0.0935 + 1.5 N / I_0) * max softmax + 1/128 per row.
+    Coarse resolution (I_0 < 64, 8-bit logits) is reported only: terms below
+    1/I_0 of the row maximum floor to zero there by construction.
+    """
+    r = np.random.default_rng(7)
+    N = 197
+    for I0, lim, check in ((4096, 32767, True), (19, 127, False)):
+        worst = 0.0
+        for _ in range(150):
+            L = np.round(r.laplace(0, 1.0, size=N) * I0).clip(-lim - 1, lim).astype(np.int64)
+            x = L / I0
+            keep = x >= x.max() - 8
+            P = oracle.shiftmax_row(L, I0) / 128.0
+            sm = np.exp(x - x.max())
+            sm /= sm.sum()
+            err = np.abs(P - sm)
+            worst = max(worst, float(err.max()))
+            if check:
+                bound = (0.0935 + 1.5 * N / I0) * sm.max() + 1 / 128
+                assert err[keep].max() <= bound, (err.max(), bound)
+        with capsys.disabled():
+            print(f"\n[fp report] Shiftmax max |P - softmax| at I0={I0}: {worst:.4f}")
+
+
+# --------------------------------------------------------------------------
+# ShiftGELU (section 3.4)
+# --------------------------------------------------------------------------
+
+def test_shiftgelu_worked_example():
+    g = _kv("shiftgelu_worked_example.txt")
+    I0, M, k_out = g["I0"][0], g["M"][0], g["k_out"][0]
+    assert oracle.recip_i0(8 / 127) == I0
+    for x, e1, e2, s in zip(g["x"], g["e1"], g["e2"], g["sigma"]):
+        Ip = g["I_p"][g["x"].index(x)]
+        m = max(Ip, 0)
+        assert oracle.shift_exp(Ip - m, I0) == e1
+        assert oracle.shift_exp(-m, I0) == e2
+        _, sig = oracle.shiftgelu_one(x, I0, M, k_out)
+        assert sig == s
+        assert oracle.shift_sigmoid(Ip, I0, M, k_out) == s
+
+
+def test_shift_sigmoid_symmetry():
+    """sigma(I_p) + sigma(-I_p) in [126, 128]: both share the denominator
+    ShiftExp(-|I_p|) + I_0, and each IntDiv floors once."""
+    for I0 in (1, 2, 5, 13, 16, 64, 1000, 40000):
+        for Ip in range(0, 401):
+            s = oracle.shift_sigmoid(Ip, I0) + oracle.shift_sigmoid(-Ip, I0)
+            assert 126 <= s <= 128, (I0, Ip, s)
+
+
+def test_shiftgelu_exhaustive_properties():
+    for I0 in (2, 5, 13, 16, 25, 64):
+        sig_prev = -1
+        for x in range(-128, 128):
+            g, sig = oracle.shiftgelu_one(x, I0, 30, 8, 1, 0)
+            assert 0 <= sig <= 128
+            assert sig >= sig_prev                # sigmoid non-decreasing in x
+            sig_prev = sig
+            # b = 1, c = 0: the requant is a plain int8 saturation of x * sigma
+            assert g == max(-128, min(127, x * sig))
+        assert oracle.shiftgelu_one(0, I0)[0] == 0
+    # large positive x: e2 underflows to 0, sigma = 128 exactly, out = 128 x
+    _, sig = oracle.shiftgelu_one(127, 2)
+    assert sig == 128
+    # large negative x: e1 underflows to 0
+    _, sig = oracle.shiftgelu_one(-127, 2)
+    assert sig == 0
+
+
+def test_shiftgelu_close_to_gelu():
+    """Reported FP check over all 256 inputs against x * Phi(x)."""
+    for S in (8 / 127, 4 / 127, 12 / 127):
+        I0 = oracle.recip_i0(S)
+        worst = 0.0
+        for x in range(-128, 128):
+            _, sig = oracle.shiftgelu_one(x, I0)
+            approx = x * S * sig / 128.0
+            exact = x * S * 0.5 * (1 + math.erf(x * S / math.sqrt(2)))
+            worst = max(worst, abs(approx - exact))
+        assert worst < 0.25, (S, worst)
+
+
+# --------------------------------------------------------------------------
+# I-LayerNorm (section 3.5)
+# --------------------------------------------------------------------------
+
+def test_isqrt_golden_cases():
+    with open(os.path.join(GOLDEN, "isqrt_cases.txt")) as f:
+        for line in f:
+            if line.strip() and not line.startswith("#"):
+                V, want = (int(t) for t in line.split())
+                assert oracle.isqrt_newton(V) == want, V
+
+
+def test_isqrt_against_textbook():
+    for V in range(1, 1 << 16):
+        s = math.isqrt(V)
+        assert oracle.isqrt_newton(V) in (s, s + 1), V
+    r = np.random.default_rng(8)
+    for V in r.integers(1, 2 ** 31, size=20000):
+        s = math.isqrt(int(V))
+        assert oracle.isqrt_newton(int(V)) in (s, s + 1)
+    for k in range(1, 31):                      # perfect squares are exact
+        assert oracle.isqrt_newton(k * k) == k
+
+
+def test_layernorm_hand_cases():
+    one = np.array([1], np.int8)
+    zero = np.array([0], np.int32)
+    # floor (not truncating) mean: [-1, 0, 0] -> mu = -1, d = [0, 1, 1], V = 0,
+    # sigma = 1, n = d * 2^23 >> 16 = 128 d -> saturates to 127
+    y = oracle.layernorm(np.array([[-1, 0, 0]], np.int8), np.ones(3, np.int8), np.zeros(3, np.int32), 7, 23, (1, 0))
+    assert list(y[0]) == [0, 127, 127]
+    # constant row: d = 0, so y = requant(beta)
+    beta = np.array([100, -300, 5, 0], np.int32)
+    y = oracle.layernorm(np.full((1, 4), 42, np.int8), np.full(4, 3, np.int8), beta, 7, 23, (1, 2))
+    assert list(y[0]) == [25, -75, 1, 0]
+    # a single column behaves the same
+    y = oracle.layernorm(np.array([[-7]], np.int8), one, np.array([64], np.int32), 7, 23, (1, 0))
+    assert list(y[0]) == [64]
+    # symmetric row: mu exact, V = 16, sigma = 4, n = d * 2^21 >> 16 = 32 d
+    y = oracle.layernorm(np.array([[-4, 4, -4, 4]], np.int8), np.ones(4, np.int8), np.zeros(4, np.int32), 7, 23,
+                         (1, 1))
+    assert list(y[0]) == [-64, 64, -64, 64]
+
+
+def test_layernorm_close_to_float():
+    """Reported FP check: dequantised output vs float LayerNorm."""
+    r = np.random.default_rng(9)
+    x = r.integers(-100, 100, size=(64, 192)).astype(np.int8)
+    gamma = np.full(192, 64, np.int8)            # S_gamma = 1/64
+    beta = np.zeros(192, np.int32)
+    # b/2^c = S_gamma 2^-7 / S_out with S_out = 4/127
+    b, c = oracle.dyadic((1 / 64) * 2 ** -7 / (4 / 127))
+    y = oracle.layernorm(x, gamma, beta, 7, 23, (b, c)) * (4 / 127)
+    xf = x.astype(np.float64)
+    ref = (xf - xf.mean(1, keepdims=True)) / xf.std(1, keepdims=True)
+    assert np.max(np.abs(y - ref)) < 0.1
+
+
+# --------------------------------------------------------------------------
+# attention (sections 3.1-3.3, Trio-ViT eqs. 1-3)
+# --------------------------------------------------------------------------
+
+def _qkv(r, B, N, H, lo=-128, hi=128):
+    return r.integers(lo, hi, size=(B * N, 3 * H * 64), dtype=np.int8)
+
+
+def test_attention_single_key():
+    r = np.random.default_rng(10)
+    qkv = _qkv(r, 3, 1, 2)
+    for I0 in (16, 17):
+        ctx = oracle.attention(qkv, 3, 1, 2, (123, 20), 8, I0, 30, 8, (1, 3))
+        p = ((2 ** 30) // I0) * I0 // 2 ** 23          # IntDiv of a single term: 128, 127
+        v = qkv[:, 2 * 128:].astype(np.int64)
+        np.testing.assert_array_equal(ctx, np.clip(np.floor_divide(p * v, 8), -128, 127))
+
+
+def test_attention_uniform_when_logits_equal():
+    r = np.random.default_rng(11)
+    B, N, H, I0 = 2, 23, 3, 29
+    qkv = _qkv(r, B, N, H)
+    ctx = oracle.attention(qkv, B, N, H, (0, 0), 8, I0, 30, 8, (1, 5))   # b_s = 0: all logits 0
+    p = ((2 ** 30) // (N * I0)) * I0 // 2 ** 23
+    D = H * 64
+    v = qkv[:, 2 * D:].astype(np.int64).reshape(B, N, D)
+    want = np.clip(np.floor_divide(p * v.sum(1, keepdims=True), 32), -128, 127)
+    np.testing.assert_array_equal(ctx.reshape(B, N, D), np.broadcast_to(want, (B, N, D)))
+
+
+def test_attention_hardmax_reduces_to_argmax():
+    """I_0 = 1 and (b_s, c_s) = (1, 0): L = clip(Q K^T), P = hard max; the
+    context is floor(128 / #argmax) * (sum of V over the arg-max keys)."""
+    r = np.random.default_rng(12)
+    B, N, H = 2, 19, 2
+    D = H * 64
+    qkv = _qkv(r, B, N, H, -3, 4)
+    for k_s in (8, 4):
+        ctx = oracle.attention(qkv, B, N, H, (1, 0), k_s, 1, 30, 8, (1, 4))
+        lim = 2 ** (k_s - 1)
+        for b in range(B):
+            rows = slice(b * N, (b + 1) * N)
+            for h in range(H):
+                q = qkv[rows, h * 64:(h + 1) * 64].astype(np.int64)
+                k = qkv[rows, D + h * 64:D + (h + 1) * 64].astype(np.int64)
+                v = qkv[rows, 2 * D + h * 64:2 * D + (h + 1) * 64].astype(np.int64)
+                L = np.clip(q @ k.T, -lim, lim - 1)
+                for i in range(N):
+                    am = L[i] == L[i].max()
+                    acc = (128 // int(am.sum())) * v[am].sum(0)
+                    want = np.clip(np.floor_divide(acc, 16), -128, 127)
+                    np.testing.assert_array_equal(ctx[b * N + i, h * 64:(h + 1) * 64], want)
+
+
+# --------------------------------------------------------------------------
+# block (section 3.1)
+# --------------------------------------------------------------------------
+
+def test_block_residual_identity():
+    """With zero output projections (W^O, W_2 and their biases) and unit skip
+    multipliers, both residual additions return their skip input: Y = X."""
+    import synthetic
+    wl = synthetic.make_workload(B=2, N=9, D=128, H=2, Dm=256, seed=3, n_cal=2)
+    p = oracle.block_params(wl.blocks[0])
+    p["w_o"] = np.zeros_like(p["w_o"]); p["bias_o"] = np.zeros_like(p["bias_o"])
+    p["w2"] = np.zeros_like(p["w2"]); p["bias2"] = np.zeros_like(p["bias2"])
+    p["res1"] = (1, 12345, 0)
+    p["res2"] = (1, 777, 0)
+    # zero accumulators requantise to 0, so the branch adds nothing
+    y = oracle.block_forward(p, wl.x, 2, 9)
+    np.testing.assert_array_equal(y, wl.x)
+
+
+def test_block_is_composition_of_ops():
+    """Consistency (not an independent pin): the block equals the chain of the
+    individually pinned operators in the order of section 3.1."""
+    import synthetic
+    B, N = 2, 13
+    wl = synthetic.make_workload(B=B, N=N, D=128, H=2, Dm=256, seed=4, n_cal=2)
+    p = oracle.block_params(wl.blocks[0])
+    x = wl.x
+    ln1 = oracle.layernorm(x, p["ln1_gamma"], p["ln1_beta"], 7, 23, p["ln1_out"])
+    qkv = oracle.linear_requant(ln1, p["w_qkv"], p["bias_qkv"], p["b_qkv"], p["c_qkv"])
+    ctx = oracle.attention(qkv, B, N, 2, p["logit"], 8, p["attn_I0"], 30, 8, p["attn_out"])
+    xh = oracle.linear_requant(ctx, p["w_o"], p["bias_o"], p["b_o"], p["c_o"], skip=x, res=p["res1"])
+    ln2 = oracle.layernorm(xh, p["ln2_gamma"], p["ln2_beta"], 7, 23, p["ln2_out"])
+    h = oracle.linear_requant(ln2, p["w1"], p["bias1"], p["b1"], p["c1"])
+    g = oracle.shiftgelu(h, p["gelu_I0"], 30, 8, p["gelu_out"])
+    y = oracle.linear_requant(g, p["w2"], p["bias2"], p["b2"], p["c2"], skip=xh, res=p["res2"])
+    np.testing.assert_array_equal(oracle.block_forward(p, x, B, N), y)
+    # the calibrated block is not degenerate: outputs use the int8 range
+    assert np.unique(y).size > 50 and np.unique(g).size > 20 and np.unique(ctx).size > 50
