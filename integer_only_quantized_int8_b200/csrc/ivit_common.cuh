@@ -1,0 +1,230 @@
+// ivit_common.cuh -- sm_100a building blocks shared by the integer ViT kernels:
+// mbarrier / TMA / tcgen05 (TMEM, UMMA) wrappers in inline PTX, bounded waits,
+// and the integer helpers of the method (dyadic requant, shift-exponential).
+//
+// Method sources: "I-ViT: Integer-only Quantization for Efficient Vision
+// Transformer Inference", sections 3.2 (dyadic arithmetic), 3.3 (Shiftmax),
+// 3.4 (ShiftGELU), 3.5 (I-LayerNorm); the Trio-ViT article, eq. (12).
+#pragma once
+
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include "../../include/ivit.h"
+
+#define IVIT_DEV __device__ __forceinline__
+
+namespace ivit {
+
+// ---------------------------------------------------------------------------
+// device status word (bounded waits report here instead of hanging)
+// ---------------------------------------------------------------------------
+enum : int { kStatusOk = 0, kStatusTimeout = 1 };
+
+// Wait budget in nanoseconds of %globaltimer: far above any legitimate wait in
+// these kernels (each finishes in well under a millisecond), far below a hang.
+constexpr uint64_t kWaitBudgetNs = 1000ull * 1000ull * 1000ull;   // 1 s
+
+IVIT_DEV uint64_t globaltimer_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+IVIT_DEV void report_timeout(int* status) {
+  if (status) atomicExch(status, kStatusTimeout);
+}
+
+// ---------------------------------------------------------------------------
+// shared-memory addresses and mbarriers
+// ---------------------------------------------------------------------------
+IVIT_DEV uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+IVIT_DEV void mbar_init(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
+}
+
+// make barrier initialisation visible to the async proxy (TMA, tensor core)
+IVIT_DEV void fence_barrier_init() {
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+IVIT_DEV void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+IVIT_DEV void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
+               : "memory");
+}
+
+IVIT_DEV void mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+IVIT_DEV bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Wait until the phase with the given parity has completed.  Gives up after
+// kWaitBudgetNs, records a timeout in *status and returns false.
+IVIT_DEV bool mbar_wait(uint64_t* bar, uint32_t parity, int* status) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  while (true) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if (globaltimer_ns() - t0 > kWaitBudgetNs) {
+      report_timeout(status);
+      return false;
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// TMA (cp.async.bulk.tensor), no multicast
+// ---------------------------------------------------------------------------
+IVIT_DEV void tma_load_2d(void* smem_dst, const CUtensorMap* map, int32_t x, int32_t y, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::"r"(
+          smem_u32(smem_dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_u32(bar))
+      : "memory");
+}
+
+IVIT_DEV void prefetch_tensormap(const CUtensorMap* map) {
+  asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
+}
+
+// ---------------------------------------------------------------------------
+// tcgen05: TMEM allocation, UMMA issue/commit, TMEM loads
+// ---------------------------------------------------------------------------
+// whole warp; writes the TMEM base address into *slot (shared memory)
+IVIT_DEV void tmem_alloc(uint32_t* slot, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(slot)),
+               "r"(ncols)
+               : "memory");
+}
+IVIT_DEV void tmem_relinquish() {
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+IVIT_DEV void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+IVIT_DEV void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+IVIT_DEV void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+// D[tmem] (+)= A[smem] * B[smem]^T, kind::i8, int32 accumulate; single thread.
+IVIT_DEV void umma_i8(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::i8 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// arrive on *bar once all previously issued tcgen05.mma of this thread complete
+IVIT_DEV void umma_commit(uint64_t* bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
+               : "memory");
+}
+
+// Instruction descriptor of tcgen05.mma kind::i8 (int32 accumulator):
+// bits 4-5 D format (2 = s32), 7-9 A format, 10-12 B format (1 = signed,
+// 0 = unsigned 8-bit), 15 / 16 A / B major (0 = K-major, 1 = MN-major),
+// 17-22 N >> 3, 24-28 M >> 4.
+__host__ __device__ constexpr uint32_t idesc_i8(int M, int N, bool a_signed, bool b_signed, bool b_mn_major) {
+  return (2u << 4) | ((a_signed ? 1u : 0u) << 7) | ((b_signed ? 1u : 0u) << 10) |
+         ((b_mn_major ? 1u : 0u) << 16) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+
+// Shared-memory matrix descriptor (sm_100 format): start address >> 4 in bits
+// 0-13, leading-dimension byte offset >> 4 in 16-29, stride-dimension byte
+// offset >> 4 in 32-45, version 1 in 46-47, layout (swizzle) in 61-63.
+enum : uint32_t { kSwizzleNone = 0, kSwizzle128B = 2, kSwizzle64B = 4, kSwizzle32B = 6 };
+
+IVIT_DEV uint64_t smem_desc(uint32_t saddr, uint32_t lbo_bytes, uint32_t sbo_bytes, uint32_t layout) {
+  return (uint64_t)((saddr >> 4) & 0x3FFFu) | ((uint64_t)((lbo_bytes >> 4) & 0x3FFFu) << 16) |
+         ((uint64_t)((sbo_bytes >> 4) & 0x3FFFu) << 32) | (1ull << 46) | ((uint64_t)layout << 61);
+}
+
+// 32 lanes x 32 consecutive 32-bit columns: thread i of the warp receives
+// lane (base lane + i), columns [col, col + 32).
+IVIT_DEV void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
+      "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+        "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+        "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr)
+      : "memory");
+}
+IVIT_DEV void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+
+// ---------------------------------------------------------------------------
+// integer arithmetic of the method
+// ---------------------------------------------------------------------------
+
+// sat_8((b * v) >> c), b >= 0, 0 <= c <= 31, with >> an arithmetic (floor) shift
+IVIT_DEV int32_t requant8(int32_t v, int32_t b, int32_t c) {
+  const int64_t p = (int64_t)b * (int64_t)v;
+  const int64_t q = p >> c;
+  return (int32_t)(q < -128 ? -128 : (q > 127 ? 127 : q));
+}
+
+IVIT_DEV int32_t requant_bits(int32_t v, int32_t b, int32_t c, int32_t lo, int32_t hi) {
+  const int64_t q = ((int64_t)b * (int64_t)v) >> c;
+  return (int32_t)(q < lo ? lo : (q > hi ? hi : q));
+}
+
+// Residual addition of two int8 tensors on a common shift:
+// sat_8((b_skip * skip + b_branch * branch) >> c)
+IVIT_DEV int32_t residual8(int32_t skip, int32_t branch, int32_t b_skip, int32_t b_branch, int32_t c) {
+  const int64_t q = ((int64_t)b_skip * skip + (int64_t)b_branch * branch) >> c;
+  return (int32_t)(q < -128 ? -128 : (q > 127 ? 127 : q));
+}
+
+// Shift-exponential of d <= 0 at scale 1/I0 (I-ViT section 3.3):
+// log2 e ~ 1.0111b (d + d/2 - d/16, floor shifts); -I_p = q I0 + r with
+// 0 <= r < I0; 2^(-r/I0) ~ 1 - r/(2 I0); then a right shift by q.
+IVIT_DEV int32_t shift_exp(int32_t d, int32_t I0) {
+  const int32_t ip = d + (d >> 1) - (d >> 4);
+  const int32_t neg = -ip;                       // >= 0
+  const int32_t q = neg / I0;                    // non-negative operands: truncation == floor
+  const int32_t r = neg - q * I0;
+  const int32_t t = I0 - ((r + 1) >> 1);         // I0 + floor(-r / 2)
+  return q >= 31 ? 0 : (t >> q);
+}
+
+// Integer sigmoid of S * I_p as a two-term Shiftmax (I-ViT section 3.4),
+// exponent offset max(I_p, 0); result scale 2^-(k_out - 1).
+IVIT_DEV int32_t shift_sigmoid(int32_t ip, int32_t I0, int32_t M, int32_t k_out) {
+  const int32_t m = ip > 0 ? ip : 0;
+  const int32_t e1 = shift_exp(ip - m, I0);
+  const int32_t e2 = shift_exp(-m, I0);
+  const uint32_t dv = (1u << M) / (uint32_t)(e1 + e2);
+  return (int32_t)((dv * (uint32_t)e1) >> (M - (k_out - 1)));
+}
+
+// ShiftGELU of one int8 input: x * sigma(1.1011b * x), requantised to int8.
+IVIT_DEV int32_t shiftgelu8(int32_t x, int32_t I0, int32_t M, int32_t k_out, int32_t b, int32_t c) {
+  const int32_t ip = x + (x >> 1) + (x >> 3) + (x >> 4);
+  const int32_t sig = shift_sigmoid(ip, I0, M, k_out);
+  return requant8(x * sig, b, c);
+}
+
+}  // namespace ivit

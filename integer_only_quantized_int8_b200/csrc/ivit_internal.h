@@ -1,0 +1,50 @@
+// ivit_internal.h -- launchers shared between the operator files and the C ABI.
+#pragma once
+
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include "../../include/ivit.h"
+
+namespace ivit {
+
+enum EpiMode : int { kEpiPlain = 0, kEpiResidual = 1, kEpiGelu = 2 };
+
+struct GeluParams {
+  int32_t I0, M, k_out;
+  ivit_dyadic out;
+};
+
+// Per-device context: SM count, the status word's device address.
+struct DeviceCtx {
+  int device;
+  int num_sms;
+  int* status;
+};
+ivit_status device_ctx(DeviceCtx* out);
+
+// Count a kernel launch (for ivit_launch_count).
+void note_launch(int n = 1);
+
+ivit_status encode_tmap_2d_u8(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer,
+                              uint64_t row_stride_bytes, uint32_t box_inner, uint32_t box_outer,
+                              CUtensorMapSwizzle swizzle);
+
+ivit_status launch_gemm(const DeviceCtx& dc, const int8_t* X, int64_t M, int32_t K, const int8_t* W, int32_t N,
+                        const int32_t* bias, const int32_t* b, const int8_t* c, int32_t out_bits, EpiMode mode,
+                        const int8_t* skip, ivit_residual res, const GeluParams* gelu, int8_t* Y,
+                        cudaStream_t stream);
+
+ivit_status launch_attention(const DeviceCtx& dc, const int8_t* qkv, int32_t B, int32_t N, int32_t H,
+                             ivit_dyadic logit, int32_t k_s, int32_t I0, int32_t M, int32_t k_out,
+                             ivit_dyadic out, int8_t* ctx, cudaStream_t stream);
+
+ivit_status launch_shiftgelu(const DeviceCtx& dc, const int8_t* x, int64_t n, const GeluParams& g, int8_t* y,
+                             cudaStream_t stream);
+
+ivit_status launch_layernorm(const DeviceCtx& dc, const int8_t* x, int64_t rows, int32_t cols,
+                             const int8_t* gamma, const int32_t* beta, int32_t F, int32_t M_ln, ivit_dyadic out,
+                             int8_t* y, cudaStream_t stream);
+
+}  // namespace ivit

@@ -1,0 +1,114 @@
+"""Host-side checks of the C ABI (no compute call needs a GPU here).
+
+- the shared library loads and exports every entry point include/ivit.h declares;
+- the host parameter helpers agree with the oracle's own implementations;
+- argument validation rejects bad calls before anything is enqueued;
+- the product parameter builder equals the oracle's, field by field.
+"""
+import math
+import os
+import re
+
+import numpy as np
+import pytest
+
+import integer_only_quantized_int8_b200 as ivit
+import oracle
+import synthetic
+from integer_only_quantized_int8_b200 import build as ivit_build
+from integer_only_quantized_int8_b200 import params as ivit_params
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module", autouse=True)
+def built():
+    ivit_build.build()
+
+
+def _declared():
+    src = open(os.path.join(ROOT, "include", "ivit.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(ivit_[a-z0-9_]+)\s*\(", src)))
+
+
+def test_exports_every_declared_symbol():
+    import ctypes
+    L = ctypes.CDLL(ivit.library_path)
+    decl = _declared()
+    assert len(decl) >= 12
+    for name in decl:
+        assert hasattr(L, name), name
+    assert sorted(decl) == sorted(ivit.EXPORTED_SYMBOLS)
+
+
+def test_status_strings():
+    assert ivit.ivit_status_string(0) == "IVIT_OK"
+    assert ivit.ivit_status_string(4) == "IVIT_ERR_TIMEOUT"
+
+
+def test_dyadic_helper_matches_oracle():
+    r = np.random.default_rng(20)
+    for s in np.exp(r.uniform(math.log(2.0 ** -24), math.log(2.0 ** 12), size=5000)):
+        assert ivit.ivit_dyadic_from_double(s) == oracle.dyadic(s)
+    for s in (0.0, 0.5, 1.0, 3.0, 2.0 ** 30):
+        assert ivit.ivit_dyadic_from_double(s) == oracle.dyadic(s)
+    for bad in (-1.0, float("nan"), float("inf"), 2.0 ** 31):
+        with pytest.raises(ivit.IvitError):
+            ivit.ivit_dyadic_from_double(bad)
+
+
+def test_residual_and_i0_helpers_match_oracle():
+    r = np.random.default_rng(21)
+    for s1, s2 in np.exp(r.uniform(-8, 4, size=(2000, 2))):
+        assert ivit.ivit_residual_from_double(s1, s2) == oracle.dyadic_pair(s1, s2)
+    for S in np.exp(r.uniform(-12, 3, size=2000)):
+        assert ivit.ivit_i0_from_scale(S) == oracle.recip_i0(S)
+    with pytest.raises(ivit.IvitError):
+        ivit.ivit_i0_from_scale(0.0)
+
+
+def test_validation_rejects_before_launch():
+    import ctypes as C
+    L = ivit.lib()
+    none = ivit.Residual(0, 0, 0)
+    # null pointers
+    assert L.ivit_linear_requant(None, 16, 16, None, 16, None, None, None, 8, None, none, None, None) == 1
+    # misaligned pointer (odd address) and bad shapes; no device pointer is touched
+    p = 0x1000
+    assert L.ivit_linear_requant(p + 1, 16, 16, p, 16, None, p, p, 8, None, none, p, None) == 1
+    assert L.ivit_linear_requant(p, 16, 24, p, 16, None, p, p, 8, None, none, p, None) == 1   # K % 16
+    assert L.ivit_linear_requant(p, 16, 16, p, 16, None, p, p, 9, None, none, p, None) == 1   # out_bits
+    d = ivit.Dyadic(1, 0)
+    assert L.ivit_attention(p, 1, 8, 1, d, 9, 4, 30, 8, d, p, None) == 1      # k_s > 8
+    assert L.ivit_attention(p, 1, 8, 1, d, 8, 0, 30, 8, d, p, None) == 1      # I0 < 1
+    assert L.ivit_attention(p, 1, 8, 1, d, 8, 4, 31, 8, d, p, None) == 1      # M > 30
+    assert L.ivit_attention(p, 1, 641, 1, d, 8, 4, 30, 8, d, p, None) == 2    # too many keys
+    assert L.ivit_attention(p, 1, 8, 1, ivit.Dyadic(1, 32), 8, 4, 30, 8, d, p, None) == 1
+    assert L.ivit_layernorm(p, 4, 24, p, p, 7, 23, d, p, None) == 1          # cols % 16
+    assert L.ivit_layernorm(p, 4, 32, p, p, 7, 24, d, p, None) == 1          # M_ln > 23
+    assert L.ivit_shiftgelu(p, 16, 0, 30, 8, d, p, None) == 1
+    # empty inputs are a successful no-op that touches nothing
+    assert L.ivit_shiftgelu(None, 0, 4, 30, 8, d, None, None) == 0
+    assert L.ivit_layernorm(None, 0, 32, None, None, 7, 23, d, None, None) == 0
+
+
+def test_workspace_bytes():
+    assert ivit.ivit_block_workspace_bytes(0, 197, 768, 3072) == 0
+    T, D, Dm = 64 * 197, 768, 3072
+    up = lambda v: (v + 255) // 256 * 256
+    assert ivit.ivit_block_workspace_bytes(64, 197, D, Dm) == up(T * D) * 3 + up(T * 3 * D) + up(T * Dm)
+
+
+def test_product_params_equal_oracle_params():
+    wl = synthetic.make_workload(B=2, N=9, D=192, H=3, Dm=768, blocks=2, seed=2, n_cal=2,
+                                 tails="laplace")
+    for q in wl.blocks:
+        a = ivit_params.integer_params(q)
+        b = oracle.block_params(q)
+        assert set(b) <= set(a)
+        for k, v in b.items():
+            if isinstance(v, np.ndarray):
+                np.testing.assert_array_equal(np.asarray(a[k]).astype(np.int64), v.astype(np.int64), err_msg=k)
+            else:
+                assert tuple(np.atleast_1d(a[k])) == tuple(np.atleast_1d(v)), k

@@ -1,0 +1,177 @@
+"""GPU parity of every operator against the CPU oracle, bit for bit.
+
+Inputs are seeded synthetic tensors (``synthetic``); each side derives its
+integer parameters from the same real scales with its own code (the library's
+host helpers vs the oracle's).  Sizes span several tiles and ragged tails;
+edge cases cover single rows/keys, empty inputs and the maximum key count.
+"""
+import numpy as np
+import pytest
+import torch
+
+import integer_only_quantized_int8_b200 as ivit
+import oracle
+import synthetic
+from integer_only_quantized_int8_b200 import build as ivit_build
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def built():
+    ivit_build.build()
+    yield
+    assert ivit.ivit_stream_status() == 0
+
+
+def dev(a, dtype):
+    return torch.from_numpy(np.ascontiguousarray(a)).to(device="cuda", dtype=dtype)
+
+
+def host(t):
+    torch.cuda.synchronize()
+    return t.cpu().numpy()
+
+
+# ---------------------------------------------------------------------------
+# INT8 linear + dyadic requant (tcgen05 GEMM)
+# ---------------------------------------------------------------------------
+
+LINEAR_SHAPES = [
+    (1, 16, 16), (5, 32, 48), (197, 192, 576), (130, 384, 384), (300, 768, 3072),
+    (256, 3072, 768), (129, 64, 272), (1000, 1024, 512),
+]
+
+
+@pytest.mark.parametrize("M,K,N", LINEAR_SHAPES)
+def test_linear_requant_parity(M, K, N):
+    lc = synthetic.linear_case(M, K, N, seed=M + K + N, with_skip=True)
+    bq = [ivit.ivit_dyadic_from_double(r) for r in lc.ratio]
+    bo = [oracle.dyadic(r) for r in lc.ratio]
+    b_d, c_d = np.array([x[0] for x in bq], np.int32), np.array([x[1] for x in bq], np.int8)
+    b_o, c_o = np.array([x[0] for x in bo], np.int32), np.array([x[1] for x in bo], np.int32)
+    X, W = dev(lc.X, torch.int8), dev(lc.W, torch.int8)
+    Y = torch.empty((M, N), dtype=torch.int8, device="cuda")
+    for use_bias in (True, False):
+        bias = lc.bias if use_bias else None
+        ivit.ivit_linear_requant(X, W, None if bias is None else dev(bias, torch.int32), dev(b_d, torch.int32),
+                                 dev(c_d, torch.int8), Y)
+        want = oracle.linear_requant(lc.X, lc.W, bias, b_o, c_o)
+        np.testing.assert_array_equal(host(Y), want)
+    # residual epilogue
+    res_d = ivit.ivit_residual_from_double(*lc.res_ratio)
+    res_o = oracle.dyadic_pair(*lc.res_ratio)
+    ivit.ivit_linear_requant(X, W, dev(lc.bias, torch.int32), dev(b_d, torch.int32), dev(c_d, torch.int8), Y,
+                             skip=dev(lc.skip, torch.int8), res=res_d)
+    want = oracle.linear_requant(lc.X, lc.W, lc.bias, b_o, c_o, skip=lc.skip, res=res_o)
+    np.testing.assert_array_equal(host(Y), want)
+    # a narrower output width
+    ivit.ivit_linear_requant(X, W, dev(lc.bias, torch.int32), dev(b_d, torch.int32), dev(c_d, torch.int8), Y,
+                             out_bits=4)
+    np.testing.assert_array_equal(host(Y), oracle.linear_requant(lc.X, lc.W, lc.bias, b_o, c_o, out_bits=4))
+
+
+def test_linear_saturation_and_extremes():
+    r = np.random.default_rng(30)
+    M, K, N = 64, 4096, 32
+    X = np.full((M, K), -128, np.int8)
+    X[1::2] = 127
+    W = r.choice(np.array([-128, 127], np.int8), size=(N, K))
+    b = np.zeros(N, np.int32); b[:] = 2 ** 31 - 1
+    c = (np.arange(N) % 32).astype(np.int32)
+    bias = r.integers(-2 ** 20, 2 ** 20, size=N).astype(np.int32)
+    Y = torch.empty((M, N), dtype=torch.int8, device="cuda")
+    ivit.ivit_linear_requant(dev(X, torch.int8), dev(W, torch.int8), dev(bias, torch.int32), dev(b, torch.int32),
+                             dev(c, torch.int8), Y)
+    np.testing.assert_array_equal(host(Y), oracle.linear_requant(X, W, bias, b, c))
+
+
+# ---------------------------------------------------------------------------
+# fused attention with Shiftmax
+# ---------------------------------------------------------------------------
+
+ATTN_CASES = [
+    (1, 1, 1, "normal", 8), (2, 5, 1, "normal", 8), (2, 197, 3, "normal", 8), (1, 577, 2, "laplace", 8),
+    (3, 130, 2, "normal", 8), (1, 128, 1, "laplace", 8), (2, 256, 1, "normal", 8), (1, 300, 1, "laplace", 8),
+    (1, 640, 1, "laplace", 8), (2, 197, 2, "laplace", 4), (1, 33, 2, "normal", 6),
+]
+
+
+@pytest.mark.parametrize("B,N,H,tails,k_s", ATTN_CASES)
+def test_attention_parity(B, N, H, tails, k_s):
+    ac = synthetic.attention_case(B, N, H, seed=B * 1000 + N + H, tails=tails, k_s=k_s)
+    logit_d, logit_o = ivit.ivit_dyadic_from_double(ac.logit_ratio), oracle.dyadic(ac.logit_ratio)
+    out_d, out_o = ivit.ivit_dyadic_from_double(ac.out_ratio), oracle.dyadic(ac.out_ratio)
+    I0_d, I0_o = ivit.ivit_i0_from_scale(ac.S_logit), oracle.recip_i0(ac.S_logit)
+    qkv = dev(ac.qkv, torch.int8)
+    ctx = torch.full((B * N, H * 64), 99, dtype=torch.int8, device="cuda")
+    ivit.ivit_attention(qkv, B, N, H, logit_d, k_s, I0_d, 30, 8, out_d, ctx)
+    want = oracle.attention(ac.qkv, B, N, H, logit_o, k_s, I0_o, 30, 8, out_o)
+    np.testing.assert_array_equal(host(ctx), want)
+
+
+@pytest.mark.parametrize("I0,M,k_out", [(1, 30, 8), (3, 20, 8), (97, 30, 5), (4096, 30, 8)])
+def test_attention_shiftmax_parameters(I0, M, k_out):
+    ac = synthetic.attention_case(2, 70, 2, seed=I0, tails="laplace")
+    qkv = dev(ac.qkv, torch.int8)
+    ctx = torch.empty((140, 128), dtype=torch.int8, device="cuda")
+    logit = oracle.dyadic(ac.logit_ratio)
+    out = oracle.dyadic(ac.out_ratio * 2 ** (8 - k_out))
+    ivit.ivit_attention(qkv, 2, 70, 2, logit, 8, I0, M, k_out, out, ctx)
+    np.testing.assert_array_equal(host(ctx), oracle.attention(ac.qkv, 2, 70, 2, logit, 8, I0, M, k_out, out))
+
+
+# ---------------------------------------------------------------------------
+# ShiftGELU
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("n", [0, 1, 15, 16, 17, 4099, 1 << 20, (1 << 20) + 13])
+def test_shiftgelu_parity(n):
+    gc = synthetic.gelu_case(max(n, 1), seed=n)
+    x = gc.x[:n]
+    I0_d, out_d = ivit.ivit_i0_from_scale(gc.S_h), ivit.ivit_dyadic_from_double(gc.out_ratio)
+    I0_o, out_o = oracle.recip_i0(gc.S_h), oracle.dyadic(gc.out_ratio)
+    xd = dev(x, torch.int8) if n else torch.empty(0, dtype=torch.int8, device="cuda")
+    y = torch.empty_like(xd)
+    ivit.ivit_shiftgelu(xd, I0_d, 30, 8, out_d, y)
+    np.testing.assert_array_equal(host(y), oracle.shiftgelu(x, I0_o, 30, 8, out_o))
+
+
+@pytest.mark.parametrize("I0", [1, 2, 5, 16, 25, 64, 1000])
+def test_shiftgelu_all_inputs(I0):
+    x = np.tile(np.arange(-128, 128, dtype=np.int8), 4)
+    out = oracle.dyadic(1.0 / 128)
+    y = torch.empty(x.size, dtype=torch.int8, device="cuda")
+    ivit.ivit_shiftgelu(dev(x, torch.int8), I0, 30, 8, out, y)
+    np.testing.assert_array_equal(host(y), oracle.shiftgelu(x, I0, 30, 8, out))
+
+
+# ---------------------------------------------------------------------------
+# I-LayerNorm
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("rows,cols", [(1, 16), (7, 192), (1000, 384), (4099, 768), (33, 1024), (9, 2048),
+                                       (5, 48)])
+def test_layernorm_parity(rows, cols):
+    nc = synthetic.layernorm_case(rows, cols, seed=rows + cols)
+    x = nc.x.copy()
+    x[0] = 17                                    # a constant row (variance 0)
+    out_d, out_o = ivit.ivit_dyadic_from_double(nc.out_ratio), oracle.dyadic(nc.out_ratio)
+    y = torch.empty((rows, cols), dtype=torch.int8, device="cuda")
+    ivit.ivit_layernorm(dev(x, torch.int8), dev(nc.gamma, torch.int8), dev(nc.beta, torch.int32), 7, 23, out_d, y)
+    np.testing.assert_array_equal(host(y), oracle.layernorm(x, nc.gamma, nc.beta, 7, 23, out_o))
+
+
+def test_layernorm_extreme_rows():
+    cols = 256
+    x = np.zeros((4, cols), np.int8)
+    x[0, ::2], x[0, 1::2] = -128, 127            # maximum spread
+    x[1, 0] = 1                                  # V floors to 0
+    x[2] = -128
+    x[3] = np.arange(cols) - 128
+    gamma = np.full(cols, -128, np.int8)
+    beta = np.arange(cols, dtype=np.int32) * 1000 - 100000
+    out = (3, 2)
+    y = torch.empty((4, cols), dtype=torch.int8, device="cuda")
+    ivit.ivit_layernorm(dev(x, torch.int8), dev(gamma, torch.int8), dev(beta, torch.int32), 7, 23, out, y)
+    np.testing.assert_array_equal(host(y), oracle.layernorm(x, gamma, beta, 7, 23, out))
