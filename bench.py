@@ -1,0 +1,518 @@
+#!/usr/bin/env python
+"""Benchmark of the integer-only ViT encoder block on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+One step = one pass of the whole block (I-LayerNorm, QKV, Shiftmax attention,
+W^O + residual, I-LayerNorm, fc1 + ShiftGELU, fc2 + residual; every block of
+the workload) over one batch of seeded synthetic int8 input that is already
+resident in HBM.  Inputs rotate over enough copies that their total exceeds
+the L2 cache.  Steps are replayed from CUDA graphs and timed with CUDA events
+on the launching stream; under torchrun each rank runs its own batch (images
+are independent: weak scaling, no collective on the data path) and rank 0
+prints one JSON line with the max time over ranks.
+
+``--impl reference`` times the CPU oracle (plain C, one core) on a bounded
+sample of the same workload instead.
+"""
+from __future__ import annotations
+
+import argparse
+import glob
+import hashlib
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+import synthetic  # noqa: E402
+
+METRIC = "int-only ViT block images/s (ViT-B, 197 tok); % INT8 TC peak & % HBM BW"
+DEFAULT_WORKLOAD = "vit_b_b64"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+INT8_PER_BF16 = 2.0  # nominal dense tensor-core ratio on B200 (4.5 vs 2.25 PFLOP/s)
+
+
+def parse_args():
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=synthetic.CONFIG_ORDER)
+    ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--no-graph", action="store_true", help="launch eagerly instead of replaying CUDA graphs")
+    ap.add_argument("--cpu-units", type=int, default=10,
+                    help="CPU-baseline sample: (image, block) units the oracle runs")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--kernel-reps", type=int, default=50)
+    return ap.parse_args()
+
+
+def ops_per_image_block(N, D):
+    """Integer ops (2 x MAC) of the method per image per block: the four
+    linears (12 N D^2 MAC) and Q K^T, P V (2 N^2 D MAC); padding not counted."""
+    return 24 * N * D * D + 4 * N * N * D
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return {k: float(p[k]) for k in ("hbm_gbs", "bf16_tflops", "bf16_tflops_sustained")}, "measured"
+    except Exception:
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle timing (reference arm and cpu_baseline)
+# ---------------------------------------------------------------------------
+
+def oracle_units(wl, units):
+    """Time the oracle on ``units`` (image, block) pairs; returns (seconds, images/s)."""
+    import oracle
+    ps = [oracle.block_params(q) for q in wl.blocks]
+    N, nb = wl.N, len(wl.blocks)
+    x_by_block = [wl.x]
+    t = 0.0
+    for u in range(units):
+        b = u % nb
+        img = (u // nb) % wl.B
+        xin = wl.x[img * N:(img + 1) * N]
+        t0 = time.perf_counter()
+        oracle.block_forward(ps[b], xin, 1, N)
+        t += time.perf_counter() - t0
+    del x_by_block
+    return t, units / (t * nb)
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    wl = synthetic.workload(args.workload, seed=args.seed)
+    import oracle
+    ps = [oracle.block_params(q) for q in wl.blocks]
+    N, nb = wl.N, len(wl.blocks)
+    times = []
+    for step in range(args.warmup + args.steps):
+        b = step % nb
+        img = (step // nb) % wl.B
+        xin = wl.x[img * N:(img + 1) * N]
+        t0 = time.perf_counter()
+        oracle.block_forward(ps[b], xin, 1, N)
+        dt = time.perf_counter() - t0
+        if step >= args.warmup:
+            times.append(dt)
+    step_s = sum(times) / len(times)
+    value = 1.0 / (step_s * nb)
+    sample = (f"each step: 1 image x 1 block of {args.workload} (block cycles over the {nb} block(s)); "
+              f"images/s = 1 / (step time x {nb} blocks)")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "images/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_s * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "int64", "data": "synthetic",
+        "config": workload_config(wl, args),
+        "cpu_baseline": {"value": value, "unit": "images/s", "cores": 1, "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": "images/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def workload_config(wl, args, extra=None):
+    cfg = {"workload": wl.name, "B": wl.B, "N": wl.N, "D": wl.D, "H": wl.H, "Dm": wl.Dm,
+           "blocks": len(wl.blocks), "seed": args.seed}
+    if extra:
+        cfg.update(extra)
+    return cfg
+
+
+# ---------------------------------------------------------------------------
+# clock sampling (NVML) during the run
+# ---------------------------------------------------------------------------
+
+_REASONS = [(0x1, "gpu_idle"), (0x2, "applications_clocks_setting"), (0x4, "sw_power_cap"),
+            (0x8, "hw_slowdown"), (0x10, "sync_boost"), (0x20, "sw_thermal_slowdown"),
+            (0x40, "hw_thermal_slowdown"), (0x80, "hw_power_brake_slowdown"), (0x100, "display_clock_setting")]
+
+
+class ClockSampler:
+    def __init__(self, device_index, period_s=0.01):
+        self.samples = []
+        self.ok = False
+        self.max_mhz = None
+        self.period = period_s
+        self._stop = threading.Event()
+        try:
+            import pynvml
+            import torch
+            pynvml.nvmlInit()
+            uuid = str(torch.cuda.get_device_properties(device_index).uuid)
+            uuid = uuid if uuid.startswith("GPU-") else "GPU-" + uuid
+            self.h = pynvml.nvmlDeviceGetHandleByUUID(uuid)
+            self.nv = pynvml
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception as e:  # pragma: no cover - depends on the box
+            self.err = repr(e)
+
+    def _reasons(self):
+        nv = self.nv
+        for fn in ("nvmlDeviceGetCurrentClocksEventReasons", "nvmlDeviceGetCurrentClocksThrottleReasons"):
+            if hasattr(nv, fn):
+                return int(getattr(nv, fn)(self.h))
+        return 0
+
+    def _run(self):
+        nv = self.nv
+        while not self._stop.is_set():
+            try:
+                self.samples.append((time.perf_counter(), nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM),
+                                     self._reasons()))
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def start(self):
+        if self.ok:
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+
+    def stop(self):
+        if self.ok:
+            self._stop.set()
+            self.t.join()
+
+    def summary(self, t0, t1):
+        if not self.ok:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0, "source": "unavailable"}
+        win = [s for s in self.samples if t0 <= s[0] <= t1]
+        busy = [s for s in win if not (s[2] & 0x1)] or win
+        if not busy:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [], "samples": 0, "source": "nvml"}
+        bits = 0
+        for s in busy:
+            bits |= s[2]
+        return {"sm_mhz": statistics.median(s[1] for s in busy), "sm_max_mhz": self.max_mhz,
+                "reasons": [n for b, n in _REASONS if bits & b and n != "gpu_idle"], "samples": len(busy),
+                "source": "nvml, every 10 ms over warm-up + timed steps"}
+
+
+# ---------------------------------------------------------------------------
+# our arm
+# ---------------------------------------------------------------------------
+
+def source_hash(paths):
+    h = hashlib.sha256()
+    for p in sorted(paths):
+        with open(p, "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def kernel_source_hash():
+    csrc = os.path.join(ROOT, "integer_only_quantized_int8_b200", "csrc")
+    return source_hash(glob.glob(os.path.join(csrc, "*.cu")) + glob.glob(os.path.join(csrc, "*.cuh")) +
+                       glob.glob(os.path.join(csrc, "*.h")))
+
+
+def load_traffic(kernel, workload):
+    """DRAM bytes per launch from a committed ncu capture, if the kernels are unchanged since."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as f:
+            tab = json.load(f)
+        ent = tab.get(f"{kernel}@{workload}")
+        if ent and ent.get("source_hash") == kernel_source_hash():
+            return float(ent["dram_bytes_per_launch"])
+    except Exception:
+        pass
+    return None
+
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+    import integer_only_quantized_int8_b200 as ivit
+    from integer_only_quantized_int8_b200 import params as ivit_params
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device (there is no CPU fallback)")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=dev)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    wl = synthetic.workload(args.workload, seed=args.seed + rank)
+    B, N, D, Dm = wl.B, wl.N, wl.D, wl.Dm
+    T = B * N
+    nblk = len(wl.blocks)
+    dps = [ivit_params.to_device(ivit_params.integer_params(q), dev) for q in wl.blocks]
+    ws = torch.empty(ivit.ivit_block_workspace_bytes(B, N, D, Dm), dtype=torch.uint8, device=dev)
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    xbytes = T * D
+    R = max(2, min(64, math.ceil(2 * l2 / xbytes)))
+    x0 = torch.from_numpy(wl.x).to(dev)
+    xs = [x0.clone() for _ in range(R)]
+    ya = torch.empty((T, D), dtype=torch.int8, device=dev)
+    yb = torch.empty((T, D), dtype=torch.int8, device=dev)
+
+    def step(r):
+        cur = xs[r]
+        for i, dp in enumerate(dps):
+            nxt = ya if i % 2 == 0 else yb
+            ivit.ivit_block_forward(dp, cur, nxt, ws, B, N)
+            cur = nxt
+        return cur
+
+    # eager warm-up (sets kernel attributes), launch accounting
+    c0 = ivit.ivit_launch_count()
+    out = step(0)
+    torch.cuda.synchronize()
+    launches_per_step = ivit.ivit_launch_count() - c0
+    assert ivit.ivit_stream_status() == 0
+
+    use_graph = not args.no_graph
+    graphs = []
+    if use_graph:
+        s = torch.cuda.Stream(device=dev)
+        s.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(s):
+            for r in range(R):
+                g = torch.cuda.CUDAGraph()
+                with torch.cuda.graph(g, stream=s):
+                    step(r)
+                graphs.append(g)
+        torch.cuda.current_stream().wait_stream(s)
+        torch.cuda.synchronize()
+
+    def run(i):
+        if use_graph:
+            graphs[i % R].replay()
+        else:
+            step(i % R)
+
+    sampler = ClockSampler(local)
+    sampler.start()
+    t_w0 = time.perf_counter()
+    for i in range(args.warmup):
+        run(i)
+    torch.cuda.synchronize()
+    barrier()
+    torch.cuda.synchronize()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ev0.record()
+    for i in range(args.steps):
+        run(args.warmup + i)
+    ev1.record()
+    torch.cuda.synchronize()
+    t_w1 = time.perf_counter()
+    barrier()
+    elapsed_ms = ev0.elapsed_time(ev1)
+    if world > 1:
+        t = torch.tensor([elapsed_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        elapsed_ms = float(t.item())
+    sampler.stop()
+    clocks = sampler.summary(t_w0, t_w1)
+    if ivit.ivit_stream_status() != 0:
+        raise SystemExit("a kernel reported a timed-out wait")
+    ms_per_step = elapsed_ms / args.steps
+    images_per_s = world * B * args.steps / (elapsed_ms / 1e3)
+
+    # ---------------- per-kernel breakdown of block 0 (CUDA events, same stream)
+    kern = kernel_breakdown(ivit, wl, dps[0], ws, xs, args.kernel_reps, dev)
+
+    # ---------------- end to end through host buffers
+    x_host = torch.from_numpy(wl.x).pin_memory()
+    y_host = torch.empty((T, D), dtype=torch.int8).pin_memory()
+    k_e2e = max(1, min(args.steps, 50))
+    for _ in range(3):
+        xs[0].copy_(x_host, non_blocking=True)
+        run(0)
+        y_host.copy_(out, non_blocking=True)
+    torch.cuda.synchronize()
+    barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(k_e2e):
+        xs[0].copy_(x_host, non_blocking=True)
+        run(0)
+        y_host.copy_(out, non_blocking=True)
+    e1.record()
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1)
+    if world > 1:
+        t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    barrier()
+    e2e_value = world * B * k_e2e / (e2e_ms / 1e3)
+
+    # release graphs before the process group goes away
+    graphs.clear()
+    if world > 1:
+        dist.destroy_process_group()
+    if rank != 0:
+        return 0
+
+    peaks, peak_src = load_peaks()
+    ops_step = world * B * nblk * ops_per_image_block(N, D)
+    eff_tops = ops_step / (ms_per_step / 1e3) / 1e12
+    int8_peak_burst = peaks["bf16_tflops"] * INT8_PER_BF16
+    int8_peak_sust = peaks["bf16_tflops_sustained"] * INT8_PER_BF16
+
+    # dominant kernel of the block by time per step
+    dom = max((k for k in kern if k["in_block"]), key=lambda k: k["ms"] * k["per_block"])
+    if dom["bound"] == "tensor":
+        achieved = dom["amount"] / (dom["ms"] / 1e3) / 1e12
+        peak, unit = int8_peak_burst, "TOP/s"
+        peak_note = f"INT8 dense = {INT8_PER_BF16:g} x bf16 burst ({peak_src})"
+    else:
+        achieved = dom["amount"] / (dom["ms"] / 1e3) / 1e9
+        peak, unit = peaks["hbm_gbs"], "GB/s"
+        peak_note = f"HBM copy ({peak_src})"
+    traffic = load_traffic(dom["name"], wl.name)
+    roofline = {"kernel": dom["name"], "bound": dom["bound"], "achieved": achieved, "peak": peak, "unit": unit,
+                "frac": achieved / peak, "traffic": traffic, "peak_source": peak_note,
+                "launch_ms": dom["ms"]}
+
+    cpu = None
+    if world == 1 and not args.no_cpu_baseline:
+        secs, ips = oracle_units(wl, args.cpu_units)
+        cpu = {"value": ips, "unit": "images/s", "cores": 1, "kind": "oracle",
+               "sample": f"{args.cpu_units} (image, block) units of {wl.name} through the single-threaded C "
+                         f"oracle ({secs:.1f} s); images/s = units / (time x {nblk} blocks)"}
+
+    line = {
+        "metric": METRIC, "value": images_per_s, "unit": "images/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "int8", "data": "synthetic",
+        "config": workload_config(wl, args, {
+            "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+            "l2": f"inputs rotate over {R} copies ({R * xbytes / 1e6:.0f} MB > {l2 / 1e6:.0f} MB L2)",
+            "graph": use_graph}),
+        "effective_tops": eff_tops,
+        "frac_int8_peak_e2e": {"burst": eff_tops / int8_peak_burst, "sustained": eff_tops / int8_peak_sust,
+                               "peak_source": f"{INT8_PER_BF16:g} x bf16 ({peak_src})"},
+        "roofline": roofline,
+        "kernels": [{k2: v for k2, v in k.items()} for k in kern],
+        "cpu_baseline": cpu,
+        "e2e": {"value": e2e_value, "unit": "images/s", "h2d_bytes_per_step": int(T * D),
+                "d2h_bytes_per_step": int(T * D), "steps": k_e2e},
+        "clocks": clocks,
+        "gpu_launches": int(launches_per_step * args.steps),
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def kernel_breakdown(ivit, wl, dp, ws, xs, reps, dev):
+    """Average device time per launch of every kernel of one block, each timed
+    alone over ``reps`` back-to-back launches with CUDA events.  Inputs are the
+    block's own intermediates (left in the workspace by a block forward)."""
+    import torch
+    B, N, D, Dm, H = wl.B, wl.N, wl.D, wl.Dm, wl.H
+    T = B * N
+    p = dp.host
+    t = dp.tensors
+    up = lambda v: (v + 255) // 256 * 256
+    w8 = ws.view(torch.int8)
+    o_ln = 0
+    o_qkv = o_ln + up(T * D)
+    o_ctx = o_qkv + up(T * 3 * D)
+    o_xh = o_ctx + up(T * D)
+    o_g = o_xh + up(T * D)
+    y = torch.empty((T, D), dtype=torch.int8, device=dev)
+    ivit.ivit_block_forward(dp, xs[0], y, ws, B, N)      # leaves ln2, qkv, ctx, xh, g in the workspace
+    torch.cuda.synchronize()
+    ln = w8[o_ln:o_ln + T * D].view(T, D).clone()
+    qkv = w8[o_qkv:o_qkv + T * 3 * D].view(T, 3 * D).clone()
+    ctx = w8[o_ctx:o_ctx + T * D].view(T, D).clone()
+    xh = w8[o_xh:o_xh + T * D].view(T, D).clone()
+    g = w8[o_g:o_g + T * Dm].view(T, Dm).clone()
+    qkv_o = torch.empty_like(qkv)
+    ctx_o = torch.empty_like(ctx)
+    h_o = torch.empty_like(g)
+    R = len(xs)
+    hs = [g.clone() for _ in range(max(2, math.ceil(2 * 126e6 / (2 * T * Dm))))]
+
+    def timed(fn):
+        for i in range(3):
+            fn(i)
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        for i in range(reps):
+            fn(i)
+        b.record()
+        torch.cuda.synchronize()
+        return a.elapsed_time(b) / reps
+
+    gemm = lambda M, K, Nn: 2 * M * K * Nn
+    out = []
+
+    def add(name, fn, bound, amount, in_block=True, per_block=1):
+        out.append({"name": name, "ms": timed(fn), "bound": bound, "amount": amount, "in_block": in_block,
+                    "per_block": per_block})
+
+    add("layernorm", lambda i: ivit.ivit_layernorm(xs[i % R], t["ln1_gamma"], t["ln1_beta"], p["ln_F"], p["ln_M"],
+                                                   p["ln1_out"], y), "hbm", 2 * T * D, per_block=2)
+    add("gemm_qkv", lambda i: ivit.ivit_linear_requant(ln, t["w_qkv"], t["bias_qkv"], t["b_qkv"], t["c_qkv"], qkv_o),
+        "tensor", gemm(T, D, 3 * D))
+    add("attention", lambda i: ivit.ivit_attention(qkv, B, N, H, p["logit"], p["k_s"], p["attn_I0"], p["attn_M"],
+                                                   p["attn_k_out"], p["attn_out"], ctx_o),
+        "tensor", 4 * B * N * N * D)
+    add("gemm_o_residual", lambda i: ivit.ivit_linear_requant(ctx, t["w_o"], t["bias_o"], t["b_o"], t["c_o"], y,
+                                                              skip=xs[i % R], res=p["res1"]),
+        "tensor", gemm(T, D, D))
+    add("gemm_fc1_shiftgelu", lambda i: ivit.ivit_linear_shiftgelu(ln, t["w1"], t["bias1"], t["b1"], t["c1"],
+                                                                   p["gelu_I0"], p["gelu_M"], p["gelu_k_out"],
+                                                                   p["gelu_out"], h_o),
+        "tensor", gemm(T, D, Dm))
+    add("gemm_fc2_residual", lambda i: ivit.ivit_linear_requant(g, t["w2"], t["bias2"], t["b2"], t["c2"], y,
+                                                                skip=xh, res=p["res2"]),
+        "tensor", gemm(T, Dm, D))
+    add("shiftgelu_standalone", lambda i: ivit.ivit_shiftgelu(hs[i % len(hs)], p["gelu_I0"], p["gelu_M"],
+                                                              p["gelu_k_out"], p["gelu_out"], h_o),
+        "hbm", 2 * T * Dm, in_block=False)
+    peaks, src = load_peaks()
+    for k in out:
+        if k["bound"] == "hbm":
+            k["achieved"] = k["amount"] / (k["ms"] / 1e3) / 1e9
+            k["unit"] = "GB/s"
+            k["frac"] = k["achieved"] / peaks["hbm_gbs"]
+        else:
+            k["achieved"] = k["amount"] / (k["ms"] / 1e3) / 1e12
+            k["unit"] = "TOP/s"
+            k["frac"] = k["achieved"] / (peaks["bf16_tflops"] * INT8_PER_BF16)
+    return out
+
+
+def main():
+    args = parse_args()
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -96,13 +96,25 @@ ivit_status ivit_i0_from_scale(double S, int32_t *out);
  *   Y_ij   = skip ? sat_8((res.b_skip * skip[i,j] + res.b_branch * o_ij) >> res.c)
  *                 : o_ij
  * X [M x K] int8; W [N x K] int8 (one output channel per row, i.e. K-major);
- * bias [N] int32 or NULL; b [N] int32 in [0, 2^31); c [N] int8 in [0, 31];
+ * bias [N] int32 or NULL, |bias| <= 2^30 (the int32 accumulator cannot
+ * overflow); b [N] int32 in [0, 2^31); c [N] int8 in [0, 31];
  * skip [M x N] int8 or NULL; Y [M x N] int8.
  * Constraints: M >= 1; 16 <= K <= 16384 and N >= 16, both multiples of 16;
  * 2 <= out_bits <= 8.  Runs on the tensor cores (tcgen05 kind::i8).      */
 ivit_status ivit_linear_requant(const int8_t *X, int64_t M, int32_t K, const int8_t *W, int32_t N,
                                 const int32_t *bias, const int32_t *b, const int8_t *c, int32_t out_bits,
                                 const int8_t *skip, ivit_residual res, int8_t *Y, ivit_stream_t stream);
+
+/* fc1 of the MLP with ShiftGELU fused into the epilogue ([IVIT] 3.1, 3.2,
+ * 3.4): Y = ShiftGELU(sat_8((b[j] * (X W^T + bias)_ij) >> c[j])), with the
+ * ShiftGELU of ivit_shiftgelu (I0 = round(1 / S_h) of the requantised fc1
+ * output, gelu_out ~ S_h 2^-(k_out-1) / S_g).  Bit-identical to
+ * ivit_linear_requant followed by ivit_shiftgelu, without the intermediate
+ * tensor in memory.  Same constraints as both.                              */
+ivit_status ivit_linear_shiftgelu(const int8_t *X, int64_t M, int32_t K, const int8_t *W, int32_t N,
+                                  const int32_t *bias, const int32_t *b, const int8_t *c, int32_t gelu_I0,
+                                  int32_t gelu_M, int32_t gelu_k_out, ivit_dyadic gelu_out, int8_t *Y,
+                                  ivit_stream_t stream);
 
 /* Multi-head attention core with Shiftmax ([IVIT] 3.1-3.3; [TRIO] eqs.
  * (1)-(3)), fused on chip (the score matrix never reaches memory):
@@ -137,8 +149,8 @@ ivit_status ivit_shiftgelu(const int8_t *x, int64_t n, int32_t I0, int32_t M, in
  *   n_i = ((x_i - mu) * floor(2^M_ln / sigma)) >> (M_ln - F)   (scale 2^-F)
  *   y_i = sat_8((out.b * (n_i * gamma_i + beta_i)) >> out.c)
  * x, y [rows x cols] int8; gamma [cols] int8 (scale S_gamma); beta [cols]
- * int32 (scale S_gamma 2^-F).  Constraints: rows >= 0; 16 <= cols <= 2048,
- * multiple of 16; 0 <= F <= M_ln <= 23.                                     */
+ * int32 (scale S_gamma 2^-F), |beta| <= 2^30.  Constraints: rows >= 0;
+ * 16 <= cols <= 2048, multiple of 16; 0 <= F <= 14; F <= M_ln <= 23.        */
 ivit_status ivit_layernorm(const int8_t *x, int64_t rows, int32_t cols, const int8_t *gamma,
                            const int32_t *beta, int32_t F, int32_t M_ln, ivit_dyadic out, int8_t *y,
                            ivit_stream_t stream);

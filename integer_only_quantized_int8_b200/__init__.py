@@ -19,7 +19,7 @@ import torch
 __all__ = [
     "IvitError", "lib", "library_path", "Dyadic", "Residual", "BlockParams",
     "ivit_status_string", "ivit_dyadic_from_double", "ivit_residual_from_double", "ivit_i0_from_scale",
-    "ivit_linear_requant", "ivit_attention", "ivit_shiftgelu", "ivit_layernorm",
+    "ivit_linear_requant", "ivit_linear_shiftgelu", "ivit_attention", "ivit_shiftgelu", "ivit_layernorm",
     "ivit_block_workspace_bytes", "ivit_block_forward", "ivit_stream_status", "ivit_launch_count",
     "EXPORTED_SYMBOLS",
 ]
@@ -31,7 +31,8 @@ _lib = None
 
 EXPORTED_SYMBOLS = (
     "ivit_status_string", "ivit_dyadic_from_double", "ivit_residual_from_double", "ivit_i0_from_scale",
-    "ivit_linear_requant", "ivit_attention", "ivit_shiftgelu", "ivit_layernorm", "ivit_block_workspace_bytes",
+    "ivit_linear_requant", "ivit_linear_shiftgelu", "ivit_attention", "ivit_shiftgelu", "ivit_layernorm",
+    "ivit_block_workspace_bytes",
     "ivit_block_forward", "ivit_stream_status", "ivit_launch_count",
 )
 
@@ -92,6 +93,8 @@ def lib() -> C.CDLL:
             L.ivit_i0_from_scale.argtypes = [C.c_double, C.POINTER(C.c_int32)]
             L.ivit_linear_requant.restype = C.c_int
             L.ivit_linear_requant.argtypes = [vp, i64, i32, vp, i32, vp, vp, vp, i32, vp, Residual, vp, vp]
+            L.ivit_linear_shiftgelu.restype = C.c_int
+            L.ivit_linear_shiftgelu.argtypes = [vp, i64, i32, vp, i32, vp, vp, vp, i32, i32, i32, Dyadic, vp, vp]
             L.ivit_attention.restype = C.c_int
             L.ivit_attention.argtypes = [vp, i32, i32, i32, Dyadic, i32, i32, i32, i32, Dyadic, vp, vp]
             L.ivit_shiftgelu.restype = C.c_int
@@ -190,6 +193,21 @@ def ivit_linear_requant(X, W, bias, b, c, Y, out_bits: int = 8, skip=None, res=N
                                    _ptr(c, torch.int8, "c"), int(out_bits), _ptr(skip, torch.int8, "skip"),
                                    _res(res), _ptr(Y, torch.int8, "Y"), _stream(stream))
     _check("ivit_linear_requant", st)
+    return Y
+
+
+def ivit_linear_shiftgelu(X, W, bias, b, c, gelu_I0: int, gelu_M: int, gelu_k_out: int, gelu_out, Y,
+                          stream=None):
+    """Y = ShiftGELU(sat_8((b_j (X W^T + bias)_ij) >> c_j)) in one kernel."""
+    M, K = X.shape
+    N = W.shape[0]
+    if W.shape[1] != K or tuple(Y.shape) != (M, N):
+        raise ValueError("shape mismatch")
+    st = lib().ivit_linear_shiftgelu(_ptr(X, torch.int8, "X"), M, K, _ptr(W, torch.int8, "W"), N,
+                                     _ptr(bias, torch.int32, "bias"), _ptr(b, torch.int32, "b"),
+                                     _ptr(c, torch.int8, "c"), int(gelu_I0), int(gelu_M), int(gelu_k_out),
+                                     _dy(gelu_out), _ptr(Y, torch.int8, "Y"), _stream(stream))
+    _check("ivit_linear_shiftgelu", st)
     return Y
 
 

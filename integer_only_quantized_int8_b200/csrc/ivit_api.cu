@@ -182,6 +182,25 @@ ivit_status ivit_linear_requant(const int8_t* X, int64_t M, int32_t K, const int
                      (cudaStream_t)stream);
 }
 
+ivit_status ivit_linear_shiftgelu(const int8_t* X, int64_t M, int32_t K, const int8_t* W, int32_t N,
+                                  const int32_t* bias, const int32_t* b, const int8_t* c, int32_t gelu_I0,
+                                  int32_t gelu_M, int32_t gelu_k_out, ivit_dyadic gelu_out, int8_t* Y,
+                                  ivit_stream_t stream) {
+  if (!X || !W || !b || !c || !Y) return IVIT_ERR_INVALID_ARG;
+  if (!aligned16(X) || !aligned16(W) || !aligned16(b) || !aligned16(c) || !aligned16(Y) ||
+      (bias && !aligned16(bias)))
+    return IVIT_ERR_INVALID_ARG;
+  if (M < 1 || K < 16 || K % 16 != 0 || N < 16 || N % 16 != 0) return IVIT_ERR_INVALID_ARG;
+  if (!valid_shiftmax(gelu_I0, gelu_M, gelu_k_out) || !valid_dyadic(gelu_out)) return IVIT_ERR_INVALID_ARG;
+  if (K > 16384 || M > 0x7fffff00LL) return IVIT_ERR_UNSUPPORTED;
+  DeviceCtx dc;
+  ivit_status st = device_ctx(&dc);
+  if (st != IVIT_OK) return st;
+  const GeluParams gp{gelu_I0, gelu_M, gelu_k_out, gelu_out};
+  return launch_gemm(dc, X, M, K, W, N, bias, b, c, 8, kEpiGelu, nullptr, ivit_residual{0, 0, 0}, &gp, Y,
+                     (cudaStream_t)stream);
+}
+
 ivit_status ivit_attention(const int8_t* qkv, int32_t B, int32_t N, int32_t H, ivit_dyadic logit, int32_t k_s,
                            int32_t I0, int32_t M, int32_t k_out, ivit_dyadic out, int8_t* ctx,
                            ivit_stream_t stream) {

@@ -50,7 +50,7 @@ def rng(seed: int, tensor: str, block: int = 0) -> np.random.Generator:
 def round_sym(v: np.ndarray, S, lim: int = 127) -> np.ndarray:
     """Round-half-away-from-zero of v / S, clipped to +-lim (symmetric)."""
     t = np.asarray(v, dtype=np.float64) / S
-    r = np.sign(t) * np.floor(np.abs(t) + 0.5)
+    r = np.copysign(np.floor(np.abs(t) + 0.5), t)
     return np.clip(r, -lim, lim)
 
 

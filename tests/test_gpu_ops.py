@@ -175,3 +175,21 @@ def test_layernorm_extreme_rows():
     y = torch.empty((4, cols), dtype=torch.int8, device="cuda")
     ivit.ivit_layernorm(dev(x, torch.int8), dev(gamma, torch.int8), dev(beta, torch.int32), 7, 23, out, y)
     np.testing.assert_array_equal(host(y), oracle.layernorm(x, gamma, beta, 7, 23, out))
+
+
+@pytest.mark.parametrize("M,K,N", [(1, 16, 16), (197, 192, 768), (300, 768, 3072), (129, 384, 1552)])
+def test_linear_shiftgelu_parity(M, K, N):
+    """fc1 with ShiftGELU in the epilogue == oracle linear, then oracle ShiftGELU."""
+    lc = synthetic.linear_case(M, K, N, seed=7 * M + N)
+    gc = synthetic.gelu_case(1024, seed=N)
+    bq = [ivit.ivit_dyadic_from_double(r) for r in lc.ratio]
+    bo = [oracle.dyadic(r) for r in lc.ratio]
+    b_d, c_d = np.array([x[0] for x in bq], np.int32), np.array([x[1] for x in bq], np.int8)
+    b_o, c_o = np.array([x[0] for x in bo], np.int32), np.array([x[1] for x in bo], np.int32)
+    I0_d, out_d = ivit.ivit_i0_from_scale(gc.S_h), ivit.ivit_dyadic_from_double(gc.out_ratio)
+    I0_o, out_o = oracle.recip_i0(gc.S_h), oracle.dyadic(gc.out_ratio)
+    Y = torch.empty((M, N), dtype=torch.int8, device="cuda")
+    ivit.ivit_linear_shiftgelu(dev(lc.X, torch.int8), dev(lc.W, torch.int8), dev(lc.bias, torch.int32),
+                               dev(b_d, torch.int32), dev(c_d, torch.int8), I0_d, 30, 8, out_d, Y)
+    h = oracle.linear_requant(lc.X, lc.W, lc.bias, b_o, c_o)
+    np.testing.assert_array_equal(host(Y), oracle.shiftgelu(h, I0_o, 30, 8, out_o))
