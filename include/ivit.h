@@ -220,6 +220,39 @@ size_t ivit_block_workspace_bytes(int32_t B, int32_t N, int32_t D, int32_t Dm);
 ivit_status ivit_block_forward(const ivit_block_params *p, const int8_t *x, int8_t *y, void *workspace,
                                size_t workspace_bytes, int32_t B, int32_t N, ivit_stream_t stream);
 
+/* Size of the device array that ivit_block_forward_static keeps its
+ * intermediates in: 32 MiB on every GPU that loads the library.            */
+#define IVIT_STATIC_SCRATCH_BYTES ((size_t)32 << 20)
+
+/* The encoder block without a workspace argument and without allocating.
+ * The pages have no counterpart: this is a deployment convenience.
+ *
+ * For callers that cannot allocate device memory at all: an inference-server
+ * plugin whose host gives it no allocator, code inside a framework whose
+ * caching allocator already holds the whole device, or a latency-critical
+ * loop that cannot pay for cudaMalloc/cudaFree (which may synchronise the
+ * device).  The intermediates that ivit_block_forward keeps in the caller's
+ * workspace live instead in one fixed array of IVIT_STATIC_SCRATCH_BYTES in
+ * device memory, defined by the library; every GPU that loads the library
+ * holds it until the process exits.  The caller still passes the inputs x,
+ * the outputs y and the parameters, exactly as for ivit_block_forward.
+ *
+ * - Returns IVIT_ERR_UNSUPPORTED, with nothing enqueued, when
+ *   ivit_block_workspace_bytes(B, N, p->D, p->Dm) exceeds
+ *   IVIT_STATIC_SCRATCH_BYTES (e.g. more than 22 images of 197 tokens at
+ *   ViT-B width); all other checks and errors are those of
+ *   ivit_block_forward.
+ * - The first call on a device looks up the array's device address
+ *   (cudaGetSymbolAddress, with that device current); make that first call
+ *   before any stream capture.  No call allocates or frees memory.
+ * - Every call on a device shares the one array, and it keeps whatever the
+ *   last call left in it (no intermediate needs to start at zero).  Calls
+ *   whose work overlaps on the GPU -- on different streams, or from different
+ *   threads without ordering -- race on the array and corrupt each other's
+ *   results; order them on one stream.                                       */
+ivit_status ivit_block_forward_static(const ivit_block_params *p, const int8_t *x, int8_t *y, int32_t B,
+                                      int32_t N, ivit_stream_t stream);
+
 /* ---------------------------------------------------------------------------
  * Status
  * ------------------------------------------------------------------------- */

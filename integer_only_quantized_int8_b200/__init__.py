@@ -21,7 +21,7 @@ __all__ = [
     "ivit_status_string", "ivit_dyadic_from_double", "ivit_residual_from_double", "ivit_i0_from_scale",
     "ivit_linear_requant", "ivit_linear_shiftgelu", "ivit_attention", "ivit_shiftgelu", "ivit_layernorm",
     "ivit_block_workspace_bytes", "ivit_block_forward", "ivit_stream_status", "ivit_launch_count",
-    "EXPORTED_SYMBOLS",
+    "ivit_block_forward_static", "STATIC_SCRATCH_BYTES", "EXPORTED_SYMBOLS",
 ]
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
@@ -34,6 +34,7 @@ EXPORTED_SYMBOLS = (
     "ivit_linear_requant", "ivit_linear_shiftgelu", "ivit_attention", "ivit_shiftgelu", "ivit_layernorm",
     "ivit_block_workspace_bytes",
     "ivit_block_forward", "ivit_stream_status", "ivit_launch_count",
+    "ivit_block_forward_static",
 )
 
 _STATUS = {0: "IVIT_OK", 1: "IVIT_ERR_INVALID_ARG", 2: "IVIT_ERR_UNSUPPORTED", 3: "IVIT_ERR_CUDA",
@@ -105,6 +106,8 @@ def lib() -> C.CDLL:
             L.ivit_block_workspace_bytes.argtypes = [i32, i32, i32, i32]
             L.ivit_block_forward.restype = C.c_int
             L.ivit_block_forward.argtypes = [C.POINTER(BlockParams), vp, vp, vp, C.c_size_t, i32, i32, vp]
+            L.ivit_block_forward_static.restype = C.c_int
+            L.ivit_block_forward_static.argtypes = [C.POINTER(BlockParams), vp, vp, i32, i32, vp]
             L.ivit_stream_status.restype = C.c_int
             L.ivit_stream_status.argtypes = [vp]
             L.ivit_launch_count.restype = C.c_uint64
@@ -253,6 +256,24 @@ def ivit_block_forward(params, x, y, workspace, B: int, N: int, stream=None):
                                   _ptr(workspace, torch.uint8, "workspace"), workspace.numel(), int(B), int(N),
                                   _stream(stream))
     _check("ivit_block_forward", st)
+    return y
+
+
+# Bytes of the library's fixed device array (IVIT_STATIC_SCRATCH_BYTES).
+STATIC_SCRATCH_BYTES = 32 << 20
+
+
+def ivit_block_forward_static(params, x, y, B: int, N: int, stream=None):
+    """One encoder block without a workspace, for callers that cannot allocate
+    device memory (plugins without an allocator, code inside a framework that
+    has reserved the whole device, loops that cannot afford cudaMalloc).  The
+    intermediates live in the library's own 32 MiB device array, shared by all
+    calls on a device: calls that overlap on the GPU race.  Larger batches
+    raise IvitError (IVIT_ERR_UNSUPPORTED)."""
+    p = params.c if hasattr(params, "c") else params
+    st = lib().ivit_block_forward_static(C.byref(p), _ptr(x, torch.int8, "x"), _ptr(y, torch.int8, "y"), int(B),
+                                         int(N), _stream(stream))
+    _check("ivit_block_forward_static", st)
     return y
 
 
