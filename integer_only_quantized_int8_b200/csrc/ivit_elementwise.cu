@@ -5,9 +5,12 @@
 // input and scalar parameters, so each CTA tabulates the 256 possible outputs
 // with the integer formula and streams 16-byte vectors through the table.
 //
-// I-LayerNorm (same page, section 3.5): one warp per row; sums of x and x^2
-// with dp4a, exact integer variance, 10 Newton steps of the integer square
-// root, then the per-element normalisation, affine and dyadic requant.
+// I-LayerNorm (same page, section 3.5): one half-warp per row, so a whole
+// activation tensor is in flight in one wave; sums of x and x^2 with dp4a,
+// exact integer variance, 10 Newton steps of the integer square root, then the
+// per-element normalisation, affine and dyadic requant.
+#include <climits>
+
 #include "ivit_common.cuh"
 #include "ivit_internal.h"
 
@@ -48,15 +51,7 @@ __global__ void __launch_bounds__(kGeluThreads)
   }
 }
 
-constexpr int kLnWarps = 8;
-constexpr int kLnMaxChunks = 4;  // 16-byte chunks per lane: cols <= 32 * 16 * 4 = 2048
-
-// floor(a / b) for b > 0
-__device__ __forceinline__ int64_t floordiv64(int64_t a, int64_t b) {
-  int64_t q = a / b;
-  if ((a % b) != 0 && a < 0) q -= 1;
-  return q;
-}
+constexpr int kLnThreads = 256;  // 16 half-warps: one row each
 
 __device__ __forceinline__ int32_t isqrt_newton10(int32_t V) {
   if (V <= 0) return 0;
@@ -67,21 +62,48 @@ __device__ __forceinline__ int32_t isqrt_newton10(int32_t V) {
   return I;
 }
 
-__global__ void __launch_bounds__(kLnWarps * 32)
+// Saturation bounds of the output requant sat_8((b acc) >> c): clamping acc to
+// [lo, hi] keeps every unsaturated result and the direction of the others,
+// and keeps (b acc) >> c inside int32.
+__device__ __forceinline__ void out_bounds(int32_t b, int32_t c, int32_t& lo, int32_t& hi) {
+  if (b == 0) {
+    lo = INT_MIN;
+    hi = INT_MAX;
+    return;
+  }
+  const int64_t p2 = (int64_t)1 << c;
+  const int64_t vhi = (127 * p2 + b - 1) / b;       // first acc with result >= 127
+  const int64_t num = -127 * p2 - 1;                 // results <= -128: b acc <= num
+  const int64_t vlo = -((-num + b - 1) / b);
+  hi = (int32_t)(vhi > INT_MAX ? INT_MAX : vhi);
+  lo = (int32_t)(vlo < INT_MIN ? INT_MIN : vlo);
+}
+
+__device__ __forceinline__ uint32_t pack_sat4_ln(int32_t y0, int32_t y1, int32_t y2, int32_t y3) {
+  uint32_t t, d;
+  asm("cvt.pack.sat.s8.s32.b32 %0, %1, %2, %3;" : "=r"(t) : "r"(y3), "r"(y2), "r"(0u));
+  asm("cvt.pack.sat.s8.s32.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(y1), "r"(y0), "r"(t));
+  return d;
+}
+
+// One row of `cols` int8 values per half-warp; lane l of the half-warp holds
+// the 16-byte chunks l, l + 16, ... (CPL of them).
+template <int CPL>
+__global__ void __launch_bounds__(kLnThreads)
     layernorm_kernel(const int8_t* __restrict__ x, int64_t rows, int32_t cols, const int8_t* __restrict__ gamma,
                      const int32_t* __restrict__ beta, int32_t F, int32_t M_ln, ivit_dyadic out,
                      int8_t* __restrict__ y) {
-  const int lane = threadIdx.x & 31;
-  const int64_t row = (int64_t)blockIdx.x * kLnWarps + (threadIdx.x >> 5);
-  if (row >= rows) return;
+  const int hl = threadIdx.x & 15;
+  const int64_t row = (int64_t)blockIdx.x * (kLnThreads / 16) + (threadIdx.x >> 4);
+  const bool active = row < rows;
   const int nchunk = cols >> 4;
-  const int8_t* xr = x + row * cols;
-  int4 v[kLnMaxChunks];
+  const int8_t* xr = x + (active ? row : 0) * cols;
+  int4 v[CPL];
   int32_t s1 = 0, s2 = 0;
 #pragma unroll
-  for (int k = 0; k < kLnMaxChunks; ++k) {
-    const int ci = lane + 32 * k;
-    if (ci < nchunk) {
+  for (int k = 0; k < CPL; ++k) {
+    const int ci = hl + 16 * k;
+    if (active && ci < nchunk) {
       v[k] = __ldcs(reinterpret_cast<const int4*>(xr) + ci);
       const int w[4] = {v[k].x, v[k].y, v[k].z, v[k].w};
 #pragma unroll
@@ -92,38 +114,47 @@ __global__ void __launch_bounds__(kLnWarps * 32)
     }
   }
 #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) {
+  for (int o = 8; o > 0; o >>= 1) {  // reduce within each half-warp
     s1 += __shfl_xor_sync(0xffffffffu, s1, o);
     s2 += __shfl_xor_sync(0xffffffffu, s2, o);
   }
-  // mu = floor(sum x / n); sum (x - mu)^2 = sum x^2 - 2 mu sum x + n mu^2 (exact)
-  const int64_t mu = floordiv64(s1, cols);
-  const int64_t sd2 = (int64_t)s2 - 2 * mu * (int64_t)s1 + (int64_t)cols * mu * mu;
-  const int32_t V = (int32_t)(sd2 / cols);  // sd2 >= 0: truncation == floor
+  if (!active) return;
+  // mu = floor(sum x / n); sum (x - mu)^2 = sum x^2 - 2 mu sum x + n mu^2, all within int32
+  int32_t mu = s1 / cols;
+  if ((s1 % cols) != 0 && s1 < 0) mu -= 1;
+  const int32_t sd2 = s2 - 2 * mu * s1 + cols * mu * mu;
+  const int32_t V = sd2 / cols;  // sd2 >= 0: truncation == floor
   int32_t sigma = isqrt_newton10(V);
   if (sigma < 1) sigma = 1;
   const int32_t f = (1 << M_ln) / sigma;
   const int sh = M_ln - F;
-  const int32_t m32 = (int32_t)mu;
+  int32_t lo, hi;
+  out_bounds(out.b, out.c, lo, hi);
   int8_t* yr = y + row * cols;
 #pragma unroll
-  for (int k = 0; k < kLnMaxChunks; ++k) {
-    const int ci = lane + 32 * k;
+  for (int k = 0; k < CPL; ++k) {
+    const int ci = hl + 16 * k;
     if (ci < nchunk) {
       const int c0 = ci * 16;
       const int4 gv = __ldg(reinterpret_cast<const int4*>(gamma + c0));
-      const int8_t* gb = reinterpret_cast<const int8_t*>(&gv);
-      const int8_t* xb = reinterpret_cast<const int8_t*>(&v[k]);
-      int32_t bt[16];
+      const uint32_t gw[4] = {(uint32_t)gv.x, (uint32_t)gv.y, (uint32_t)gv.z, (uint32_t)gv.w};
+      const uint32_t xw[4] = {(uint32_t)v[k].x, (uint32_t)v[k].y, (uint32_t)v[k].z, (uint32_t)v[k].w};
+      uint32_t o[4];
 #pragma unroll
-      for (int q = 0; q < 4; ++q) *reinterpret_cast<int4*>(&bt[4 * q]) = __ldg(reinterpret_cast<const int4*>(beta + c0) + q);
-      uint32_t o[4] = {0, 0, 0, 0};
+      for (int q = 0; q < 4; ++q) {
+        const int4 bt = __ldg(reinterpret_cast<const int4*>(beta + c0) + q);
+        const int32_t bb[4] = {bt.x, bt.y, bt.z, bt.w};
+        int32_t r[4];
 #pragma unroll
-      for (int e = 0; e < 16; ++e) {
-        const int32_t d = (int32_t)xb[e] - m32;
-        const int32_t nv = (d * f) >> sh;
-        const int32_t acc = nv * (int32_t)gb[e] + bt[e];
-        o[e >> 2] |= ((uint32_t)requant8(acc, out.b, out.c) & 0xFFu) << (8 * (e & 3));
+        for (int e = 0; e < 4; ++e) {
+          const int32_t d = (int32_t)(int8_t)(uint8_t)(xw[q] >> (8 * e)) - mu;
+          const int32_t nv = (d * f) >> sh;
+          const int32_t acc = nv * (int32_t)(int8_t)(uint8_t)(gw[q] >> (8 * e)) + bb[e];
+          const int32_t a = min(max(acc, lo), hi);
+          const int64_t pr = (int64_t)out.b * a;  // (b a) >> c fits int32: one funnel shift
+          r[e] = (int32_t)__funnelshift_r((uint32_t)pr, (uint32_t)(pr >> 32), (uint32_t)out.c);
+        }
+        o[q] = pack_sat4_ln(r[0], r[1], r[2], r[3]);
       }
       __stcs(reinterpret_cast<int4*>(yr) + ci, make_int4((int)o[0], (int)o[1], (int)o[2], (int)o[3]));
     }
@@ -150,9 +181,20 @@ ivit_status launch_layernorm(const DeviceCtx& dc, const int8_t* x, int64_t rows,
                              int8_t* y, cudaStream_t stream) {
   (void)dc;
   if (rows == 0) return IVIT_OK;
-  const int64_t blocks = (rows + kLnWarps - 1) / kLnWarps;
+  const int64_t blocks = (rows + kLnThreads / 16 - 1) / (kLnThreads / 16);
   if (blocks > 0x7fffffff) return IVIT_ERR_UNSUPPORTED;
-  layernorm_kernel<<<(unsigned)blocks, kLnWarps * 32, 0, stream>>>(x, rows, cols, gamma, beta, F, M_ln, out, y);
+  const unsigned g = (unsigned)blocks;
+  const int nchunk = cols / 16;
+  if (nchunk <= 16)
+    layernorm_kernel<1><<<g, kLnThreads, 0, stream>>>(x, rows, cols, gamma, beta, F, M_ln, out, y);
+  else if (nchunk <= 32)
+    layernorm_kernel<2><<<g, kLnThreads, 0, stream>>>(x, rows, cols, gamma, beta, F, M_ln, out, y);
+  else if (nchunk <= 48)
+    layernorm_kernel<3><<<g, kLnThreads, 0, stream>>>(x, rows, cols, gamma, beta, F, M_ln, out, y);
+  else if (nchunk <= 64)
+    layernorm_kernel<4><<<g, kLnThreads, 0, stream>>>(x, rows, cols, gamma, beta, F, M_ln, out, y);
+  else
+    layernorm_kernel<8><<<g, kLnThreads, 0, stream>>>(x, rows, cols, gamma, beta, F, M_ln, out, y);
   note_launch();
   return cudaGetLastError() == cudaSuccess ? IVIT_OK : IVIT_ERR_CUDA;
 }

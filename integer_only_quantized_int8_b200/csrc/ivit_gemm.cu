@@ -6,29 +6,39 @@
 // Efficient Vision Transformer Inference", sections 3.1, 3.2 and 3.4; the
 // Trio-ViT article, eqs. (1) and (12)).
 //
-// Design (one CTA per SM, persistent over 128 x BN output tiles):
-//   warp 0      TMA producer: 128 x 128 A and BN x 128 B k-slices, 128B swizzle,
+// The accumulator is computed transposed, D = W X^T: the UMMA M dimension
+// (TMEM lanes) runs over 128 output channels and N over BN tokens.  Every
+// epilogue thread therefore owns one output channel of the tile and keeps that
+// channel's multiplier, shift, bias and saturation bounds in registers; the
+// per-element work is a clamp, one 32x32->64 multiply-add, one funnel shift
+// and a saturating byte pack.  A 4 x 4 byte transpose across lanes turns the
+// channel-major bytes into token-major 4-byte words for coalesced stores.
+//
+// Roles (one CTA per SM, persistent over 128 x BN tiles):
+//   warp 0      TMA producer: W and X k-slices of 128 bytes, 128B swizzle,
 //               into a STAGES-deep ring guarded by full/empty mbarriers;
-//   warp 1      allocates TMEM (2 x BN columns) and one lane issues
+//   warp 1      allocates TMEM (two BN-column accumulators) and one lane issues
 //               tcgen05.mma M=128 N=BN K=32; tcgen05.commit frees smem stages
 //               and publishes finished accumulators;
-//   warps 2-5   epilogue: tcgen05.ld 32 columns at a time, bias, dyadic
-//               requant, saturation, optional residual / GELU table, 16-byte
-//               stores.  Two accumulators let the epilogue of tile t overlap
-//               the MMAs of tile t+1.
+//   warps 2-9   epilogue: two warps per TMEM lane quarter split the tile's
+//               token chunks; the accumulator of tile t drains while the
+//               MMAs of tile t+1 run.
+#include <climits>
+
 #include "ivit_common.cuh"
 #include "ivit_internal.h"
 
 namespace ivit {
 namespace {
 
-constexpr int kBM = 128;
+constexpr int kBM = 128;  // output channels per tile
 constexpr int kBK = 128;  // bytes = int8 elements per k-slice (one 128-byte swizzle row)
-constexpr int kGemmThreads = 192;
+constexpr int kEpiWarps = 8;  // two per TMEM lane quarter
+constexpr int kGemmThreads = 64 + 32 * kEpiWarps;
 
 struct GemmArgs {
-  int64_t M;
-  int32_t N, K;
+  int64_t M;       // tokens (rows of X and Y)
+  int32_t N, K;    // output channels, reduction length
   const int32_t* bias;
   const int32_t* b;
   const int8_t* c;
@@ -51,11 +61,178 @@ struct GemmLayout {
   static constexpr int kGeluOff = kSlotOff + 16;
   static constexpr int kBytes = kGeluOff + 256;
   static constexpr int kAlloc = kBytes + 1024;  // slack to align the base to 1024 bytes
+  static constexpr int kTmemCols = (2 * BN <= 256) ? 256 : 512;
 };
 
-template <int BN, int STAGES, int EPI>
+IVIT_DEV int32_t sat_i32(int64_t v) {
+  return (int32_t)(v < (int64_t)INT_MIN ? (int64_t)INT_MIN : (v > (int64_t)INT_MAX ? (int64_t)INT_MAX : v));
+}
+
+// Per-channel constants of the requant sat((b (acc + bias)) >> c), b >= 0.
+// With v = acc + bias the result floor(b v / 2^c) is monotone in v.  With
+// bl = bit length of b, s = bl - 1 - c (so 2^s <= b / 2^c < 2^(s+1)) and
+// u = 128 / 2^s (u = 1 once s >= 7), v = u gives a result >= 128 and v = -u
+// one <= -128, while every v in [-u, u] gives a result of magnitude at most
+// max(256, b / 2^c) < 2^31.  Clamping acc to [-u - bias, u - bias] therefore
+// changes no result inside the int8 range (nor any narrower range), sends
+// everything beyond to a value that saturates the same way, and keeps the
+// shifted result within int32: the saturating byte pack then finishes the
+// job.  When even the largest possible |acc + bias| (2^14 K + |bias|) keeps
+// |b (acc + bias)| below 2^(30 + c), the shifted result always fits int32 and
+// the clamp is skipped.
+struct ChanConst {
+  int32_t b, c, lo_acc, hi_acc;
+  int64_t bb;       // b * bias
+  bool needs_clamp;
+};
+
+IVIT_DEV ChanConst chan_const(int32_t b, int32_t c, int32_t bias, int32_t K) {
+  ChanConst k;
+  k.b = b;
+  k.c = c;
+  k.bb = (int64_t)b * bias;
+  if (b == 0) {
+    k.lo_acc = INT_MIN;
+    k.hi_acc = INT_MAX;
+    k.needs_clamp = false;
+    return k;
+  }
+  const int bl = 32 - __clz(b);
+  const int s = bl - 1 - c;                                   // 2^s <= b / 2^c < 2^(s+1)
+  const int64_t u = s >= 7 ? 1 : (s >= 0 ? (128 >> s) : ((int64_t)128 << (-s)));
+  const int64_t hi = u - bias, lo = -u - bias;
+  k.hi_acc = sat_i32(hi);
+  k.lo_acc = sat_i32(lo);
+  const int64_t vmax = (int64_t)K * 16384 + (bias < 0 ? -(int64_t)bias : (int64_t)bias);
+  k.needs_clamp = vmax * (int64_t)b >= ((int64_t)1 << (30 + c));
+  return k;
+}
+
+// floor(b (acc + bias) / 2^c) for acc within the bounds above; fits int32, so
+// the low word of the 64-bit shift is one funnel shift (c <= 31)
+template <bool CLAMP>
+IVIT_DEV int32_t requant_clamped(int32_t acc, const ChanConst& k) {
+  const int32_t a = CLAMP ? min(max(acc, k.lo_acc), k.hi_acc) : acc;
+  const int64_t v = (int64_t)k.b * a + k.bb;
+  return (int32_t)__funnelshift_r((uint32_t)v, (uint32_t)(v >> 32), (uint32_t)k.c);
+}
+
+// bytes [sat8(y0), sat8(y1), sat8(y2), sat8(y3)]
+IVIT_DEV uint32_t pack_sat4(int32_t y0, int32_t y1, int32_t y2, int32_t y3) {
+  uint32_t t, d;
+  asm("cvt.pack.sat.s8.s32.b32 %0, %1, %2, %3;" : "=r"(t) : "r"(y3), "r"(y2), "r"(0u));
+  asm("cvt.pack.sat.s8.s32.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(y1), "r"(y0), "r"(t));
+  return d;
+}
+
+// sign-extended byte i of w
+IVIT_DEV int32_t sbyte(uint32_t w, int i) { return (int32_t)(int8_t)(uint8_t)(w >> (8 * i)); }
+
+// 4 x 4 byte transpose among lanes 4g..4g+3: lane l enters with byte i =
+// element (i, l) and leaves with byte i = element (l, i).  sel2 / sel1 are
+// the lane's byte selectors, (lane & 2) ? 0x3276 : 0x5410 and
+// (lane & 1) ? 0x3715 : 0x6240.
+IVIT_DEV uint32_t transpose4x4(uint32_t w, uint32_t sel2, uint32_t sel1) {
+  uint32_t o = __shfl_xor_sync(0xffffffffu, w, 2);
+  w = __byte_perm(w, o, sel2);
+  o = __shfl_xor_sync(0xffffffffu, w, 1);
+  return __byte_perm(w, o, sel1);
+}
+
+// One 32-token chunk of one epilogue warp: requant the 32 accumulators of this
+// thread's channel, pack, transpose to token-major words, apply the residual
+// if any, and store.  r holds TMEM columns [32 cc, 32 cc + 32) of lane ch.
+template <int EPI, bool NARROW, bool CLAMP>
+IVIT_DEV void epi_chunk(const uint32_t (&r)[32], const ChanConst& kc, const GemmArgs& args, const int8_t* gelu_tab,
+                        int64_t tok0, int ch4, int sub, uint32_t sel2, uint32_t sel1, bool fast_res) {
+  const int64_t M = args.M;
+  const int N = args.N;
+  uint32_t w[8];
+#pragma unroll
+  for (int k = 0; k < 8; ++k) {
+    int32_t y[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      int32_t v = requant_clamped<CLAMP>((int32_t)r[4 * k + i], kc);
+      if (EPI == kEpiGelu) {
+        v = min(max(v, -128), 127);
+        v = gelu_tab[v + 128];
+      } else if (NARROW) {
+        v = min(max(v, args.lo), args.hi);
+      }
+      y[i] = v;
+    }
+    w[k] = transpose4x4(pack_sat4(y[0], y[1], y[2], y[3]), sel2, sel1);
+  }
+  // lane (4 grp + sub) now holds, for k = 0..7, token tok0 + 4k + sub, channels ch4..ch4+3
+  if (ch4 >= N) return;
+  // word k goes to token tok0 + 4k + sub: a fixed stride of 4N bytes
+  const int64_t off0 = (tok0 + sub) * N + ch4;
+  const int64_t stride = 4 * (int64_t)N;
+  const bool full = tok0 + 32 <= M;
+  if (EPI == kEpiResidual) {
+    // all eight skip words are requested before any store, so their latencies overlap
+    uint32_t s[8];
+    const int8_t* sp = args.skip + off0;
+#pragma unroll
+    for (int k = 0; k < 8; ++k)
+      s[k] = (full || tok0 + 4 * k + sub < M) ? __ldg(reinterpret_cast<const uint32_t*>(sp + k * stride)) : 0u;
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      int32_t z[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int64_t sum = (int64_t)args.res.b_skip * sbyte(s[k], i) + (int64_t)args.res.b_branch * sbyte(w[k], i);
+        if (fast_res) {
+          z[i] = (int32_t)__funnelshift_r((uint32_t)sum, (uint32_t)(sum >> 32), (uint32_t)args.res.c);
+        } else {
+          const int64_t q = sum >> args.res.c;
+          z[i] = (int32_t)(q < -128 ? -128 : (q > 127 ? 127 : q));
+        }
+      }
+      w[k] = pack_sat4(z[0], z[1], z[2], z[3]);
+    }
+  }
+  int8_t* yp = args.Y + off0;
+  if (full) {
+#pragma unroll
+    for (int k = 0; k < 8; ++k) *reinterpret_cast<uint32_t*>(yp + k * stride) = w[k];
+  } else {
+#pragma unroll
+    for (int k = 0; k < 8; ++k)
+      if (tok0 + 4 * k + sub < M) *reinterpret_cast<uint32_t*>(yp + k * stride) = w[k];
+  }
+}
+
+// The chunks [c_begin, c_end) of one tile, with the next chunk's TMEM load in
+// flight while the current chunk is processed.
+template <int EPI, bool NARROW, bool CLAMP>
+IVIT_DEV void epi_tile(uint32_t tbase, int c_begin, int c_end, int64_t tok_base, const ChanConst& kc,
+                       const GemmArgs& args, const int8_t* gelu_tab, int ch4, int sub, uint32_t sel2, uint32_t sel1,
+                       bool fast_res) {
+  const int64_t M = args.M;
+  int n = c_end - c_begin;  // chunks that hold at least one valid token
+  while (n > 0 && tok_base + 32 * (c_begin + n - 1) >= M) --n;
+  if (n <= 0) return;
+  uint32_t ra[32], rb[32];
+  tmem_ld32(tbase + (uint32_t)(32 * c_begin), ra);
+  for (int i = 0; i < n; i += 2) {
+    const int ca = c_begin + i;
+    tmem_ld_wait();
+    if (i + 1 < n) tmem_ld32(tbase + (uint32_t)(32 * (ca + 1)), rb);
+    epi_chunk<EPI, NARROW, CLAMP>(ra, kc, args, gelu_tab, tok_base + 32 * ca, ch4, sub, sel2, sel1, fast_res);
+    if (i + 1 < n) {
+      tmem_ld_wait();
+      if (i + 2 < n) tmem_ld32(tbase + (uint32_t)(32 * (ca + 2)), ra);
+      epi_chunk<EPI, NARROW, CLAMP>(rb, kc, args, gelu_tab, tok_base + 32 * (ca + 1), ch4, sub, sel2, sel1,
+                                    fast_res);
+    }
+  }
+}
+
+template <int BN, int STAGES, int EPI, bool NARROW>
 __global__ void __launch_bounds__(kGemmThreads, 1)
-    gemm_i8_requant_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+    gemm_i8_requant_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX,
                            const GemmArgs args) {
   using L = GemmLayout<BN, STAGES>;
   extern __shared__ uint8_t smem_raw[];
@@ -72,9 +249,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   const int lane = threadIdx.x & 31;
   const int64_t M = args.M;
   const int N = args.N;
-  const int m_tiles = (int)((M + kBM - 1) / kBM);
-  const int n_tiles = (N + BN - 1) / BN;
-  const int num_tiles = m_tiles * n_tiles;
+  const int ch_tiles = (N + kBM - 1) / kBM;
+  const int tok_tiles = (int)((M + BN - 1) / BN);
+  const int num_tiles = ch_tiles * tok_tiles;
   const int num_kb = (args.K + kBK - 1) / kBK;
 
   if (threadIdx.x == 0) {
@@ -84,12 +261,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&tfull[a], 1);
-      mbar_init(&tempty[a], 128);
+      mbar_init(&tempty[a], kEpiWarps);
     }
     mbar_init(drain, 1);
     fence_barrier_init();
-    prefetch_tensormap(&tmA);
-    prefetch_tensormap(&tmB);
+    prefetch_tensormap(&tmW);
+    prefetch_tensormap(&tmX);
   }
   if (EPI == kEpiGelu) {
     for (int i = threadIdx.x; i < 256; i += blockDim.x)
@@ -98,7 +275,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   }
   if (warp == 1) {
     __syncwarp();
-    tmem_alloc(tslot, 2 * BN);
+    tmem_alloc(tslot, L::kTmemCols);
     tmem_relinquish();
   }
   tc_fence_before();
@@ -114,7 +291,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       bool ok = true;
       int issued = 0;
       for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
-        const int mb = t / n_tiles, nb = t % n_tiles;
+        const int cb = t % ch_tiles, tb = t / ch_tiles;
         for (int kb = 0; kb < num_kb; ++kb) {
           if (!mbar_wait(&empty[stage], phase ^ 1, args.status)) {
             ok = false;
@@ -122,8 +299,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           }
           mbar_arrive_expect_tx(&full[stage], L::kStageBytes);
           uint8_t* sa = smem + stage * L::kStageBytes;
-          tma_load_2d(sa, &tmA, kb * kBK, mb * kBM, &full[stage]);
-          tma_load_2d(sa + L::kABytes, &tmB, kb * kBK, nb * BN, &full[stage]);
+          tma_load_2d(sa, &tmW, kb * kBK, cb * kBM, &full[stage]);
+          tma_load_2d(sa + L::kABytes, &tmX, kb * kBK, tb * BN, &full[stage]);
           ++issued;
           if (++stage == STAGES) {
             stage = 0;
@@ -184,73 +361,45 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     }
   } else {
     // ------------------------------------------------------------ epilogue
-    const int quarter = warp & 3;  // TMEM lanes [32 * quarter, 32 * quarter + 32)
-    const int row_local = quarter * 32 + lane;
+    constexpr int kChunks = BN / 32;
+    constexpr int kPerQuarter = kEpiWarps / 4;
+    const int e = warp - 2;
+    const int quarter = warp & 3;  // TMEM lanes [32 q, 32 q + 32) = channels of this warp
+    const int part = e >> 2;       // which of the quarter's warps: splits the token chunks
+    const int c_begin = (kChunks * part) / kPerQuarter;
+    const int c_end = (kChunks * (part + 1)) / kPerQuarter;
+    const uint32_t sel2 = (lane & 2) ? 0x3276u : 0x5410u;
+    const uint32_t sel1 = (lane & 1) ? 0x3715u : 0x6240u;
+    const int sub = lane & 3;               // token offset within a transposed 4 x 4 block
+    const int grp = lane >> 2;              // channel group of 4 within the warp's 32 channels
+    const bool fast_res = args.res.c >= 9;  // |b_skip s + b_branch y| < 2^39: the shifted sum fits int32
     int acc = 0;
     uint32_t acc_phase = 0;
     for (int t = blockIdx.x; t < num_tiles; t += gridDim.x) {
-      const int mb = t / n_tiles, nb = t % n_tiles;
+      const int cb = t % ch_tiles, tb = t / ch_tiles;
+      const int ch = cb * kBM + quarter * 32 + lane;      // this thread's output channel
+      const int ch4 = cb * kBM + quarter * 32 + grp * 4;  // first channel of the stored word
+      ChanConst kc;
+      if (ch < N)
+        kc = chan_const(__ldg(args.b + ch), (int32_t)__ldg(args.c + ch), args.bias ? __ldg(args.bias + ch) : 0,
+                        args.K);
+      else
+        kc = chan_const(0, 0, 0, args.K);
+      const bool clamp = __any_sync(0xffffffffu, kc.needs_clamp);  // warp-uniform path choice
       const bool got = mbar_wait(&tfull[acc], acc_phase, args.status);
       if (!__all_sync(0xffffffffu, got)) break;  // warp-uniform give-up
       tc_fence_after();
-      const int64_t row = (int64_t)mb * kBM + row_local;
       const uint32_t tbase = tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(acc * BN);
-#pragma unroll 1
-      for (int ch = 0; ch < BN / 32; ++ch) {
-        const int col0 = nb * BN + ch * 32;
-        if (col0 >= N) break;  // warp-uniform
-        uint32_t r[32];
-        __syncwarp();
-        tmem_ld32(tbase + (uint32_t)(ch * 32), r);
-        tmem_ld_wait();
-        if (row < M) {
-#pragma unroll
-          for (int half = 0; half < 2; ++half) {
-            const int col = col0 + half * 16;
-            if (col < N) {
-              int32_t bb[16], bi[16];
-              int8_t cc[16];
-              *reinterpret_cast<int4*>(&bb[0]) = __ldg(reinterpret_cast<const int4*>(args.b + col));
-              *reinterpret_cast<int4*>(&bb[4]) = __ldg(reinterpret_cast<const int4*>(args.b + col + 4));
-              *reinterpret_cast<int4*>(&bb[8]) = __ldg(reinterpret_cast<const int4*>(args.b + col + 8));
-              *reinterpret_cast<int4*>(&bb[12]) = __ldg(reinterpret_cast<const int4*>(args.b + col + 12));
-              if (args.bias) {
-                *reinterpret_cast<int4*>(&bi[0]) = __ldg(reinterpret_cast<const int4*>(args.bias + col));
-                *reinterpret_cast<int4*>(&bi[4]) = __ldg(reinterpret_cast<const int4*>(args.bias + col + 4));
-                *reinterpret_cast<int4*>(&bi[8]) = __ldg(reinterpret_cast<const int4*>(args.bias + col + 8));
-                *reinterpret_cast<int4*>(&bi[12]) = __ldg(reinterpret_cast<const int4*>(args.bias + col + 12));
-              } else {
-#pragma unroll
-                for (int i = 0; i < 16; ++i) bi[i] = 0;
-              }
-              *reinterpret_cast<int4*>(&cc[0]) = __ldg(reinterpret_cast<const int4*>(args.c + col));
-              int4 sk = make_int4(0, 0, 0, 0);
-              if (EPI == kEpiResidual)
-                sk = __ldg(reinterpret_cast<const int4*>(args.skip + row * N + col));
-              const int8_t* skb = reinterpret_cast<const int8_t*>(&sk);
-              uint32_t packed[4];
-#pragma unroll
-              for (int w = 0; w < 4; ++w) {
-                uint32_t word = 0;
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                  const int i = w * 4 + e;
-                  const int32_t v = (int32_t)r[half * 16 + i] + bi[i];
-                  int32_t y = requant_bits(v, bb[i], (int32_t)cc[i], args.lo, args.hi);
-                  if (EPI == kEpiResidual) y = residual8(skb[i], y, args.res.b_skip, args.res.b_branch, args.res.c);
-                  if (EPI == kEpiGelu) y = gelu_tab[y + 128];
-                  word |= ((uint32_t)y & 0xFFu) << (8 * e);
-                }
-                packed[w] = word;
-              }
-              *reinterpret_cast<int4*>(args.Y + row * N + col) =
-                  make_int4((int)packed[0], (int)packed[1], (int)packed[2], (int)packed[3]);
-            }
-          }
-        }
-      }
+      __syncwarp();
+      if (clamp)
+        epi_tile<EPI, NARROW, true>(tbase, c_begin, c_end, (int64_t)tb * BN, kc, args, gelu_tab, ch4, sub, sel2, sel1,
+                                    fast_res);
+      else
+        epi_tile<EPI, NARROW, false>(tbase, c_begin, c_end, (int64_t)tb * BN, kc, args, gelu_tab, ch4, sub, sel2,
+                                     sel1, fast_res);
       tc_fence_before();
-      mbar_arrive(&tempty[acc]);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&tempty[acc]);
       acc ^= 1;
       if (acc == 0) acc_phase ^= 1;
     }
@@ -261,43 +410,71 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   if (warp == 1) {
     __syncwarp();
     tc_fence_after();
-    tmem_dealloc(tmem_base, 2 * BN);
+    tmem_dealloc(tmem_base, L::kTmemCols);
   }
 }
 
-template <int BN, int STAGES, int EPI>
+template <int BN, int STAGES, int EPI, bool NARROW>
 ivit_status run_gemm(const DeviceCtx& dc, const int8_t* X, const int8_t* W, const GemmArgs& a,
                      cudaStream_t stream) {
   using L = GemmLayout<BN, STAGES>;
   static_assert(L::kAlloc <= 227 * 1024, "shared memory budget");
-  CUtensorMap tmA, tmB;
-  ivit_status st = encode_tmap_2d_u8(&tmA, X, (uint64_t)a.K, (uint64_t)a.M, (uint64_t)a.K, kBK, kBM,
+  CUtensorMap tmW, tmX;
+  ivit_status st = encode_tmap_2d_u8(&tmW, W, (uint64_t)a.K, (uint64_t)a.N, (uint64_t)a.K, kBK, kBM,
                                      CU_TENSOR_MAP_SWIZZLE_128B);
   if (st != IVIT_OK) return st;
-  st = encode_tmap_2d_u8(&tmB, W, (uint64_t)a.K, (uint64_t)a.N, (uint64_t)a.K, kBK, BN,
+  st = encode_tmap_2d_u8(&tmX, X, (uint64_t)a.K, (uint64_t)a.M, (uint64_t)a.K, kBK, BN,
                          CU_TENSOR_MAP_SWIZZLE_128B);
   if (st != IVIT_OK) return st;
-  auto kern = gemm_i8_requant_kernel<BN, STAGES, EPI>;
+  auto kern = gemm_i8_requant_kernel<BN, STAGES, EPI, NARROW>;
   static bool attr_done = false;  // benign race: the attribute value is the same
   if (!attr_done) {
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAlloc) != cudaSuccess)
       return IVIT_ERR_CUDA;
     attr_done = true;
   }
-  const int m_tiles = (int)((a.M + kBM - 1) / kBM);
-  const int n_tiles = (a.N + BN - 1) / BN;
-  const int tiles = m_tiles * n_tiles;
+  const int tiles = ((a.N + kBM - 1) / kBM) * (int)((a.M + BN - 1) / BN);
   const int grid = tiles < dc.num_sms ? tiles : dc.num_sms;
-  kern<<<grid, kGemmThreads, L::kAlloc, stream>>>(tmA, tmB, a);
+  kern<<<grid, kGemmThreads, L::kAlloc, stream>>>(tmW, tmX, a);
   note_launch();
   return cudaGetLastError() == cudaSuccess ? IVIT_OK : IVIT_ERR_CUDA;
 }
 
-template <int EPI>
+// Token-tile width: fewest rounds of tiles over the SMs, weighted by the tile
+// width plus a fixed per-tile cost, so narrower tiles win only when they save
+// a round.
+int pick_bn(int64_t M, int N, int num_sms) {
+  static const int cands[] = {256, 224, 192, 160, 128};
+  const int ch_tiles = (N + kBM - 1) / kBM;
+  int best = 256;
+  int64_t best_cost = INT64_MAX;
+  for (int bn : cands) {
+    const int64_t tiles = (int64_t)ch_tiles * ((M + bn - 1) / bn);
+    const int64_t rounds = (tiles + num_sms - 1) / num_sms;
+    const int64_t cost = rounds * (bn + 32);
+    if (cost < best_cost) {
+      best_cost = cost;
+      best = bn;
+    }
+  }
+  return best;
+}
+
+template <int EPI, bool NARROW>
 ivit_status dispatch_bn(const DeviceCtx& dc, const int8_t* X, const int8_t* W, const GemmArgs& a,
                         cudaStream_t stream) {
-  if (a.N % 256 == 0) return run_gemm<256, 4, EPI>(dc, X, W, a, stream);
-  return run_gemm<128, 6, EPI>(dc, X, W, a, stream);
+  switch (pick_bn(a.M, a.N, dc.num_sms)) {
+    case 256:
+      return run_gemm<256, 4, EPI, NARROW>(dc, X, W, a, stream);
+    case 224:
+      return run_gemm<224, 5, EPI, NARROW>(dc, X, W, a, stream);
+    case 192:
+      return run_gemm<192, 5, EPI, NARROW>(dc, X, W, a, stream);
+    case 160:
+      return run_gemm<160, 6, EPI, NARROW>(dc, X, W, a, stream);
+    default:
+      return run_gemm<128, 7, EPI, NARROW>(dc, X, W, a, stream);
+  }
 }
 
 }  // namespace
@@ -320,13 +497,16 @@ ivit_status launch_gemm(const DeviceCtx& dc, const int8_t* X, int64_t M, int32_t
   a.Y = Y;
   a.gelu = gelu ? *gelu : GeluParams{1, 30, 8, {0, 0}};
   a.status = dc.status;
+  const bool narrow = out_bits < 8;
   switch (mode) {
     case kEpiPlain:
-      return dispatch_bn<kEpiPlain>(dc, X, W, a, stream);
+      return narrow ? dispatch_bn<kEpiPlain, true>(dc, X, W, a, stream)
+                    : dispatch_bn<kEpiPlain, false>(dc, X, W, a, stream);
     case kEpiResidual:
-      return dispatch_bn<kEpiResidual>(dc, X, W, a, stream);
+      return narrow ? dispatch_bn<kEpiResidual, true>(dc, X, W, a, stream)
+                    : dispatch_bn<kEpiResidual, false>(dc, X, W, a, stream);
     case kEpiGelu:
-      return dispatch_bn<kEpiGelu>(dc, X, W, a, stream);
+      return dispatch_bn<kEpiGelu, false>(dc, X, W, a, stream);
   }
   return IVIT_ERR_INTERNAL;
 }
