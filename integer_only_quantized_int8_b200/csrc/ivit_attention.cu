@@ -36,6 +36,7 @@ struct AttnArgs {
   int32_t logit_b, logit_c, ks_lo, ks_hi, k_s;
   int32_t I0, M, k_out;
   int32_t out_b, out_c;
+  int32_t o_lo, o_hi;  // accumulator clamp of the output requant (see out_clamp)
   int8_t* ctx;
   int* status;
 };
@@ -278,39 +279,56 @@ __global__ void __launch_bounds__(kAttnThreads)
 }
 
 // ---------------------------------------------------------------------------
-// Short sequences (N <= 256 keys): the whole score row stays in TMEM.
+// Short sequences (N <= 256 keys): persistent, warp-specialised kernel.
 //
-// 8 warps; warps w and w + 4 read the same TMEM lanes (query rows) and split
-// the key columns in two halves.  Pass 1 takes the row maximum of the raw
-// int32 scores (the logit requant is monotone, so max L = requant(max S)).
-// Pass 2 requantises each score, looks up ShiftExp(L - max L) in a table
-// replicated once per shared-memory bank (lane l reads copy l: no bank
-// conflicts), accumulates the row sum and writes the exponentials back into
-// TMEM in place.  Pass 3 turns them into u8 P = (Dv e) >> (M - k_out + 1),
-// written straight into the 128B-swizzled K-major operand of the P V MMA.
+// One CTA per SM walks the work items (128-query tile, head, image) with
+// stride gridDim.x.  Warp 0 issues the TMA loads of Q, K and V of the next
+// items into a two-stage shared-memory ring; warp 1 issues the tcgen05 MMAs
+// -- S = Q K^T of item i+1 into one of two 256-column TMEM buffers while the
+// softmax warps still work on item i, then P V of item i -- and warps 2-9
+// run Shiftmax and the output requant.  Within an item the score row never
+// leaves TMEM: pass 1 takes the row maximum of the raw int32 scores (the
+// logit requant is monotone, so max L = requant(max S)); pass 2 requantises
+// each score, looks up ShiftExp(L - max L) in a table replicated once per
+// shared-memory bank (lane l reads copy l, so lookups never conflict), sums
+// the row and writes the exponentials back into TMEM in place; pass 3 turns
+// them into u8 P = (Dv e) >> (M - k_out + 1), written straight into the
+// 128B-swizzled K-major operand of the P V MMA.  Warps w and w + 4 share TMEM
+// lanes (query rows) and split the key columns; their partial maxima and sums
+// meet in shared memory behind a named barrier of the 256 softmax threads.
 // ---------------------------------------------------------------------------
-constexpr int kShortThreads = 256;
 constexpr int kShortMaxKeys = 256;
+constexpr int kSoftWarps = 8;    // per softmax group
+constexpr int kSoftGroups = 2;   // groups take alternate items, one TMEM buffer each
+constexpr int kPersistThreads = 64 + 32 * kSoftWarps * kSoftGroups;
 
-struct ShortLayout {
+struct PersistLayout {
   int n64, n32, kblocks;
-  int r0_bytes, v_off, tab_off, part_off, bar_off, total;
+  int r0_bytes, stage_bytes, tab_off, part_off, bar_off, total;
 };
 
-__host__ __device__ inline ShortLayout short_layout(int N) {
-  ShortLayout L;
+__host__ __device__ inline PersistLayout persist_layout(int N) {
+  PersistLayout L;
   L.n64 = (N + 63) / 64 * 64;
   L.n32 = (N + 31) / 32 * 32;
   L.kblocks = (L.n32 + 127) / 128;
   const int qk = kQTile * kHeadDim + L.n64 * kHeadDim;
   const int p = L.kblocks * 128 * 128;
   L.r0_bytes = ((qk > p ? qk : p) + 1023) / 1024 * 1024;
-  L.v_off = L.r0_bytes;
-  L.tab_off = L.v_off + (L.n64 * kHeadDim + 1023) / 1024 * 1024;
+  L.stage_bytes = L.r0_bytes + (L.n64 * kHeadDim + 1023) / 1024 * 1024;  // R0 (Q, K, later P) + V
+  L.tab_off = 2 * L.stage_bytes;
   L.part_off = L.tab_off + 256 * 32 * 4;
-  L.bar_off = L.part_off + 2 * 2 * kQTile * 4;
-  L.total = L.bar_off + 64;
+  L.bar_off = L.part_off + kSoftGroups * 2 * 2 * kQTile * 4;
+  L.total = L.bar_off + 16 * 8 + 16;
   return L;
+}
+
+// bytes [sat8(y0), sat8(y1), sat8(y2), sat8(y3)]
+IVIT_DEV uint32_t pack_sat4_attn(int32_t y0, int32_t y1, int32_t y2, int32_t y3) {
+  uint32_t t, d;
+  asm("cvt.pack.sat.s8.s32.b32 %0, %1, %2, %3;" : "=r"(t) : "r"(y3), "r"(y2), "r"(0u));
+  asm("cvt.pack.sat.s8.s32.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(y1), "r"(y0), "r"(t));
+  return d;
 }
 
 // sat_ks(floor(b S / 2^c)): one mul.hi when b 2^(32-c) fits a positive int32
@@ -324,245 +342,321 @@ IVIT_DEV int32_t logit_requant(int32_t S, int32_t bq, int32_t b, int32_t c, int3
   }
 }
 
+// bounded wait that also gives up at once when another thread has aborted
+IVIT_DEV bool wait_or_abort(uint64_t* bar, uint32_t parity, int* status, volatile int* abort_flag) {
+  if (*abort_flag) return false;
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  while (true) {
+    if (mbar_try_wait_sleep(bar, parity)) return true;
+    if (*abort_flag) return false;
+    if (globaltimer_ns() - t0 > kWaitBudgetNs) {
+      report_timeout(status);
+      *abort_flag = 1;
+      return false;
+    }
+  }
+}
+
+// named barrier of one softmax group (ids 1 and 2; 256 threads each)
+IVIT_DEV void softmax_bar(int group) { asm volatile("bar.sync %0, %1;" ::"r"(1 + group), "n"(32 * kSoftWarps) : "memory"); }
+
 template <bool FASTQ>
-__global__ void __launch_bounds__(kShortThreads, 2)
-    attention_short_kernel(const __grid_constant__ CUtensorMap tm, const AttnArgs a, const int32_t bq) {
+__global__ void __launch_bounds__(kPersistThreads, 1)
+    attention_persist_kernel(const __grid_constant__ CUtensorMap tm, const AttnArgs a, const int32_t bq) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int N = a.N;
-  const ShortLayout L = short_layout(N);
-  uint8_t* sQ = smem;
-  uint8_t* sK = smem + kQTile * kHeadDim;
-  uint8_t* sP = smem;
-  uint8_t* sV = smem + L.v_off;
+  const PersistLayout L = persist_layout(N);
   int32_t* tab = reinterpret_cast<int32_t*>(smem + L.tab_off);
-  int32_t* part = reinterpret_cast<int32_t*>(smem + L.part_off);  // [half][max, sum][128 rows]
-  uint64_t* bar_qk = reinterpret_cast<uint64_t*>(smem + L.bar_off);
-  uint64_t* bar_v = bar_qk + 1;
-  uint64_t* bar_s = bar_qk + 2;
-  uint64_t* bar_o = bar_qk + 3;
-  uint32_t* tslot = reinterpret_cast<uint32_t*>(bar_qk + 4);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L.bar_off);
+  uint64_t* qk_full = bars + 0;       // [2] Q and K landed
+  uint64_t* v_full = bars + 2;        // [2] V landed
+  uint64_t* s_full = bars + 4;        // [2] S in TMEM
+  uint64_t* p_full = bars + 6;        // [2] P in shared memory (one arrival per softmax warp)
+  uint64_t* o_full = bars + 8;        // [2] P V in TMEM
+  uint64_t* stage_empty = bars + 10;  // [2] ring stage reusable
+  uint64_t* tmem_empty = bars + 12;   // [2] TMEM buffer reusable (one arrival per softmax warp)
+  uint32_t* tslot = reinterpret_cast<uint32_t*>(bars + 14);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 15);
 
   const int tid = threadIdx.x;
   const int warp = tid >> 5;
   const int lane = tid & 31;
-  const int quarter = warp & 3;
-  const int half = warp >> 2;
-  const int row = quarter * 32 + lane;  // query row of the tile = TMEM lane
-  const int q0 = blockIdx.x * kQTile;
-  const int h = blockIdx.y;
-  const int img = blockIdx.z;
   const int D = a.H * kHeadDim;
-  const int row0 = img * N;
+  const int qtiles = (N + kQTile - 1) / kQTile;
+  const int n_items = qtiles * a.H * a.B;
   const int nload = L.n64 / 64;
-  const int hcols = L.n32 / 2;  // key columns per half (multiple of 16)
+  const int hcols = L.n32 / 2;  // key columns per softmax half (multiple of 16)
 
   if (tid == 0) {
-    mbar_init(bar_qk, 1);
-    mbar_init(bar_v, 1);
-    mbar_init(bar_s, 1);
-    mbar_init(bar_o, 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&qk_full[s], 1);
+      mbar_init(&v_full[s], 1);
+      mbar_init(&s_full[s], 1);
+      mbar_init(&p_full[s], kSoftWarps);
+      mbar_init(&o_full[s], 1);
+      mbar_init(&stage_empty[s], 1);
+      mbar_init(&tmem_empty[s], kSoftWarps);
+    }
+    *abort_flag = 0;
     fence_barrier_init();
     prefetch_tensormap(&tm);
   }
-  if (warp == 0) {
+  // replicated ShiftExp table, tab[t * 32 + l] = ShiftExp(-t) for every lane l:
+  // one evaluation per entry (staged in the partials area), then copies in
+  // consecutive 16-byte chunks
+  int32_t* stage_t = reinterpret_cast<int32_t*>(smem + L.part_off);
+  if (tid < (1 << a.k_s)) stage_t[tid] = shift_exp(-tid, a.I0);
+  if (warp == 1) {
     __syncwarp();
-    tmem_alloc(tslot, kTmemCols);
+    tmem_alloc(tslot, 512);
     tmem_relinquish();
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  const uint32_t tmem = *tslot;
-
-  if (tid == 0) {
-    mbar_arrive_expect_tx(bar_qk, (uint32_t)(kQTile * kHeadDim + nload * 64 * kHeadDim));
-    tma_load_2d(sQ, &tm, h * kHeadDim, row0 + q0, bar_qk);
-    tma_load_2d(sQ + 64 * kHeadDim, &tm, h * kHeadDim, row0 + q0 + 64, bar_qk);
-    for (int i = 0; i < nload; ++i) tma_load_2d(sK + i * 64 * kHeadDim, &tm, D + h * kHeadDim, row0 + 64 * i, bar_qk);
-    mbar_arrive_expect_tx(bar_v, (uint32_t)(nload * 64 * kHeadDim));
-    for (int i = 0; i < nload; ++i)
-      tma_load_2d(sV + i * 64 * kHeadDim, &tm, 2 * D + h * kHeadDim, row0 + 64 * i, bar_v);
-  }
-  // replicated ShiftExp table: tab[t * 32 + l] = ShiftExp(-t) for every lane l.
-  // One evaluation per entry into part[] (free until pass 1), then copies
-  // written as consecutive 16-byte chunks by consecutive threads (no bank
-  // conflicts).
-  if (tid < (1 << a.k_s)) part[tid] = shift_exp(-tid, a.I0);
-  __syncthreads();
-  for (int i4 = tid; i4 < (8 << a.k_s); i4 += kShortThreads) {
-    const int32_t e = part[i4 >> 3];
+  for (int i4 = tid; i4 < (8 << a.k_s); i4 += kPersistThreads) {
+    const int32_t e = stage_t[i4 >> 3];
     reinterpret_cast<int4*>(tab)[i4] = make_int4(e, e, e, e);
   }
-
-  bool ok = true;
-  if (tid == 0) {
-    if (!mbar_wait(bar_qk, 0, a.status)) ok = false;
-    if (ok) {
-      tc_fence_after();
-      const uint32_t idesc = idesc_i8(kQTile, L.n32, true, true, false);
-      const uint32_t qa = smem_u32(sQ);
-      const uint32_t kb = smem_u32(sK);
-#pragma unroll
-      for (int k = 0; k < kHeadDim / 32; ++k)
-        umma_i8(tmem, smem_desc(qa + k * 32, 16, 512, kSwizzle64B), smem_desc(kb + k * 32, 16, 512, kSwizzle64B),
-                idesc, k != 0);
-    }
-    umma_commit(bar_s);
-  }
-  __syncthreads();  // exp table complete
-  if (!mbar_wait(bar_s, 0, a.status)) ok = false;
-  ok = __all_sync(0xffffffffu, ok);
-  tc_fence_after();
-  const uint32_t t_row = tmem + ((uint32_t)(quarter * 32) << 16);
-  const int cbase = half * hcols;
-
-  // Warps whose 32 query rows all lie past the image's last token skip the
-  // three passes (their P rows feed only outputs that are never stored).
-  const bool rows_live = q0 + quarter * 32 < N;
-  const bool work = ok && rows_live;
-  const int nchunk = hcols / 16;
-
-  // Each pass streams this thread's key columns in 16-column TMEM chunks with
-  // the next chunk's load in flight while the current one is processed.
-#define IVIT_STREAM_CHUNKS(BODY)                                          \
-  {                                                                       \
-    uint32_t ra[16], rb[16];                                              \
-    tmem_ld16(t_row + (uint32_t)cbase, ra);                               \
-    for (int k = 0; k < nchunk; k += 2) {                                 \
-      tmem_ld_wait();                                                     \
-      if (k + 1 < nchunk) tmem_ld16(t_row + (uint32_t)(cbase + 16 * (k + 1)), rb); \
-      { uint32_t(&r)[16] = ra; const int col = cbase + 16 * k; BODY }     \
-      if (k + 1 < nchunk) {                                               \
-        tmem_ld_wait();                                                   \
-        if (k + 2 < nchunk) tmem_ld16(t_row + (uint32_t)(cbase + 16 * (k + 2)), ra); \
-        { uint32_t(&r)[16] = rb; const int col = cbase + 16 * (k + 1); BODY } \
-      }                                                                   \
-    }                                                                     \
-  }
-
-  // ---- pass 1: row maximum of the raw scores over the valid keys
-  int32_t smax = INT_MIN;
-  if (work) {
-    IVIT_STREAM_CHUNKS({
-      const int lim = N - col;
-      if (lim >= 16) {
-#pragma unroll
-        for (int i = 0; i < 16; ++i) smax = max(smax, (int32_t)r[i]);
-      } else {
-#pragma unroll
-        for (int i = 0; i < 16; ++i)
-          if (i < lim) smax = max(smax, (int32_t)r[i]);
-      }
-    })
-  }
-  part[half * 256 + row] = smax;
   __syncthreads();
-  smax = max(part[row], part[256 + row]);
-  const int32_t lmax = logit_requant<FASTQ>(smax, bq, a.logit_b, a.logit_c, a.ks_lo, a.ks_hi);
+  const uint32_t tmem = *tslot;
 
-  // ---- pass 2: e = ShiftExp(L - max L) back into TMEM, row sum
-  uint32_t sum = 0;
-  // tb[-32 L] = ShiftExp(L - max L) from this lane's copy of the table
-  const int32_t* tb = tab + lane + lmax * 32;
-  if (work) {
-    IVIT_STREAM_CHUNKS({
-      const int lim = N - col;
-      if (lim >= 16) {
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const int32_t l = logit_requant<FASTQ>((int32_t)r[i], bq, a.logit_b, a.logit_c, a.ks_lo, a.ks_hi);
-          const uint32_t e = (uint32_t)tb[-32 * l];
-          sum += e;
-          r[i] = e;
-        }
-      } else {
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const int32_t l = logit_requant<FASTQ>((int32_t)r[i], bq, a.logit_b, a.logit_c, a.ks_lo, a.ks_hi);
-          const uint32_t e = (i < lim) ? (uint32_t)tb[-32 * l] : 0u;
-          sum += e;
-          r[i] = e;
-        }
-      }
-      tmem_st16(t_row + (uint32_t)col, r);
-    })
-    tmem_st_wait();
-  }
-  part[half * 256 + 128 + row] = (int32_t)sum;
-  __syncthreads();
-  sum = (uint32_t)part[128 + row] + (uint32_t)part[256 + 128 + row];
-  if (sum == 0) sum = 1;  // rows that skipped the passes
-  const uint32_t dv = (1u << a.M) / sum;
-  const int pshift = a.M - (a.k_out - 1);
-
-  // ---- pass 3: P = (Dv e) >> (M - k_out + 1) into the swizzled operand
-  fence_proxy_async_smem();
-  if (work) {
-    const int rlo = row & 7;
-    uint8_t* prow = sP + (row >> 3) * 1024 + rlo * 128;
-    IVIT_STREAM_CHUNKS({
-      uint32_t w[4];
-#pragma unroll
-      for (int q = 0; q < 4; ++q)
-        w[q] = ((dv * r[4 * q]) >> pshift) + ((dv * r[4 * q + 1]) >> pshift) * 256u +
-               ((dv * r[4 * q + 2]) >> pshift) * 65536u + ((dv * r[4 * q + 3]) >> pshift) * 16777216u;
-      *reinterpret_cast<int4*>(prow + (col >> 7) * 16384 + ((((col & 127) >> 4) ^ rlo) << 4)) =
-          make_int4((int)w[0], (int)w[1], (int)w[2], (int)w[3]);
-    })
-  }
-#undef IVIT_STREAM_CHUNKS
-  fence_proxy_async_smem();
-  tc_fence_before();
-  __syncthreads();
-
-  // ---- O = P V
-  if (tid == 0) {
-    if (ok && mbar_wait(bar_v, 0, a.status)) {
-      tc_fence_after();
-      const uint32_t idesc = idesc_i8(kQTile, kHeadDim, false, true, true);
-      const uint32_t pa = smem_u32(sP);
-      const uint32_t va = smem_u32(sV);
-      for (int k = 0; k < L.n32 / 32; ++k) {
-        const uint64_t da = smem_desc(pa + (k >> 2) * 16384 + (k & 3) * 32, 16, 1024, kSwizzle128B);
-        const uint64_t db = smem_desc(va + k * 32 * kHeadDim, 512, 512, kSwizzle64B);
-        umma_i8(tmem, da, db, idesc, k != 0);
-      }
-    }
-    umma_commit(bar_o);
-  }
-  if (!mbar_wait(bar_o, 0, a.status)) ok = false;
-  ok = __all_sync(0xffffffffu, ok);
-  tc_fence_after();
-
-  // ---- ctx = sat_8((b_o O) >> c_o); warp half h writes columns [32 h, 32 h + 32)
-  {
-    uint32_t r[32];
-    tmem_ld32(t_row + (uint32_t)(half * 32), r);
-    tmem_ld_wait();
-    const int q = q0 + row;
-    if (ok && q < N) {
-      int8_t* dst = a.ctx + (int64_t)(row0 + q) * D + h * kHeadDim + half * 32;
-      uint32_t packed[8];
-#pragma unroll
-      for (int wd = 0; wd < 8; ++wd) {
-        uint32_t word = 0;
-#pragma unroll
-        for (int e = 0; e < 4; ++e)
-          word |= ((uint32_t)requant8((int32_t)r[wd * 4 + e], a.out_b, a.out_c) & 0xFFu) << (8 * e);
-        packed[wd] = word;
-      }
-      reinterpret_cast<int4*>(dst)[0] = make_int4(packed[0], packed[1], packed[2], packed[3]);
-      reinterpret_cast<int4*>(dst)[1] = make_int4(packed[4], packed[5], packed[6], packed[7]);
-    }
-  }
-
-  tc_fence_before();
-  __syncthreads();
   if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      int i = 0;
+      for (int item = blockIdx.x; item < n_items; item += gridDim.x, ++i) {
+        const int s = i & 1;
+        const uint32_t ph = (uint32_t)((i >> 1) & 1);
+        if (!wait_or_abort(&stage_empty[s], ph ^ 1, a.status, abort_flag)) break;
+        const int qt = item % qtiles, h = (item / qtiles) % a.H, img = item / (qtiles * a.H);
+        const int row0 = img * N;
+        uint8_t* st = smem + s * L.stage_bytes;
+        uint8_t* sV = st + L.r0_bytes;
+        mbar_arrive_expect_tx(&qk_full[s], (uint32_t)(kQTile * kHeadDim + nload * 64 * kHeadDim));
+        tma_load_2d(st, &tm, h * kHeadDim, row0 + qt * kQTile, &qk_full[s]);
+        tma_load_2d(st + 64 * kHeadDim, &tm, h * kHeadDim, row0 + qt * kQTile + 64, &qk_full[s]);
+        for (int j = 0; j < nload; ++j)
+          tma_load_2d(st + kQTile * kHeadDim + j * 64 * kHeadDim, &tm, D + h * kHeadDim, row0 + 64 * j, &qk_full[s]);
+        mbar_arrive_expect_tx(&v_full[s], (uint32_t)(nload * 64 * kHeadDim));
+        for (int j = 0; j < nload; ++j)
+          tma_load_2d(sV + j * 64 * kHeadDim, &tm, 2 * D + h * kHeadDim, row0 + 64 * j, &v_full[s]);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      const uint32_t idesc_s = idesc_i8(kQTile, L.n32, true, true, false);
+      const uint32_t idesc_o = idesc_i8(kQTile, kHeadDim, false, true, true);
+      const int n_local = n_items > (int)blockIdx.x ? (n_items - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
+      // S = Q K^T of local item j into TMEM buffer j & 1
+      auto issue_s = [&](int j) -> bool {
+        const int s = j & 1;
+        const uint32_t ph = (uint32_t)((j >> 1) & 1);
+        if (!wait_or_abort(&tmem_empty[s], ph ^ 1, a.status, abort_flag)) return false;
+        if (!wait_or_abort(&qk_full[s], ph, a.status, abort_flag)) return false;
+        tc_fence_after();
+        const uint32_t qa = smem_u32(smem + s * L.stage_bytes);
+        const uint32_t ka = qa + kQTile * kHeadDim;
+#pragma unroll
+        for (int k = 0; k < kHeadDim / 32; ++k)
+          umma_i8(tmem + (uint32_t)(s * 256), smem_desc(qa + k * 32, 16, 512, kSwizzle64B),
+                  smem_desc(ka + k * 32, 16, 512, kSwizzle64B), idesc_s, k != 0);
+        umma_commit(&s_full[s]);
+        return true;
+      };
+      bool ok = n_local == 0 || issue_s(0);
+      for (int j = 0; j < n_local && ok; ++j) {
+        if (j + 1 < n_local && !issue_s(j + 1)) break;
+        const int s = j & 1;
+        const uint32_t ph = (uint32_t)((j >> 1) & 1);
+        if (!wait_or_abort(&p_full[s], ph, a.status, abort_flag)) break;
+        if (!wait_or_abort(&v_full[s], ph, a.status, abort_flag)) break;
+        tc_fence_after();
+        const uint32_t pa = smem_u32(smem + s * L.stage_bytes);
+        const uint32_t va = pa + L.r0_bytes;
+        for (int k = 0; k < L.n32 / 32; ++k)
+          umma_i8(tmem + (uint32_t)(s * 256), smem_desc(pa + (k >> 2) * 16384 + (k & 3) * 32, 16, 1024, kSwizzle128B),
+                  smem_desc(va + k * 32 * kHeadDim, 512, 512, kSwizzle64B), idesc_o, k != 0);
+        umma_commit(&o_full[s]);
+        umma_commit(&stage_empty[s]);
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ softmax warps
+    const int group = (warp - 2) / kSoftWarps;          // handles local items i with i % 2 == group
+    const int quarter = warp & 3;
+    const int half = ((warp - 2) >> 2) & 1;
+    const int row = quarter * 32 + lane;  // query row of the tile = TMEM lane
+    const int cbase = half * hcols;
+    const int nchunk = hcols / 16;
+    const int rlo = row & 7;
+    int32_t* part = reinterpret_cast<int32_t*>(smem + L.part_off) + group * 512;  // [half][max, sum][128 rows]
+    bool ok = true;
+    int i = group;
+    for (int item = blockIdx.x + group * gridDim.x; item < n_items; item += 2 * gridDim.x, i += 2) {
+      const int s = i & 1;
+      const uint32_t ph = (uint32_t)((i >> 1) & 1);
+      const int qt = item % qtiles, h = (item / qtiles) % a.H, img = item / (qtiles * a.H);
+      const int q0 = qt * kQTile;
+      if (ok) ok = wait_or_abort(&s_full[s], ph, a.status, abort_flag);
+      ok = __all_sync(0xffffffffu, ok);
+      tc_fence_after();
+      const uint32_t t_row = tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(s * 256);
+      // warps whose rows all lie past the image's last token skip the passes
+      const bool work = ok && (q0 + quarter * 32 < N);
+
+#define IVIT_STREAM_CHUNKS(BODY)                                                      \
+  {                                                                                   \
+    uint32_t ra[16], rb[16];                                                          \
+    tmem_ld16(t_row + (uint32_t)cbase, ra);                                           \
+    for (int k = 0; k < nchunk; k += 2) {                                             \
+      tmem_ld_wait();                                                                 \
+      if (k + 1 < nchunk) tmem_ld16(t_row + (uint32_t)(cbase + 16 * (k + 1)), rb);    \
+      {                                                                               \
+        uint32_t(&r)[16] = ra;                                                        \
+        const int col = cbase + 16 * k;                                               \
+        BODY                                                                          \
+      }                                                                               \
+      if (k + 1 < nchunk) {                                                           \
+        tmem_ld_wait();                                                               \
+        if (k + 2 < nchunk) tmem_ld16(t_row + (uint32_t)(cbase + 16 * (k + 2)), ra);  \
+        {                                                                             \
+          uint32_t(&r)[16] = rb;                                                      \
+          const int col = cbase + 16 * (k + 1);                                       \
+          BODY                                                                        \
+        }                                                                             \
+      }                                                                               \
+    }                                                                                 \
+  }
+
+      // ---- pass 1: row maximum of the raw scores over the valid keys
+      // (independent running maxima keep the dependency chains short)
+      int32_t m4[4] = {INT_MIN, INT_MIN, INT_MIN, INT_MIN};
+      if (work) {
+        IVIT_STREAM_CHUNKS({
+          const int lim = N - col;
+          if (lim >= 16) {
+#pragma unroll
+            for (int e = 0; e < 16; ++e) m4[e & 3] = max(m4[e & 3], (int32_t)r[e]);
+          } else {
+#pragma unroll
+            for (int e = 0; e < 16; ++e)
+              if (e < lim) m4[e & 3] = max(m4[e & 3], (int32_t)r[e]);
+          }
+        })
+      }
+      int32_t smax = max(max(m4[0], m4[1]), max(m4[2], m4[3]));
+      part[half * 256 + row] = smax;
+      softmax_bar(group);
+      smax = max(part[row], part[256 + row]);
+      const int32_t lmax = logit_requant<FASTQ>(smax, bq, a.logit_b, a.logit_c, a.ks_lo, a.ks_hi);
+
+      // ---- pass 2: e = ShiftExp(L - max L) back into TMEM, row sum (four partial sums)
+      uint32_t s4[4] = {0u, 0u, 0u, 0u};
+      const int32_t* tb = tab + lane + lmax * 32;  // tb[-32 L] = ShiftExp(L - max L)
+      if (work) {
+        IVIT_STREAM_CHUNKS({
+          const int lim = N - col;
+          if (lim >= 16) {
+#pragma unroll
+            for (int e = 0; e < 16; ++e) {
+              const int32_t l = logit_requant<FASTQ>((int32_t)r[e], bq, a.logit_b, a.logit_c, a.ks_lo, a.ks_hi);
+              const uint32_t x = (uint32_t)tb[-32 * l];
+              s4[e & 3] += x;
+              r[e] = x;
+            }
+          } else {
+#pragma unroll
+            for (int e = 0; e < 16; ++e) {
+              const int32_t l = logit_requant<FASTQ>((int32_t)r[e], bq, a.logit_b, a.logit_c, a.ks_lo, a.ks_hi);
+              const uint32_t x = (e < lim) ? (uint32_t)tb[-32 * l] : 0u;
+              s4[e & 3] += x;
+              r[e] = x;
+            }
+          }
+          tmem_st16(t_row + (uint32_t)col, r);
+        })
+        tmem_st_wait();
+      }
+      uint32_t sum = (s4[0] + s4[1]) + (s4[2] + s4[3]);
+      part[half * 256 + 128 + row] = (int32_t)sum;
+      softmax_bar(group);
+      sum = (uint32_t)part[128 + row] + (uint32_t)part[256 + 128 + row];
+      if (sum == 0) sum = 1;  // rows that skipped the passes
+      const uint32_t dv = (1u << a.M) / sum;
+      const int pshift = a.M - (a.k_out - 1);
+
+      // ---- pass 3: P = (Dv e) >> (M - k_out + 1) into the swizzled operand of stage s
+      if (work) {
+        uint8_t* prow = smem + s * L.stage_bytes + (row >> 3) * 1024 + rlo * 128;
+        // (Dv e) >> pshift is one mul.hi by Dv 2^(32 - pshift) when that fits 32 bits
+        const bool hip = __all_sync(0xffffffffu, pshift <= 32 && (uint64_t)dv < ((uint64_t)1 << pshift));
+        const uint32_t dvh = hip ? dv << (32 - pshift) : 0u;
+        IVIT_STREAM_CHUNKS({
+          uint32_t w[4];
+          if (hip) {
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+              w[q] = __umulhi(dvh, r[4 * q]) + __umulhi(dvh, r[4 * q + 1]) * 256u +
+                     __umulhi(dvh, r[4 * q + 2]) * 65536u + __umulhi(dvh, r[4 * q + 3]) * 16777216u;
+          } else {
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+              w[q] = ((dv * r[4 * q]) >> pshift) + ((dv * r[4 * q + 1]) >> pshift) * 256u +
+                     ((dv * r[4 * q + 2]) >> pshift) * 65536u + ((dv * r[4 * q + 3]) >> pshift) * 16777216u;
+          }
+          *reinterpret_cast<int4*>(prow + (col >> 7) * 16384 + ((((col & 127) >> 4) ^ rlo) << 4)) =
+              make_int4((int)w[0], (int)w[1], (int)w[2], (int)w[3]);
+        })
+      }
+#undef IVIT_STREAM_CHUNKS
+      fence_proxy_async_smem();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&p_full[s]);
+
+      // ---- ctx = sat_8((b_o O) >> c_o); half h writes columns [32 h, 32 h + 32)
+      if (ok) ok = wait_or_abort(&o_full[s], ph, a.status, abort_flag);
+      ok = __all_sync(0xffffffffu, ok);
+      tc_fence_after();
+      if (ok) {
+        uint32_t r[32];
+        tmem_ld32(t_row + (uint32_t)(half * 32), r);
+        tmem_ld_wait();
+        const int q = q0 + row;
+        if (q < N) {
+          int8_t* dst = a.ctx + (int64_t)(img * N + q) * D + h * kHeadDim + half * 32;
+          uint32_t packed[8];
+#pragma unroll
+          for (int wd = 0; wd < 8; ++wd) {
+            int32_t y[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const int32_t acc = min(max((int32_t)r[wd * 4 + e], a.o_lo), a.o_hi);
+              const int64_t v = (int64_t)a.out_b * acc;  // |v >> c| < 2^31 after the clamp
+              y[e] = (int32_t)__funnelshift_r((uint32_t)v, (uint32_t)(v >> 32), (uint32_t)a.out_c);
+            }
+            packed[wd] = pack_sat4_attn(y[0], y[1], y[2], y[3]);
+          }
+          reinterpret_cast<int4*>(dst)[0] = make_int4(packed[0], packed[1], packed[2], packed[3]);
+          reinterpret_cast<int4*>(dst)[1] = make_int4(packed[4], packed[5], packed[6], packed[7]);
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&tmem_empty[s]);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
     __syncwarp();
     tc_fence_after();
-    tmem_dealloc(tmem, kTmemCols);
+    tmem_dealloc(tmem, 512);
   }
 }
 
@@ -593,28 +687,47 @@ ivit_status launch_attention(const DeviceCtx& dc, const int8_t* qkv, int32_t B, 
   a.k_out = k_out;
   a.out_b = out.b;
   a.out_c = out.c;
+  {
+    // acc in [-u, u] with u = 128 / 2^s (2^s <= b / 2^c < 2^(s+1)) keeps every
+    // unsaturated result, saturates the rest the same way and keeps
+    // (b acc) >> c within int32
+    if (out.b == 0) {
+      a.o_lo = INT_MIN;
+      a.o_hi = INT_MAX;
+    } else {
+      int bl = 0;
+      while (bl < 31 && (out.b >> bl) != 0) ++bl;
+      const int sh = bl - 1 - out.c;
+      const int64_t u = sh >= 7 ? 1 : (sh >= 0 ? (128 >> sh) : ((int64_t)128 << (-sh)));
+      a.o_hi = (int32_t)(u > INT_MAX ? INT_MAX : u);
+      a.o_lo = -a.o_hi;
+    }
+  }
   a.ctx = ctx;
   a.status = dc.status;
   dim3 grid((unsigned)((N + kQTile - 1) / kQTile), (unsigned)H, (unsigned)B);
   if (N <= kShortMaxKeys) {
-    const ShortLayout S = short_layout(N);
-    const int smem = S.total + 1024;  // >= 80 KB: at most two CTAs (2 x 256 TMEM columns) per SM
+    const PersistLayout P = persist_layout(N);
+    const int smem = P.total + 1024;
     // bq = b 2^(32 - c) when it fits a positive int32: the logit requant is then one mul.hi
     const bool fastq = logit.c >= 1 && (int64_t)logit.b < ((int64_t)1 << (logit.c - 1));
     const int32_t bq = fastq ? (int32_t)((int64_t)logit.b << (32 - logit.c)) : 0;
-    static bool attr_short = false;
-    if (!attr_short) {
-      if (cudaFuncSetAttribute(attention_short_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    static bool attr_persist = false;
+    if (!attr_persist) {
+      if (cudaFuncSetAttribute(attention_persist_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                227 * 1024) != cudaSuccess ||
-          cudaFuncSetAttribute(attention_short_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+          cudaFuncSetAttribute(attention_persist_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                227 * 1024) != cudaSuccess)
         return IVIT_ERR_CUDA;
-      attr_short = true;
+      attr_persist = true;
     }
+    const int64_t items = (int64_t)((N + kQTile - 1) / kQTile) * H * B;
+    if (items > 0x7fffffff) return IVIT_ERR_UNSUPPORTED;
+    const unsigned pgrid = (unsigned)(items < dc.num_sms ? items : dc.num_sms);
     if (fastq)
-      attention_short_kernel<true><<<grid, kShortThreads, smem, stream>>>(tm, a, bq);
+      attention_persist_kernel<true><<<pgrid, kPersistThreads, smem, stream>>>(tm, a, bq);
     else
-      attention_short_kernel<false><<<grid, kShortThreads, smem, stream>>>(tm, a, bq);
+      attention_persist_kernel<false><<<pgrid, kPersistThreads, smem, stream>>>(tm, a, bq);
     note_launch();
     return cudaGetLastError() == cudaSuccess ? IVIT_OK : IVIT_ERR_CUDA;
   }
