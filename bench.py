@@ -37,8 +37,15 @@ import synthetic  # noqa: E402
 
 METRIC = "int-only ViT block images/s (ViT-B, 197 tok); % INT8 TC peak & % HBM BW"
 DEFAULT_WORKLOAD = "vit_b_b64"
-FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "sm_max_mhz": 1965.0}
 INT8_PER_BF16 = 2.0  # nominal dense tensor-core ratio on B200 (4.5 vs 2.25 PFLOP/s)
+# Integer operations the method specifies per attention score (Shiftmax, section 3.3 of the
+# I-ViT notes): logit requant (multiply, shift, two-sided saturation: 4), row max (1),
+# I_delta = L - max (1), I_p = I_delta + (I_delta >> 1) - (I_delta >> 4) (4), q and r by one
+# division, one multiply and one subtraction (3), (I_0 + ((-r) >> 1)) >> q (3), row sum (1),
+# P = (Dv e) >> (M - k_out + 1) (2).
+SHIFTMAX_OPS_PER_SCORE = 19
+INT_LANES_PER_SM = 128  # 4 sub-partitions x 32 lanes, one integer instruction per lane per clock
 
 
 def parse_args():
@@ -63,14 +70,42 @@ def ops_per_image_block(N, D):
     return 24 * N * D * D + 4 * N * N * D
 
 
+def max_over_ranks(x: float, world: int, device=None) -> float:
+    """Largest value of x over all ranks (the timing rule: the slowest rank counts)."""
+    if world == 1:
+        return float(x)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_images_per_s(world: int, images_per_rank: int, steps: int, elapsed_ms: float) -> float:
+    """Images all ranks processed per second of the slowest rank's device time."""
+    return world * images_per_rank * steps / (elapsed_ms / 1e3)
+
+
 def load_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
         with open(path) as f:
             p = json.load(f)
-        return {k: float(p[k]) for k in ("hbm_gbs", "bf16_tflops", "bf16_tflops_sustained")}, "measured"
+        out = {k: float(p[k]) for k in ("hbm_gbs", "bf16_tflops", "bf16_tflops_sustained")}
+        out["sm_max_mhz"] = float(p.get("sm_max_mhz", FALLBACK_PEAKS["sm_max_mhz"]))
+        return out, "measured"
     except Exception:
         return dict(FALLBACK_PEAKS), "fallback"
+
+
+def peak_for(bound, peaks, num_sms):
+    """(peak, unit, note) of a roofline bound."""
+    if bound == "tensor":
+        return peaks["bf16_tflops"] * INT8_PER_BF16, "TOP/s", f"INT8 dense = {INT8_PER_BF16:g} x bf16 burst"
+    if bound == "alu":
+        pk = num_sms * INT_LANES_PER_SM * peaks["sm_max_mhz"] * 1e6 / 1e12
+        return pk, "TOP/s", f"{num_sms} SMs x {INT_LANES_PER_SM} integer lanes x {peaks['sm_max_mhz']:.0f} MHz"
+    return peaks["hbm_gbs"], "GB/s", "HBM copy"
 
 
 # ---------------------------------------------------------------------------
@@ -82,7 +117,6 @@ def oracle_units(wl, units):
     import oracle
     ps = [oracle.block_params(q) for q in wl.blocks]
     N, nb = wl.N, len(wl.blocks)
-    x_by_block = [wl.x]
     t = 0.0
     for u in range(units):
         b = u % nb
@@ -91,7 +125,6 @@ def oracle_units(wl, units):
         t0 = time.perf_counter()
         oracle.block_forward(ps[b], xin, 1, N)
         t += time.perf_counter() - t0
-    del x_by_block
     return t, units / (t * nb)
 
 
@@ -326,17 +359,13 @@ def run_ours(args):
     torch.cuda.synchronize()
     t_w1 = time.perf_counter()
     barrier()
-    elapsed_ms = ev0.elapsed_time(ev1)
-    if world > 1:
-        t = torch.tensor([elapsed_ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        elapsed_ms = float(t.item())
+    elapsed_ms = max_over_ranks(ev0.elapsed_time(ev1), world, dev)
     sampler.stop()
     clocks = sampler.summary(t_w0, t_w1)
     if ivit.ivit_stream_status() != 0:
         raise SystemExit("a kernel reported a timed-out wait")
     ms_per_step = elapsed_ms / args.steps
-    images_per_s = world * B * args.steps / (elapsed_ms / 1e3)
+    images_per_s = whole_job_images_per_s(world, B, args.steps, elapsed_ms)
 
     # ---------------- per-kernel breakdown of block 0 (CUDA events, same stream)
     kern = kernel_breakdown(ivit, wl, dps[0], ws, xs, args.kernel_reps, dev)
@@ -359,13 +388,9 @@ def run_ours(args):
         y_host.copy_(out, non_blocking=True)
     e1.record()
     torch.cuda.synchronize()
-    e2e_ms = e0.elapsed_time(e1)
-    if world > 1:
-        t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
     barrier()
-    e2e_value = world * B * k_e2e / (e2e_ms / 1e3)
+    e2e_value = whole_job_images_per_s(world, B, k_e2e, e2e_ms)
 
     # release graphs before the process group goes away
     graphs.clear()
@@ -382,18 +407,11 @@ def run_ours(args):
 
     # dominant kernel of the block by time per step
     dom = max((k for k in kern if k["in_block"]), key=lambda k: k["ms"] * k["per_block"])
-    if dom["bound"] == "tensor":
-        achieved = dom["amount"] / (dom["ms"] / 1e3) / 1e12
-        peak, unit = int8_peak_burst, "TOP/s"
-        peak_note = f"INT8 dense = {INT8_PER_BF16:g} x bf16 burst ({peak_src})"
-    else:
-        achieved = dom["amount"] / (dom["ms"] / 1e3) / 1e9
-        peak, unit = peaks["hbm_gbs"], "GB/s"
-        peak_note = f"HBM copy ({peak_src})"
     traffic = load_traffic(dom["name"], wl.name)
-    roofline = {"kernel": dom["name"], "bound": dom["bound"], "achieved": achieved, "peak": peak, "unit": unit,
-                "frac": achieved / peak, "traffic": traffic, "peak_source": peak_note,
-                "launch_ms": dom["ms"]}
+    roofline = {"kernel": dom["name"], "bound": dom["bound"], "achieved": dom["achieved"], "peak": dom["peak"],
+                "unit": dom["unit"], "frac": dom["frac"], "traffic": traffic,
+                "peak_source": f"{dom['peak_note']} ({peak_src})", "launch_ms": dom["ms"],
+                "algorithmic_per_launch": dom["amount"], "algorithmic_unit": dom["amount_unit"]}
 
     cpu = None
     if world == 1 and not args.no_cpu_baseline:
@@ -456,15 +474,27 @@ def kernel_breakdown(ivit, wl, dp, ws, xs, reps, dev):
     hs = [g.clone() for _ in range(max(2, math.ceil(2 * 126e6 / (2 * T * Dm))))]
 
     def timed(fn):
+        # reps launches captured in one CUDA graph and replayed, so host launch
+        # overhead does not enter the per-launch device time
         for i in range(3):
             fn(i)
         torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        s = torch.cuda.Stream(device=dev)
+        s.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(s):
+            with torch.cuda.graph(g, stream=s):
+                for i in range(reps):
+                    fn(i)
+        torch.cuda.current_stream().wait_stream(s)
+        g.replay()
+        torch.cuda.synchronize()
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a.record()
-        for i in range(reps):
-            fn(i)
+        g.replay()
         b.record()
         torch.cuda.synchronize()
+        del g
         return a.elapsed_time(b) / reps
 
     gemm = lambda M, K, Nn: 2 * M * K * Nn
@@ -480,7 +510,7 @@ def kernel_breakdown(ivit, wl, dp, ws, xs, reps, dev):
         "tensor", gemm(T, D, 3 * D))
     add("attention", lambda i: ivit.ivit_attention(qkv, B, N, H, p["logit"], p["k_s"], p["attn_I0"], p["attn_M"],
                                                    p["attn_k_out"], p["attn_out"], ctx_o),
-        "tensor", 4 * B * N * N * D)
+        "alu", SHIFTMAX_OPS_PER_SCORE * B * H * N * N)
     add("gemm_o_residual", lambda i: ivit.ivit_linear_requant(ctx, t["w_o"], t["bias_o"], t["b_o"], t["c_o"], y,
                                                               skip=xs[i % R], res=p["res1"]),
         "tensor", gemm(T, D, D))
@@ -495,15 +525,14 @@ def kernel_breakdown(ivit, wl, dp, ws, xs, reps, dev):
                                                               p["gelu_k_out"], p["gelu_out"], h_o),
         "hbm", 2 * T * Dm, in_block=False)
     peaks, src = load_peaks()
+    num_sms = torch.cuda.get_device_properties(dev).multi_processor_count
     for k in out:
-        if k["bound"] == "hbm":
-            k["achieved"] = k["amount"] / (k["ms"] / 1e3) / 1e9
-            k["unit"] = "GB/s"
-            k["frac"] = k["achieved"] / peaks["hbm_gbs"]
-        else:
-            k["achieved"] = k["amount"] / (k["ms"] / 1e3) / 1e12
-            k["unit"] = "TOP/s"
-            k["frac"] = k["achieved"] / (peaks["bf16_tflops"] * INT8_PER_BF16)
+        k["peak"], k["unit"], k["peak_note"] = peak_for(k["bound"], peaks, num_sms)
+        scale = 1e9 if k["bound"] == "hbm" else 1e12
+        k["achieved"] = k["amount"] / (k["ms"] / 1e3) / scale
+        k["frac"] = k["achieved"] / k["peak"]
+        k["amount_unit"] = {"hbm": "bytes", "tensor": "int8 ops (2 x MAC)",
+                            "alu": "Shiftmax integer ops (19 per score)"}[k["bound"]]
     return out
 
 
