@@ -10,6 +10,7 @@
 // exact integer variance, 10 Newton steps of the integer square root, then the
 // per-element normalisation, affine and dyadic requant.
 #include <climits>
+#include <cmath>
 
 #include "ivit_common.cuh"
 #include "ivit_internal.h"
@@ -86,9 +87,18 @@ __device__ __forceinline__ uint32_t pack_sat4_ln(int32_t y0, int32_t y1, int32_t
   return d;
 }
 
+// byte i of w, sign-extended (prmt in sign-replicate mode)
+__device__ __forceinline__ int32_t sext_byte(uint32_t w, int i) {
+  int32_t r;
+  const uint32_t sel = (uint32_t)i | ((uint32_t)(8 | i) << 4) | ((uint32_t)(8 | i) << 8) | ((uint32_t)(8 | i) << 12);
+  asm("prmt.b32 %0, %1, 0, %2;" : "=r"(r) : "r"(w), "r"(sel));
+  return r;
+}
+
 // One row of `cols` int8 values per half-warp; lane l of the half-warp holds
-// the 16-byte chunks l, l + 16, ... (CPL of them).
-template <int CPL>
+// the 16-byte chunks l, l + 16, ... (CPL of them).  CLAMP = false when the host
+// has shown that (b acc) >> c fits int32 for every reachable acc.
+template <int CPL, bool CLAMP>
 __global__ void __launch_bounds__(kLnThreads)
     layernorm_kernel(const int8_t* __restrict__ x, int64_t rows, int32_t cols, const int8_t* __restrict__ gamma,
                      const int32_t* __restrict__ beta, int32_t F, int32_t M_ln, ivit_dyadic out,
@@ -128,8 +138,9 @@ __global__ void __launch_bounds__(kLnThreads)
   if (sigma < 1) sigma = 1;
   const int32_t f = (1 << M_ln) / sigma;
   const int sh = M_ln - F;
-  int32_t lo, hi;
-  out_bounds(out.b, out.c, lo, hi);
+  const int32_t muf = mu * f;  // (x - mu) f = x f - mu f, exact in 32-bit arithmetic (|(x - mu) f| < 2^31)
+  int32_t lo = INT_MIN, hi = INT_MAX;
+  if (CLAMP) out_bounds(out.b, out.c, lo, hi);
   int8_t* yr = y + row * cols;
 #pragma unroll
   for (int k = 0; k < CPL; ++k) {
@@ -147,11 +158,10 @@ __global__ void __launch_bounds__(kLnThreads)
         int32_t r[4];
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-          const int32_t d = (int32_t)(int8_t)(uint8_t)(xw[q] >> (8 * e)) - mu;
-          const int32_t nv = (d * f) >> sh;
-          const int32_t acc = nv * (int32_t)(int8_t)(uint8_t)(gw[q] >> (8 * e)) + bb[e];
-          const int32_t a = min(max(acc, lo), hi);
-          const int64_t pr = (int64_t)out.b * a;  // (b a) >> c fits int32: one funnel shift
+          const int32_t nv = (sext_byte(xw[q], e) * f - muf) >> sh;
+          int32_t acc = nv * sext_byte(gw[q], e) + bb[e];
+          if (CLAMP) acc = min(max(acc, lo), hi);
+          const int64_t pr = (int64_t)out.b * acc;  // (b acc) >> c fits int32: one funnel shift
           r[e] = (int32_t)__funnelshift_r((uint32_t)pr, (uint32_t)(pr >> 32), (uint32_t)out.c);
         }
         o[q] = pack_sat4_ln(r[0], r[1], r[2], r[3]);
@@ -185,16 +195,24 @@ ivit_status launch_layernorm(const DeviceCtx& dc, const int8_t* x, int64_t rows,
   if (blocks > 0x7fffffff) return IVIT_ERR_UNSUPPORTED;
   const unsigned g = (unsigned)blocks;
   const int nchunk = cols / 16;
+  // |n| <= 255 2^F, |gamma| <= 128, |beta| <= 2^30: when b times that bound stays
+  // below 2^(30 + c), (b acc) >> c always fits int32 and the clamp is not needed
+  const double amax = 255.0 * 128.0 * std::ldexp(1.0, F) + std::ldexp(1.0, 30);
+  const bool clamp = amax * (double)out.b >= std::ldexp(1.0, 30 + out.c);
+#define IVIT_LN_LAUNCH(CPL)                                                                                 \
+  (clamp ? layernorm_kernel<CPL, true><<<g, kLnThreads, 0, stream>>>(x, rows, cols, gamma, beta, F, M_ln, out, y) \
+         : layernorm_kernel<CPL, false><<<g, kLnThreads, 0, stream>>>(x, rows, cols, gamma, beta, F, M_ln, out, y))
   if (nchunk <= 16)
-    layernorm_kernel<1><<<g, kLnThreads, 0, stream>>>(x, rows, cols, gamma, beta, F, M_ln, out, y);
+    IVIT_LN_LAUNCH(1);
   else if (nchunk <= 32)
-    layernorm_kernel<2><<<g, kLnThreads, 0, stream>>>(x, rows, cols, gamma, beta, F, M_ln, out, y);
+    IVIT_LN_LAUNCH(2);
   else if (nchunk <= 48)
-    layernorm_kernel<3><<<g, kLnThreads, 0, stream>>>(x, rows, cols, gamma, beta, F, M_ln, out, y);
+    IVIT_LN_LAUNCH(3);
   else if (nchunk <= 64)
-    layernorm_kernel<4><<<g, kLnThreads, 0, stream>>>(x, rows, cols, gamma, beta, F, M_ln, out, y);
+    IVIT_LN_LAUNCH(4);
   else
-    layernorm_kernel<8><<<g, kLnThreads, 0, stream>>>(x, rows, cols, gamma, beta, F, M_ln, out, y);
+    IVIT_LN_LAUNCH(8);
+#undef IVIT_LN_LAUNCH
   note_launch();
   return cudaGetLastError() == cudaSuccess ? IVIT_OK : IVIT_ERR_CUDA;
 }

@@ -386,6 +386,28 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       else
         kc = chan_const(0, 0, 0, args.K);
       const bool clamp = __any_sync(0xffffffffu, kc.needs_clamp);  // warp-uniform path choice
+      if (EPI == kEpiResidual) {
+        // pull this warp's skip rows of the next tile into L2 while the MMAs of
+        // this one run (one 32-byte sector per token row of each chunk)
+        const int tn = t + (int)gridDim.x;
+        if (tn < num_tiles) {
+          const int64_t tok_n = (int64_t)(tn / ch_tiles) * BN + lane;
+          const int ch_n = (tn % ch_tiles) * kBM + quarter * 32;
+          if (ch_n < N)
+            for (int cc = c_begin; cc < c_end; ++cc) {
+              const int64_t tok = tok_n + 32 * cc;
+              if (tok < M) asm volatile("prefetch.global.L2 [%0];" ::"l"(args.skip + tok * N + ch_n));
+            }
+        }
+        if (t == (int)blockIdx.x) {  // the first tile prefetches its own rows
+          const int64_t tok_c = (int64_t)tb * BN + lane;
+          if (quarter * 32 + cb * kBM < N)
+            for (int cc = c_begin; cc < c_end; ++cc) {
+              const int64_t tok = tok_c + 32 * cc;
+              if (tok < M) asm volatile("prefetch.global.L2 [%0];" ::"l"(args.skip + tok * N + cb * kBM + quarter * 32));
+            }
+        }
+      }
       const bool got = mbar_wait(&tfull[acc], acc_phase, args.status);
       if (!__all_sync(0xffffffffu, got)) break;  // warp-uniform give-up
       tc_fence_after();

@@ -177,6 +177,26 @@ def test_layernorm_extreme_rows():
     np.testing.assert_array_equal(host(y), oracle.layernorm(x, gamma, beta, 7, 23, out))
 
 
+@pytest.mark.parametrize("F", [0, 7, 14])
+@pytest.mark.parametrize("side", [0.9, 1.1])
+def test_layernorm_extreme_beta(F, side):
+    """|beta| at its limit 2^30 and an output ratio on either side of the point
+    where the product b acc can leave int32 (the kernel then clamps acc first)."""
+    cols, rows = 64, 6
+    rng = np.random.default_rng(F + int(10 * side))
+    x = rng.integers(-128, 128, (rows, cols)).astype(np.int8)
+    x[0, ::2], x[0, 1::2] = -128, 127
+    gamma = np.where(np.arange(cols) % 2 == 0, -128, 127).astype(np.int8)
+    beta = np.where(np.arange(cols) % 3 == 0, 1 << 30, -(1 << 30)).astype(np.int32)
+    beta[5] = 0
+    amax = 255.0 * 128.0 * 2.0**F + 2.0**30
+    ratio = side * 2.0**30 / amax
+    out_d, out_o = ivit.ivit_dyadic_from_double(ratio), oracle.dyadic(ratio)
+    y = torch.empty((rows, cols), dtype=torch.int8, device="cuda")
+    ivit.ivit_layernorm(dev(x, torch.int8), dev(gamma, torch.int8), dev(beta, torch.int32), F, 23, out_d, y)
+    np.testing.assert_array_equal(host(y), oracle.layernorm(x, gamma, beta, F, 23, out_o))
+
+
 @pytest.mark.parametrize("M,K,N", [(1, 16, 16), (197, 192, 768), (300, 768, 3072), (129, 384, 1552)])
 def test_linear_shiftgelu_parity(M, K, N):
     """fc1 with ShiftGELU in the epilogue == oracle linear, then oracle ShiftGELU."""
