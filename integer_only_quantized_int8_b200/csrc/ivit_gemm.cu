@@ -9,10 +9,11 @@
 // The accumulator is computed transposed, D = W X^T: the UMMA M dimension
 // (TMEM lanes) runs over 128 output channels and N over BN tokens.  Every
 // epilogue thread therefore owns one output channel of the tile and keeps that
-// channel's multiplier, shift, bias and saturation bounds in registers; the
-// per-element work is a clamp, one 32x32->64 multiply-add, one funnel shift
-// and a saturating byte pack.  A 4 x 4 byte transpose across lanes turns the
-// channel-major bytes into token-major 4-byte words for coalesced stores.
+// channel's multiplier, shift, bias and saturation bounds in registers.  When
+// b_j < 2^(c_j - 1) (a requant scale below one half, the usual case) the
+// requant floor(b (acc + bias) / 2^c) is one mul.hi by b 2^(32 - c); the
+// saturating byte pack then clips.  A 4 x 4 byte transpose across lanes turns
+// the channel-major bytes into token-major 4-byte words for coalesced stores.
 //
 // Roles (one CTA per SM, persistent over 128 x BN tiles):
 //   warp 0      TMA producer: W and X k-slices of 128 bytes, 128B swizzle,
@@ -20,8 +21,8 @@
 //   warp 1      allocates TMEM (two BN-column accumulators) and one lane issues
 //               tcgen05.mma M=128 N=BN K=32; tcgen05.commit frees smem stages
 //               and publishes finished accumulators;
-//   warps 2-9   epilogue: two warps per TMEM lane quarter split the tile's
-//               token chunks; the accumulator of tile t drains while the
+//   warps 2-13  epilogue: three warps per TMEM lane quarter split the tile's
+//               16-token chunks; the accumulator of tile t drains while the
 //               MMAs of tile t+1 run.
 #include <climits>
 
@@ -33,7 +34,8 @@ namespace {
 
 constexpr int kBM = 128;  // output channels per tile
 constexpr int kBK = 128;  // bytes = int8 elements per k-slice (one 128-byte swizzle row)
-constexpr int kEpiWarps = 8;  // two per TMEM lane quarter
+constexpr int kEpiWarps = 12;  // three per TMEM lane quarter
+constexpr int kEpiParts = kEpiWarps / 4;
 constexpr int kGemmThreads = 64 + 32 * kEpiWarps;
 
 struct GemmArgs {
@@ -80,17 +82,26 @@ IVIT_DEV int32_t sat_i32(int64_t v) {
 // job.  When even the largest possible |acc + bias| (2^14 K + |bias|) keeps
 // |b (acc + bias)| below 2^(30 + c), the shifted result always fits int32 and
 // the clamp is skipped.
+//
+// Fast form: when b < 2^(c - 1), bq = b 2^(32 - c) is a positive int32 and
+// floor(b v / 2^c) = floor(bq v / 2^32) = mul.hi(bq, v) exactly, for every
+// int32 v; acc + bias stays within int32 because |acc| <= 2^14 K <= 2^28 and
+// |bias| <= 2^30.  b = 0 takes the fast form with bq = 0.
 struct ChanConst {
   int32_t b, c, lo_acc, hi_acc;
+  int32_t bias, bq;
   int64_t bb;       // b * bias
-  bool needs_clamp;
+  bool fast, needs_clamp;
 };
 
 IVIT_DEV ChanConst chan_const(int32_t b, int32_t c, int32_t bias, int32_t K) {
   ChanConst k;
   k.b = b;
   k.c = c;
+  k.bias = bias;
   k.bb = (int64_t)b * bias;
+  k.fast = b == 0 || (c >= 1 && (int64_t)b < ((int64_t)1 << (c - 1)));
+  k.bq = (k.fast && b != 0) ? (int32_t)((uint32_t)b << (32 - c)) : 0;
   if (b == 0) {
     k.lo_acc = INT_MIN;
     k.hi_acc = INT_MAX;
@@ -108,11 +119,16 @@ IVIT_DEV ChanConst chan_const(int32_t b, int32_t c, int32_t bias, int32_t K) {
   return k;
 }
 
-// floor(b (acc + bias) / 2^c) for acc within the bounds above; fits int32, so
-// the low word of the 64-bit shift is one funnel shift (c <= 31)
-template <bool CLAMP>
-IVIT_DEV int32_t requant_clamped(int32_t acc, const ChanConst& k) {
-  const int32_t a = CLAMP ? min(max(acc, k.lo_acc), k.hi_acc) : acc;
+// Requant forms, chosen per warp and tile: every channel of the warp fast, or
+// the 64-bit product with or without the accumulator clamp.
+enum ReqForm : int { kReqFast = 0, kReqWide = 1, kReqWideClamp = 2 };
+
+// floor(b (acc + bias) / 2^c); in the wide forms the result fits int32 (see
+// above), so the low word of the 64-bit shift is one funnel shift (c <= 31)
+template <int REQ>
+IVIT_DEV int32_t requant_acc(int32_t acc, const ChanConst& k) {
+  if (REQ == kReqFast) return __mulhi(k.bq, acc + k.bias);
+  const int32_t a = REQ == kReqWideClamp ? min(max(acc, k.lo_acc), k.hi_acc) : acc;
   const int64_t v = (int64_t)k.b * a + k.bb;
   return (int32_t)__funnelshift_r((uint32_t)v, (uint32_t)(v >> 32), (uint32_t)k.c);
 }
@@ -125,8 +141,16 @@ IVIT_DEV uint32_t pack_sat4(int32_t y0, int32_t y1, int32_t y2, int32_t y3) {
   return d;
 }
 
-// sign-extended byte i of w
-IVIT_DEV int32_t sbyte(uint32_t w, int i) { return (int32_t)(int8_t)(uint8_t)(w >> (8 * i)); }
+// sign-extended byte I of w: one prmt in sign-replicate mode (the __byte_perm
+// intrinsic keeps only the low three bits of each selector nibble, so the
+// instruction is written out)
+template <int I>
+IVIT_DEV int32_t sbyte(uint32_t w) {
+  constexpr uint32_t sel = (uint32_t)I | ((8u | I) << 4) | ((8u | I) << 8) | ((8u | I) << 12);
+  int32_t r;
+  asm("prmt.b32 %0, %1, 0, %2;" : "=r"(r) : "r"(w), "n"(sel));
+  return r;
+}
 
 // 4 x 4 byte transpose among lanes 4g..4g+3: lane l enters with byte i =
 // element (i, l) and leaves with byte i = element (l, i).  sel2 / sel1 are
@@ -139,21 +163,46 @@ IVIT_DEV uint32_t transpose4x4(uint32_t w, uint32_t sel2, uint32_t sel1) {
   return __byte_perm(w, o, sel1);
 }
 
-// One 32-token chunk of one epilogue warp: requant the 32 accumulators of this
+// sat_8((b_skip s + b_branch y) >> c) on the four bytes of two words.  The
+// sum is below 2^39 in magnitude, so once c >= 9 the shifted value fits int32:
+// the low word of the funnel shift is exact and the saturating pack clips it.
+template <bool FAST_RES>
+IVIT_DEV uint32_t residual_word(uint32_t s, uint32_t y, const ivit_residual& res) {
+  int32_t z[4];
+#define IVIT_RES_BYTE(I)                                                                      \
+  {                                                                                           \
+    int64_t t = (int64_t)res.b_skip * sbyte<I>(s);                                            \
+    t += (int64_t)res.b_branch * sbyte<I>(y);                                                 \
+    if (FAST_RES) {                                                                           \
+      z[I] = (int32_t)__funnelshift_r((uint32_t)t, (uint32_t)(t >> 32), (uint32_t)res.c);     \
+    } else {                                                                                  \
+      const int64_t q = t >> res.c;                                                           \
+      z[I] = (int32_t)(q < -128 ? -128 : (q > 127 ? 127 : q));                                \
+    }                                                                                         \
+  }
+  IVIT_RES_BYTE(0)
+  IVIT_RES_BYTE(1)
+  IVIT_RES_BYTE(2)
+  IVIT_RES_BYTE(3)
+#undef IVIT_RES_BYTE
+  return pack_sat4(z[0], z[1], z[2], z[3]);
+}
+
+// One 16-token chunk of one epilogue warp: requant the 16 accumulators of this
 // thread's channel, pack, transpose to token-major words, apply the residual
-// if any, and store.  r holds TMEM columns [32 cc, 32 cc + 32) of lane ch.
-template <int EPI, bool NARROW, bool CLAMP>
-IVIT_DEV void epi_chunk(const uint32_t (&r)[32], const ChanConst& kc, const GemmArgs& args, const int8_t* gelu_tab,
-                        int64_t tok0, int ch4, int sub, uint32_t sel2, uint32_t sel1, bool fast_res) {
+// if any, and store.  r holds TMEM columns [16 cc, 16 cc + 16) of lane ch.
+template <int EPI, bool NARROW, int REQ>
+IVIT_DEV void epi_chunk(const uint32_t (&r)[16], const ChanConst& kc, const GemmArgs& args, const int8_t* gelu_tab,
+                        int64_t tok0, int ch4, int sub, uint32_t sel2, uint32_t sel1) {
   const int64_t M = args.M;
   const int N = args.N;
-  uint32_t w[8];
+  uint32_t w[4];
 #pragma unroll
-  for (int k = 0; k < 8; ++k) {
+  for (int k = 0; k < 4; ++k) {
     int32_t y[4];
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-      int32_t v = requant_clamped<CLAMP>((int32_t)r[4 * k + i], kc);
+      int32_t v = requant_acc<REQ>((int32_t)r[4 * k + i], kc);
       if (EPI == kEpiGelu) {
         v = min(max(v, -128), 127);
         v = gelu_tab[v + 128];
@@ -164,68 +213,59 @@ IVIT_DEV void epi_chunk(const uint32_t (&r)[32], const ChanConst& kc, const Gemm
     }
     w[k] = transpose4x4(pack_sat4(y[0], y[1], y[2], y[3]), sel2, sel1);
   }
-  // lane (4 grp + sub) now holds, for k = 0..7, token tok0 + 4k + sub, channels ch4..ch4+3
+  // lane (4 grp + sub) now holds, for k = 0..3, token tok0 + 4k + sub, channels ch4..ch4+3
   if (ch4 >= N) return;
   // word k goes to token tok0 + 4k + sub: a fixed stride of 4N bytes
   const int64_t off0 = (tok0 + sub) * N + ch4;
   const int64_t stride = 4 * (int64_t)N;
-  const bool full = tok0 + 32 <= M;
+  const bool full = tok0 + 16 <= M;
   if (EPI == kEpiResidual) {
-    // all eight skip words are requested before any store, so their latencies overlap
-    uint32_t s[8];
+    // all four skip words are requested before any store, so their latencies overlap
+    uint32_t s[4];
     const int8_t* sp = args.skip + off0;
 #pragma unroll
-    for (int k = 0; k < 8; ++k)
+    for (int k = 0; k < 4; ++k)
       s[k] = (full || tok0 + 4 * k + sub < M) ? __ldg(reinterpret_cast<const uint32_t*>(sp + k * stride)) : 0u;
+    if (args.res.c >= 9) {
 #pragma unroll
-    for (int k = 0; k < 8; ++k) {
-      int32_t z[4];
+      for (int k = 0; k < 4; ++k) w[k] = residual_word<true>(s[k], w[k], args.res);
+    } else {
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const int64_t sum = (int64_t)args.res.b_skip * sbyte(s[k], i) + (int64_t)args.res.b_branch * sbyte(w[k], i);
-        if (fast_res) {
-          z[i] = (int32_t)__funnelshift_r((uint32_t)sum, (uint32_t)(sum >> 32), (uint32_t)args.res.c);
-        } else {
-          const int64_t q = sum >> args.res.c;
-          z[i] = (int32_t)(q < -128 ? -128 : (q > 127 ? 127 : q));
-        }
-      }
-      w[k] = pack_sat4(z[0], z[1], z[2], z[3]);
+      for (int k = 0; k < 4; ++k) w[k] = residual_word<false>(s[k], w[k], args.res);
     }
   }
   int8_t* yp = args.Y + off0;
   if (full) {
 #pragma unroll
-    for (int k = 0; k < 8; ++k) *reinterpret_cast<uint32_t*>(yp + k * stride) = w[k];
+    for (int k = 0; k < 4; ++k) *reinterpret_cast<uint32_t*>(yp + k * stride) = w[k];
   } else {
 #pragma unroll
-    for (int k = 0; k < 8; ++k)
+    for (int k = 0; k < 4; ++k)
       if (tok0 + 4 * k + sub < M) *reinterpret_cast<uint32_t*>(yp + k * stride) = w[k];
   }
 }
 
-// The chunks [c_begin, c_end) of one tile, with the next chunk's TMEM load in
-// flight while the current chunk is processed.
-template <int EPI, bool NARROW, bool CLAMP>
+// The 16-token chunks [c_begin, c_end) of one tile, with the next chunk's TMEM
+// load in flight while the current chunk is processed.
+template <int EPI, bool NARROW, int REQ>
 IVIT_DEV void epi_tile(uint32_t tbase, int c_begin, int c_end, int64_t tok_base, const ChanConst& kc,
-                       const GemmArgs& args, const int8_t* gelu_tab, int ch4, int sub, uint32_t sel2, uint32_t sel1,
-                       bool fast_res) {
+                       const GemmArgs& args, const int8_t* gelu_tab, int ch4, int sub, uint32_t sel2,
+                       uint32_t sel1) {
   const int64_t M = args.M;
   int n = c_end - c_begin;  // chunks that hold at least one valid token
-  while (n > 0 && tok_base + 32 * (c_begin + n - 1) >= M) --n;
+  while (n > 0 && tok_base + 16 * (c_begin + n - 1) >= M) --n;
   if (n <= 0) return;
-  uint32_t ra[32], rb[32];
-  tmem_ld32(tbase + (uint32_t)(32 * c_begin), ra);
+  uint32_t ra[16], rb[16];
+  tmem_ld16(tbase + (uint32_t)(16 * c_begin), ra);
   for (int i = 0; i < n; i += 2) {
     const int ca = c_begin + i;
     tmem_ld_wait();
-    if (i + 1 < n) tmem_ld32(tbase + (uint32_t)(32 * (ca + 1)), rb);
-    epi_chunk<EPI, NARROW, CLAMP>(ra, kc, args, gelu_tab, tok_base + 32 * ca, ch4, sub, sel2, sel1, fast_res);
+    if (i + 1 < n) tmem_ld16(tbase + (uint32_t)(16 * (ca + 1)), rb);
+    epi_chunk<EPI, NARROW, REQ>(ra, kc, args, gelu_tab, tok_base + 16 * ca, ch4, sub, sel2, sel1);
     if (i + 1 < n) {
       tmem_ld_wait();
-      if (i + 2 < n) tmem_ld32(tbase + (uint32_t)(32 * (ca + 2)), ra);
-      epi_chunk<EPI, NARROW, CLAMP>(rb, kc, args, gelu_tab, tok_base + 32 * (ca + 1), ch4, sub, sel2, sel1,
-                                    fast_res);
+      if (i + 2 < n) tmem_ld16(tbase + (uint32_t)(16 * (ca + 2)), ra);
+      epi_chunk<EPI, NARROW, REQ>(rb, kc, args, gelu_tab, tok_base + 16 * (ca + 1), ch4, sub, sel2, sel1);
     }
   }
 }
@@ -361,18 +401,16 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     }
   } else {
     // ------------------------------------------------------------ epilogue
-    constexpr int kChunks = BN / 32;
-    constexpr int kPerQuarter = kEpiWarps / 4;
+    constexpr int kChunks = BN / 16;
     const int e = warp - 2;
     const int quarter = warp & 3;  // TMEM lanes [32 q, 32 q + 32) = channels of this warp
     const int part = e >> 2;       // which of the quarter's warps: splits the token chunks
-    const int c_begin = (kChunks * part) / kPerQuarter;
-    const int c_end = (kChunks * (part + 1)) / kPerQuarter;
+    const int c_begin = (kChunks * part) / kEpiParts;
+    const int c_end = (kChunks * (part + 1)) / kEpiParts;
     const uint32_t sel2 = (lane & 2) ? 0x3276u : 0x5410u;
     const uint32_t sel1 = (lane & 1) ? 0x3715u : 0x6240u;
-    const int sub = lane & 3;               // token offset within a transposed 4 x 4 block
-    const int grp = lane >> 2;              // channel group of 4 within the warp's 32 channels
-    const bool fast_res = args.res.c >= 9;  // |b_skip s + b_branch y| < 2^39: the shifted sum fits int32
+    const int sub = lane & 3;   // token offset within a transposed 4 x 4 block
+    const int grp = lane >> 2;  // channel group of 4 within the warp's 32 channels
     int acc = 0;
     uint32_t acc_phase = 0;
     for (int t = blockIdx.x; t < num_tiles; t += gridDim.x) {
@@ -385,26 +423,31 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                         args.K);
       else
         kc = chan_const(0, 0, 0, args.K);
-      const bool clamp = __any_sync(0xffffffffu, kc.needs_clamp);  // warp-uniform path choice
+      // warp-uniform requant form
+      const int req = __all_sync(0xffffffffu, kc.fast) ? kReqFast
+                      : (__any_sync(0xffffffffu, kc.needs_clamp) ? kReqWideClamp : kReqWide);
       if (EPI == kEpiResidual) {
         // pull this warp's skip rows of the next tile into L2 while the MMAs of
-        // this one run (one 32-byte sector per token row of each chunk)
+        // this one run (one 32-byte sector per token row)
         const int tn = t + (int)gridDim.x;
         if (tn < num_tiles) {
-          const int64_t tok_n = (int64_t)(tn / ch_tiles) * BN + lane;
+          const int64_t tok_n = (int64_t)(tn / ch_tiles) * BN + 16 * c_begin + lane;
           const int ch_n = (tn % ch_tiles) * kBM + quarter * 32;
           if (ch_n < N)
-            for (int cc = c_begin; cc < c_end; ++cc) {
-              const int64_t tok = tok_n + 32 * cc;
-              if (tok < M) asm volatile("prefetch.global.L2 [%0];" ::"l"(args.skip + tok * N + ch_n));
+            for (int tk = 0; tk < 16 * (c_end - c_begin); tk += 32) {
+              const int64_t tok = tok_n + tk;
+              if (lane + tk < 16 * (c_end - c_begin) && tok < M)
+                asm volatile("prefetch.global.L2 [%0];" ::"l"(args.skip + tok * N + ch_n));
             }
         }
         if (t == (int)blockIdx.x) {  // the first tile prefetches its own rows
-          const int64_t tok_c = (int64_t)tb * BN + lane;
-          if (quarter * 32 + cb * kBM < N)
-            for (int cc = c_begin; cc < c_end; ++cc) {
-              const int64_t tok = tok_c + 32 * cc;
-              if (tok < M) asm volatile("prefetch.global.L2 [%0];" ::"l"(args.skip + tok * N + cb * kBM + quarter * 32));
+          const int64_t tok_c = (int64_t)tb * BN + 16 * c_begin + lane;
+          const int ch_c = cb * kBM + quarter * 32;
+          if (ch_c < N)
+            for (int tk = 0; tk < 16 * (c_end - c_begin); tk += 32) {
+              const int64_t tok = tok_c + tk;
+              if (lane + tk < 16 * (c_end - c_begin) && tok < M)
+                asm volatile("prefetch.global.L2 [%0];" ::"l"(args.skip + tok * N + ch_c));
             }
         }
       }
@@ -413,12 +456,14 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       tc_fence_after();
       const uint32_t tbase = tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(acc * BN);
       __syncwarp();
-      if (clamp)
-        epi_tile<EPI, NARROW, true>(tbase, c_begin, c_end, (int64_t)tb * BN, kc, args, gelu_tab, ch4, sub, sel2, sel1,
-                                    fast_res);
+      const int64_t tok_base = (int64_t)tb * BN;
+      if (req == kReqFast)
+        epi_tile<EPI, NARROW, kReqFast>(tbase, c_begin, c_end, tok_base, kc, args, gelu_tab, ch4, sub, sel2, sel1);
+      else if (req == kReqWide)
+        epi_tile<EPI, NARROW, kReqWide>(tbase, c_begin, c_end, tok_base, kc, args, gelu_tab, ch4, sub, sel2, sel1);
       else
-        epi_tile<EPI, NARROW, false>(tbase, c_begin, c_end, (int64_t)tb * BN, kc, args, gelu_tab, ch4, sub, sel2,
-                                     sel1, fast_res);
+        epi_tile<EPI, NARROW, kReqWideClamp>(tbase, c_begin, c_end, tok_base, kc, args, gelu_tab, ch4, sub, sel2,
+                                             sel1);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&tempty[acc]);
