@@ -282,29 +282,38 @@ __global__ void __launch_bounds__(kAttnThreads)
 // Short sequences (N <= 256 keys): persistent, warp-specialised kernel.
 //
 // One CTA per SM walks the work items (128-query tile, head, image) with
-// stride gridDim.x.  Warp 0 issues the TMA loads of Q, K and V of the next
-// items into a two-stage shared-memory ring; warp 1 issues the tcgen05 MMAs
-// -- S = Q K^T of item i+1 into one of two 256-column TMEM buffers while the
-// softmax warps still work on item i, then P V of item i -- and warps 2-9
-// run Shiftmax and the output requant.  Within an item the score row never
-// leaves TMEM: pass 1 takes the row maximum of the raw int32 scores (the
-// logit requant is monotone, so max L = requant(max S)); pass 2 requantises
-// each score, looks up ShiftExp(L - max L) in a table replicated once per
-// shared-memory bank (lane l reads copy l, so lookups never conflict), sums
-// the row and writes the exponentials back into TMEM in place; pass 3 turns
-// them into u8 P = (Dv e) >> (M - k_out + 1), written straight into the
-// 128B-swizzled K-major operand of the P V MMA.  Warps w and w + 4 share TMEM
+// stride gridDim.x; local item j of a CTA belongs to softmax group j & 1.
+//   warp 0      TMA producer: Q, K and V of item j into stage j % 3 of a
+//               three-stage ring; a stage is released when P V of its item
+//               has completed, so loads run up to two items ahead;
+//   warp 1      MMA issuer: S = Q K^T of item j into TMEM buffer j & 1 once
+//               that buffer is free and the stage has landed, and P V of item
+//               j once its P is in shared memory.  It polls both conditions
+//               without blocking, so neither softmax group waits behind the
+//               other;
+//   warps 2-17  two softmax groups of eight warps.
+// Within an item the score row never leaves TMEM: pass 1 takes the row
+// maximum of the raw int32 scores (the logit requant is monotone, so
+// max L = requant(max S)); pass 2 requantises each score, looks up
+// ShiftExp(L - max L) in a table replicated once per shared-memory bank (lane
+// l reads copy l, so lookups never conflict), sums the row and writes the
+// exponentials back into TMEM in place; pass 3 turns them into
+// u8 P = (Dv e) >> (M - k_out + 1), written into the group's own
+// 128B-swizzled K-major P operand.  Warps w and w + 4 of a group share TMEM
 // lanes (query rows) and split the key columns; their partial maxima and sums
-// meet in shared memory behind a named barrier of the 256 softmax threads.
+// meet in shared memory behind a named barrier of the group's 256 threads.
+// P V lands in the first 64 columns of the item's S buffer, dead by then.
 // ---------------------------------------------------------------------------
 constexpr int kShortMaxKeys = 256;
 constexpr int kSoftWarps = 8;    // per softmax group
 constexpr int kSoftGroups = 2;   // groups take alternate items, one TMEM buffer each
+constexpr int kLoadStages = 3;
 constexpr int kPersistThreads = 64 + 32 * kSoftWarps * kSoftGroups;
 
 struct PersistLayout {
   int n64, n32, kblocks;
-  int r0_bytes, stage_bytes, tab_off, part_off, bar_off, total;
+  int k_off, v_off, stage_bytes;  // Q at 0, K, V within a stage
+  int p_off, p_bytes, tab_off, part_off, bar_off, total;
 };
 
 __host__ __device__ inline PersistLayout persist_layout(int N) {
@@ -312,14 +321,15 @@ __host__ __device__ inline PersistLayout persist_layout(int N) {
   L.n64 = (N + 63) / 64 * 64;
   L.n32 = (N + 31) / 32 * 32;
   L.kblocks = (L.n32 + 127) / 128;
-  const int qk = kQTile * kHeadDim + L.n64 * kHeadDim;
-  const int p = L.kblocks * 128 * 128;
-  L.r0_bytes = ((qk > p ? qk : p) + 1023) / 1024 * 1024;
-  L.stage_bytes = L.r0_bytes + (L.n64 * kHeadDim + 1023) / 1024 * 1024;  // R0 (Q, K, later P) + V
-  L.tab_off = 2 * L.stage_bytes;
+  L.k_off = kQTile * kHeadDim;             // 8 KB
+  L.v_off = L.k_off + L.n64 * kHeadDim;    // + a multiple of 4 KB
+  L.stage_bytes = L.v_off + L.n64 * kHeadDim;
+  L.p_off = kLoadStages * L.stage_bytes;   // a multiple of 4 KB
+  L.p_bytes = L.kblocks * 128 * 128;       // 16 KB per 128 keys
+  L.tab_off = L.p_off + kSoftGroups * L.p_bytes;
   L.part_off = L.tab_off + 256 * 32 * 4;
   L.bar_off = L.part_off + kSoftGroups * 2 * 2 * kQTile * 4;
-  L.total = L.bar_off + 16 * 8 + 16;
+  L.total = L.bar_off + 24 * 8;
   return L;
 }
 
@@ -331,15 +341,13 @@ IVIT_DEV uint32_t pack_sat4_attn(int32_t y0, int32_t y1, int32_t y2, int32_t y3)
   return d;
 }
 
-// sat_ks(floor(b S / 2^c)): one mul.hi when b 2^(32-c) fits a positive int32
+// floor(b S / 2^c) before the k_s-bit saturation: one mul.hi when
+// bq = b 2^(32 - c) fits a positive int32
 template <bool FASTQ>
-IVIT_DEV int32_t logit_requant(int32_t S, int32_t bq, int32_t b, int32_t c, int32_t lo, int32_t hi) {
-  if (FASTQ) {
-    const int32_t v = __mulhi(bq, S);  // floor(bq S / 2^32), bq = b 2^(32 - c)
-    return min(max(v, lo), hi);
-  } else {
-    return requant_bits(S, b, c, lo, hi);
-  }
+IVIT_DEV int32_t logit_unclamped(int32_t S, int32_t bq, int32_t b, int32_t c) {
+  if (FASTQ) return __mulhi(bq, S);
+  const int64_t q = ((int64_t)b * (int64_t)S) >> c;
+  return (int32_t)(q < (int64_t)INT_MIN ? (int64_t)INT_MIN : (q > (int64_t)INT_MAX ? (int64_t)INT_MAX : q));
 }
 
 // bounded wait that also gives up at once when another thread has aborted
@@ -361,6 +369,56 @@ IVIT_DEV bool wait_or_abort(uint64_t* bar, uint32_t parity, int* status, volatil
 // named barrier of one softmax group (ids 1 and 2; 256 threads each)
 IVIT_DEV void softmax_bar(int group) { asm volatile("bar.sync %0, %1;" ::"r"(1 + group), "n"(32 * kSoftWarps) : "memory"); }
 
+// Streams n 16-column chunks of this warp's TMEM lanes starting at taddr,
+// body(r, k) on chunk k.  Single-buffered: with eighteen warps a thread has
+// at most 96 registers, and the other softmax warps cover the load latency.
+template <typename F>
+IVIT_DEV void tmem_stream16(uint32_t taddr, int n, F&& body) {
+  uint32_t r[16];
+  for (int k = 0; k < n; ++k) {
+    tmem_ld16(taddr + (uint32_t)(16 * k), r);
+    tmem_ld_wait();
+    body(r, k);
+  }
+}
+
+// Pass 2 of one half row: e = ShiftExp(L - max L) by table, written back to
+// TMEM in place; returns the partial row sum.  tb = table + lane + 32 lmax,
+// so tb[-32 L] = ShiftExp(L - lmax).  UPPER: some row of the warp has a raw
+// logit maximum above the k_s-bit range, so the upper saturation is needed
+// (otherwise every logit of the row is at most lmax already).
+template <bool FASTQ, bool UPPER>
+IVIT_DEV uint32_t shiftmax_pass2(uint32_t t_row, int cbase, int nvalid, int N, const int32_t* tb, int32_t lmax,
+                                 int32_t bq, const AttnArgs& a) {
+  uint32_t s4[4] = {0u, 0u, 0u, 0u};
+  tmem_stream16(t_row + (uint32_t)cbase, nvalid, [&](uint32_t(&r)[16], int k) {
+    const int col = cbase + 16 * k;
+    const int lim = N - col;
+    if (lim >= 16) {
+#pragma unroll
+      for (int e = 0; e < 16; ++e) {
+        int32_t l = max(logit_unclamped<FASTQ>((int32_t)r[e], bq, a.logit_b, a.logit_c), a.ks_lo);
+        if (UPPER || !FASTQ) l = min(l, a.ks_hi);
+        const uint32_t x = (uint32_t)tb[-32 * l];
+        s4[e & 3] += x;
+        r[e] = x;
+      }
+    } else {
+#pragma unroll
+      for (int e = 0; e < 16; ++e) {
+        // padding keys: any index in range, then masked
+        const int32_t l = min(max(logit_unclamped<FASTQ>((int32_t)r[e], bq, a.logit_b, a.logit_c), a.ks_lo), lmax);
+        const uint32_t x = e < lim ? (uint32_t)tb[-32 * l] : 0u;
+        s4[e & 3] += x;
+        r[e] = x;
+      }
+    }
+    tmem_st16(t_row + (uint32_t)col, r);
+  });
+  tmem_st_wait();
+  return (s4[0] + s4[1]) + (s4[2] + s4[3]);
+}
+
 template <bool FASTQ>
 __global__ void __launch_bounds__(kPersistThreads, 1)
     attention_persist_kernel(const __grid_constant__ CUtensorMap tm, const AttnArgs a, const int32_t bq) {
@@ -370,15 +428,15 @@ __global__ void __launch_bounds__(kPersistThreads, 1)
   const PersistLayout L = persist_layout(N);
   int32_t* tab = reinterpret_cast<int32_t*>(smem + L.tab_off);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L.bar_off);
-  uint64_t* qk_full = bars + 0;       // [2] Q and K landed
-  uint64_t* v_full = bars + 2;        // [2] V landed
-  uint64_t* s_full = bars + 4;        // [2] S in TMEM
-  uint64_t* p_full = bars + 6;        // [2] P in shared memory (one arrival per softmax warp)
-  uint64_t* o_full = bars + 8;        // [2] P V in TMEM
-  uint64_t* stage_empty = bars + 10;  // [2] ring stage reusable
-  uint64_t* tmem_empty = bars + 12;   // [2] TMEM buffer reusable (one arrival per softmax warp)
-  uint32_t* tslot = reinterpret_cast<uint32_t*>(bars + 14);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 15);
+  uint64_t* qkv_full = bars + 0;      // [3] Q, K and V of a stage landed
+  uint64_t* stage_empty = bars + 3;   // [3] stage reusable (P V of its item done)
+  uint64_t* s_full = bars + 6;        // [2] S in TMEM buffer g
+  uint64_t* p_full = bars + 8;        // [2] P of group g in shared memory (one arrival per warp)
+  uint64_t* o_full = bars + 10;       // [2] P V in TMEM buffer g
+  uint64_t* tmem_empty = bars + 12;   // [2] TMEM buffer g reusable (one arrival per warp)
+  uint64_t* drain = bars + 14;        // all MMAs of the CTA complete
+  uint32_t* tslot = reinterpret_cast<uint32_t*>(bars + 15);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 16);
 
   const int tid = threadIdx.x;
   const int warp = tid >> 5;
@@ -387,18 +445,19 @@ __global__ void __launch_bounds__(kPersistThreads, 1)
   const int qtiles = (N + kQTile - 1) / kQTile;
   const int n_items = qtiles * a.H * a.B;
   const int nload = L.n64 / 64;
-  const int hcols = L.n32 / 2;  // key columns per softmax half (multiple of 16)
 
   if (tid == 0) {
-    for (int s = 0; s < 2; ++s) {
-      mbar_init(&qk_full[s], 1);
-      mbar_init(&v_full[s], 1);
-      mbar_init(&s_full[s], 1);
-      mbar_init(&p_full[s], kSoftWarps);
-      mbar_init(&o_full[s], 1);
+    for (int s = 0; s < kLoadStages; ++s) {
+      mbar_init(&qkv_full[s], 1);
       mbar_init(&stage_empty[s], 1);
-      mbar_init(&tmem_empty[s], kSoftWarps);
     }
+    for (int g = 0; g < kSoftGroups; ++g) {
+      mbar_init(&s_full[g], 1);
+      mbar_init(&p_full[g], kSoftWarps);
+      mbar_init(&o_full[g], 1);
+      mbar_init(&tmem_empty[g], kSoftWarps);
+    }
+    mbar_init(drain, 1);
     *abort_flag = 0;
     fence_barrier_init();
     prefetch_tensormap(&tm);
@@ -426,23 +485,21 @@ __global__ void __launch_bounds__(kPersistThreads, 1)
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
-      int i = 0;
-      for (int item = blockIdx.x; item < n_items; item += gridDim.x, ++i) {
-        const int s = i & 1;
-        const uint32_t ph = (uint32_t)((i >> 1) & 1);
+      int j = 0;
+      for (int item = blockIdx.x; item < n_items; item += gridDim.x, ++j) {
+        const int s = j % kLoadStages;
+        const uint32_t ph = (uint32_t)((j / kLoadStages) & 1);
         if (!wait_or_abort(&stage_empty[s], ph ^ 1, a.status, abort_flag)) break;
         const int qt = item % qtiles, h = (item / qtiles) % a.H, img = item / (qtiles * a.H);
         const int row0 = img * N;
         uint8_t* st = smem + s * L.stage_bytes;
-        uint8_t* sV = st + L.r0_bytes;
-        mbar_arrive_expect_tx(&qk_full[s], (uint32_t)(kQTile * kHeadDim + nload * 64 * kHeadDim));
-        tma_load_2d(st, &tm, h * kHeadDim, row0 + qt * kQTile, &qk_full[s]);
-        tma_load_2d(st + 64 * kHeadDim, &tm, h * kHeadDim, row0 + qt * kQTile + 64, &qk_full[s]);
-        for (int j = 0; j < nload; ++j)
-          tma_load_2d(st + kQTile * kHeadDim + j * 64 * kHeadDim, &tm, D + h * kHeadDim, row0 + 64 * j, &qk_full[s]);
-        mbar_arrive_expect_tx(&v_full[s], (uint32_t)(nload * 64 * kHeadDim));
-        for (int j = 0; j < nload; ++j)
-          tma_load_2d(sV + j * 64 * kHeadDim, &tm, 2 * D + h * kHeadDim, row0 + 64 * j, &v_full[s]);
+        mbar_arrive_expect_tx(&qkv_full[s], (uint32_t)(kQTile * kHeadDim + 2 * nload * 64 * kHeadDim));
+        tma_load_2d(st, &tm, h * kHeadDim, row0 + qt * kQTile, &qkv_full[s]);
+        tma_load_2d(st + 64 * kHeadDim, &tm, h * kHeadDim, row0 + qt * kQTile + 64, &qkv_full[s]);
+        for (int i = 0; i < nload; ++i)
+          tma_load_2d(st + L.k_off + i * 64 * kHeadDim, &tm, D + h * kHeadDim, row0 + 64 * i, &qkv_full[s]);
+        for (int i = 0; i < nload; ++i)
+          tma_load_2d(st + L.v_off + i * 64 * kHeadDim, &tm, 2 * D + h * kHeadDim, row0 + 64 * i, &qkv_full[s]);
       }
     }
   } else if (warp == 1) {
@@ -451,93 +508,92 @@ __global__ void __launch_bounds__(kPersistThreads, 1)
       const uint32_t idesc_s = idesc_i8(kQTile, L.n32, true, true, false);
       const uint32_t idesc_o = idesc_i8(kQTile, kHeadDim, false, true, true);
       const int n_local = n_items > (int)blockIdx.x ? (n_items - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
-      // S = Q K^T of local item j into TMEM buffer j & 1
-      auto issue_s = [&](int j) -> bool {
-        const int s = j & 1;
-        const uint32_t ph = (uint32_t)((j >> 1) & 1);
-        if (!wait_or_abort(&tmem_empty[s], ph ^ 1, a.status, abort_flag)) return false;
-        if (!wait_or_abort(&qk_full[s], ph, a.status, abort_flag)) return false;
-        tc_fence_after();
-        const uint32_t qa = smem_u32(smem + s * L.stage_bytes);
-        const uint32_t ka = qa + kQTile * kHeadDim;
+      int js = 0, jp = 0;  // next S, next P V (in item order each)
+      uint64_t t_last = globaltimer_ns();
+      while (jp < n_local) {
+        bool progress = false;
+        if (js < n_local && js < jp + kSoftGroups) {
+          const int g = js & 1, s = js % kLoadStages;
+          if (mbar_test(&tmem_empty[g], (uint32_t)(((js >> 1) & 1) ^ 1)) &&
+              mbar_test(&qkv_full[s], (uint32_t)((js / kLoadStages) & 1))) {
+            tc_fence_after();
+            const uint32_t qa = smem_u32(smem + s * L.stage_bytes);
+            const uint32_t ka = qa + L.k_off;
 #pragma unroll
-        for (int k = 0; k < kHeadDim / 32; ++k)
-          umma_i8(tmem + (uint32_t)(s * 256), smem_desc(qa + k * 32, 16, 512, kSwizzle64B),
-                  smem_desc(ka + k * 32, 16, 512, kSwizzle64B), idesc_s, k != 0);
-        umma_commit(&s_full[s]);
-        return true;
-      };
-      bool ok = n_local == 0 || issue_s(0);
-      for (int j = 0; j < n_local && ok; ++j) {
-        if (j + 1 < n_local && !issue_s(j + 1)) break;
-        const int s = j & 1;
-        const uint32_t ph = (uint32_t)((j >> 1) & 1);
-        if (!wait_or_abort(&p_full[s], ph, a.status, abort_flag)) break;
-        if (!wait_or_abort(&v_full[s], ph, a.status, abort_flag)) break;
-        tc_fence_after();
-        const uint32_t pa = smem_u32(smem + s * L.stage_bytes);
-        const uint32_t va = pa + L.r0_bytes;
-        for (int k = 0; k < L.n32 / 32; ++k)
-          umma_i8(tmem + (uint32_t)(s * 256), smem_desc(pa + (k >> 2) * 16384 + (k & 3) * 32, 16, 1024, kSwizzle128B),
-                  smem_desc(va + k * 32 * kHeadDim, 512, 512, kSwizzle64B), idesc_o, k != 0);
-        umma_commit(&o_full[s]);
-        umma_commit(&stage_empty[s]);
+            for (int k = 0; k < kHeadDim / 32; ++k)
+              umma_i8(tmem + (uint32_t)(g * 256), smem_desc(qa + k * 32, 16, 512, kSwizzle64B),
+                      smem_desc(ka + k * 32, 16, 512, kSwizzle64B), idesc_s, k != 0);
+            umma_commit(&s_full[g]);
+            ++js;
+            progress = true;
+          }
+        }
+        if (jp < js) {
+          const int g = jp & 1, s = jp % kLoadStages;
+          if (mbar_test(&p_full[g], (uint32_t)((jp >> 1) & 1))) {
+            tc_fence_after();
+            const uint32_t pa = smem_u32(smem + L.p_off + g * L.p_bytes);
+            const uint32_t va = smem_u32(smem + s * L.stage_bytes + L.v_off);
+            for (int k = 0; k < L.n32 / 32; ++k)
+              umma_i8(tmem + (uint32_t)(g * 256),
+                      smem_desc(pa + (k >> 2) * 16384 + (k & 3) * 32, 16, 1024, kSwizzle128B),
+                      smem_desc(va + k * 32 * kHeadDim, 512, 512, kSwizzle64B), idesc_o, k != 0);
+            umma_commit(&o_full[g]);
+            umma_commit(&stage_empty[s]);
+            ++jp;
+            progress = true;
+          }
+        }
+        if (progress) {
+          t_last = globaltimer_ns();
+        } else {
+          if (*abort_flag) break;
+          if (globaltimer_ns() - t_last > kWaitBudgetNs) {
+            report_timeout(a.status);
+            *abort_flag = 1;
+            break;
+          }
+          __nanosleep(32);
+        }
       }
+      // every MMA of this CTA has completed before TMEM is released
+      umma_commit(drain);
+      mbar_wait(drain, 0, a.status);
     }
   } else {
     // ------------------------------------------------------------ softmax warps
-    const int group = (warp - 2) / kSoftWarps;          // handles local items i with i % 2 == group
+    const int sw = warp - 2;
+    const int group = sw / kSoftWarps;   // handles local items j with j % 2 == group
     const int quarter = warp & 3;
-    const int half = ((warp - 2) >> 2) & 1;
+    const int half = (sw >> 2) & 1;
     const int row = quarter * 32 + lane;  // query row of the tile = TMEM lane
+    const int hcols = L.n32 / 2;          // key columns per half (a multiple of 16)
     const int cbase = half * hcols;
-    const int nchunk = hcols / 16;
-    const int rlo = row & 7;
+    const int nch = hcols / 16;
+    int nvalid = 0;  // chunks of this half that hold at least one real key
+    while (nvalid < nch && cbase + 16 * nvalid < N) ++nvalid;
     int32_t* part = reinterpret_cast<int32_t*>(smem + L.part_off) + group * 512;  // [half][max, sum][128 rows]
+    const int rlo = row & 7;
+    uint8_t* prow = smem + L.p_off + group * L.p_bytes + (row >> 3) * 1024 + rlo * 128;
+    const uint32_t t_row = tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(group * 256);
+    const int pshift = a.M - (a.k_out - 1);
     bool ok = true;
-    int i = group;
-    for (int item = blockIdx.x + group * gridDim.x; item < n_items; item += 2 * gridDim.x, i += 2) {
-      const int s = i & 1;
-      const uint32_t ph = (uint32_t)((i >> 1) & 1);
+    int j = group;
+    for (int item = blockIdx.x + group * gridDim.x; item < n_items; item += kSoftGroups * gridDim.x, j += 2) {
+      const uint32_t ph = (uint32_t)((j >> 1) & 1);
       const int qt = item % qtiles, h = (item / qtiles) % a.H, img = item / (qtiles * a.H);
       const int q0 = qt * kQTile;
-      if (ok) ok = wait_or_abort(&s_full[s], ph, a.status, abort_flag);
+      if (ok) ok = wait_or_abort(&s_full[group], ph, a.status, abort_flag);
       ok = __all_sync(0xffffffffu, ok);
       tc_fence_after();
-      const uint32_t t_row = tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(s * 256);
       // warps whose rows all lie past the image's last token skip the passes
       const bool work = ok && (q0 + quarter * 32 < N);
 
-#define IVIT_STREAM_CHUNKS(BODY)                                                      \
-  {                                                                                   \
-    uint32_t ra[16], rb[16];                                                          \
-    tmem_ld16(t_row + (uint32_t)cbase, ra);                                           \
-    for (int k = 0; k < nchunk; k += 2) {                                             \
-      tmem_ld_wait();                                                                 \
-      if (k + 1 < nchunk) tmem_ld16(t_row + (uint32_t)(cbase + 16 * (k + 1)), rb);    \
-      {                                                                               \
-        uint32_t(&r)[16] = ra;                                                        \
-        const int col = cbase + 16 * k;                                               \
-        BODY                                                                          \
-      }                                                                               \
-      if (k + 1 < nchunk) {                                                           \
-        tmem_ld_wait();                                                               \
-        if (k + 2 < nchunk) tmem_ld16(t_row + (uint32_t)(cbase + 16 * (k + 2)), ra);  \
-        {                                                                             \
-          uint32_t(&r)[16] = rb;                                                      \
-          const int col = cbase + 16 * (k + 1);                                       \
-          BODY                                                                        \
-        }                                                                             \
-      }                                                                               \
-    }                                                                                 \
-  }
-
-      // ---- pass 1: row maximum of the raw scores over the valid keys
-      // (independent running maxima keep the dependency chains short)
+      // ---- pass 1: row maximum of the raw scores over the real keys
       int32_t m4[4] = {INT_MIN, INT_MIN, INT_MIN, INT_MIN};
       if (work) {
-        IVIT_STREAM_CHUNKS({
-          const int lim = N - col;
+        tmem_stream16(t_row + (uint32_t)cbase, nvalid, [&](uint32_t(&r)[16], int k) {
+          const int lim = N - (cbase + 16 * k);
           if (lim >= 16) {
 #pragma unroll
             for (int e = 0; e < 16; ++e) m4[e & 3] = max(m4[e & 3], (int32_t)r[e]);
@@ -546,56 +602,39 @@ __global__ void __launch_bounds__(kPersistThreads, 1)
             for (int e = 0; e < 16; ++e)
               if (e < lim) m4[e & 3] = max(m4[e & 3], (int32_t)r[e]);
           }
-        })
+        });
       }
       int32_t smax = max(max(m4[0], m4[1]), max(m4[2], m4[3]));
       part[half * 256 + row] = smax;
       softmax_bar(group);
       smax = max(part[row], part[256 + row]);
-      const int32_t lmax = logit_requant<FASTQ>(smax, bq, a.logit_b, a.logit_c, a.ks_lo, a.ks_hi);
+      const int32_t vmax = logit_unclamped<FASTQ>(smax, bq, a.logit_b, a.logit_c);
+      const int32_t lmax = min(max(vmax, a.ks_lo), a.ks_hi);
 
-      // ---- pass 2: e = ShiftExp(L - max L) back into TMEM, row sum (four partial sums)
-      uint32_t s4[4] = {0u, 0u, 0u, 0u};
-      const int32_t* tb = tab + lane + lmax * 32;  // tb[-32 L] = ShiftExp(L - max L)
+      // ---- pass 2: e = ShiftExp(L - max L) back into TMEM, row sum
+      uint32_t sum = 0;
       if (work) {
-        IVIT_STREAM_CHUNKS({
-          const int lim = N - col;
-          if (lim >= 16) {
-#pragma unroll
-            for (int e = 0; e < 16; ++e) {
-              const int32_t l = logit_requant<FASTQ>((int32_t)r[e], bq, a.logit_b, a.logit_c, a.ks_lo, a.ks_hi);
-              const uint32_t x = (uint32_t)tb[-32 * l];
-              s4[e & 3] += x;
-              r[e] = x;
-            }
-          } else {
-#pragma unroll
-            for (int e = 0; e < 16; ++e) {
-              const int32_t l = logit_requant<FASTQ>((int32_t)r[e], bq, a.logit_b, a.logit_c, a.ks_lo, a.ks_hi);
-              const uint32_t x = (e < lim) ? (uint32_t)tb[-32 * l] : 0u;
-              s4[e & 3] += x;
-              r[e] = x;
-            }
-          }
-          tmem_st16(t_row + (uint32_t)col, r);
-        })
-        tmem_st_wait();
+        const int32_t* tb = tab + lane + lmax * 32;
+        if (__any_sync(0xffffffffu, vmax > a.ks_hi))
+          sum = shiftmax_pass2<FASTQ, true>(t_row, cbase, nvalid, N, tb, lmax, bq, a);
+        else
+          sum = shiftmax_pass2<FASTQ, false>(t_row, cbase, nvalid, N, tb, lmax, bq, a);
       }
-      uint32_t sum = (s4[0] + s4[1]) + (s4[2] + s4[3]);
       part[half * 256 + 128 + row] = (int32_t)sum;
       softmax_bar(group);
       sum = (uint32_t)part[128 + row] + (uint32_t)part[256 + 128 + row];
       if (sum == 0) sum = 1;  // rows that skipped the passes
       const uint32_t dv = (1u << a.M) / sum;
-      const int pshift = a.M - (a.k_out - 1);
 
-      // ---- pass 3: P = (Dv e) >> (M - k_out + 1) into the swizzled operand of stage s
+      // ---- pass 3: P = (Dv e) >> (M - k_out + 1) into the group's swizzled operand
+      // (the previous P of this group was consumed by a P V that completed
+      // before the o_full wait of the previous item)
       if (work) {
-        uint8_t* prow = smem + s * L.stage_bytes + (row >> 3) * 1024 + rlo * 128;
-        // (Dv e) >> pshift is one mul.hi by Dv 2^(32 - pshift) when that fits 32 bits
-        const bool hip = __all_sync(0xffffffffu, pshift <= 32 && (uint64_t)dv < ((uint64_t)1 << pshift));
+        // (Dv e) >> pshift is one mul.hi by Dv 2^(32 - pshift) when Dv < 2^pshift
+        const bool hip = pshift >= 1 && __all_sync(0xffffffffu, (uint64_t)dv < ((uint64_t)1 << pshift));
         const uint32_t dvh = hip ? dv << (32 - pshift) : 0u;
-        IVIT_STREAM_CHUNKS({
+        tmem_stream16(t_row + (uint32_t)cbase, nvalid, [&](uint32_t(&r)[16], int k) {
+          const int col = cbase + 16 * k;
           uint32_t w[4];
           if (hip) {
 #pragma unroll
@@ -610,19 +649,24 @@ __global__ void __launch_bounds__(kPersistThreads, 1)
           }
           *reinterpret_cast<int4*>(prow + (col >> 7) * 16384 + ((((col & 127) >> 4) ^ rlo) << 4)) =
               make_int4((int)w[0], (int)w[1], (int)w[2], (int)w[3]);
-        })
+        });
       }
-#undef IVIT_STREAM_CHUNKS
+      // chunks of padding keys (and every chunk of a skipped warp): P = 0
+      for (int k = work ? nvalid : 0; k < nch; ++k) {
+        const int col = cbase + 16 * k;
+        *reinterpret_cast<int4*>(prow + (col >> 7) * 16384 + ((((col & 127) >> 4) ^ rlo) << 4)) =
+            make_int4(0, 0, 0, 0);
+      }
       fence_proxy_async_smem();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&p_full[s]);
+      if (lane == 0) mbar_arrive(&p_full[group]);
 
       // ---- ctx = sat_8((b_o O) >> c_o); half h writes columns [32 h, 32 h + 32)
-      if (ok) ok = wait_or_abort(&o_full[s], ph, a.status, abort_flag);
+      if (ok) ok = wait_or_abort(&o_full[group], ph, a.status, abort_flag);
       ok = __all_sync(0xffffffffu, ok);
       tc_fence_after();
-      if (ok) {
+      if (ok && work) {
         uint32_t r[32];
         tmem_ld32(t_row + (uint32_t)(half * 32), r);
         tmem_ld_wait();
@@ -647,7 +691,7 @@ __global__ void __launch_bounds__(kPersistThreads, 1)
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&tmem_empty[s]);
+      if (lane == 0) mbar_arrive(&tmem_empty[group]);
     }
   }
 

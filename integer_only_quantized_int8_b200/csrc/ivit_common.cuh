@@ -77,6 +77,20 @@ IVIT_DEV bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
+// Non-blocking test of phase completion (never suspends the thread), for a
+// thread that polls several barriers in turn.
+IVIT_DEV bool mbar_test(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
 // As mbar_try_wait, but the thread may be suspended in hardware for up to
 // kSuspendHintNs while the phase is incomplete (it resumes as soon as the
 // phase completes), so a waiting warp does not spin on the issue slots.
