@@ -69,7 +69,7 @@ __host__ __device__ inline AttnLayout attn_layout(int N) {
 __global__ void __launch_bounds__(kAttnThreads)
     attention_shiftmax_kernel(const __grid_constant__ CUtensorMap tm, const AttnArgs a) {
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* smem = align_smem_1024(smem_raw);
   const int N = a.N;
   const AttnLayout L = attn_layout(N);
   uint8_t* r0 = smem;
@@ -423,7 +423,7 @@ template <bool FASTQ>
 __global__ void __launch_bounds__(kPersistThreads, 1)
     attention_persist_kernel(const __grid_constant__ CUtensorMap tm, const AttnArgs a, const int32_t bq) {
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* smem = align_smem_1024(smem_raw);
   const int N = a.N;
   const PersistLayout L = persist_layout(N);
   int32_t* tab = reinterpret_cast<int32_t*>(smem + L.tab_off);

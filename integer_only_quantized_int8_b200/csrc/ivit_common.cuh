@@ -43,6 +43,15 @@ IVIT_DEV uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
 
+// The first 1024-byte-aligned byte of a dynamic shared-memory array, found by
+// pointer arithmetic on the array itself: the compiler then still knows that
+// the result points into shared memory, so accesses through it stay 32-bit
+// ld/st.shared (a round trip through an integer makes them generic accesses
+// with 64-bit address arithmetic).
+IVIT_DEV uint8_t* align_smem_1024(uint8_t* raw) {
+  return raw + ((1024u - (smem_u32(raw) & 1023u)) & 1023u);
+}
+
 IVIT_DEV void mbar_init(uint64_t* bar, uint32_t count) {
   asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
 }
