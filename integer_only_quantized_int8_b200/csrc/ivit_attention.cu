@@ -37,6 +37,8 @@ struct AttnArgs {
   int32_t I0, M, k_out;
   int32_t out_b, out_c;
   int32_t o_lo, o_hi;  // accumulator clamp of the output requant (see out_clamp)
+  int32_t out_bq;      // b_o 2^(32 - c_o) when that fits a positive int32 (then the requant is one mul.hi), else 0
+  int32_t out_fast;
   int8_t* ctx;
   int* status;
 };
@@ -286,12 +288,12 @@ __global__ void __launch_bounds__(kAttnThreads)
 //   warp 0      TMA producer: Q, K and V of item j into stage j % 3 of a
 //               three-stage ring; a stage is released when P V of its item
 //               has completed, so loads run up to two items ahead;
-//   warp 1      MMA issuer: S = Q K^T of item j into TMEM buffer j & 1 once
-//               that buffer is free and the stage has landed, and P V of item
-//               j once its P is in shared memory.  It polls both conditions
-//               without blocking, so neither softmax group waits behind the
-//               other;
-//   warps 2-17  two softmax groups of eight warps.
+//   warp 1      S issuer: S = Q K^T of item j into TMEM buffer j & 1 once
+//               that buffer is free and the stage has landed;
+//   warp 2      P V issuer: P V of item j once its P is in shared memory.
+//               Two issuing threads, each blocked on its own next event, so
+//               neither softmax group waits behind the other;
+//   warps 3-18  two softmax groups of eight warps.
 // Within an item the score row never leaves TMEM: pass 1 takes the row
 // maximum of the raw int32 scores (the logit requant is monotone, so
 // max L = requant(max S)); pass 2 requantises each score, looks up
@@ -308,7 +310,7 @@ constexpr int kShortMaxKeys = 256;
 constexpr int kSoftWarps = 8;    // per softmax group
 constexpr int kSoftGroups = 2;   // groups take alternate items, one TMEM buffer each
 constexpr int kLoadStages = 3;
-constexpr int kPersistThreads = 64 + 32 * kSoftWarps * kSoftGroups;
+constexpr int kPersistThreads = 96 + 32 * kSoftWarps * kSoftGroups;
 
 struct PersistLayout {
   int n64, n32, kblocks;
@@ -434,7 +436,7 @@ __global__ void __launch_bounds__(kPersistThreads, 1)
   uint64_t* p_full = bars + 8;        // [2] P of group g in shared memory (one arrival per warp)
   uint64_t* o_full = bars + 10;       // [2] P V in TMEM buffer g
   uint64_t* tmem_empty = bars + 12;   // [2] TMEM buffer g reusable (one arrival per warp)
-  uint64_t* drain = bars + 14;        // all MMAs of the CTA complete
+  uint64_t* drain = bars + 14;        // all MMAs of the CTA complete (one commit per issuer)
   uint32_t* tslot = reinterpret_cast<uint32_t*>(bars + 15);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 16);
 
@@ -457,7 +459,7 @@ __global__ void __launch_bounds__(kPersistThreads, 1)
       mbar_init(&o_full[g], 1);
       mbar_init(&tmem_empty[g], kSoftWarps);
     }
-    mbar_init(drain, 1);
+    mbar_init(drain, 2);
     *abort_flag = 0;
     fence_barrier_init();
     prefetch_tensormap(&tm);
@@ -503,66 +505,49 @@ __global__ void __launch_bounds__(kPersistThreads, 1)
       }
     }
   } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
+    // ------------------------------------------------------------ S issuer
     if (lane == 0) {
       const uint32_t idesc_s = idesc_i8(kQTile, L.n32, true, true, false);
-      const uint32_t idesc_o = idesc_i8(kQTile, kHeadDim, false, true, true);
       const int n_local = n_items > (int)blockIdx.x ? (n_items - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
-      int js = 0, jp = 0;  // next S, next P V (in item order each)
-      uint64_t t_last = globaltimer_ns();
-      while (jp < n_local) {
-        bool progress = false;
-        if (js < n_local && js < jp + kSoftGroups) {
-          const int g = js & 1, s = js % kLoadStages;
-          if (mbar_test(&tmem_empty[g], (uint32_t)(((js >> 1) & 1) ^ 1)) &&
-              mbar_test(&qkv_full[s], (uint32_t)((js / kLoadStages) & 1))) {
-            tc_fence_after();
-            const uint32_t qa = smem_u32(smem + s * L.stage_bytes);
-            const uint32_t ka = qa + L.k_off;
+      for (int j = 0; j < n_local; ++j) {
+        const int g = j & 1, s = j % kLoadStages;
+        if (!wait_or_abort(&tmem_empty[g], (uint32_t)(((j >> 1) & 1) ^ 1), a.status, abort_flag)) break;
+        if (!wait_or_abort(&qkv_full[s], (uint32_t)((j / kLoadStages) & 1), a.status, abort_flag)) break;
+        tc_fence_after();
+        const uint32_t qa = smem_u32(smem + s * L.stage_bytes);
+        const uint32_t ka = qa + L.k_off;
 #pragma unroll
-            for (int k = 0; k < kHeadDim / 32; ++k)
-              umma_i8(tmem + (uint32_t)(g * 256), smem_desc(qa + k * 32, 16, 512, kSwizzle64B),
-                      smem_desc(ka + k * 32, 16, 512, kSwizzle64B), idesc_s, k != 0);
-            umma_commit(&s_full[g]);
-            ++js;
-            progress = true;
-          }
-        }
-        if (jp < js) {
-          const int g = jp & 1, s = jp % kLoadStages;
-          if (mbar_test(&p_full[g], (uint32_t)((jp >> 1) & 1))) {
-            tc_fence_after();
-            const uint32_t pa = smem_u32(smem + L.p_off + g * L.p_bytes);
-            const uint32_t va = smem_u32(smem + s * L.stage_bytes + L.v_off);
-            for (int k = 0; k < L.n32 / 32; ++k)
-              umma_i8(tmem + (uint32_t)(g * 256),
-                      smem_desc(pa + (k >> 2) * 16384 + (k & 3) * 32, 16, 1024, kSwizzle128B),
-                      smem_desc(va + k * 32 * kHeadDim, 512, 512, kSwizzle64B), idesc_o, k != 0);
-            umma_commit(&o_full[g]);
-            umma_commit(&stage_empty[s]);
-            ++jp;
-            progress = true;
-          }
-        }
-        if (progress) {
-          t_last = globaltimer_ns();
-        } else {
-          if (*abort_flag) break;
-          if (globaltimer_ns() - t_last > kWaitBudgetNs) {
-            report_timeout(a.status);
-            *abort_flag = 1;
-            break;
-          }
-          __nanosleep(32);
-        }
+        for (int k = 0; k < kHeadDim / 32; ++k)
+          umma_i8(tmem + (uint32_t)(g * 256), smem_desc(qa + k * 32, 16, 512, kSwizzle64B),
+                  smem_desc(ka + k * 32, 16, 512, kSwizzle64B), idesc_s, k != 0);
+        umma_commit(&s_full[g]);
       }
-      // every MMA of this CTA has completed before TMEM is released
+      // every MMA of this thread has completed before TMEM is released
       umma_commit(drain);
       mbar_wait(drain, 0, a.status);
     }
+  } else if (warp == 2) {
+    // ------------------------------------------------------------ P V issuer
+    if (lane == 0) {
+      const uint32_t idesc_o = idesc_i8(kQTile, kHeadDim, false, true, true);
+      const int n_local = n_items > (int)blockIdx.x ? (n_items - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
+      for (int j = 0; j < n_local; ++j) {
+        const int g = j & 1, s = j % kLoadStages;
+        if (!wait_or_abort(&p_full[g], (uint32_t)((j >> 1) & 1), a.status, abort_flag)) break;
+        tc_fence_after();
+        const uint32_t pa = smem_u32(smem + L.p_off + g * L.p_bytes);
+        const uint32_t va = smem_u32(smem + s * L.stage_bytes + L.v_off);
+        for (int k = 0; k < L.n32 / 32; ++k)
+          umma_i8(tmem + (uint32_t)(g * 256), smem_desc(pa + (k >> 2) * 16384 + (k & 3) * 32, 16, 1024, kSwizzle128B),
+                  smem_desc(va + k * 32 * kHeadDim, 512, 512, kSwizzle64B), idesc_o, k != 0);
+        umma_commit(&o_full[g]);
+        umma_commit(&stage_empty[s]);
+      }
+      umma_commit(drain);
+    }
   } else {
     // ------------------------------------------------------------ softmax warps
-    const int sw = warp - 2;
+    const int sw = warp - 3;
     const int group = sw / kSoftWarps;   // handles local items j with j % 2 == group
     const int quarter = warp & 3;
     const int half = (sw >> 2) & 1;
@@ -679,9 +664,13 @@ __global__ void __launch_bounds__(kPersistThreads, 1)
             int32_t y[4];
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
-              const int32_t acc = min(max((int32_t)r[wd * 4 + e], a.o_lo), a.o_hi);
-              const int64_t v = (int64_t)a.out_b * acc;  // |v >> c| < 2^31 after the clamp
-              y[e] = (int32_t)__funnelshift_r((uint32_t)v, (uint32_t)(v >> 32), (uint32_t)a.out_c);
+              if (a.out_fast) {
+                y[e] = __mulhi(a.out_bq, (int32_t)r[wd * 4 + e]);  // floor(b_o acc / 2^c_o), exact
+              } else {
+                const int32_t acc = min(max((int32_t)r[wd * 4 + e], a.o_lo), a.o_hi);
+                const int64_t v = (int64_t)a.out_b * acc;  // |v >> c| < 2^31 after the clamp
+                y[e] = (int32_t)__funnelshift_r((uint32_t)v, (uint32_t)(v >> 32), (uint32_t)a.out_c);
+              }
             }
             packed[wd] = pack_sat4_attn(y[0], y[1], y[2], y[3]);
           }
@@ -747,6 +736,8 @@ ivit_status launch_attention(const DeviceCtx& dc, const int8_t* qkv, int32_t B, 
       a.o_lo = -a.o_hi;
     }
   }
+  a.out_fast = out.c >= 1 && (int64_t)out.b < ((int64_t)1 << (out.c - 1));
+  a.out_bq = a.out_fast ? (int32_t)((int64_t)out.b << (32 - out.c)) : 0;
   a.ctx = ctx;
   a.status = dc.status;
   dim3 grid((unsigned)((N + kQTile - 1) / kQTile), (unsigned)H, (unsigned)B);

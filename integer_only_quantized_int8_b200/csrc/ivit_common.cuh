@@ -131,7 +131,7 @@ IVIT_DEV bool mbar_wait(uint64_t* bar, uint32_t parity, int* status) {
 }
 
 // ---------------------------------------------------------------------------
-// TMA (cp.async.bulk.tensor), no multicast
+// TMA (cp.async.bulk.tensor): every copy fills or drains this CTA's own shared memory
 // ---------------------------------------------------------------------------
 IVIT_DEV void tma_load_2d(void* smem_dst, const CUtensorMap* map, int32_t x, int32_t y, uint64_t* bar) {
   asm volatile(
@@ -140,6 +140,19 @@ IVIT_DEV void tma_load_2d(void* smem_dst, const CUtensorMap* map, int32_t x, int
       "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_u32(bar))
       : "memory");
 }
+
+// shared -> global tile store, tracked in the issuing thread's bulk groups
+IVIT_DEV void tma_store_2d(const CUtensorMap* map, int32_t x, int32_t y, const void* smem_src) {
+  asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%1, %2}], [%3];" ::"l"(
+                   reinterpret_cast<uint64_t>(map)),
+               "r"(x), "r"(y), "r"(smem_u32(smem_src))
+               : "memory");
+}
+IVIT_DEV void bulk_commit_group() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// every committed store of this thread has finished reading shared memory
+IVIT_DEV void bulk_wait_read_all() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+// every committed store of this thread has completed
+IVIT_DEV void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 
 IVIT_DEV void prefetch_tensormap(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");

@@ -9,11 +9,15 @@
 // The accumulator is computed transposed, D = W X^T: the UMMA M dimension
 // (TMEM lanes) runs over 128 output channels and N over BN tokens.  Every
 // epilogue thread therefore owns one output channel of the tile and keeps that
-// channel's multiplier, shift, bias and saturation bounds in registers.  When
-// b_j < 2^(c_j - 1) (a requant scale below one half, the usual case) the
-// requant floor(b (acc + bias) / 2^c) is one mul.hi by b 2^(32 - c); the
-// saturating byte pack then clips.  A 4 x 4 byte transpose across lanes turns
-// the channel-major bytes into token-major 4-byte words for coalesced stores.
+// channel's multiplier and shift in registers.  The bias is not added per
+// element: each accumulator buffer is preloaded with its next tile's bias
+// (tcgen05.st) before the MMAs accumulate onto it.  When b_j < 2^(c_j - 1) (a
+// requant scale below one half, the usual case) the requant
+// floor(b acc / 2^c) is then one mul.hi by b 2^(32 - c); the saturating byte
+// pack clips.  A 4 x 4 byte transpose across lanes turns channel-major bytes
+// into token-major 4-byte words, which go to a shared-memory staging slot per
+// 16-token chunk and leave by TMA store (the residual's skip tile arrives the
+// same way).
 //
 // Roles (one CTA per SM, persistent over 128 x BN tiles):
 //   warp 0      TMA producer: W and X k-slices of 128 bytes, 128B swizzle,
@@ -37,6 +41,7 @@ constexpr int kBK = 128;  // bytes = int8 elements per k-slice (one 128-byte swi
 constexpr int kEpiWarps = 12;  // three per TMEM lane quarter
 constexpr int kEpiParts = kEpiWarps / 4;
 constexpr int kGemmThreads = 64 + 32 * kEpiWarps;
+constexpr int kSlotBytes = 16 * 32;  // one staged chunk: 16 tokens x 32 channels
 
 struct GemmArgs {
   int64_t M;       // tokens (rows of X and Y)
@@ -45,9 +50,7 @@ struct GemmArgs {
   const int32_t* b;
   const int8_t* c;
   int32_t lo, hi;  // saturation range of the requantised output
-  const int8_t* skip;
   ivit_residual res;
-  int8_t* Y;
   GeluParams gelu;
   int* status;
 };
@@ -57,8 +60,13 @@ struct GemmLayout {
   static constexpr int kABytes = kBM * kBK;
   static constexpr int kBBytes = BN * kBK;
   static constexpr int kStageBytes = kABytes + kBBytes;
-  static constexpr int kBarOff = STAGES * kStageBytes;
-  static constexpr int kNumBars = 2 * STAGES + 5;  // full, empty, tmem full x2, tmem empty x2, drain
+  static constexpr int kChunks = BN / 16;
+  static constexpr int kMaxPart = (kChunks + kEpiParts - 1) / kEpiParts;  // chunks of the largest part
+  static constexpr int kOutOff = STAGES * kStageBytes;
+  static constexpr int kWarpSlots = kMaxPart * kSlotBytes;
+  static constexpr int kBarOff = kOutOff + kEpiWarps * kWarpSlots;
+  // full, empty (STAGES each), tmem full x2, tmem empty x2, drain, one skip barrier per epilogue warp
+  static constexpr int kNumBars = 2 * STAGES + 5 + kEpiWarps;
   static constexpr int kSlotOff = kBarOff + kNumBars * 8;
   static constexpr int kGeluOff = kSlotOff + 16;
   static constexpr int kBytes = kGeluOff + 256;
@@ -70,27 +78,24 @@ IVIT_DEV int32_t sat_i32(int64_t v) {
   return (int32_t)(v < (int64_t)INT_MIN ? (int64_t)INT_MIN : (v > (int64_t)INT_MAX ? (int64_t)INT_MAX : v));
 }
 
-// Per-channel constants of the requant sat((b (acc + bias)) >> c), b >= 0.
-// With v = acc + bias the result floor(b v / 2^c) is monotone in v.  With
+// Per-channel constants of the requant sat((b acc) >> c), b >= 0, where acc
+// already holds the bias.  floor(b acc / 2^c) is monotone in acc.  With
 // bl = bit length of b, s = bl - 1 - c (so 2^s <= b / 2^c < 2^(s+1)) and
-// u = 128 / 2^s (u = 1 once s >= 7), v = u gives a result >= 128 and v = -u
-// one <= -128, while every v in [-u, u] gives a result of magnitude at most
-// max(256, b / 2^c) < 2^31.  Clamping acc to [-u - bias, u - bias] therefore
-// changes no result inside the int8 range (nor any narrower range), sends
-// everything beyond to a value that saturates the same way, and keeps the
-// shifted result within int32: the saturating byte pack then finishes the
-// job.  When even the largest possible |acc + bias| (2^14 K + |bias|) keeps
-// |b (acc + bias)| below 2^(30 + c), the shifted result always fits int32 and
-// the clamp is skipped.
+// u = 128 / 2^s (u = 1 once s >= 7), acc = u gives a result >= 128 and
+// acc = -u one <= -128, while every acc in [-u, u] gives a result of magnitude
+// at most max(256, b / 2^c) < 2^31.  Clamping acc to [-u, u] therefore changes
+// no result inside the int8 range (nor any narrower range), sends everything
+// beyond to a value that saturates the same way, and keeps the shifted result
+// within int32: the saturating byte pack then finishes the job.  When even
+// the largest possible |acc| (2^14 K + |bias|) keeps |b acc| below 2^(30 + c),
+// the shifted result always fits int32 and the clamp is skipped.
 //
 // Fast form: when b < 2^(c - 1), bq = b 2^(32 - c) is a positive int32 and
-// floor(b v / 2^c) = floor(bq v / 2^32) = mul.hi(bq, v) exactly, for every
-// int32 v; acc + bias stays within int32 because |acc| <= 2^14 K <= 2^28 and
-// |bias| <= 2^30.  b = 0 takes the fast form with bq = 0.
+// floor(b acc / 2^c) = floor(bq acc / 2^32) = mul.hi(bq, acc) exactly, for
+// every int32 acc; acc stays within int32 because |acc| <= 2^14 K + |bias| <=
+// 2^28 + 2^30.  b = 0 takes the fast form with bq = 0.
 struct ChanConst {
-  int32_t b, c, lo_acc, hi_acc;
-  int32_t bias, bq;
-  int64_t bb;       // b * bias
+  int32_t b, c, lim, bq;
   bool fast, needs_clamp;
 };
 
@@ -98,22 +103,17 @@ IVIT_DEV ChanConst chan_const(int32_t b, int32_t c, int32_t bias, int32_t K) {
   ChanConst k;
   k.b = b;
   k.c = c;
-  k.bias = bias;
-  k.bb = (int64_t)b * bias;
   k.fast = b == 0 || (c >= 1 && (int64_t)b < ((int64_t)1 << (c - 1)));
   k.bq = (k.fast && b != 0) ? (int32_t)((uint32_t)b << (32 - c)) : 0;
   if (b == 0) {
-    k.lo_acc = INT_MIN;
-    k.hi_acc = INT_MAX;
+    k.lim = INT_MAX;
     k.needs_clamp = false;
     return k;
   }
   const int bl = 32 - __clz(b);
-  const int s = bl - 1 - c;                                   // 2^s <= b / 2^c < 2^(s+1)
+  const int s = bl - 1 - c;  // 2^s <= b / 2^c < 2^(s+1)
   const int64_t u = s >= 7 ? 1 : (s >= 0 ? (128 >> s) : ((int64_t)128 << (-s)));
-  const int64_t hi = u - bias, lo = -u - bias;
-  k.hi_acc = sat_i32(hi);
-  k.lo_acc = sat_i32(lo);
+  k.lim = sat_i32(u);
   const int64_t vmax = (int64_t)K * 16384 + (bias < 0 ? -(int64_t)bias : (int64_t)bias);
   k.needs_clamp = vmax * (int64_t)b >= ((int64_t)1 << (30 + c));
   return k;
@@ -123,13 +123,13 @@ IVIT_DEV ChanConst chan_const(int32_t b, int32_t c, int32_t bias, int32_t K) {
 // the 64-bit product with or without the accumulator clamp.
 enum ReqForm : int { kReqFast = 0, kReqWide = 1, kReqWideClamp = 2 };
 
-// floor(b (acc + bias) / 2^c); in the wide forms the result fits int32 (see
-// above), so the low word of the 64-bit shift is one funnel shift (c <= 31)
+// floor(b acc / 2^c); in the wide forms the result fits int32 (see above), so
+// the low word of the 64-bit shift is one funnel shift (c <= 31)
 template <int REQ>
 IVIT_DEV int32_t requant_acc(int32_t acc, const ChanConst& k) {
-  if (REQ == kReqFast) return __mulhi(k.bq, acc + k.bias);
-  const int32_t a = REQ == kReqWideClamp ? min(max(acc, k.lo_acc), k.hi_acc) : acc;
-  const int64_t v = (int64_t)k.b * a + k.bb;
+  if (REQ == kReqFast) return __mulhi(k.bq, acc);
+  const int32_t a = REQ == kReqWideClamp ? min(max(acc, -k.lim), k.lim) : acc;
+  const int64_t v = (int64_t)k.b * a;
   return (int32_t)__funnelshift_r((uint32_t)v, (uint32_t)(v >> 32), (uint32_t)k.c);
 }
 
@@ -189,13 +189,14 @@ IVIT_DEV uint32_t residual_word(uint32_t s, uint32_t y, const ivit_residual& res
 }
 
 // One 16-token chunk of one epilogue warp: requant the 16 accumulators of this
-// thread's channel, pack, transpose to token-major words, apply the residual
-// if any, and store.  r holds TMEM columns [16 cc, 16 cc + 16) of lane ch.
+// thread's channel (r = TMEM columns of the chunk), pack, transpose to
+// token-major words, apply the residual (its skip words were staged in the
+// same slot) and leave the result in the slot.  slot_w points at the lane's
+// word of the slot: word k (token 4k + sub, channels 4 grp .. 4 grp + 3) sits
+// at byte (4k + sub) * 32 + 4 grp, i.e. slot_w[32 k].
 template <int EPI, bool NARROW, int REQ>
 IVIT_DEV void epi_chunk(const uint32_t (&r)[16], const ChanConst& kc, const GemmArgs& args, const int8_t* gelu_tab,
-                        int64_t tok0, int ch4, int sub, uint32_t sel2, uint32_t sel1) {
-  const int64_t M = args.M;
-  const int N = args.N;
+                        uint32_t* slot_w, uint32_t sel2, uint32_t sel1) {
   uint32_t w[4];
 #pragma unroll
   for (int k = 0; k < 4; ++k) {
@@ -213,19 +214,10 @@ IVIT_DEV void epi_chunk(const uint32_t (&r)[16], const ChanConst& kc, const Gemm
     }
     w[k] = transpose4x4(pack_sat4(y[0], y[1], y[2], y[3]), sel2, sel1);
   }
-  // lane (4 grp + sub) now holds, for k = 0..3, token tok0 + 4k + sub, channels ch4..ch4+3
-  if (ch4 >= N) return;
-  // word k goes to token tok0 + 4k + sub: a fixed stride of 4N bytes
-  const int64_t off0 = (tok0 + sub) * N + ch4;
-  const int64_t stride = 4 * (int64_t)N;
-  const bool full = tok0 + 16 <= M;
   if (EPI == kEpiResidual) {
-    // all four skip words are requested before any store, so their latencies overlap
     uint32_t s[4];
-    const int8_t* sp = args.skip + off0;
 #pragma unroll
-    for (int k = 0; k < 4; ++k)
-      s[k] = (full || tok0 + 4 * k + sub < M) ? __ldg(reinterpret_cast<const uint32_t*>(sp + k * stride)) : 0u;
+    for (int k = 0; k < 4; ++k) s[k] = slot_w[32 * k];
     if (args.res.c >= 9) {
 #pragma unroll
       for (int k = 0; k < 4; ++k) w[k] = residual_word<true>(s[k], w[k], args.res);
@@ -234,45 +226,35 @@ IVIT_DEV void epi_chunk(const uint32_t (&r)[16], const ChanConst& kc, const Gemm
       for (int k = 0; k < 4; ++k) w[k] = residual_word<false>(s[k], w[k], args.res);
     }
   }
-  int8_t* yp = args.Y + off0;
-  if (full) {
 #pragma unroll
-    for (int k = 0; k < 4; ++k) *reinterpret_cast<uint32_t*>(yp + k * stride) = w[k];
-  } else {
-#pragma unroll
-    for (int k = 0; k < 4; ++k)
-      if (tok0 + 4 * k + sub < M) *reinterpret_cast<uint32_t*>(yp + k * stride) = w[k];
+  for (int k = 0; k < 4; ++k) slot_w[32 * k] = w[k];
+}
+
+// The chunks [c_begin, c_begin + n) of one tile into the warp's slots.
+template <int EPI, bool NARROW, int REQ>
+IVIT_DEV void epi_tile(uint32_t tbase, int c_begin, int n, const ChanConst& kc, const GemmArgs& args,
+                       const int8_t* gelu_tab, uint32_t* slot_w, uint32_t sel2, uint32_t sel1) {
+  for (int i = 0; i < n; ++i) {
+    uint32_t r[16];
+    tmem_ld16(tbase + (uint32_t)(16 * (c_begin + i)), r);
+    tmem_ld_wait();
+    epi_chunk<EPI, NARROW, REQ>(r, kc, args, gelu_tab, slot_w + i * (kSlotBytes / 4), sel2, sel1);
   }
 }
 
-// The 16-token chunks [c_begin, c_end) of one tile, with the next chunk's TMEM
-// load in flight while the current chunk is processed.
-template <int EPI, bool NARROW, int REQ>
-IVIT_DEV void epi_tile(uint32_t tbase, int c_begin, int c_end, int64_t tok_base, const ChanConst& kc,
-                       const GemmArgs& args, const int8_t* gelu_tab, int ch4, int sub, uint32_t sel2,
-                       uint32_t sel1) {
-  const int64_t M = args.M;
-  int n = c_end - c_begin;  // chunks that hold at least one valid token
-  while (n > 0 && tok_base + 16 * (c_begin + n - 1) >= M) --n;
-  if (n <= 0) return;
-  uint32_t ra[16], rb[16];
-  tmem_ld16(tbase + (uint32_t)(16 * c_begin), ra);
-  for (int i = 0; i < n; i += 2) {
-    const int ca = c_begin + i;
-    tmem_ld_wait();
-    if (i + 1 < n) tmem_ld16(tbase + (uint32_t)(16 * (ca + 1)), rb);
-    epi_chunk<EPI, NARROW, REQ>(ra, kc, args, gelu_tab, tok_base + 16 * ca, ch4, sub, sel2, sel1);
-    if (i + 1 < n) {
-      tmem_ld_wait();
-      if (i + 2 < n) tmem_ld16(tbase + (uint32_t)(16 * (ca + 2)), ra);
-      epi_chunk<EPI, NARROW, REQ>(rb, kc, args, gelu_tab, tok_base + 16 * (ca + 1), ch4, sub, sel2, sel1);
-    }
-  }
+// Preload TMEM columns [16 c_begin, 16 c_end) of this warp's lanes in one
+// accumulator buffer with the bias of the lane's output channel.
+IVIT_DEV void bias_fill(uint32_t tbase, int c_begin, int c_end, int32_t bias) {
+  uint32_t v[16];
+#pragma unroll
+  for (int i = 0; i < 16; ++i) v[i] = (uint32_t)bias;
+  for (int cc = c_begin; cc < c_end; ++cc) tmem_st16(tbase + (uint32_t)(16 * cc), v);
 }
 
 template <int BN, int STAGES, int EPI, bool NARROW>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     gemm_i8_requant_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX,
+                           const __grid_constant__ CUtensorMap tmY, const __grid_constant__ CUtensorMap tmS,
                            const GemmArgs args) {
   using L = GemmLayout<BN, STAGES>;
   extern __shared__ uint8_t smem_raw[];
@@ -282,6 +264,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   uint64_t* tfull = empty + STAGES;
   uint64_t* tempty = tfull + 2;
   uint64_t* drain = tempty + 2;
+  uint64_t* skip_full = drain + 1;  // [kEpiWarps]
   uint32_t* tslot = reinterpret_cast<uint32_t*>(smem + L::kSlotOff);
   int8_t* gelu_tab = reinterpret_cast<int8_t*>(smem + L::kGeluOff);
 
@@ -304,9 +287,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       mbar_init(&tempty[a], kEpiWarps);
     }
     mbar_init(drain, 1);
+    for (int e = 0; e < kEpiWarps; ++e) mbar_init(&skip_full[e], 1);
     fence_barrier_init();
     prefetch_tensormap(&tmW);
     prefetch_tensormap(&tmX);
+    prefetch_tensormap(&tmY);
+    if (EPI == kEpiResidual) prefetch_tensormap(&tmS);
   }
   if (EPI == kEpiGelu) {
     for (int i = threadIdx.x; i < 256; i += blockDim.x)
@@ -329,7 +315,6 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       int stage = 0;
       uint32_t phase = 0;
       bool ok = true;
-      int issued = 0;
       for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
         const int cb = t % ch_tiles, tb = t / ch_tiles;
         for (int kb = 0; kb < num_kb; ++kb) {
@@ -341,19 +326,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           uint8_t* sa = smem + stage * L::kStageBytes;
           tma_load_2d(sa, &tmW, kb * kBK, cb * kBM, &full[stage]);
           tma_load_2d(sa + L::kABytes, &tmX, kb * kBK, tb * BN, &full[stage]);
-          ++issued;
           if (++stage == STAGES) {
             stage = 0;
             phase ^= 1;
           }
-        }
-      }
-      if (!ok) {
-        // let the copies already in flight land before the CTA exits
-        for (int i = 0; i < STAGES && i < issued; ++i) {
-          stage = (stage + STAGES - 1) % STAGES;
-          if (stage == STAGES - 1) phase ^= 1;
-          mbar_wait(&full[stage], phase, args.status);
         }
       }
     }
@@ -367,7 +343,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       uint32_t acc_phase = 0;
       bool ok = true;
       for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
-        if (!mbar_wait(&tempty[acc], acc_phase ^ 1, args.status)) break;
+        // the buffer holds this tile's bias once the epilogue has drained it
+        if (!mbar_wait(&tempty[acc], acc_phase, args.status)) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BN);
         for (int kb = 0; kb < num_kb; ++kb) {
@@ -382,7 +359,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           for (int k = 0; k < kBK / 32; ++k) {
             const uint64_t da = smem_desc(sa + k * 32, 16, 1024, kSwizzle128B);
             const uint64_t db = smem_desc(sb + k * 32, 16, 1024, kSwizzle128B);
-            umma_i8(d_tmem, da, db, idesc, (kb | k) != 0 ? 1u : 0u);
+            umma_i8(d_tmem, da, db, idesc, 1u);  // accumulate onto the preloaded bias
           }
           umma_commit(&empty[stage]);
           if (++stage == STAGES) {
@@ -401,7 +378,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     }
   } else {
     // ------------------------------------------------------------ epilogue
-    constexpr int kChunks = BN / 16;
+    constexpr int kChunks = L::kChunks;
     const int e = warp - 2;
     const int quarter = warp & 3;  // TMEM lanes [32 q, 32 q + 32) = channels of this warp
     const int part = e >> 2;       // which of the quarter's warps: splits the token chunks
@@ -411,65 +388,82 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     const uint32_t sel1 = (lane & 1) ? 0x3715u : 0x6240u;
     const int sub = lane & 3;   // token offset within a transposed 4 x 4 block
     const int grp = lane >> 2;  // channel group of 4 within the warp's 32 channels
+    uint8_t* slots = smem + L::kOutOff + e * L::kWarpSlots;
+    uint32_t* slot_w = reinterpret_cast<uint32_t*>(slots) + sub * 8 + grp;
+    uint64_t* sbar = &skip_full[e];
+    const uint32_t tlane = tmem_base + ((uint32_t)(quarter * 32) << 16);
+    auto bias_of = [&](int t) -> int32_t {
+      const int ch = (t % ch_tiles) * kBM + quarter * 32 + lane;
+      return (args.bias && ch < N) ? __ldg(args.bias + ch) : 0;
+    };
+    // both accumulator buffers start out holding the bias of their first tile
+    for (int a = 0; a < 2; ++a) {
+      const int t = (int)blockIdx.x + a * (int)gridDim.x;
+      if (t < num_tiles) bias_fill(tlane + (uint32_t)(a * BN), c_begin, c_end, bias_of(t));
+      tmem_st_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&tempty[a]);
+    }
     int acc = 0;
     uint32_t acc_phase = 0;
+    uint32_t skip_phase = 0;
     for (int t = blockIdx.x; t < num_tiles; t += gridDim.x) {
       const int cb = t % ch_tiles, tb = t / ch_tiles;
-      const int ch = cb * kBM + quarter * 32 + lane;      // this thread's output channel
-      const int ch4 = cb * kBM + quarter * 32 + grp * 4;  // first channel of the stored word
-      ChanConst kc;
-      if (ch < N)
-        kc = chan_const(__ldg(args.b + ch), (int32_t)__ldg(args.c + ch), args.bias ? __ldg(args.bias + ch) : 0,
-                        args.K);
-      else
-        kc = chan_const(0, 0, 0, args.K);
+      const int ch0 = cb * kBM + quarter * 32;  // first channel of this warp
+      const int ch = ch0 + lane;                // this thread's output channel
+      const ChanConst kc = ch < N ? chan_const(__ldg(args.b + ch), (int32_t)__ldg(args.c + ch),
+                                               args.bias ? __ldg(args.bias + ch) : 0, args.K)
+                                  : chan_const(0, 0, 0, args.K);
       // warp-uniform requant form
       const int req = __all_sync(0xffffffffu, kc.fast) ? kReqFast
                       : (__any_sync(0xffffffffu, kc.needs_clamp) ? kReqWideClamp : kReqWide);
-      if (EPI == kEpiResidual) {
-        // pull this warp's skip rows of the next tile into L2 while the MMAs of
-        // this one run (one 32-byte sector per token row)
-        const int tn = t + (int)gridDim.x;
-        if (tn < num_tiles) {
-          const int64_t tok_n = (int64_t)(tn / ch_tiles) * BN + 16 * c_begin + lane;
-          const int ch_n = (tn % ch_tiles) * kBM + quarter * 32;
-          if (ch_n < N)
-            for (int tk = 0; tk < 16 * (c_end - c_begin); tk += 32) {
-              const int64_t tok = tok_n + tk;
-              if (lane + tk < 16 * (c_end - c_begin) && tok < M)
-                asm volatile("prefetch.global.L2 [%0];" ::"l"(args.skip + tok * N + ch_n));
-            }
-        }
-        if (t == (int)blockIdx.x) {  // the first tile prefetches its own rows
-          const int64_t tok_c = (int64_t)tb * BN + 16 * c_begin + lane;
-          const int ch_c = cb * kBM + quarter * 32;
-          if (ch_c < N)
-            for (int tk = 0; tk < 16 * (c_end - c_begin); tk += 32) {
-              const int64_t tok = tok_c + tk;
-              if (lane + tk < 16 * (c_end - c_begin) && tok < M)
-                asm volatile("prefetch.global.L2 [%0];" ::"l"(args.skip + tok * N + ch_c));
-            }
-        }
+      const int64_t tok_base = (int64_t)tb * BN;
+      int n = c_end - c_begin;  // chunks that hold at least one real token
+      while (n > 0 && tok_base + 16 * (c_begin + n - 1) >= M) --n;
+      const bool live = n > 0 && ch0 < N;
+      // the slots are free again once the stores of the previous tile have read them
+      if (lane == 0) bulk_wait_read_all();
+      __syncwarp();
+      if (EPI == kEpiResidual && live && lane == 0) {
+        mbar_arrive_expect_tx(sbar, (uint32_t)(n * kSlotBytes));
+        for (int i = 0; i < n; ++i)
+          tma_load_2d(slots + i * kSlotBytes, &tmS, ch0, (int32_t)(tok_base + 16 * (c_begin + i)), sbar);
       }
-      const bool got = mbar_wait(&tfull[acc], acc_phase, args.status);
+      bool got = mbar_wait(&tfull[acc], acc_phase, args.status);
+      if (EPI == kEpiResidual && live) {
+        got = mbar_wait(sbar, skip_phase, args.status) && got;
+        skip_phase ^= 1;
+      }
       if (!__all_sync(0xffffffffu, got)) break;  // warp-uniform give-up
       tc_fence_after();
-      const uint32_t tbase = tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(acc * BN);
-      __syncwarp();
-      const int64_t tok_base = (int64_t)tb * BN;
+      const uint32_t tbase = tlane + (uint32_t)(acc * BN);
       if (req == kReqFast)
-        epi_tile<EPI, NARROW, kReqFast>(tbase, c_begin, c_end, tok_base, kc, args, gelu_tab, ch4, sub, sel2, sel1);
+        epi_tile<EPI, NARROW, kReqFast>(tbase, c_begin, n, kc, args, gelu_tab, slot_w, sel2, sel1);
       else if (req == kReqWide)
-        epi_tile<EPI, NARROW, kReqWide>(tbase, c_begin, c_end, tok_base, kc, args, gelu_tab, ch4, sub, sel2, sel1);
+        epi_tile<EPI, NARROW, kReqWide>(tbase, c_begin, n, kc, args, gelu_tab, slot_w, sel2, sel1);
       else
-        epi_tile<EPI, NARROW, kReqWideClamp>(tbase, c_begin, c_end, tok_base, kc, args, gelu_tab, ch4, sub, sel2,
-                                             sel1);
+        epi_tile<EPI, NARROW, kReqWideClamp>(tbase, c_begin, n, kc, args, gelu_tab, slot_w, sel2, sel1);
+      // staged words -> global by TMA (rows past M and channels past N are clipped)
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (live && lane == 0) {
+        for (int i = 0; i < n; ++i)
+          tma_store_2d(&tmY, ch0, (int32_t)(tok_base + 16 * (c_begin + i)), slots + i * kSlotBytes);
+        bulk_commit_group();
+      }
+      // preload the bias of the tile that next accumulates in this buffer
+      const int t2 = t + 2 * (int)gridDim.x;
+      if (t2 < num_tiles) bias_fill(tbase, c_begin, c_end, bias_of(t2));
+      tmem_st_wait();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&tempty[acc]);
       acc ^= 1;
       if (acc == 0) acc_phase ^= 1;
     }
+    if (lane == 0) bulk_wait_all();
+    __syncwarp();
   }
 
   tc_fence_before();
@@ -482,17 +476,26 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 }
 
 template <int BN, int STAGES, int EPI, bool NARROW>
-ivit_status run_gemm(const DeviceCtx& dc, const int8_t* X, const int8_t* W, const GemmArgs& a,
-                     cudaStream_t stream) {
+ivit_status run_gemm(const DeviceCtx& dc, const int8_t* X, const int8_t* W, const int8_t* skip, int8_t* Y,
+                     const GemmArgs& a, cudaStream_t stream) {
   using L = GemmLayout<BN, STAGES>;
   static_assert(L::kAlloc <= 227 * 1024, "shared memory budget");
-  CUtensorMap tmW, tmX;
+  CUtensorMap tmW, tmX, tmY, tmS;
   ivit_status st = encode_tmap_2d_u8(&tmW, W, (uint64_t)a.K, (uint64_t)a.N, (uint64_t)a.K, kBK, kBM,
                                      CU_TENSOR_MAP_SWIZZLE_128B);
   if (st != IVIT_OK) return st;
   st = encode_tmap_2d_u8(&tmX, X, (uint64_t)a.K, (uint64_t)a.M, (uint64_t)a.K, kBK, BN,
                          CU_TENSOR_MAP_SWIZZLE_128B);
   if (st != IVIT_OK) return st;
+  st = encode_tmap_2d_u8(&tmY, Y, (uint64_t)a.N, (uint64_t)a.M, (uint64_t)a.N, 32, 16, CU_TENSOR_MAP_SWIZZLE_NONE);
+  if (st != IVIT_OK) return st;
+  if (EPI == kEpiResidual) {
+    st = encode_tmap_2d_u8(&tmS, skip, (uint64_t)a.N, (uint64_t)a.M, (uint64_t)a.N, 32, 16,
+                           CU_TENSOR_MAP_SWIZZLE_NONE);
+    if (st != IVIT_OK) return st;
+  } else {
+    tmS = tmY;  // unused
+  }
   auto kern = gemm_i8_requant_kernel<BN, STAGES, EPI, NARROW>;
   static bool attr_done = false;  // benign race: the attribute value is the same
   if (!attr_done) {
@@ -502,7 +505,7 @@ ivit_status run_gemm(const DeviceCtx& dc, const int8_t* X, const int8_t* W, cons
   }
   const int tiles = ((a.N + kBM - 1) / kBM) * (int)((a.M + BN - 1) / BN);
   const int grid = tiles < dc.num_sms ? tiles : dc.num_sms;
-  kern<<<grid, kGemmThreads, L::kAlloc, stream>>>(tmW, tmX, a);
+  kern<<<grid, kGemmThreads, L::kAlloc, stream>>>(tmW, tmX, tmY, tmS, a);
   note_launch();
   return cudaGetLastError() == cudaSuccess ? IVIT_OK : IVIT_ERR_CUDA;
 }
@@ -528,19 +531,19 @@ int pick_bn(int64_t M, int N, int num_sms) {
 }
 
 template <int EPI, bool NARROW>
-ivit_status dispatch_bn(const DeviceCtx& dc, const int8_t* X, const int8_t* W, const GemmArgs& a,
-                        cudaStream_t stream) {
+ivit_status dispatch_bn(const DeviceCtx& dc, const int8_t* X, const int8_t* W, const int8_t* skip, int8_t* Y,
+                        const GemmArgs& a, cudaStream_t stream) {
   switch (pick_bn(a.M, a.N, dc.num_sms)) {
     case 256:
-      return run_gemm<256, 4, EPI, NARROW>(dc, X, W, a, stream);
+      return run_gemm<256, 3, EPI, NARROW>(dc, X, W, skip, Y, a, stream);
     case 224:
-      return run_gemm<224, 5, EPI, NARROW>(dc, X, W, a, stream);
+      return run_gemm<224, 4, EPI, NARROW>(dc, X, W, skip, Y, a, stream);
     case 192:
-      return run_gemm<192, 5, EPI, NARROW>(dc, X, W, a, stream);
+      return run_gemm<192, 5, EPI, NARROW>(dc, X, W, skip, Y, a, stream);
     case 160:
-      return run_gemm<160, 6, EPI, NARROW>(dc, X, W, a, stream);
+      return run_gemm<160, 5, EPI, NARROW>(dc, X, W, skip, Y, a, stream);
     default:
-      return run_gemm<128, 7, EPI, NARROW>(dc, X, W, a, stream);
+      return run_gemm<128, 6, EPI, NARROW>(dc, X, W, skip, Y, a, stream);
   }
 }
 
@@ -559,21 +562,19 @@ ivit_status launch_gemm(const DeviceCtx& dc, const int8_t* X, int64_t M, int32_t
   a.c = c;
   a.lo = -(1 << (out_bits - 1));
   a.hi = (1 << (out_bits - 1)) - 1;
-  a.skip = skip;
   a.res = res;
-  a.Y = Y;
   a.gelu = gelu ? *gelu : GeluParams{1, 30, 8, {0, 0}};
   a.status = dc.status;
   const bool narrow = out_bits < 8;
   switch (mode) {
     case kEpiPlain:
-      return narrow ? dispatch_bn<kEpiPlain, true>(dc, X, W, a, stream)
-                    : dispatch_bn<kEpiPlain, false>(dc, X, W, a, stream);
+      return narrow ? dispatch_bn<kEpiPlain, true>(dc, X, W, skip, Y, a, stream)
+                    : dispatch_bn<kEpiPlain, false>(dc, X, W, skip, Y, a, stream);
     case kEpiResidual:
-      return narrow ? dispatch_bn<kEpiResidual, true>(dc, X, W, a, stream)
-                    : dispatch_bn<kEpiResidual, false>(dc, X, W, a, stream);
+      return narrow ? dispatch_bn<kEpiResidual, true>(dc, X, W, skip, Y, a, stream)
+                    : dispatch_bn<kEpiResidual, false>(dc, X, W, skip, Y, a, stream);
     case kEpiGelu:
-      return dispatch_bn<kEpiGelu, false>(dc, X, W, a, stream);
+      return dispatch_bn<kEpiGelu, false>(dc, X, W, skip, Y, a, stream);
   }
   return IVIT_ERR_INTERNAL;
 }
