@@ -115,6 +115,8 @@ __global__ void __launch_bounds__(kAttnThreads)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tslot;
+  pdl_wait();  // Q, K and V come from the previous kernel
+  pdl_launch_dependents();
 
   if (tid == 0) {
     mbar_arrive_expect_tx(bar_qk, (uint32_t)(kQTile * kHeadDim + nload * 64 * kHeadDim));
@@ -483,6 +485,8 @@ __global__ void __launch_bounds__(kPersistThreads, 1)
   }
   __syncthreads();
   const uint32_t tmem = *tslot;
+  pdl_wait();  // Q, K and V come from the previous kernel
+  pdl_launch_dependents();
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
@@ -759,12 +763,12 @@ ivit_status launch_attention(const DeviceCtx& dc, const int8_t* qkv, int32_t B, 
     const int64_t items = (int64_t)((N + kQTile - 1) / kQTile) * H * B;
     if (items > 0x7fffffff) return IVIT_ERR_UNSUPPORTED;
     const unsigned pgrid = (unsigned)(items < dc.num_sms ? items : dc.num_sms);
-    if (fastq)
-      attention_persist_kernel<true><<<pgrid, kPersistThreads, smem, stream>>>(tm, a, bq);
-    else
-      attention_persist_kernel<false><<<pgrid, kPersistThreads, smem, stream>>>(tm, a, bq);
+    const cudaError_t e =
+        fastq ? launch_pdl(attention_persist_kernel<true>, dim3(pgrid), dim3(kPersistThreads), smem, stream, tm, a, bq)
+              : launch_pdl(attention_persist_kernel<false>, dim3(pgrid), dim3(kPersistThreads), smem, stream, tm, a,
+                           bq);
     note_launch();
-    return cudaGetLastError() == cudaSuccess ? IVIT_OK : IVIT_ERR_CUDA;
+    return e == cudaSuccess ? IVIT_OK : IVIT_ERR_CUDA;
   }
   const AttnLayout L = attn_layout(N);
   // at most two CTAs per SM, so that their TMEM (256 columns each) always fits
@@ -777,9 +781,9 @@ ivit_status launch_attention(const DeviceCtx& dc, const int8_t* qkv, int32_t B, 
       return IVIT_ERR_CUDA;
     attr_bytes = 227 * 1024;
   }
-  attention_shiftmax_kernel<<<grid, kAttnThreads, smem, stream>>>(tm, a);
+  const cudaError_t e = launch_pdl(attention_shiftmax_kernel, grid, dim3(kAttnThreads), smem, stream, tm, a);
   note_launch();
-  return cudaGetLastError() == cudaSuccess ? IVIT_OK : IVIT_ERR_CUDA;
+  return e == cudaSuccess ? IVIT_OK : IVIT_ERR_CUDA;
 }
 
 }  // namespace ivit

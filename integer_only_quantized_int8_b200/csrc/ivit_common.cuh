@@ -131,6 +131,18 @@ IVIT_DEV bool mbar_wait(uint64_t* bar, uint32_t parity, int* status) {
 }
 
 // ---------------------------------------------------------------------------
+// programmatic dependent launch
+// ---------------------------------------------------------------------------
+// Every kernel of this library is launched so that the next kernel of the
+// stream may start (and run its prologue) while this one finishes.  A kernel
+// therefore calls pdl_wait() before it first touches memory that an earlier
+// kernel of the stream writes, and before its own first global write; the
+// wait returns once every earlier kernel has completed and its writes are
+// visible.  pdl_launch_dependents() lets the next kernel be scheduled.
+IVIT_DEV void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+IVIT_DEV void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
+// ---------------------------------------------------------------------------
 // TMA (cp.async.bulk.tensor): every copy fills or drains this CTA's own shared memory
 // ---------------------------------------------------------------------------
 IVIT_DEV void tma_load_2d(void* smem_dst, const CUtensorMap* map, int32_t x, int32_t y, uint64_t* bar) {

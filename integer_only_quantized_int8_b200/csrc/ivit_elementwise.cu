@@ -26,6 +26,8 @@ __global__ void __launch_bounds__(kGeluThreads)
   for (int i = threadIdx.x; i < 256; i += blockDim.x)
     tab[i] = (int8_t)shiftgelu8(i - 128, g.I0, g.M, g.k_out, g.out.b, g.out.c);
   __syncthreads();
+  pdl_wait();  // x comes from an earlier kernel
+  pdl_launch_dependents();
   const int64_t nvec = n >> 4;
   const int4* xv = reinterpret_cast<const int4*>(x);
   int4* yv = reinterpret_cast<int4*>(y);
@@ -54,12 +56,27 @@ __global__ void __launch_bounds__(kGeluThreads)
 
 constexpr int kLnThreads = 256;  // 16 half-warps: one row each
 
+// floor(a / d) for 0 <= a < 2^24 and 1 <= d < 2^24.  The fp32 quotient
+// a * rcp(d) has a relative error below 2^-23, so it is within 2 / d of a / d
+// (exact when d is a power of two): its floor is the true quotient or off by
+// one, and one integer correction in each direction settles it.
+__device__ __forceinline__ int32_t udiv_small(int32_t a, int32_t d) {
+  int32_t q = (int32_t)((float)a * __frcp_rn((float)d));
+  const int32_t r = a - q * d;
+  if (r < 0) q -= 1;
+  else if (r >= d) q += 1;
+  return q;
+}
+
+// Integer square root by exactly 10 Newton steps I <- (I + floor(V / I)) / 2
+// from I_0 = 2^floor(bits(V) / 2) (I-ViT section 3.5).  V is the variance of
+// int8 values, below 2^16, so every quotient takes the fast exact division.
 __device__ __forceinline__ int32_t isqrt_newton10(int32_t V) {
   if (V <= 0) return 0;
   const int bits = 32 - __clz(V);
   int32_t I = 1 << (bits >> 1);
 #pragma unroll
-  for (int it = 0; it < 10; ++it) I = (I + V / I) >> 1;
+  for (int it = 0; it < 10; ++it) I = (I + udiv_small(V, I)) >> 1;
   return I;
 }
 
@@ -98,11 +115,13 @@ __device__ __forceinline__ int32_t sext_byte(uint32_t w, int i) {
 // One row of `cols` int8 values per half-warp; lane l of the half-warp holds
 // the 16-byte chunks l, l + 16, ... (CPL of them).  CLAMP = false when the host
 // has shown that (b acc) >> c fits int32 for every reachable acc.
-template <int CPL, bool CLAMP>
+template <int CPL, bool CLAMP, bool FASTQ>
 __global__ void __launch_bounds__(kLnThreads)
     layernorm_kernel(const int8_t* __restrict__ x, int64_t rows, int32_t cols, const int8_t* __restrict__ gamma,
-                     const int32_t* __restrict__ beta, int32_t F, int32_t M_ln, ivit_dyadic out,
+                     const int32_t* __restrict__ beta, int32_t F, int32_t M_ln, ivit_dyadic out, int32_t out_bq,
                      int8_t* __restrict__ y) {
+  pdl_wait();  // x comes from an earlier kernel
+  pdl_launch_dependents();
   const int hl = threadIdx.x & 15;
   const int64_t row = (int64_t)blockIdx.x * (kLnThreads / 16) + (threadIdx.x >> 4);
   const bool active = row < rows;
@@ -136,7 +155,7 @@ __global__ void __launch_bounds__(kLnThreads)
   const int32_t V = sd2 / cols;  // sd2 >= 0: truncation == floor
   int32_t sigma = isqrt_newton10(V);
   if (sigma < 1) sigma = 1;
-  const int32_t f = (1 << M_ln) / sigma;
+  const int32_t f = udiv_small(1 << M_ln, sigma);  // M_ln <= 23
   const int sh = M_ln - F;
   const int32_t muf = mu * f;  // (x - mu) f = x f - mu f, exact in 32-bit arithmetic (|(x - mu) f| < 2^31)
   int32_t lo = INT_MIN, hi = INT_MAX;
@@ -160,9 +179,13 @@ __global__ void __launch_bounds__(kLnThreads)
         for (int e = 0; e < 4; ++e) {
           const int32_t nv = (sext_byte(xw[q], e) * f - muf) >> sh;
           int32_t acc = nv * sext_byte(gw[q], e) + bb[e];
-          if (CLAMP) acc = min(max(acc, lo), hi);
-          const int64_t pr = (int64_t)out.b * acc;  // (b acc) >> c fits int32: one funnel shift
-          r[e] = (int32_t)__funnelshift_r((uint32_t)pr, (uint32_t)(pr >> 32), (uint32_t)out.c);
+          if (FASTQ) {
+            r[e] = __mulhi(out_bq, acc);  // floor(b acc / 2^c) with bq = b 2^(32 - c), exact
+          } else {
+            if (CLAMP) acc = min(max(acc, lo), hi);
+            const int64_t pr = (int64_t)out.b * acc;  // (b acc) >> c fits int32: one funnel shift
+            r[e] = (int32_t)__funnelshift_r((uint32_t)pr, (uint32_t)(pr >> 32), (uint32_t)out.c);
+          }
         }
         o[q] = pack_sat4_ln(r[0], r[1], r[2], r[3]);
       }
@@ -181,9 +204,9 @@ ivit_status launch_shiftgelu(const DeviceCtx& dc, const int8_t* x, int64_t n, co
   const int64_t cap = (int64_t)dc.num_sms * 8;
   if (blocks > cap) blocks = cap;
   if (blocks < 1) blocks = 1;
-  shiftgelu_kernel<<<(unsigned)blocks, kGeluThreads, 0, stream>>>(x, n, g, y);
+  const cudaError_t e = launch_pdl(shiftgelu_kernel, dim3((unsigned)blocks), dim3(kGeluThreads), 0, stream, x, n, g, y);
   note_launch();
-  return cudaGetLastError() == cudaSuccess ? IVIT_OK : IVIT_ERR_CUDA;
+  return e == cudaSuccess ? IVIT_OK : IVIT_ERR_CUDA;
 }
 
 ivit_status launch_layernorm(const DeviceCtx& dc, const int8_t* x, int64_t rows, int32_t cols,
@@ -199,22 +222,28 @@ ivit_status launch_layernorm(const DeviceCtx& dc, const int8_t* x, int64_t rows,
   // below 2^(30 + c), (b acc) >> c always fits int32 and the clamp is not needed
   const double amax = 255.0 * 128.0 * std::ldexp(1.0, F) + std::ldexp(1.0, 30);
   const bool clamp = amax * (double)out.b >= std::ldexp(1.0, 30 + out.c);
-#define IVIT_LN_LAUNCH(CPL)                                                                                 \
-  (clamp ? layernorm_kernel<CPL, true><<<g, kLnThreads, 0, stream>>>(x, rows, cols, gamma, beta, F, M_ln, out, y) \
-         : layernorm_kernel<CPL, false><<<g, kLnThreads, 0, stream>>>(x, rows, cols, gamma, beta, F, M_ln, out, y))
+  // the output requant is one mul.hi by b 2^(32 - c) when that fits a positive int32
+  const bool fastq = out.c >= 1 && (int64_t)out.b < ((int64_t)1 << (out.c - 1));
+  const int32_t bq = fastq ? (int32_t)((int64_t)out.b << (32 - out.c)) : 0;
+#define IVIT_LN_LAUNCH(CPL)                                                                                \
+  launch_pdl(fastq   ? layernorm_kernel<CPL, false, true>                                                      \
+             : clamp ? layernorm_kernel<CPL, true, false>                                                      \
+                     : layernorm_kernel<CPL, false, false>,                                                    \
+             dim3(g), dim3(kLnThreads), 0, stream, x, rows, cols, gamma, beta, F, M_ln, out, bq, y)
+  cudaError_t e;
   if (nchunk <= 16)
-    IVIT_LN_LAUNCH(1);
+    e = IVIT_LN_LAUNCH(1);
   else if (nchunk <= 32)
-    IVIT_LN_LAUNCH(2);
+    e = IVIT_LN_LAUNCH(2);
   else if (nchunk <= 48)
-    IVIT_LN_LAUNCH(3);
+    e = IVIT_LN_LAUNCH(3);
   else if (nchunk <= 64)
-    IVIT_LN_LAUNCH(4);
+    e = IVIT_LN_LAUNCH(4);
   else
-    IVIT_LN_LAUNCH(8);
+    e = IVIT_LN_LAUNCH(8);
 #undef IVIT_LN_LAUNCH
   note_launch();
-  return cudaGetLastError() == cudaSuccess ? IVIT_OK : IVIT_ERR_CUDA;
+  return e == cudaSuccess ? IVIT_OK : IVIT_ERR_CUDA;
 }
 
 }  // namespace ivit

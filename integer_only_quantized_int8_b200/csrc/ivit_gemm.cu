@@ -308,6 +308,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tslot;
+  pdl_wait();  // X and the skip tensor come from earlier kernels
+  pdl_launch_dependents();
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
@@ -505,9 +507,9 @@ ivit_status run_gemm(const DeviceCtx& dc, const int8_t* X, const int8_t* W, cons
   }
   const int tiles = ((a.N + kBM - 1) / kBM) * (int)((a.M + BN - 1) / BN);
   const int grid = tiles < dc.num_sms ? tiles : dc.num_sms;
-  kern<<<grid, kGemmThreads, L::kAlloc, stream>>>(tmW, tmX, tmY, tmS, a);
+  const cudaError_t e = launch_pdl(kern, dim3(grid), dim3(kGemmThreads), L::kAlloc, stream, tmW, tmX, tmY, tmS, a);
   note_launch();
-  return cudaGetLastError() == cudaSuccess ? IVIT_OK : IVIT_ERR_CUDA;
+  return e == cudaSuccess ? IVIT_OK : IVIT_ERR_CUDA;
 }
 
 // Token-tile width: fewest rounds of tiles over the SMs, weighted by the tile

@@ -177,6 +177,27 @@ def test_layernorm_extreme_rows():
     np.testing.assert_array_equal(host(y), oracle.layernorm(x, gamma, beta, 7, 23, out))
 
 
+def test_layernorm_variance_sweep():
+    """Rows of two values a apart (half each, a = 0..255) have variance
+    floor(a^2 / 4), from 0 up to 16256, the largest an int8 row can have: the
+    Newton square root and the reciprocal 2^M / sigma are checked across the
+    whole range, with M_ln = 23 and with a small M_ln."""
+    cols = 64
+    amp = np.arange(256)
+    x = np.zeros((256, cols), np.int16)
+    x[:, ::2] = -128
+    x[:, 1::2] = (-128 + amp)[:, None]
+    x = x.astype(np.int8)
+    rng = np.random.default_rng(3)
+    gamma = rng.integers(-128, 128, cols).astype(np.int8)
+    beta = rng.integers(-(1 << 20), 1 << 20, cols).astype(np.int32)
+    out = ivit.ivit_dyadic_from_double(1.0 / 3000.0)
+    for F, M_ln in ((7, 23), (3, 9)):
+        y = torch.empty((256, cols), dtype=torch.int8, device="cuda")
+        ivit.ivit_layernorm(dev(x, torch.int8), dev(gamma, torch.int8), dev(beta, torch.int32), F, M_ln, out, y)
+        np.testing.assert_array_equal(host(y), oracle.layernorm(x, gamma, beta, F, M_ln, oracle.dyadic(1.0 / 3000.0)))
+
+
 @pytest.mark.parametrize("F", [0, 7, 14])
 @pytest.mark.parametrize("side", [0.9, 1.1])
 def test_layernorm_extreme_beta(F, side):
