@@ -339,6 +339,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       const uint32_t idesc = idesc_i8(kBM, BN, true, true, false);
+      // descriptors of stage 0, k-step 0: a stage adds kStageBytes >> 4 to the
+      // low half, the B tile kABytes >> 4 and a 32-byte k-step 2, so the issue
+      // loop stays a handful of instructions per MMA (this thread shares its
+      // sub-partition with three busy epilogue warps)
+      const uint64_t d0 = smem_desc(smem_u32(smem), 16, 1024, kSwizzle128B);
+      const uint32_t d_lo0 = (uint32_t)d0, d_hi = (uint32_t)(d0 >> 32);
       int stage = 0;
       uint32_t phase = 0;
       int acc = 0;
@@ -355,14 +361,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             break;
           }
           tc_fence_after();
-          const uint32_t sa = smem_u32(smem + stage * L::kStageBytes);
-          const uint32_t sb = sa + L::kABytes;
+          const uint32_t a_lo = d_lo0 + (uint32_t)(stage * (L::kStageBytes >> 4));
+          const uint32_t b_lo = a_lo + (uint32_t)(L::kABytes >> 4);
 #pragma unroll
-          for (int k = 0; k < kBK / 32; ++k) {
-            const uint64_t da = smem_desc(sa + k * 32, 16, 1024, kSwizzle128B);
-            const uint64_t db = smem_desc(sb + k * 32, 16, 1024, kSwizzle128B);
-            umma_i8(d_tmem, da, db, idesc, 1u);  // accumulate onto the preloaded bias
-          }
+          for (int k = 0; k < kBK / 32; ++k)  // accumulate onto the preloaded bias
+            umma_i8_acc(d_tmem, a_lo + 2 * k, d_hi, b_lo + 2 * k, d_hi, idesc);
           umma_commit(&empty[stage]);
           if (++stage == STAGES) {
             stage = 0;
