@@ -296,6 +296,7 @@ __global__ void __launch_bounds__(kAttnThreads)
 //               Two issuing threads, each blocked on its own next event, so
 //               neither softmax group waits behind the other;
 //   warps 3-18  two softmax groups of eight warps.
+// S = Q K^T is N = round16(N) columns wide.
 // Within an item the score row never leaves TMEM: pass 1 takes the row
 // maximum of the raw int32 scores (the logit requant is monotone, so
 // max L = requant(max S)); pass 2 requantises each score, looks up
@@ -315,7 +316,9 @@ constexpr int kLoadStages = 3;
 constexpr int kPersistThreads = 96 + 32 * kSoftWarps * kSoftGroups;
 
 struct PersistLayout {
-  int n64, n32, kblocks;
+  int n64, n32, n16, kblocks;
+  int sbuf;    // TMEM column stride of the two S buffers
+  int o_col;   // first TMEM column of the P V output when it has a region of its own, else -1
   int k_off, v_off, stage_bytes;  // Q at 0, K, V within a stage
   int p_off, p_bytes, tab_off, part_off, bar_off, total;
 };
@@ -324,7 +327,15 @@ __host__ __device__ inline PersistLayout persist_layout(int N) {
   PersistLayout L;
   L.n64 = (N + 63) / 64 * 64;
   L.n32 = (N + 31) / 32 * 32;
+  L.n16 = (N + 15) / 16 * 16;
   L.kblocks = (L.n32 + 127) / 128;
+  // Two S buffers of n32 columns and a 64-column region for P V fit the 512
+  // TMEM columns while n32 <= 224: a group then frees its S buffer as soon as
+  // P is written, and the next S MMA overlaps P V and the output requant.
+  // Beyond that P V lands in the first 64 columns of the item's S buffer.
+  const bool sep = 2 * L.n32 + kHeadDim <= 512;
+  L.sbuf = sep ? L.n32 : 256;
+  L.o_col = sep ? 2 * L.n32 : -1;
   L.k_off = kQTile * kHeadDim;             // 8 KB
   L.v_off = L.k_off + L.n64 * kHeadDim;    // + a multiple of 4 KB
   L.stage_bytes = L.v_off + L.n64 * kHeadDim;
@@ -436,11 +447,13 @@ __global__ void __launch_bounds__(kPersistThreads, 1)
   uint64_t* stage_empty = bars + 3;   // [3] stage reusable (P V of its item done)
   uint64_t* s_full = bars + 6;        // [2] S in TMEM buffer g
   uint64_t* p_full = bars + 8;        // [2] P of group g in shared memory (one arrival per warp)
-  uint64_t* o_full = bars + 10;       // [2] P V in TMEM buffer g
-  uint64_t* tmem_empty = bars + 12;   // [2] TMEM buffer g reusable (one arrival per warp)
+  uint64_t* o_full = bars + 10;       // [2] P V of group g's item in TMEM
+  uint64_t* tmem_empty = bars + 12;   // [2] S buffer g reusable (one arrival per warp)
   uint64_t* drain = bars + 14;        // all MMAs of the CTA complete (one commit per issuer)
   uint32_t* tslot = reinterpret_cast<uint32_t*>(bars + 15);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 16);
+  uint64_t* o_empty = bars + 17;      // separate P V region read out (one arrival per warp)
+  const bool sep_o = L.o_col >= 0;
 
   const int tid = threadIdx.x;
   const int warp = tid >> 5;
@@ -462,6 +475,7 @@ __global__ void __launch_bounds__(kPersistThreads, 1)
       mbar_init(&tmem_empty[g], kSoftWarps);
     }
     mbar_init(drain, 2);
+    mbar_init(o_empty, kSoftWarps);
     *abort_flag = 0;
     fence_barrier_init();
     prefetch_tensormap(&tm);
@@ -511,7 +525,7 @@ __global__ void __launch_bounds__(kPersistThreads, 1)
   } else if (warp == 1) {
     // ------------------------------------------------------------ S issuer
     if (lane == 0) {
-      const uint32_t idesc_s = idesc_i8(kQTile, L.n32, true, true, false);
+      const uint32_t idesc_s = idesc_i8(kQTile, L.n16, true, true, false);
       const int n_local = n_items > (int)blockIdx.x ? (n_items - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
       for (int j = 0; j < n_local; ++j) {
         const int g = j & 1, s = j % kLoadStages;
@@ -522,7 +536,7 @@ __global__ void __launch_bounds__(kPersistThreads, 1)
         const uint32_t ka = qa + L.k_off;
 #pragma unroll
         for (int k = 0; k < kHeadDim / 32; ++k)
-          umma_i8(tmem + (uint32_t)(g * 256), smem_desc(qa + k * 32, 16, 512, kSwizzle64B),
+          umma_i8(tmem + (uint32_t)(g * L.sbuf), smem_desc(qa + k * 32, 16, 512, kSwizzle64B),
                   smem_desc(ka + k * 32, 16, 512, kSwizzle64B), idesc_s, k != 0);
         umma_commit(&s_full[g]);
       }
@@ -538,11 +552,14 @@ __global__ void __launch_bounds__(kPersistThreads, 1)
       for (int j = 0; j < n_local; ++j) {
         const int g = j & 1, s = j % kLoadStages;
         if (!wait_or_abort(&p_full[g], (uint32_t)((j >> 1) & 1), a.status, abort_flag)) break;
+        // the shared P V region is free once the previous item's output is read
+        if (sep_o && j > 0 && !wait_or_abort(o_empty, (uint32_t)((j - 1) & 1), a.status, abort_flag)) break;
         tc_fence_after();
         const uint32_t pa = smem_u32(smem + L.p_off + g * L.p_bytes);
         const uint32_t va = smem_u32(smem + s * L.stage_bytes + L.v_off);
+        const uint32_t d_o = tmem + (uint32_t)(sep_o ? L.o_col : g * L.sbuf);
         for (int k = 0; k < L.n32 / 32; ++k)
-          umma_i8(tmem + (uint32_t)(g * 256), smem_desc(pa + (k >> 2) * 16384 + (k & 3) * 32, 16, 1024, kSwizzle128B),
+          umma_i8(d_o, smem_desc(pa + (k >> 2) * 16384 + (k & 3) * 32, 16, 1024, kSwizzle128B),
                   smem_desc(va + k * 32 * kHeadDim, 512, 512, kSwizzle64B), idesc_o, k != 0);
         umma_commit(&o_full[g]);
         umma_commit(&stage_empty[s]);
@@ -564,13 +581,18 @@ __global__ void __launch_bounds__(kPersistThreads, 1)
     int32_t* part = reinterpret_cast<int32_t*>(smem + L.part_off) + group * 512;  // [half][max, sum][128 rows]
     const int rlo = row & 7;
     uint8_t* prow = smem + L.p_off + group * L.p_bytes + (row >> 3) * 1024 + rlo * 128;
-    const uint32_t t_row = tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(group * 256);
+    const uint32_t t_row = tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(group * L.sbuf);
+    const uint32_t t_out = sep_o ? tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)L.o_col : t_row;
     const int pshift = a.M - (a.k_out - 1);
     bool ok = true;
     int j = group;
-    for (int item = blockIdx.x + group * gridDim.x; item < n_items; item += kSoftGroups * gridDim.x, j += 2) {
+    // item = qt + qtiles (h + H img), advanced by a fixed step without divisions
+    const int first = blockIdx.x + group * gridDim.x;
+    const int step = kSoftGroups * gridDim.x;
+    int qt = first % qtiles, h = (first / qtiles) % a.H, img = first / (qtiles * a.H);
+    const int st_q = step % qtiles, st_h = (step / qtiles) % a.H, st_i = step / (qtiles * a.H);
+    for (int item = first; item < n_items; item += step, j += 2) {
       const uint32_t ph = (uint32_t)((j >> 1) & 1);
-      const int qt = item % qtiles, h = (item / qtiles) % a.H, img = item / (qtiles * a.H);
       const int q0 = qt * kQTile;
       if (ok) ok = wait_or_abort(&s_full[group], ph, a.status, abort_flag);
       ok = __all_sync(0xffffffffu, ok);
@@ -649,7 +671,10 @@ __global__ void __launch_bounds__(kPersistThreads, 1)
       fence_proxy_async_smem();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&p_full[group]);
+      if (lane == 0) {
+        mbar_arrive(&p_full[group]);
+        if (sep_o) mbar_arrive(&tmem_empty[group]);  // S is consumed: the next S may land
+      }
 
       // ---- ctx = sat_8((b_o O) >> c_o); half h writes columns [32 h, 32 h + 32)
       if (ok) ok = wait_or_abort(&o_full[group], ph, a.status, abort_flag);
@@ -657,7 +682,7 @@ __global__ void __launch_bounds__(kPersistThreads, 1)
       tc_fence_after();
       if (ok && work) {
         uint32_t r[32];
-        tmem_ld32(t_row + (uint32_t)(half * 32), r);
+        tmem_ld32(t_out + (uint32_t)(half * 32), r);
         tmem_ld_wait();
         const int q = q0 + row;
         if (q < N) {
@@ -684,7 +709,18 @@ __global__ void __launch_bounds__(kPersistThreads, 1)
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&tmem_empty[group]);
+      if (lane == 0) mbar_arrive(sep_o ? o_empty : &tmem_empty[group]);
+      qt += st_q;
+      if (qt >= qtiles) {
+        qt -= qtiles;
+        ++h;
+      }
+      h += st_h;
+      if (h >= a.H) {
+        h -= a.H;
+        ++img;
+      }
+      img += st_i;
     }
   }
 

@@ -56,11 +56,12 @@ __global__ void __launch_bounds__(kGeluThreads)
 
 constexpr int kLnThreads = 256;  // 16 half-warps: one row each
 
-// floor(a / d) for 0 <= a < 2^24 and 1 <= d < 2^24.  The fp32 quotient
-// a * rcp(d) has a relative error below 2^-23, so it is within 2 / d of a / d
-// (exact when d is a power of two): its floor is the true quotient or off by
+// floor(a / d) for 0 <= a < 2^30, d >= 1 and a quotient below 2^22.  Each of
+// the conversions of a, the reciprocal of d and the product rounds with a
+// relative error of at most 2^-24, so the fp32 quotient is within
+// 3.01 * 2^-24 * 2^22 < 1 of a / d: its floor is the true quotient or off by
 // one, and one integer correction in each direction settles it.
-__device__ __forceinline__ int32_t udiv_small(int32_t a, int32_t d) {
+__device__ __forceinline__ int32_t udiv_fast(int32_t a, int32_t d) {
   int32_t q = (int32_t)((float)a * __frcp_rn((float)d));
   const int32_t r = a - q * d;
   if (r < 0) q -= 1;
@@ -69,15 +70,31 @@ __device__ __forceinline__ int32_t udiv_small(int32_t a, int32_t d) {
 }
 
 // Integer square root by exactly 10 Newton steps I <- (I + floor(V / I)) / 2
-// from I_0 = 2^floor(bits(V) / 2) (I-ViT section 3.5).  V is the variance of
-// int8 values, below 2^16, so every quotient takes the fast exact division.
-__device__ __forceinline__ int32_t isqrt_newton10(int32_t V) {
+// from I_0 = 2^floor(bits(V) / 2) (I-ViT section 3.5).
+__host__ __device__ constexpr int32_t isqrt_newton10_exact(int32_t V) {
   if (V <= 0) return 0;
-  const int bits = 32 - __clz(V);
+  int bits = 0;
+  for (int32_t x = V; x; x >>= 1) ++bits;
   int32_t I = 1 << (bits >> 1);
-#pragma unroll
-  for (int it = 0; it < 10; ++it) I = (I + udiv_small(V, I)) >> 1;
+  for (int it = 0; it < 10; ++it) I = (I + V / I) >> 1;
   return I;
+}
+
+// The variance of int8 values is at most 127.5^2 < 16384, so the 10-step root
+// of every reachable V is tabulated at compile time (each entry <= 128).
+constexpr int kIsqrtTab = 16384;
+struct IsqrtTable {
+  uint8_t v[kIsqrtTab];
+};
+__host__ __device__ constexpr IsqrtTable make_isqrt_table() {
+  IsqrtTable t{};
+  for (int V = 0; V < kIsqrtTab; ++V) t.v[V] = (uint8_t)isqrt_newton10_exact(V);
+  return t;
+}
+__device__ constexpr IsqrtTable g_isqrt10 = make_isqrt_table();
+
+__device__ __forceinline__ int32_t isqrt_newton10(int32_t V) {
+  return V < kIsqrtTab ? (int32_t)g_isqrt10.v[V] : isqrt_newton10_exact(V);
 }
 
 // Saturation bounds of the output requant sat_8((b acc) >> c): clamping acc to
@@ -148,14 +165,16 @@ __global__ void __launch_bounds__(kLnThreads)
     s2 += __shfl_xor_sync(0xffffffffu, s2, o);
   }
   if (!active) return;
-  // mu = floor(sum x / n); sum (x - mu)^2 = sum x^2 - 2 mu sum x + n mu^2, all within int32
-  int32_t mu = s1 / cols;
-  if ((s1 % cols) != 0 && s1 < 0) mu -= 1;
+  // mu = floor(sum x / n) (|sum x| <= 2^18); sum (x - mu)^2 = sum x^2 - 2 mu sum x + n mu^2,
+  // all within int32 (at most 2^27)
+  const int32_t as1 = s1 < 0 ? -s1 : s1;
+  const int32_t q1 = udiv_fast(as1, cols);
+  const int32_t mu = s1 >= 0 ? q1 : -q1 - (as1 - q1 * cols != 0 ? 1 : 0);
   const int32_t sd2 = s2 - 2 * mu * s1 + cols * mu * mu;
-  const int32_t V = sd2 / cols;  // sd2 >= 0: truncation == floor
+  const int32_t V = udiv_fast(sd2, cols);  // sd2 >= 0, quotient <= 16256
   int32_t sigma = isqrt_newton10(V);
   if (sigma < 1) sigma = 1;
-  const int32_t f = udiv_small(1 << M_ln, sigma);  // M_ln <= 23
+  const int32_t f = udiv_fast(1 << M_ln, sigma);  // M_ln <= 23: quotient 2^M_ln exact for sigma = 1
   const int sh = M_ln - F;
   const int32_t muf = mu * f;  // (x - mu) f = x f - mu f, exact in 32-bit arithmetic (|(x - mu) f| < 2^31)
   int32_t lo = INT_MIN, hi = INT_MAX;
