@@ -80,21 +80,52 @@ __host__ __device__ constexpr int32_t isqrt_newton10_exact(int32_t V) {
   return I;
 }
 
-// The variance of int8 values is at most 127.5^2 < 16384, so the 10-step root
-// of every reachable V is tabulated at compile time (each entry <= 128).
-constexpr int kIsqrtTab = 16384;
-struct IsqrtTable {
-  uint8_t v[kIsqrtTab];
-};
-__host__ __device__ constexpr IsqrtTable make_isqrt_table() {
-  IsqrtTable t{};
-  for (int V = 0; V < kIsqrtTab; ++V) t.v[V] = (uint8_t)isqrt_newton10_exact(V);
-  return t;
+// floor(sqrt(V)) by bisection, for the compile-time check below.
+__host__ __device__ constexpr int32_t isqrt_floor_exact(int32_t V) {
+  int32_t lo = 0, hi = 46341;  // hi^2 > INT32_MAX
+  while (hi - lo > 1) {
+    const int32_t m = (lo + hi) / 2;
+    if ((int64_t)m * m <= V) lo = m; else hi = m;
+  }
+  return lo;
 }
-__device__ constexpr IsqrtTable g_isqrt10 = make_isqrt_table();
+
+// The variance of int8 values is at most 127.5^2 < 16384.  Over that range the
+// 10-step root equals floor(sqrt(V)) except at some V = s^2 - 1, where the
+// iteration, which alternates between s - 1 and s there, stops on s.  Those s
+// (all <= 128) are marked in a bit mask built at compile time from the
+// iteration itself, and the whole range is checked against root-plus-mask.
+constexpr int kIsqrtRange = 16384;
+struct IsqrtMask {
+  uint32_t w[5];  // bit s: the 10-step root of s^2 - 1 is s
+};
+__host__ __device__ constexpr IsqrtMask make_isqrt_mask() {
+  IsqrtMask m{};
+  for (int s = 1; s * s - 1 < kIsqrtRange; ++s)
+    if (isqrt_newton10_exact(s * s - 1) == s) m.w[s >> 5] |= 1u << (s & 31);
+  return m;
+}
+constexpr IsqrtMask kIsqrtMask = make_isqrt_mask();
+__host__ __device__ constexpr bool isqrt_mask_matches() {
+  for (int32_t V = 0; V < kIsqrtRange; ++V) {
+    const int32_t r = isqrt_floor_exact(V), s = r + 1;
+    const bool up = V + 1 == s * s && ((kIsqrtMask.w[s >> 5] >> (s & 31)) & 1u);
+    if (isqrt_newton10_exact(V) != r + (up ? 1 : 0)) return false;
+  }
+  return true;
+}
+static_assert(isqrt_mask_matches(), "10-step root = floor(sqrt) + mask over int8 variances");
 
 __device__ __forceinline__ int32_t isqrt_newton10(int32_t V) {
-  return V < kIsqrtTab ? (int32_t)g_isqrt10.v[V] : isqrt_newton10_exact(V);
+  if (V >= kIsqrtRange) return isqrt_newton10_exact(V);
+  // V < 2^22: the correctly rounded single-precision root of an integer V never
+  // rounds up to the next integer, so truncation gives floor(sqrt(V))
+  const int32_t r = (int32_t)__fsqrt_rn((float)V), s = r + 1;  // s <= 128
+  constexpr uint32_t m0 = kIsqrtMask.w[0], m1 = kIsqrtMask.w[1], m2 = kIsqrtMask.w[2], m3 = kIsqrtMask.w[3],
+                     m4 = kIsqrtMask.w[4];
+  const int wi = s >> 5;
+  const uint32_t word = wi == 0 ? m0 : wi == 1 ? m1 : wi == 2 ? m2 : wi == 3 ? m3 : m4;
+  return (V + 1 == s * s && ((word >> (s & 31)) & 1u)) ? s : r;
 }
 
 // Saturation bounds of the output requant sat_8((b acc) >> c): clamping acc to

@@ -22,12 +22,29 @@
 // Roles (one CTA per SM, persistent over 128 x BN tiles):
 //   warp 0      TMA producer: W and X k-slices of 128 bytes, 128B swizzle,
 //               into a STAGES-deep ring guarded by full/empty mbarriers;
-//   warp 1      allocates TMEM (two BN-column accumulators) and one lane issues
-//               tcgen05.mma M=128 N=BN K=32; tcgen05.commit frees smem stages
-//               and publishes finished accumulators;
-//   warps 2-13  epilogue: three warps per TMEM lane quarter split the tile's
+//   warps 1-2   MMA issue: warp 1 allocates TMEM (two BN-column accumulators);
+//               lane 0 issues tcgen05.mma M=128 N=BN K=32.  With an even ring
+//               depth lane 0 of warp 2 issues too: the two threads take
+//               alternate k-slices (the even and the odd ones of the CTA's
+//               whole sequence), both into the same accumulator;
+//               tcgen05.commit frees smem stages and, from every issuing
+//               thread, publishes finished accumulators;
+//   warps 3-14  epilogue: three warps per TMEM lane quarter split the tile's
 //               16-token chunks; the accumulator of tile t drains while the
 //               MMAs of tile t+1 run.
+//
+// Why two issuing threads: one thread spends about 480 SM cycles per k-slice
+// on its mbarrier wait, the four MMA issues and the commit, whatever BN is,
+// while the four MMAs take 2 BN cycles on the tensor core; below BN = 256 a
+// single issuer leaves the tensor core idle.  Two threads overlap that
+// bookkeeping.  The integer accumulation is exact and every MMA accumulates
+// (the bias is preloaded), so the order in which the two threads' MMAs land
+// on the accumulator does not change the result.  The ring depth must be even
+// so that each thread owns the stages of its k-slice parity: a thread then
+// waits on a stage's full barrier only after its own previous use of the
+// stage, never two phases ahead of it (TMA loads may complete out of order,
+// and a parity wait cannot tell phase p from phase p + 2).  At BN = 256 the
+// ring is three deep and a single thread keeps the tensor core busy.
 #include <climits>
 
 #include "ivit_common.cuh"
@@ -40,7 +57,7 @@ constexpr int kBM = 128;  // output channels per tile
 constexpr int kBK = 128;  // bytes = int8 elements per k-slice (one 128-byte swizzle row)
 constexpr int kEpiWarps = 12;  // three per TMEM lane quarter
 constexpr int kEpiParts = kEpiWarps / 4;
-constexpr int kGemmThreads = 64 + 32 * kEpiWarps;
+constexpr int kGemmThreads = 96 + 32 * kEpiWarps;
 constexpr int kSlotBytes = 16 * 32;  // one staged chunk: 16 tokens x 32 channels
 
 struct GemmArgs {
@@ -57,6 +74,8 @@ struct GemmArgs {
 
 template <int BN, int STAGES>
 struct GemmLayout {
+  // MMA-issuing threads: two when each can own half of the ring's stages
+  static constexpr int kIssuers = (STAGES % 2 == 0) ? 2 : 1;
   static constexpr int kABytes = kBM * kBK;
   static constexpr int kBBytes = BN * kBK;
   static constexpr int kStageBytes = kABytes + kBBytes;
@@ -283,10 +302,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       mbar_init(&empty[s], 1);
     }
     for (int a = 0; a < 2; ++a) {
-      mbar_init(&tfull[a], 1);
+      mbar_init(&tfull[a], L::kIssuers);  // one commit per issuing thread
       mbar_init(&tempty[a], kEpiWarps);
     }
-    mbar_init(drain, 1);
+    mbar_init(drain, L::kIssuers);
     for (int e = 0; e < kEpiWarps; ++e) mbar_init(&skip_full[e], 1);
     fence_barrier_init();
     prefetch_tensormap(&tmW);
@@ -335,18 +354,22 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         }
       }
     }
-  } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
+  } else if (warp <= 2) {
+    // ------------------------------------------------------------ MMA issuers
+    if (lane == 0 && warp <= L::kIssuers) {
+      constexpr int kStep = L::kIssuers;
       const uint32_t idesc = idesc_i8(kBM, BN, true, true, false);
       // descriptors of stage 0, k-step 0: a stage adds kStageBytes >> 4 to the
       // low half, the B tile kABytes >> 4 and a 32-byte k-step 2, so the issue
-      // loop stays a handful of instructions per MMA (this thread shares its
-      // sub-partition with three busy epilogue warps)
+      // loop stays a handful of instructions per MMA
       const uint64_t d0 = smem_desc(smem_u32(smem), 16, 1024, kSwizzle128B);
       const uint32_t d_lo0 = (uint32_t)d0, d_hi = (uint32_t)(d0 >> 32);
-      int stage = 0;
+      // this thread takes every kStep-th k-slice of the CTA's sequence,
+      // starting with slice warp - 1; the ring position advances kStep stages
+      // per slice
+      int stage = warp - 1;
       uint32_t phase = 0;
+      int kb0 = warp - 1;  // this thread's first k-slice within the current tile
       int acc = 0;
       uint32_t acc_phase = 0;
       bool ok = true;
@@ -355,7 +378,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         if (!mbar_wait(&tempty[acc], acc_phase, args.status)) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BN);
-        for (int kb = 0; kb < num_kb; ++kb) {
+        int kb = kb0;
+        for (; kb < num_kb; kb += kStep) {
           if (!mbar_wait(&full[stage], phase, args.status)) {
             ok = false;
             break;
@@ -367,12 +391,15 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           for (int k = 0; k < kBK / 32; ++k)  // accumulate onto the preloaded bias
             umma_i8_acc(d_tmem, a_lo + 2 * k, d_hi, b_lo + 2 * k, d_hi, idesc);
           umma_commit(&empty[stage]);
-          if (++stage == STAGES) {
-            stage = 0;
+          stage += kStep;
+          if (stage >= STAGES) {
+            stage -= STAGES;
             phase ^= 1;
           }
         }
         if (!ok) break;
+        kb0 = kb - num_kb;
+        // arrives once this thread's MMAs of the tile (possibly none) are done
         umma_commit(&tfull[acc]);
         acc ^= 1;
         if (acc == 0) acc_phase ^= 1;
@@ -384,7 +411,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   } else {
     // ------------------------------------------------------------ epilogue
     constexpr int kChunks = L::kChunks;
-    const int e = warp - 2;
+    const int e = warp - 3;
     const int quarter = warp & 3;  // TMEM lanes [32 q, 32 q + 32) = channels of this warp
     const int part = e >> 2;       // which of the quarter's warps: splits the token chunks
     const int c_begin = (kChunks * part) / kEpiParts;
@@ -544,9 +571,9 @@ ivit_status dispatch_bn(const DeviceCtx& dc, const int8_t* X, const int8_t* W, c
     case 224:
       return run_gemm<224, 4, EPI, NARROW>(dc, X, W, skip, Y, a, stream);
     case 192:
-      return run_gemm<192, 5, EPI, NARROW>(dc, X, W, skip, Y, a, stream);
+      return run_gemm<192, 4, EPI, NARROW>(dc, X, W, skip, Y, a, stream);
     case 160:
-      return run_gemm<160, 5, EPI, NARROW>(dc, X, W, skip, Y, a, stream);
+      return run_gemm<160, 4, EPI, NARROW>(dc, X, W, skip, Y, a, stream);
     default:
       return run_gemm<128, 6, EPI, NARROW>(dc, X, W, skip, Y, a, stream);
   }
