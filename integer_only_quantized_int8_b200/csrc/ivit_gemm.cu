@@ -15,9 +15,12 @@
 // requant scale below one half, the usual case) the requant
 // floor(b acc / 2^c) is then one mul.hi by b 2^(32 - c); the saturating byte
 // pack clips.  A 4 x 4 byte transpose across lanes turns channel-major bytes
-// into token-major 4-byte words, which go to a shared-memory staging slot per
-// 16-token chunk and leave by TMA store (the residual's skip tile arrives the
-// same way).
+// into token-major 4-byte words.  The four warps that cover the tile's 128
+// channels for the same tokens (one per TMEM lane quarter: a "part") fill one
+// 16-token x 128-channel staging slot per chunk, 128B-swizzled, and one thread
+// of the part sends it out with a single TMA store: 16 rows of 128 bytes
+// instead of four boxes of 16 rows of 32 bytes, which the TMA unit drains four
+// times faster.  The residual's skip tile arrives the same way.
 //
 // Roles (one CTA per SM, persistent over 128 x BN tiles):
 //   warp 0      TMA producer: W and X k-slices of 128 bytes, 128B swizzle,
@@ -58,7 +61,7 @@ constexpr int kBK = 128;  // bytes = int8 elements per k-slice (one 128-byte swi
 constexpr int kEpiWarps = 12;  // three per TMEM lane quarter
 constexpr int kEpiParts = kEpiWarps / 4;
 constexpr int kGemmThreads = 96 + 32 * kEpiWarps;
-constexpr int kSlotBytes = 16 * 32;  // one staged chunk: 16 tokens x 32 channels
+constexpr int kSlotBytes = 16 * kBM;  // one staged chunk: 16 tokens x 128 channels
 
 struct GemmArgs {
   int64_t M;       // tokens (rows of X and Y)
@@ -82,10 +85,10 @@ struct GemmLayout {
   static constexpr int kChunks = BN / 16;
   static constexpr int kMaxPart = (kChunks + kEpiParts - 1) / kEpiParts;  // chunks of the largest part
   static constexpr int kOutOff = STAGES * kStageBytes;
-  static constexpr int kWarpSlots = kMaxPart * kSlotBytes;
-  static constexpr int kBarOff = kOutOff + kEpiWarps * kWarpSlots;
-  // full, empty (STAGES each), tmem full x2, tmem empty x2, drain, one skip barrier per epilogue warp
-  static constexpr int kNumBars = 2 * STAGES + 5 + kEpiWarps;
+  static constexpr int kPartSlots = kMaxPart * kSlotBytes;  // 1024-byte aligned, as the swizzle needs
+  static constexpr int kBarOff = kOutOff + kEpiParts * kPartSlots;
+  // full, empty (STAGES each), tmem full x2, tmem empty x2, drain, one skip barrier per part
+  static constexpr int kNumBars = 2 * STAGES + 5 + kEpiParts;
   static constexpr int kSlotOff = kBarOff + kNumBars * 8;
   static constexpr int kGeluOff = kSlotOff + 16;
   static constexpr int kBytes = kGeluOff + 256;
@@ -207,15 +210,23 @@ IVIT_DEV uint32_t residual_word(uint32_t s, uint32_t y, const ivit_residual& res
   return pack_sat4(z[0], z[1], z[2], z[3]);
 }
 
+// Byte offset of the lane's word k (token 4k + sub of the chunk, the lane's
+// channel group of four) in a 128B-swizzled 16 x 128-byte slot: 16-byte
+// column c of row r sits at column c ^ (r & 7).  ofs_even / ofs_odd are the
+// offsets for k = 0 and k = 1; words 2 and 3 lie 8 rows (1024 bytes) further.
+IVIT_DEV uint32_t slot_ofs(int sub, int quarter, int grp, int k01) {
+  const int r = 4 * k01 + sub;
+  const int c = 2 * quarter + (grp >> 2);
+  return (uint32_t)(r * 128 + ((c ^ (r & 7)) << 4) + ((grp & 3) << 2));
+}
+
 // One 16-token chunk of one epilogue warp: requant the 16 accumulators of this
 // thread's channel (r = TMEM columns of the chunk), pack, transpose to
 // token-major words, apply the residual (its skip words were staged in the
-// same slot) and leave the result in the slot.  slot_w points at the lane's
-// word of the slot: word k (token 4k + sub, channels 4 grp .. 4 grp + 3) sits
-// at byte (4k + sub) * 32 + 4 grp, i.e. slot_w[32 k].
+// same slot) and leave the result in the slot at the lane's offsets.
 template <int EPI, bool NARROW, int REQ>
 IVIT_DEV void epi_chunk(const uint32_t (&r)[16], const ChanConst& kc, const GemmArgs& args, const int8_t* gelu_tab,
-                        uint32_t* slot_w, uint32_t sel2, uint32_t sel1) {
+                        uint8_t* slot, uint32_t ofs_even, uint32_t ofs_odd, uint32_t sel2, uint32_t sel1) {
   uint32_t w[4];
 #pragma unroll
   for (int k = 0; k < 4; ++k) {
@@ -236,7 +247,7 @@ IVIT_DEV void epi_chunk(const uint32_t (&r)[16], const ChanConst& kc, const Gemm
   if (EPI == kEpiResidual) {
     uint32_t s[4];
 #pragma unroll
-    for (int k = 0; k < 4; ++k) s[k] = slot_w[32 * k];
+    for (int k = 0; k < 4; ++k) s[k] = *reinterpret_cast<const uint32_t*>(slot + (k >> 1) * 1024 + ((k & 1) ? ofs_odd : ofs_even));
     if (args.res.c >= 9) {
 #pragma unroll
       for (int k = 0; k < 4; ++k) w[k] = residual_word<true>(s[k], w[k], args.res);
@@ -246,28 +257,52 @@ IVIT_DEV void epi_chunk(const uint32_t (&r)[16], const ChanConst& kc, const Gemm
     }
   }
 #pragma unroll
-  for (int k = 0; k < 4; ++k) slot_w[32 * k] = w[k];
+  for (int k = 0; k < 4; ++k) *reinterpret_cast<uint32_t*>(slot + (k >> 1) * 1024 + ((k & 1) ? ofs_odd : ofs_even)) = w[k];
 }
 
-// The chunks [c_begin, c_begin + n) of one tile into the warp's slots.
+// The chunks [c_begin, c_begin + n) of one tile into the part's slots, two
+// chunks' TMEM loads per wait.
 template <int EPI, bool NARROW, int REQ>
 IVIT_DEV void epi_tile(uint32_t tbase, int c_begin, int n, const ChanConst& kc, const GemmArgs& args,
-                       const int8_t* gelu_tab, uint32_t* slot_w, uint32_t sel2, uint32_t sel1) {
-  for (int i = 0; i < n; ++i) {
-    uint32_t r[16];
-    tmem_ld16(tbase + (uint32_t)(16 * (c_begin + i)), r);
-    tmem_ld_wait();
-    epi_chunk<EPI, NARROW, REQ>(r, kc, args, gelu_tab, slot_w + i * (kSlotBytes / 4), sel2, sel1);
+                       const int8_t* gelu_tab, uint8_t* slots, uint32_t ofs_even, uint32_t ofs_odd, uint32_t sel2,
+                       uint32_t sel1) {
+  const uint32_t t0 = tbase + (uint32_t)(16 * c_begin);
+  int i = 0;
+  for (; i + 1 < n; i += 2) {
+    uint32_t ra[16], rb[16];
+    tmem_ld16(t0 + (uint32_t)(16 * i), ra);
+    tmem_ld16(t0 + (uint32_t)(16 * (i + 1)), rb);
+    tmem_ld_wait_regs2(ra, rb);
+    epi_chunk<EPI, NARROW, REQ>(ra, kc, args, gelu_tab, slots + i * kSlotBytes, ofs_even, ofs_odd, sel2, sel1);
+    epi_chunk<EPI, NARROW, REQ>(rb, kc, args, gelu_tab, slots + (i + 1) * kSlotBytes, ofs_even, ofs_odd, sel2, sel1);
   }
+  if (i < n) {
+    uint32_t r[16];
+    tmem_ld16(t0 + (uint32_t)(16 * i), r);
+    tmem_ld_wait_regs(r);
+    epi_chunk<EPI, NARROW, REQ>(r, kc, args, gelu_tab, slots + i * kSlotBytes, ofs_even, ofs_odd, sel2, sel1);
+  }
+}
+
+// Named barrier of the four warps of one part (ids 1..kEpiParts) that also
+// returns the AND of every thread's v, so the part gives up together.
+IVIT_DEV bool part_bar_and(int part, bool v) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 q, %1, 0;\n\t"
+      "bar.red.and.pred p, %2, 128, q;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(r)
+      : "r"((uint32_t)v), "r"(1 + part)
+      : "memory");
+  return r != 0;
 }
 
 // Preload TMEM columns [16 c_begin, 16 c_end) of this warp's lanes in one
 // accumulator buffer with the bias of the lane's output channel.
 IVIT_DEV void bias_fill(uint32_t tbase, int c_begin, int c_end, int32_t bias) {
-  uint32_t v[16];
-#pragma unroll
-  for (int i = 0; i < 16; ++i) v[i] = (uint32_t)bias;
-  for (int cc = c_begin; cc < c_end; ++cc) tmem_st16(tbase + (uint32_t)(16 * cc), v);
+  for (int cc = c_begin; cc < c_end; ++cc) tmem_st16_fill(tbase + (uint32_t)(16 * cc), (uint32_t)bias);
 }
 
 template <int BN, int STAGES, int EPI, bool NARROW>
@@ -283,7 +318,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   uint64_t* tfull = empty + STAGES;
   uint64_t* tempty = tfull + 2;
   uint64_t* drain = tempty + 2;
-  uint64_t* skip_full = drain + 1;  // [kEpiWarps]
+  uint64_t* skip_full = drain + 1;  // [kEpiParts]
   uint32_t* tslot = reinterpret_cast<uint32_t*>(smem + L::kSlotOff);
   int8_t* gelu_tab = reinterpret_cast<int8_t*>(smem + L::kGeluOff);
 
@@ -306,7 +341,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       mbar_init(&tempty[a], kEpiWarps);
     }
     mbar_init(drain, L::kIssuers);
-    for (int e = 0; e < kEpiWarps; ++e) mbar_init(&skip_full[e], 1);
+    for (int e = 0; e < kEpiParts; ++e) mbar_init(&skip_full[e], 1);
     fence_barrier_init();
     prefetch_tensormap(&tmW);
     prefetch_tensormap(&tmX);
@@ -420,9 +455,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     const uint32_t sel1 = (lane & 1) ? 0x3715u : 0x6240u;
     const int sub = lane & 3;   // token offset within a transposed 4 x 4 block
     const int grp = lane >> 2;  // channel group of 4 within the warp's 32 channels
-    uint8_t* slots = smem + L::kOutOff + e * L::kWarpSlots;
-    uint32_t* slot_w = reinterpret_cast<uint32_t*>(slots) + sub * 8 + grp;
-    uint64_t* sbar = &skip_full[e];
+    // the part's first warp stages its skip tiles and stores its outputs
+    const bool part_lead = (e & 3) == 0 && lane == 0;
+    uint8_t* slots = smem + L::kOutOff + part * L::kPartSlots;
+    const uint32_t ofs_even = slot_ofs(sub, quarter, grp, 0), ofs_odd = slot_ofs(sub, quarter, grp, 1);
+    uint64_t* sbar = &skip_full[part];
     const uint32_t tlane = tmem_base + ((uint32_t)(quarter * 32) << 16);
     auto bias_of = [&](int t) -> int32_t {
       const int ch = (t % ch_tiles) * kBM + quarter * 32 + lane;
@@ -451,42 +488,48 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       const int req = __all_sync(0xffffffffu, kc.fast) ? kReqFast
                       : (__any_sync(0xffffffffu, kc.needs_clamp) ? kReqWideClamp : kReqWide);
       const int64_t tok_base = (int64_t)tb * BN;
+      const int32_t next_bias = bias_of(t + 2 * (int)gridDim.x);
       int n = c_end - c_begin;  // chunks that hold at least one real token
       while (n > 0 && tok_base + 16 * (c_begin + n - 1) >= M) --n;
-      const bool live = n > 0 && ch0 < N;
-      // the slots are free again once the stores of the previous tile have read them
-      if (lane == 0) bulk_wait_read_all();
-      __syncwarp();
-      if (EPI == kEpiResidual && live && lane == 0) {
-        mbar_arrive_expect_tx(sbar, (uint32_t)(n * kSlotBytes));
-        for (int i = 0; i < n; ++i)
-          tma_load_2d(slots + i * kSlotBytes, &tmS, ch0, (int32_t)(tok_base + 16 * (c_begin + i)), sbar);
+      const bool live = n > 0;  // the same for the part's four warps
+      const int tile_ch = cb * kBM;
+      if (part_lead) {
+        // the slots are free again once the stores of the previous tile have read them
+        bulk_wait_read_all();
+        if (EPI == kEpiResidual && live) {
+          mbar_arrive_expect_tx(sbar, (uint32_t)(n * kSlotBytes));
+          for (int i = 0; i < n; ++i)
+            tma_load_2d(slots + i * kSlotBytes, &tmS, tile_ch, (int32_t)(tok_base + 16 * (c_begin + i)), sbar);
+        }
       }
-      bool got = mbar_wait(&tfull[acc], acc_phase, args.status);
+      const bool got = mbar_wait(&tfull[acc], acc_phase, args.status);
+      // the whole part has its accumulator and free slots, or gives up together
+      if (!part_bar_and(part, got)) break;
+      bool got_skip = true;
       if (EPI == kEpiResidual && live) {
-        got = mbar_wait(sbar, skip_phase, args.status) && got;
+        got_skip = mbar_wait(sbar, skip_phase, args.status);
         skip_phase ^= 1;
       }
-      if (!__all_sync(0xffffffffu, got)) break;  // warp-uniform give-up
       tc_fence_after();
       const uint32_t tbase = tlane + (uint32_t)(acc * BN);
       if (req == kReqFast)
-        epi_tile<EPI, NARROW, kReqFast>(tbase, c_begin, n, kc, args, gelu_tab, slot_w, sel2, sel1);
+        epi_tile<EPI, NARROW, kReqFast>(tbase, c_begin, n, kc, args, gelu_tab, slots, ofs_even, ofs_odd, sel2, sel1);
       else if (req == kReqWide)
-        epi_tile<EPI, NARROW, kReqWide>(tbase, c_begin, n, kc, args, gelu_tab, slot_w, sel2, sel1);
+        epi_tile<EPI, NARROW, kReqWide>(tbase, c_begin, n, kc, args, gelu_tab, slots, ofs_even, ofs_odd, sel2, sel1);
       else
-        epi_tile<EPI, NARROW, kReqWideClamp>(tbase, c_begin, n, kc, args, gelu_tab, slot_w, sel2, sel1);
-      // staged words -> global by TMA (rows past M and channels past N are clipped)
+        epi_tile<EPI, NARROW, kReqWideClamp>(tbase, c_begin, n, kc, args, gelu_tab, slots, ofs_even, ofs_odd, sel2,
+                                             sel1);
+      // staged words -> global by TMA once the part's four warps have written
+      // them (rows past M and channels past N are clipped)
       fence_proxy_async_smem();
-      __syncwarp();
-      if (live && lane == 0) {
+      if (!part_bar_and(part, got_skip)) break;
+      if (live && part_lead) {
         for (int i = 0; i < n; ++i)
-          tma_store_2d(&tmY, ch0, (int32_t)(tok_base + 16 * (c_begin + i)), slots + i * kSlotBytes);
+          tma_store_2d(&tmY, tile_ch, (int32_t)(tok_base + 16 * (c_begin + i)), slots + i * kSlotBytes);
         bulk_commit_group();
       }
       // preload the bias of the tile that next accumulates in this buffer
-      const int t2 = t + 2 * (int)gridDim.x;
-      if (t2 < num_tiles) bias_fill(tbase, c_begin, c_end, bias_of(t2));
+      if (t + 2 * (int)gridDim.x < num_tiles) bias_fill(tbase, c_begin, c_end, next_bias);
       tmem_st_wait();
       tc_fence_before();
       __syncwarp();
@@ -494,7 +537,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       acc ^= 1;
       if (acc == 0) acc_phase ^= 1;
     }
-    if (lane == 0) bulk_wait_all();
+    if (part_lead) bulk_wait_all();
     __syncwarp();
   }
 
@@ -519,11 +562,11 @@ ivit_status run_gemm(const DeviceCtx& dc, const int8_t* X, const int8_t* W, cons
   st = encode_tmap_2d_u8(&tmX, X, (uint64_t)a.K, (uint64_t)a.M, (uint64_t)a.K, kBK, BN,
                          CU_TENSOR_MAP_SWIZZLE_128B);
   if (st != IVIT_OK) return st;
-  st = encode_tmap_2d_u8(&tmY, Y, (uint64_t)a.N, (uint64_t)a.M, (uint64_t)a.N, 32, 16, CU_TENSOR_MAP_SWIZZLE_NONE);
+  st = encode_tmap_2d_u8(&tmY, Y, (uint64_t)a.N, (uint64_t)a.M, (uint64_t)a.N, kBM, 16, CU_TENSOR_MAP_SWIZZLE_128B);
   if (st != IVIT_OK) return st;
   if (EPI == kEpiResidual) {
-    st = encode_tmap_2d_u8(&tmS, skip, (uint64_t)a.N, (uint64_t)a.M, (uint64_t)a.N, 32, 16,
-                           CU_TENSOR_MAP_SWIZZLE_NONE);
+    st = encode_tmap_2d_u8(&tmS, skip, (uint64_t)a.N, (uint64_t)a.M, (uint64_t)a.N, kBM, 16,
+                           CU_TENSOR_MAP_SWIZZLE_128B);
     if (st != IVIT_OK) return st;
   } else {
     tmS = tmY;  // unused
