@@ -392,7 +392,28 @@ IVIT_DEV void tmem_stream16(uint32_t taddr, int n, F&& body) {
   uint32_t r[16];
   for (int k = 0; k < n; ++k) {
     tmem_ld16(taddr + (uint32_t)(16 * k), r);
-    tmem_ld_wait();
+    tmem_ld_wait_regs(r);
+    body(r, k);
+  }
+}
+
+// As tmem_stream16 with two chunks' loads per wait, for the passes whose
+// per-chunk work is light enough to keep 32 columns in registers.
+template <typename F>
+IVIT_DEV void tmem_stream16x2(uint32_t taddr, int n, F&& body) {
+  int k = 0;
+  for (; k + 1 < n; k += 2) {
+    uint32_t ra[16], rb[16];
+    tmem_ld16(taddr + (uint32_t)(16 * k), ra);
+    tmem_ld16(taddr + (uint32_t)(16 * (k + 1)), rb);
+    tmem_ld_wait_regs2(ra, rb);
+    body(ra, k);
+    body(rb, k + 1);
+  }
+  if (k < n) {
+    uint32_t r[16];
+    tmem_ld16(taddr + (uint32_t)(16 * k), r);
+    tmem_ld_wait_regs(r);
     body(r, k);
   }
 }
@@ -603,7 +624,7 @@ __global__ void __launch_bounds__(kPersistThreads, 1)
       // ---- pass 1: row maximum of the raw scores over the real keys
       int32_t m4[4] = {INT_MIN, INT_MIN, INT_MIN, INT_MIN};
       if (work) {
-        tmem_stream16(t_row + (uint32_t)cbase, nvalid, [&](uint32_t(&r)[16], int k) {
+        tmem_stream16x2(t_row + (uint32_t)cbase, nvalid, [&](uint32_t(&r)[16], int k) {
           const int lim = N - (cbase + 16 * k);
           if (lim >= 16) {
 #pragma unroll
@@ -644,7 +665,7 @@ __global__ void __launch_bounds__(kPersistThreads, 1)
         // (Dv e) >> pshift is one mul.hi by Dv 2^(32 - pshift) when Dv < 2^pshift
         const bool hip = pshift >= 1 && __all_sync(0xffffffffu, (uint64_t)dv < ((uint64_t)1 << pshift));
         const uint32_t dvh = hip ? dv << (32 - pshift) : 0u;
-        tmem_stream16(t_row + (uint32_t)cbase, nvalid, [&](uint32_t(&r)[16], int k) {
+        tmem_stream16x2(t_row + (uint32_t)cbase, nvalid, [&](uint32_t(&r)[16], int k) {
           const int col = cbase + 16 * k;
           uint32_t w[4];
           if (hip) {
