@@ -565,6 +565,14 @@ def kernel_breakdown(ivit, wl, dp, ws, xs, reps, dev):
     add("attention", lambda i: ivit.ivit_attention(qkv, B, N, H, p["logit"], p["k_s"], p["attn_I0"], p["attn_M"],
                                                    p["attn_k_out"], p["attn_out"], ctx_o),
         "alu", SHIFTMAX_OPS_PER_SCORE * B * H * N * N)
+    # the same attention with 16-bit logits (ShiftExp computed per score): the
+    # logit scale of the 8-bit block re-derived for a 16-bit grid
+    S_l16 = (1.0 / p["attn_I0"]) * 255.0 / 65535.0
+    logit16 = ivit.ivit_dyadic_from_double(p["logit"][0] / 2.0 ** p["logit"][1] * 65535.0 / 255.0)
+    I0_16 = ivit.ivit_i0_from_scale(S_l16)
+    add("attention_logits16", lambda i: ivit.ivit_attention(qkv, B, N, H, logit16, 16, I0_16, p["attn_M"],
+                                                            p["attn_k_out"], p["attn_out"], ctx_o),
+        "alu", SHIFTMAX_OPS_PER_SCORE * B * H * N * N, in_block=False)
     add("gemm_o_residual", lambda i: ivit.ivit_linear_requant(ctx, t["w_o"], t["bias_o"], t["b_o"], t["c_o"], y,
                                                               skip=xs[i % R], res=p["res1"]),
         "tensor", gemm(T, D, D))

@@ -126,8 +126,12 @@ ivit_status ivit_linear_shiftgelu(const int8_t *X, int64_t M, int32_t K, const i
  *   ctx_id = sat_8((out.b * sum_j P_ij V_jd) >> out.c) out ~ S_v 2^-(k_out-1) / S_ctx
  * qkv [B*N x 3*H*64] int8: columns [0, D) are Q (head h at h*64), [D, 2D) K,
  * [2D, 3D) V, D = H*64.  ctx [B*N x D] int8, heads concatenated.
- * Constraints: B, H >= 1; 1 <= N <= 640; 2 <= k_s <= 8; I0 >= 1;
- * k_out - 1 <= M <= 30; 1 <= k_out <= 8.                                   */
+ * Constraints: B, H >= 1; 1 <= N <= 640; 2 <= k_s <= 16; I0 >= 1;
+ * k_out - 1 <= M <= 30; 1 <= k_out <= 8.  Logits of up to 8 bits take
+ * ShiftExp from a table; wider ones (k_s > 8) compute it per score and need
+ * N <= 256 and n_max * I0 < 2^32, where n_max = m + ceil(m/2) - ceil(m/16)
+ * with m = 2^k_s - 1 is the largest -I_p (the floor division by I0 is then
+ * one exact mul.hi); otherwise IVIT_ERR_UNSUPPORTED, nothing enqueued.     */
 ivit_status ivit_attention(const int8_t *qkv, int32_t B, int32_t N, int32_t H, ivit_dyadic logit, int32_t k_s,
                            int32_t I0, int32_t M, int32_t k_out, ivit_dyadic out, int8_t *ctx,
                            ivit_stream_t stream);

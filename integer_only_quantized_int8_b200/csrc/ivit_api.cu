@@ -205,10 +205,11 @@ ivit_status ivit_attention(const int8_t* qkv, int32_t B, int32_t N, int32_t H, i
                            int32_t I0, int32_t M, int32_t k_out, ivit_dyadic out, int8_t* ctx,
                            ivit_stream_t stream) {
   if (!qkv || !ctx || !aligned16(qkv) || !aligned16(ctx)) return IVIT_ERR_INVALID_ARG;
-  if (B < 0 || N < 0 || H < 1 || k_s < 2 || k_s > 8 || !valid_shiftmax(I0, M, k_out) || !valid_dyadic(logit) ||
+  if (B < 0 || N < 0 || H < 1 || k_s < 2 || k_s > 16 || !valid_shiftmax(I0, M, k_out) || !valid_dyadic(logit) ||
       !valid_dyadic(out))
     return IVIT_ERR_INVALID_ARG;
-  if (N > 640 || (int64_t)B * N > 0x7fffff00LL || H > 4096) return IVIT_ERR_UNSUPPORTED;
+  if (N > 640 || (int64_t)B * N > 0x7fffff00LL || H > 4096 || !attention_config_supported(N, k_s, I0))
+    return IVIT_ERR_UNSUPPORTED;
   if (B == 0 || N == 0) return IVIT_OK;
   DeviceCtx dc;
   ivit_status st = device_ctx(&dc);
@@ -265,12 +266,13 @@ ivit_status ivit_block_forward(const ivit_block_params* p, const int8_t* x, int8
   if (!p->ln1_gamma || !p->ln1_beta || !p->w_qkv || !p->b_qkv || !p->c_qkv || !p->w_o || !p->b_o || !p->c_o ||
       !p->ln2_gamma || !p->ln2_beta || !p->w1 || !p->b1 || !p->c1 || !p->w2 || !p->b2 || !p->c2)
     return IVIT_ERR_INVALID_ARG;
-  if (p->k_s < 2 || p->k_s > 8 || !valid_shiftmax(p->attn_I0, p->attn_M, p->attn_k_out) ||
+  if (p->k_s < 2 || p->k_s > 16 || !valid_shiftmax(p->attn_I0, p->attn_M, p->attn_k_out) ||
       !valid_shiftmax(p->gelu_I0, p->gelu_M, p->gelu_k_out) || !valid_dyadic(p->logit) ||
       !valid_dyadic(p->attn_out) || !valid_dyadic(p->gelu_out) || !valid_dyadic(p->ln1_out) ||
       !valid_dyadic(p->ln2_out) || !valid_residual(p->res1) || !valid_residual(p->res2) || p->ln_F < 0 ||
       p->ln_F > 14 || p->ln_M < p->ln_F || p->ln_M > 23)
     return IVIT_ERR_INVALID_ARG;
+  if (!attention_config_supported(N, p->k_s, p->attn_I0)) return IVIT_ERR_UNSUPPORTED;
   DeviceCtx dc;
   ivit_status st = device_ctx(&dc);
   if (st != IVIT_OK) return st;

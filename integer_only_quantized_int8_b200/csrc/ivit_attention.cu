@@ -39,6 +39,7 @@ struct AttnArgs {
   int32_t o_lo, o_hi;  // accumulator clamp of the output requant (see out_clamp)
   int32_t out_bq;      // b_o 2^(32 - c_o) when that fits a positive int32 (then the requant is one mul.hi), else 0
   int32_t out_fast;
+  uint32_t exp_magic;  // ceil(2^32 / I0) for the arithmetic ShiftExp of logits wider than 8 bits (0 when I0 = 1)
   int8_t* ctx;
   int* status;
 };
@@ -310,6 +311,17 @@ __global__ void __launch_bounds__(kAttnThreads)
 // P V lands in the first 64 columns of the item's S buffer, dead by then.
 // ---------------------------------------------------------------------------
 constexpr int kShortMaxKeys = 256;
+constexpr int kTableMaxBits = 8;  // ShiftExp by table up to 8-bit logits, computed beyond
+
+// The arithmetic ShiftExp divides n = -I_p by I0 with one mul.hi, exact while
+// n I0 < 2^32.  Over k_s-bit logits |L - max L| <= 2^k_s - 1 = m, and
+// -I_p = m' + ceil(m'/2) - ceil(m'/16) at |d| = m' never decreases in m', so
+// its largest value is at m' = m.
+inline bool shift_exp_alu_exact(int32_t k_s, int32_t I0) {
+  const int64_t m = ((int64_t)1 << k_s) - 1;
+  const int64_t nmax = m + (m + 1) / 2 - (m + 15) / 16;
+  return nmax * (int64_t)I0 < ((int64_t)1 << 32);
+}
 constexpr int kSoftWarps = 8;    // per softmax group
 constexpr int kSoftGroups = 2;   // groups take alternate items, one TMEM buffer each
 constexpr int kLoadStages = 3;
@@ -418,12 +430,26 @@ IVIT_DEV void tmem_stream16x2(uint32_t taddr, int n, F&& body) {
   }
 }
 
-// Pass 2 of one half row: e = ShiftExp(L - max L) by table, written back to
-// TMEM in place; returns the partial row sum.  tb = table + lane + 32 lmax,
-// so tb[-32 L] = ShiftExp(L - lmax).  UPPER: some row of the warp has a raw
-// logit maximum above the k_s-bit range, so the upper saturation is needed
-// (otherwise every logit of the row is at most lmax already).
-template <bool FASTQ, bool UPPER>
+// ShiftExp(d), d <= 0, computed: the same steps as shift_exp, with the floor
+// division of n = -I_p by I0 done as one mul.hi by ceil(2^32 / I0), which is
+// exact while n I0 < 2^32 (the host checks that bound for the logit width;
+// I0 = 1 divides by itself).
+IVIT_DEV uint32_t shift_exp_alu(int32_t d, int32_t I0, uint32_t magic) {
+  const int32_t ip = d + (d >> 1) - (d >> 4);
+  const uint32_t n = (uint32_t)(-ip);
+  const uint32_t q = magic != 0u ? __umulhi(n, magic) : n;
+  const int32_t r = (int32_t)(n - q * (uint32_t)I0);
+  const int32_t t = I0 - ((r + 1) >> 1);  // I0 + floor(-r / 2) >= 1
+  return (uint32_t)t >> min(q, 31u);      // t < 2^31: a shift by 31 gives 0, as every q >= 31 must
+}
+
+// Pass 2 of one half row: e = ShiftExp(L - max L) by table (ALU: computed),
+// written back to TMEM in place; returns the partial row sum.  tb = table +
+// lane + 32 lmax, so tb[-32 L] = ShiftExp(L - lmax).  UPPER: some row of the
+// warp has a raw logit maximum above the k_s-bit range, so the upper
+// saturation is needed (otherwise every logit of the row is at most lmax
+// already).
+template <bool FASTQ, bool UPPER, bool ALU>
 IVIT_DEV uint32_t shiftmax_pass2(uint32_t t_row, int cbase, int nvalid, int N, const int32_t* tb, int32_t lmax,
                                  int32_t bq, const AttnArgs& a) {
   uint32_t s4[4] = {0u, 0u, 0u, 0u};
@@ -435,7 +461,7 @@ IVIT_DEV uint32_t shiftmax_pass2(uint32_t t_row, int cbase, int nvalid, int N, c
       for (int e = 0; e < 16; ++e) {
         int32_t l = max(logit_unclamped<FASTQ>((int32_t)r[e], bq, a.logit_b, a.logit_c), a.ks_lo);
         if (UPPER || !FASTQ) l = min(l, a.ks_hi);
-        const uint32_t x = (uint32_t)tb[-32 * l];
+        const uint32_t x = ALU ? shift_exp_alu(l - lmax, a.I0, a.exp_magic) : (uint32_t)tb[-32 * l];
         s4[e & 3] += x;
         r[e] = x;
       }
@@ -444,7 +470,7 @@ IVIT_DEV uint32_t shiftmax_pass2(uint32_t t_row, int cbase, int nvalid, int N, c
       for (int e = 0; e < 16; ++e) {
         // padding keys: any index in range, then masked
         const int32_t l = min(max(logit_unclamped<FASTQ>((int32_t)r[e], bq, a.logit_b, a.logit_c), a.ks_lo), lmax);
-        const uint32_t x = e < lim ? (uint32_t)tb[-32 * l] : 0u;
+        const uint32_t x = e < lim ? (ALU ? shift_exp_alu(l - lmax, a.I0, a.exp_magic) : (uint32_t)tb[-32 * l]) : 0u;
         s4[e & 3] += x;
         r[e] = x;
       }
@@ -455,7 +481,9 @@ IVIT_DEV uint32_t shiftmax_pass2(uint32_t t_row, int cbase, int nvalid, int N, c
   return (s4[0] + s4[1]) + (s4[2] + s4[3]);
 }
 
-template <bool FASTQ>
+// ALU: logits wider than 8 bits, ShiftExp computed per score instead of
+// looked up (the table would not fit).
+template <bool FASTQ, bool ALU>
 __global__ void __launch_bounds__(kPersistThreads, 1)
     attention_persist_kernel(const __grid_constant__ CUtensorMap tm, const AttnArgs a, const int32_t bq) {
   extern __shared__ uint8_t smem_raw[];
@@ -505,7 +533,7 @@ __global__ void __launch_bounds__(kPersistThreads, 1)
   // one evaluation per entry (staged in the partials area), then copies in
   // consecutive 16-byte chunks
   int32_t* stage_t = reinterpret_cast<int32_t*>(smem + L.part_off);
-  if (tid < (1 << a.k_s)) stage_t[tid] = shift_exp(-tid, a.I0);
+  if (!ALU && tid < (1 << a.k_s)) stage_t[tid] = shift_exp(-tid, a.I0);
   if (warp == 1) {
     __syncwarp();
     tmem_alloc(tslot, 512);
@@ -514,7 +542,7 @@ __global__ void __launch_bounds__(kPersistThreads, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  for (int i4 = tid; i4 < (8 << a.k_s); i4 += kPersistThreads) {
+  for (int i4 = tid; !ALU && i4 < (8 << a.k_s); i4 += kPersistThreads) {
     const int32_t e = stage_t[i4 >> 3];
     reinterpret_cast<int4*>(tab)[i4] = make_int4(e, e, e, e);
   }
@@ -648,9 +676,9 @@ __global__ void __launch_bounds__(kPersistThreads, 1)
       if (work) {
         const int32_t* tb = tab + lane + lmax * 32;
         if (__any_sync(0xffffffffu, vmax > a.ks_hi))
-          sum = shiftmax_pass2<FASTQ, true>(t_row, cbase, nvalid, N, tb, lmax, bq, a);
+          sum = shiftmax_pass2<FASTQ, true, ALU>(t_row, cbase, nvalid, N, tb, lmax, bq, a);
         else
-          sum = shiftmax_pass2<FASTQ, false>(t_row, cbase, nvalid, N, tb, lmax, bq, a);
+          sum = shiftmax_pass2<FASTQ, false, ALU>(t_row, cbase, nvalid, N, tb, lmax, bq, a);
       }
       part[half * 256 + 128 + row] = (int32_t)sum;
       softmax_bar(group);
@@ -756,6 +784,11 @@ __global__ void __launch_bounds__(kPersistThreads, 1)
 
 }  // namespace
 
+bool attention_config_supported(int32_t N, int32_t k_s, int32_t I0) {
+  if (N > kMaxKeys) return false;
+  return k_s <= kTableMaxBits || (N <= kShortMaxKeys && shift_exp_alu_exact(k_s, I0));
+}
+
 ivit_status launch_attention(const DeviceCtx& dc, const int8_t* qkv, int32_t B, int32_t N, int32_t H,
                              ivit_dyadic logit, int32_t k_s, int32_t I0, int32_t M, int32_t k_out,
                              ivit_dyadic out, int8_t* ctx, cudaStream_t stream) {
@@ -799,6 +832,10 @@ ivit_status launch_attention(const DeviceCtx& dc, const int8_t* qkv, int32_t B, 
   }
   a.out_fast = out.c >= 1 && (int64_t)out.b < ((int64_t)1 << (out.c - 1));
   a.out_bq = a.out_fast ? (int32_t)((int64_t)out.b << (32 - out.c)) : 0;
+  // logits wider than 8 bits: arithmetic ShiftExp on the short-sequence path only
+  const bool alu = k_s > kTableMaxBits;
+  if (!attention_config_supported(N, k_s, I0)) return IVIT_ERR_UNSUPPORTED;
+  a.exp_magic = I0 > 1 ? (uint32_t)((((uint64_t)1 << 32) + (uint64_t)I0 - 1) / (uint64_t)I0) : 0u;
   a.ctx = ctx;
   a.status = dc.status;
   dim3 grid((unsigned)((N + kQTile - 1) / kQTile), (unsigned)H, (unsigned)B);
@@ -810,9 +847,13 @@ ivit_status launch_attention(const DeviceCtx& dc, const int8_t* qkv, int32_t B, 
     const int32_t bq = fastq ? (int32_t)((int64_t)logit.b << (32 - logit.c)) : 0;
     static bool attr_persist = false;
     if (!attr_persist) {
-      if (cudaFuncSetAttribute(attention_persist_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+      if (cudaFuncSetAttribute(attention_persist_kernel<true, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                227 * 1024) != cudaSuccess ||
-          cudaFuncSetAttribute(attention_persist_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+          cudaFuncSetAttribute(attention_persist_kernel<false, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               227 * 1024) != cudaSuccess ||
+          cudaFuncSetAttribute(attention_persist_kernel<true, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               227 * 1024) != cudaSuccess ||
+          cudaFuncSetAttribute(attention_persist_kernel<false, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                227 * 1024) != cudaSuccess)
         return IVIT_ERR_CUDA;
       attr_persist = true;
@@ -820,10 +861,9 @@ ivit_status launch_attention(const DeviceCtx& dc, const int8_t* qkv, int32_t B, 
     const int64_t items = (int64_t)((N + kQTile - 1) / kQTile) * H * B;
     if (items > 0x7fffffff) return IVIT_ERR_UNSUPPORTED;
     const unsigned pgrid = (unsigned)(items < dc.num_sms ? items : dc.num_sms);
-    const cudaError_t e =
-        fastq ? launch_pdl(attention_persist_kernel<true>, dim3(pgrid), dim3(kPersistThreads), smem, stream, tm, a, bq)
-              : launch_pdl(attention_persist_kernel<false>, dim3(pgrid), dim3(kPersistThreads), smem, stream, tm, a,
-                           bq);
+    auto kern = fastq ? (alu ? attention_persist_kernel<true, true> : attention_persist_kernel<true, false>)
+                      : (alu ? attention_persist_kernel<false, true> : attention_persist_kernel<false, false>);
+    const cudaError_t e = launch_pdl(kern, dim3(pgrid), dim3(kPersistThreads), smem, stream, tm, a, bq);
     note_launch();
     return e == cudaSuccess ? IVIT_OK : IVIT_ERR_CUDA;
   }

@@ -55,6 +55,11 @@ ivit_status launch_gemm(const DeviceCtx& dc, const int8_t* X, int64_t M, int32_t
                         const int8_t* skip, ivit_residual res, const GeluParams* gelu, int8_t* Y,
                         cudaStream_t stream);
 
+// Whether the attention kernels take (N, k_s, I0): up to 640 keys; logits
+// wider than 8 bits (ShiftExp computed, not looked up) on up to 256 keys and
+// with (largest -I_p) * I0 < 2^32.
+bool attention_config_supported(int32_t N, int32_t k_s, int32_t I0);
+
 ivit_status launch_attention(const DeviceCtx& dc, const int8_t* qkv, int32_t B, int32_t N, int32_t H,
                              ivit_dyadic logit, int32_t k_s, int32_t I0, int32_t M, int32_t k_out,
                              ivit_dyadic out, int8_t* ctx, cudaStream_t stream);

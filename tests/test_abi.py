@@ -80,7 +80,9 @@ def test_validation_rejects_before_launch():
     assert L.ivit_linear_requant(p, 16, 24, p, 16, None, p, p, 8, None, none, p, None) == 1   # K % 16
     assert L.ivit_linear_requant(p, 16, 16, p, 16, None, p, p, 9, None, none, p, None) == 1   # out_bits
     d = ivit.Dyadic(1, 0)
-    assert L.ivit_attention(p, 1, 8, 1, d, 9, 4, 30, 8, d, p, None) == 1      # k_s > 8
+    assert L.ivit_attention(p, 1, 8, 1, d, 17, 4, 30, 8, d, p, None) == 1     # k_s > 16
+    assert L.ivit_attention(p, 1, 300, 1, d, 12, 4, 30, 8, d, p, None) == 2   # wide logits past 256 keys
+    assert L.ivit_attention(p, 1, 8, 1, d, 16, 50000, 30, 8, d, p, None) == 2  # n_max * I0 >= 2^32
     assert L.ivit_attention(p, 1, 8, 1, d, 8, 0, 30, 8, d, p, None) == 1      # I0 < 1
     assert L.ivit_attention(p, 1, 8, 1, d, 8, 4, 31, 8, d, p, None) == 1      # M > 30
     assert L.ivit_attention(p, 1, 641, 1, d, 8, 4, 30, 8, d, p, None) == 2    # too many keys

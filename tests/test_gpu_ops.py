@@ -94,6 +94,9 @@ ATTN_CASES = [
     (1, 1, 1, "normal", 8), (2, 5, 1, "normal", 8), (2, 197, 3, "normal", 8), (1, 577, 2, "laplace", 8),
     (3, 130, 2, "normal", 8), (1, 128, 1, "laplace", 8), (2, 256, 1, "normal", 8), (1, 300, 1, "laplace", 8),
     (1, 640, 1, "laplace", 8), (2, 197, 2, "laplace", 4), (1, 33, 2, "normal", 6),
+    # logits wider than 8 bits: ShiftExp computed per score
+    (2, 197, 3, "normal", 16), (1, 256, 2, "laplace", 16), (2, 5, 1, "normal", 12), (3, 130, 2, "laplace", 12),
+    (1, 33, 2, "normal", 10),
 ]
 
 
@@ -108,6 +111,19 @@ def test_attention_parity(B, N, H, tails, k_s):
     ivit.ivit_attention(qkv, B, N, H, logit_d, k_s, I0_d, 30, 8, out_d, ctx)
     want = oracle.attention(ac.qkv, B, N, H, logit_o, k_s, I0_o, 30, 8, out_o)
     np.testing.assert_array_equal(host(ctx), want)
+
+
+@pytest.mark.parametrize("k_s", [8, 12, 16])
+def test_attention_hardmax_wide_logits(k_s):
+    """I_0 = 1 (the division by I_0 is the identity) and (b_s, c_s) = (1, 0):
+    every key below the row maximum gets ShiftExp 0, at any logit width."""
+    r = np.random.default_rng(40 + k_s)
+    B, N, H = 2, 61, 2
+    D = H * 64
+    qkv = r.integers(-3, 5, size=(B * N, 3 * D)).astype(np.int8)
+    ctx = torch.full((B * N, D), 99, dtype=torch.int8, device="cuda")
+    ivit.ivit_attention(dev(qkv, torch.int8), B, N, H, (1, 0), k_s, 1, 30, 8, (1, 4), ctx)
+    np.testing.assert_array_equal(host(ctx), oracle.attention(qkv, B, N, H, (1, 0), k_s, 1, 30, 8, (1, 4)))
 
 
 @pytest.mark.parametrize("I0,M,k_out", [(1, 30, 8), (3, 20, 8), (97, 30, 5), (4096, 30, 8)])

@@ -402,7 +402,7 @@ def test_attention_hardmax_reduces_to_argmax():
     B, N, H = 2, 19, 2
     D = H * 64
     qkv = _qkv(r, B, N, H, -3, 4)
-    for k_s in (8, 4):
+    for k_s in (8, 4, 16):
         ctx = oracle.attention(qkv, B, N, H, (1, 0), k_s, 1, 30, 8, (1, 4))
         lim = 2 ** (k_s - 1)
         for b in range(B):
