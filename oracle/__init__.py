@@ -111,6 +111,14 @@ def lib():
             L.orc_layernorm.restype = None
             L.orc_layernorm.argtypes = [C.c_void_p, C.c_int64, C.c_int32, C.c_void_p, C.c_void_p,
                                         C.c_int32, C.c_int32, C.c_int32, C.c_int32, C.c_void_p]
+            L.orc_patch_embed.restype = C.c_int
+            L.orc_patch_embed.argtypes = [C.c_void_p, C.c_int32, C.c_int32, C.c_int32, C.c_int32, C.c_int32,
+                                          C.c_void_p, C.c_void_p, C.c_void_p, C.c_void_p, C.c_int32,
+                                          C.c_void_p, C.c_void_p, C.c_int32, C.c_int32, C.c_int32, C.c_void_p]
+            L.orc_head.restype = C.c_int
+            L.orc_head.argtypes = [C.c_void_p, C.c_int32, C.c_int32, C.c_int32, C.c_void_p, C.c_void_p,
+                                   C.c_int32, C.c_int32, C.c_int32, C.c_int32, C.c_void_p, C.c_int32,
+                                   C.c_void_p, C.c_void_p, C.c_void_p, C.c_void_p]
             L.orc_block_forward.restype = C.c_int
             L.orc_block_forward.argtypes = [C.POINTER(BlockParamsC), C.c_void_p, C.c_void_p,
                                             C.c_int32, C.c_int32]
@@ -316,3 +324,54 @@ def block_forward(p, x, B: int, N: int):
     if rc != 0:
         raise MemoryError("oracle block forward could not allocate scratch")
     return y
+
+
+# ---------------------------------------------------------------------------
+# steps either side of the blocks
+# ---------------------------------------------------------------------------
+
+def patch_embed(img, P: int, W, bias, b, c, cls, pos, add):
+    """img [B x C x Hi x Wi] int8 -> tokens [B*(Np+1) x D] int8.
+
+    Flattened P x P patches through an int8 linear layer (W [D x C*P*P]),
+    the class token first, then the position embedding added with the
+    two-scale dyadic pair ``add`` = (b_u, b_v, c)."""
+    img = np.ascontiguousarray(img, dtype=np.int8)
+    B, Cin, Hi, Wi = img.shape
+    W = np.ascontiguousarray(W, dtype=np.int8)
+    D = W.shape[0]
+    assert W.shape[1] == Cin * P * P and Hi % P == 0 and Wi % P == 0
+    Np = (Hi // P) * (Wi // P)
+    bias = None if bias is None else np.ascontiguousarray(bias, dtype=np.int32)
+    b = np.ascontiguousarray(b, dtype=np.int32)
+    c = np.ascontiguousarray(c, dtype=np.int32)
+    cls = np.ascontiguousarray(cls, dtype=np.int8)
+    pos = np.ascontiguousarray(pos, dtype=np.int8)
+    assert cls.shape == (D,) and pos.shape == (Np + 1, D)
+    x = np.zeros((B * (Np + 1), D), dtype=np.int8)
+    if lib().orc_patch_embed(img.ctypes.data, B, Cin, Hi, Wi, P, W.ctypes.data,
+                             None if bias is None else bias.ctypes.data, b.ctypes.data, c.ctypes.data, D,
+                             cls.ctypes.data, pos.ctypes.data, int(add[0]), int(add[1]), int(add[2]),
+                             x.ctypes.data) != 0:
+        raise MemoryError("orc_patch_embed")
+    return x
+
+
+def head(x, B: int, Ntok: int, gamma, beta, F: int, M_ln: int, ln_out, W, bias, b, c):
+    """x [B*Ntok x D] int8 -> logits [B x Ncls] int8 (class token, LN, linear)."""
+    x = np.ascontiguousarray(x, dtype=np.int8)
+    D = x.shape[1]
+    W = np.ascontiguousarray(W, dtype=np.int8)
+    Ncls = W.shape[0]
+    gamma = np.ascontiguousarray(gamma, dtype=np.int8)
+    beta = np.ascontiguousarray(beta, dtype=np.int32)
+    bias = None if bias is None else np.ascontiguousarray(bias, dtype=np.int32)
+    b = np.ascontiguousarray(b, dtype=np.int32)
+    c = np.ascontiguousarray(c, dtype=np.int32)
+    out = np.zeros((B, Ncls), dtype=np.int8)
+    if lib().orc_head(x.ctypes.data, B, Ntok, D, gamma.ctypes.data, beta.ctypes.data, int(F), int(M_ln),
+                      int(ln_out[0]), int(ln_out[1]), W.ctypes.data, Ncls,
+                      None if bias is None else bias.ctypes.data, b.ctypes.data, c.ctypes.data,
+                      out.ctypes.data) != 0:
+        raise MemoryError("orc_head")
+    return out

@@ -482,3 +482,90 @@ int orc_block_forward(const orc_block_params *p, const int8_t *x, int8_t *y,
     free(ln); free(qkv); free(ctx); free(xh); free(h); free(g);
     return 0;
 }
+
+/* ------------------------------------------------------------------------ */
+/* Steps either side of the encoder blocks: patch embedding and classifier  */
+/* head.  [IVIT] 3.1 quantises every linear layer of the ViT with the same  */
+/* int8 x int8 -> int32 -> dyadic scheme; READING: the patch projection (a  */
+/* P x P convolution with stride P, i.e. a linear layer over flattened      */
+/* patches) and the classifier are two more such layers, and the position   */
+/* embedding joins the tokens through the same two-scale dyadic addition as */
+/* the residual connections.                                                */
+/* ------------------------------------------------------------------------ */
+
+/*
+ * Patch embedding of int8 images img [B x C x Hi x Wi] (NCHW; Hi, Wi
+ * multiples of P), Np = (Hi/P)(Wi/P) patches in row-major patch order.  The
+ * patch at (py, px) flattens to z[(ch * P + ky) * P + kx] =
+ * img[b, ch, py P + ky, px P + kx] (the [D x C x P x P] layout of a
+ * convolution weight), and
+ *   e[b, p] = linear_requant(z, W [D x C P P], bias, b_e, c_e)   (int8)
+ * The Np + 1 tokens of image b are
+ *   x[b, 0]     = sat_8((b_u cls      + b_v pos[0])     >> c_add)
+ *   x[b, 1 + p] = sat_8((b_u e[b, p]  + b_v pos[1 + p]) >> c_add)
+ * READING: the class token cls [D] is held at the embedding scale, so one
+ * dyadic pair serves both rows; pos is [(Np + 1) x D] int8 at its own scale.
+ * Returns 0, or -1 if scratch allocation failed.
+ */
+int orc_patch_embed(const int8_t *img, int32_t B, int32_t C, int32_t Hi, int32_t Wi,
+                    int32_t P, const int8_t *W, const int32_t *bias, const int32_t *b_e,
+                    const int32_t *c_e, int32_t D, const int8_t *cls, const int8_t *pos,
+                    int32_t b_u, int32_t b_v, int32_t c_add, int8_t *x)
+{
+    const int32_t gy = Hi / P, gx = Wi / P, Np = gy * gx, K = C * P * P;
+    int8_t *z = (int8_t *)malloc((size_t)Np * (size_t)K);
+    int8_t *e = (int8_t *)malloc((size_t)Np * (size_t)D);
+    if (!z || !e) {
+        free(z); free(e);
+        return -1;
+    }
+    for (int32_t bi = 0; bi < B; ++bi) {
+        for (int32_t py = 0; py < gy; ++py)
+            for (int32_t px = 0; px < gx; ++px)
+                for (int32_t ch = 0; ch < C; ++ch)
+                    for (int32_t ky = 0; ky < P; ++ky)
+                        for (int32_t kx = 0; kx < P; ++kx) {
+                            const int64_t src = (((int64_t)bi * C + ch) * Hi + py * P + ky) * Wi +
+                                                px * P + kx;
+                            z[(int64_t)(py * gx + px) * K + (ch * P + ky) * P + kx] = img[src];
+                        }
+        orc_linear_requant(z, Np, K, W, D, bias, b_e, c_e, 8, NULL, 0, 0, 0, e);
+        int8_t *xb = x + (int64_t)bi * (Np + 1) * D;
+        for (int32_t t = 0; t <= Np; ++t)
+            for (int32_t j = 0; j < D; ++j) {
+                const int64_t u = t == 0 ? cls[j] : e[(int64_t)(t - 1) * D + j];
+                const int64_t v = pos[(int64_t)t * D + j];
+                xb[(int64_t)t * D + j] =
+                    (int8_t)sat_bits(shr_floor((int64_t)b_u * u + (int64_t)b_v * v, c_add), 8);
+            }
+    }
+    free(z);
+    free(e);
+    return 0;
+}
+
+/*
+ * Classifier head: the class token of every image (row 0 of its Ntok rows
+ * in x [B*Ntok x D]), I-LayerNorm, then an int8 linear layer to Ncls int8
+ * logits [B x Ncls].  Returns 0, or -1 if scratch allocation failed.
+ */
+int orc_head(const int8_t *x, int32_t B, int32_t Ntok, int32_t D, const int8_t *gamma,
+             const int32_t *beta, int32_t F, int32_t M_ln, int32_t ln_b, int32_t ln_c,
+             const int8_t *W, int32_t Ncls, const int32_t *bias, const int32_t *b,
+             const int32_t *c, int8_t *logits)
+{
+    int8_t *t = (int8_t *)malloc((size_t)B * (size_t)D);
+    int8_t *n = (int8_t *)malloc((size_t)B * (size_t)D);
+    if (!t || !n) {
+        free(t); free(n);
+        return -1;
+    }
+    for (int32_t bi = 0; bi < B; ++bi)
+        for (int32_t j = 0; j < D; ++j)
+            t[(int64_t)bi * D + j] = x[(int64_t)bi * Ntok * D + j];
+    orc_layernorm(t, B, D, gamma, beta, F, M_ln, ln_b, ln_c, n);
+    orc_linear_requant(n, B, D, W, Ncls, bias, b, c, 8, NULL, 0, 0, 0, logits);
+    free(t);
+    free(n);
+    return 0;
+}

@@ -457,3 +457,73 @@ def test_block_is_composition_of_ops():
     np.testing.assert_array_equal(oracle.block_forward(p, x, B, N), y)
     # the calibrated block is not degenerate: outputs use the int8 range
     assert np.unique(y).size > 50 and np.unique(g).size > 20 and np.unique(ctx).size > 50
+
+
+# ---------------------------------------------------------------------------
+# steps either side of the blocks: patch embedding and classifier head
+# ---------------------------------------------------------------------------
+
+def test_patch_embed_is_a_strided_convolution():
+    """The patch path equals a P x P convolution with stride P computed
+    directly from the image (weights viewed as [D x C x P x P]), requantised by
+    a power-of-two shift; with the position term off (b_v = 0, c = 0, b_u = 1)
+    the tokens are the class token then the patches in row-major order."""
+    r = np.random.default_rng(31)
+    B, Cin, Hi, Wi, P, D = 2, 3, 32, 48, 16, 32
+    img = r.integers(-128, 128, (B, Cin, Hi, Wi), dtype=np.int8)
+    W = r.integers(-4, 5, (D, Cin * P * P), dtype=np.int8)
+    bias = r.integers(-3000, 3000, D).astype(np.int32)
+    sh = 9
+    cls = r.integers(-128, 128, D, dtype=np.int8)
+    pos = r.integers(-128, 128, ((Hi // P) * (Wi // P) + 1, D), dtype=np.int8)
+    x = oracle.patch_embed(img, P, W, bias, np.ones(D, np.int32), np.full(D, sh, np.int32), cls, pos, (1, 0, 0))
+    Wc = W.reshape(D, Cin, P, P).astype(np.int64)
+    Np = (Hi // P) * (Wi // P)
+    xs = x.reshape(B, Np + 1, D)
+    for b in range(B):
+        np.testing.assert_array_equal(xs[b, 0], cls)
+        for py in range(Hi // P):
+            for px in range(Wi // P):
+                blk = img[b, :, py * P:(py + 1) * P, px * P:(px + 1) * P].astype(np.int64)
+                acc = np.einsum("cyx,dcyx->d", blk, Wc) + bias
+                want = np.clip(np.right_shift(acc, sh), -128, 127)
+                np.testing.assert_array_equal(xs[b, 1 + py * (Wi // P) + px], want)
+
+
+def test_patch_embed_position_term_closed_forms():
+    """W = 0, bias = 0 and a zero class token make every embedding 0, so the
+    tokens are sat_8((b_v pos) >> c): b_v = 2^c gives pos itself for every
+    image; with b_u = b_v = 2^c and W = 0 the class row is sat_8(cls + pos)."""
+    r = np.random.default_rng(32)
+    B, Cin, P, D = 3, 3, 16, 48
+    img = r.integers(-128, 128, (B, Cin, 32, 32), dtype=np.int8)
+    W = np.zeros((D, Cin * P * P), np.int8)
+    pos = r.integers(-128, 128, (5, D), dtype=np.int8)
+    ones, zc = np.ones(D, np.int32), np.zeros(D, np.int32)
+    x = oracle.patch_embed(img, P, W, None, ones, zc, np.zeros(D, np.int8), pos, (5, 8, 3))
+    np.testing.assert_array_equal(x.reshape(B, 5, D), np.broadcast_to(pos, (B, 5, D)))
+    cls = r.integers(-128, 128, D, dtype=np.int8)
+    x = oracle.patch_embed(img, P, W, None, ones, zc, cls, pos, (4, 4, 2))
+    want0 = np.clip(cls.astype(np.int64) + pos[0], -128, 127)
+    for b in range(B):
+        np.testing.assert_array_equal(x[b * 5], want0)
+        np.testing.assert_array_equal(x[b * 5 + 1:(b + 1) * 5], pos[1:])
+
+
+def test_head_takes_class_tokens_through_layernorm_and_linear():
+    """I-LayerNorm works row by row, so normalising every token and keeping
+    the class rows gives what the head computes on the class rows alone; the
+    head's linear layer is the pinned linear layer on those rows."""
+    r = np.random.default_rng(33)
+    B, Ntok, D, Ncls = 3, 7, 64, 48
+    x = r.integers(-128, 128, (B * Ntok, D), dtype=np.int8)
+    gamma = r.integers(-128, 128, D, dtype=np.int8)
+    beta = r.integers(-5000, 5000, D).astype(np.int32)
+    W = r.integers(-128, 128, (Ncls, D), dtype=np.int8)
+    bias = r.integers(-5000, 5000, Ncls).astype(np.int32)
+    b = r.integers(1, 1 << 20, Ncls).astype(np.int32)
+    c = np.full(Ncls, 27, np.int32)
+    got = oracle.head(x, B, Ntok, gamma, beta, 7, 23, (3, 12), W, bias, b, c)
+    ln_all = oracle.layernorm(x, gamma, beta, 7, 23, (3, 12))
+    want = oracle.linear_requant(ln_all[::Ntok], W, bias, b, c)
+    np.testing.assert_array_equal(got, want)
