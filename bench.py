@@ -61,6 +61,8 @@ def parse_args():
                     help="CPU-baseline sample: (image, block) units the oracle runs")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--kernel-reps", type=int, default=50)
+    ap.add_argument("--model-blocks", type=int, default=12,
+                    help="blocks of the whole-model timing (ViT-B workload only; 0 skips it)")
     return ap.parse_args()
 
 
@@ -374,6 +376,11 @@ def run_ours(args):
     # ---------------- per-kernel breakdown of block 0 (CUDA events, same stream)
     kern = kernel_breakdown(ivit, wl, dps[0], ws, xs, args.kernel_reps, dev)
 
+    # ---------------- a whole model on synthetic weights (rank 0, not part of the metric)
+    model = None
+    if world == 1 and args.model_blocks > 0 and wl.name == "vit_b_b64":
+        model = model_forward_timing(ivit, args.model_blocks, wl.B, dev)
+
     # ---------------- end to end through host buffers
     # Every step copies its batch from pinned host memory to the device, runs
     # the block(s) through the public API and copies the result back to pinned
@@ -493,8 +500,57 @@ def run_ours(args):
         "clocks": clocks,
         "gpu_launches": int(launches_per_step * args.steps),
     }
+    if model is not None:
+        line["model"] = model
     print(json.dumps(line), flush=True)
     return 0
+
+
+def model_forward_timing(ivit, n_blocks, B, dev, reps=10):
+    """Images/s of a whole ViT-B/16 at 224 x 224 on synthetic weights: patch
+    embedding, n_blocks encoder blocks with independent weights, classifier
+    head (1000 classes padded to 1008), one ivit_model_forward per batch,
+    replayed from a CUDA graph with the image batch resident on the device."""
+    import torch
+    import synthetic
+    from integer_only_quantized_int8_b200 import params as ivit_params
+    t0 = time.perf_counter()
+    mc = synthetic.model_case(B=B, Hi=224, Wi=224, P=16, D=768, H=12, Dm=3072, blocks=n_blocks, Ncls=1000, seed=3)
+    dm = ivit_params.model_to_device(ivit_params.model_integer_params(mc), dev)
+    setup_s = time.perf_counter() - t0
+    img = torch.from_numpy(mc.img).to(dev)
+    ws = torch.empty(ivit.ivit_model_workspace_bytes(dm, B, 224, 224), dtype=torch.uint8, device=dev)
+    logits = torch.empty((B, mc.w_head.shape[0]), dtype=torch.int8, device=dev)
+    for _ in range(3):
+        ivit.ivit_model_forward(dm, img, ws, logits)
+    torch.cuda.synchronize()
+    n0 = ivit.ivit_launch_count()
+    ivit.ivit_model_forward(dm, img, ws, logits)
+    launches = ivit.ivit_launch_count() - n0
+    g = torch.cuda.CUDAGraph()
+    s = torch.cuda.Stream(device=dev)
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        with torch.cuda.graph(g, stream=s):
+            ivit.ivit_model_forward(dm, img, ws, logits)
+    torch.cuda.current_stream().wait_stream(s)
+    for _ in range(3):
+        g.replay()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(reps):
+        g.replay()
+    b.record()
+    torch.cuda.synchronize()
+    if ivit.ivit_stream_status() != 0:
+        raise SystemExit("a kernel reported a timed-out wait")
+    ms = a.elapsed_time(b) / reps
+    del g
+    return {"workload": f"ViT-B/16 224x224, {n_blocks} blocks, batch {B}, 1000 classes (padded to 1008)",
+            "images_per_s": B / (ms / 1e3), "ms_per_batch": ms, "gpu_launches_per_batch": int(launches),
+            "data": "synthetic (seeded image and independent random-init weights per block)",
+            "setup_s": setup_s}
 
 
 def kernel_breakdown(ivit, wl, dp, ws, xs, reps, dev):

@@ -258,6 +258,83 @@ ivit_status ivit_block_forward_static(const ivit_block_params *p, const int8_t *
                                       int32_t N, ivit_stream_t stream);
 
 /* ---------------------------------------------------------------------------
+ * Steps either side of the blocks.  [IVIT] 3.1 quantises every linear layer
+ * of the ViT with the same int8 x int8 -> int32 -> dyadic scheme; READING:
+ * the patch projection (a P x P convolution with stride P, i.e. a linear
+ * layer over flattened patches) and the classifier are two more such layers,
+ * and the position embedding joins the tokens through the same two-scale
+ * dyadic addition as the residual connections.
+ * ------------------------------------------------------------------------- */
+
+/* Bytes of device workspace ivit_patch_embed needs (flattened patches and
+ * their embeddings; 256-byte aligned sub-buffers).                         */
+size_t ivit_patch_embed_workspace_bytes(int32_t B, int32_t C, int32_t Hi, int32_t Wi, int32_t P, int32_t D);
+
+/* Patch embedding.  img [B x C x Hi x Wi] int8 (NCHW), Np = (Hi/P)(Wi/P)
+ * patches in row-major patch order.  The patch at (py, px) flattens to
+ * z[(ch P + ky) P + kx] = img[b, ch, py P + ky, px P + kx] (the [D x C x P x P]
+ * layout of a convolution weight) and
+ *   e[b, p] = sat_8((b_j * (sum_k z_k W_jk + bias_j)) >> c_j)   W [D x C P P]
+ * x [B*(Np+1) x D] int8 gets, per image, the class token then the patches:
+ *   x[b, 0]     = sat_8((pos_add.b_skip * cls_j    + pos_add.b_branch * pos[0, j])     >> pos_add.c)
+ *   x[b, 1 + p] = sat_8((pos_add.b_skip * e[b,p]_j + pos_add.b_branch * pos[1 + p, j]) >> pos_add.c)
+ * cls [D] int8 is held at the embedding scale; pos [(Np+1) x D] int8.
+ * workspace: ivit_patch_embed_workspace_bytes(...) bytes, 256-byte aligned,
+ * caller-owned.  Constraints: Hi, Wi multiples of P; C P P and D multiples
+ * of 16, each <= 16384; pointers 16-byte aligned.  Errors as for
+ * ivit_linear_requant, nothing enqueued on a failed check.                 */
+ivit_status ivit_patch_embed(const int8_t *img, int32_t B, int32_t C, int32_t Hi, int32_t Wi, int32_t P,
+                             const int8_t *W, int32_t D, const int32_t *bias, const int32_t *b, const int8_t *c,
+                             const int8_t *cls, const int8_t *pos, ivit_residual pos_add, void *workspace,
+                             size_t workspace_bytes, int8_t *x, ivit_stream_t stream);
+
+/* Bytes of device workspace ivit_head needs (the class tokens, normalised). */
+size_t ivit_head_workspace_bytes(int32_t B, int32_t D);
+
+/* Classifier head: the class token of every image (row 0 of its Ntok rows
+ * in x [B*Ntok x D]), I-LayerNorm (as ivit_layernorm), then an int8 linear
+ * layer W [Ncls x D] to int8 logits [B x Ncls] (as ivit_linear_requant).
+ * Ncls a multiple of 16 (pad a class count with zero rows of W).          */
+ivit_status ivit_head(const int8_t *x, int32_t B, int32_t Ntok, int32_t D, const int8_t *gamma,
+                      const int32_t *beta, int32_t F, int32_t M_ln, ivit_dyadic ln_out, const int8_t *W,
+                      int32_t Ncls, const int32_t *bias, const int32_t *b, const int8_t *c, void *workspace,
+                      size_t workspace_bytes, int8_t *logits, ivit_stream_t stream);
+
+/* A whole ViT: patch embedding, n_blocks encoder blocks, classifier head.
+ * Device pointers as above; `blocks` is a host array of n_blocks entries
+ * (each with the model width D).                                           */
+typedef struct {
+  int32_t C, P, D, n_blocks, Ncls;
+  /* patch embedding: W [D x C P P], bias / b / c [D], class token, position embedding */
+  const int8_t *w_pe;
+  const int32_t *bias_pe;
+  const int32_t *b_pe;
+  const int8_t *c_pe;
+  const int8_t *cls;
+  const int8_t *pos;
+  ivit_residual pos_add;
+  const ivit_block_params *blocks;
+  /* head: I-LayerNorm then W [Ncls x D] */
+  const int8_t *head_gamma;
+  const int32_t *head_beta;
+  int32_t head_ln_F, head_ln_M;
+  ivit_dyadic head_ln_out;
+  const int8_t *w_head;
+  const int32_t *bias_head;
+  const int32_t *b_head;
+  const int8_t *c_head;
+} ivit_model_params;
+
+/* Bytes of device workspace ivit_model_forward needs for B images of
+ * Hi x Wi pixels (two token buffers and the largest step's workspace).     */
+size_t ivit_model_workspace_bytes(const ivit_model_params *m, int32_t B, int32_t Hi, int32_t Wi);
+
+/* img [B x C x Hi x Wi] int8 -> logits [B x Ncls] int8.  Every check of
+ * every step runs before anything is enqueued.                             */
+ivit_status ivit_model_forward(const ivit_model_params *m, const int8_t *img, int32_t B, int32_t Hi, int32_t Wi,
+                               void *workspace, size_t workspace_bytes, int8_t *logits, ivit_stream_t stream);
+
+/* ---------------------------------------------------------------------------
  * Status
  * ------------------------------------------------------------------------- */
 

@@ -22,6 +22,8 @@ __all__ = [
     "ivit_linear_requant", "ivit_linear_shiftgelu", "ivit_attention", "ivit_shiftgelu", "ivit_layernorm",
     "ivit_block_workspace_bytes", "ivit_block_forward", "ivit_stream_status", "ivit_launch_count",
     "ivit_block_forward_static", "STATIC_SCRATCH_BYTES", "EXPORTED_SYMBOLS",
+    "ModelParams", "ivit_patch_embed_workspace_bytes", "ivit_patch_embed", "ivit_head_workspace_bytes", "ivit_head",
+    "ivit_model_workspace_bytes", "ivit_model_forward",
 ]
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
@@ -35,6 +37,8 @@ EXPORTED_SYMBOLS = (
     "ivit_block_workspace_bytes",
     "ivit_block_forward", "ivit_stream_status", "ivit_launch_count",
     "ivit_block_forward_static",
+    "ivit_patch_embed_workspace_bytes", "ivit_patch_embed", "ivit_head_workspace_bytes", "ivit_head",
+    "ivit_model_workspace_bytes", "ivit_model_forward",
 )
 
 _STATUS = {0: "IVIT_OK", 1: "IVIT_ERR_INVALID_ARG", 2: "IVIT_ERR_UNSUPPORTED", 3: "IVIT_ERR_CUDA",
@@ -74,6 +78,20 @@ class BlockParams(C.Structure):
     ]
 
 
+class ModelParams(C.Structure):
+    """Mirror of ``ivit_model_params`` (``blocks`` points at a ctypes array of
+    :class:`BlockParams` that the caller keeps alive)."""
+    _fields_ = [
+        ("C", C.c_int32), ("P", C.c_int32), ("D", C.c_int32), ("n_blocks", C.c_int32), ("Ncls", C.c_int32),
+        ("w_pe", C.c_void_p), ("bias_pe", C.c_void_p), ("b_pe", C.c_void_p), ("c_pe", C.c_void_p),
+        ("cls", C.c_void_p), ("pos", C.c_void_p), ("pos_add", Residual),
+        ("blocks", C.POINTER(BlockParams)),
+        ("head_gamma", C.c_void_p), ("head_beta", C.c_void_p), ("head_ln_F", C.c_int32), ("head_ln_M", C.c_int32),
+        ("head_ln_out", Dyadic),
+        ("w_head", C.c_void_p), ("bias_head", C.c_void_p), ("b_head", C.c_void_p), ("c_head", C.c_void_p),
+    ]
+
+
 def lib() -> C.CDLL:
     """Load the shared library (raises if it was not built)."""
     global _lib
@@ -108,6 +126,20 @@ def lib() -> C.CDLL:
             L.ivit_block_forward.argtypes = [C.POINTER(BlockParams), vp, vp, vp, C.c_size_t, i32, i32, vp]
             L.ivit_block_forward_static.restype = C.c_int
             L.ivit_block_forward_static.argtypes = [C.POINTER(BlockParams), vp, vp, i32, i32, vp]
+            L.ivit_patch_embed_workspace_bytes.restype = C.c_size_t
+            L.ivit_patch_embed_workspace_bytes.argtypes = [i32, i32, i32, i32, i32, i32]
+            L.ivit_patch_embed.restype = C.c_int
+            L.ivit_patch_embed.argtypes = [vp, i32, i32, i32, i32, i32, vp, i32, vp, vp, vp, vp, vp, Residual, vp,
+                                           C.c_size_t, vp, vp]
+            L.ivit_head_workspace_bytes.restype = C.c_size_t
+            L.ivit_head_workspace_bytes.argtypes = [i32, i32]
+            L.ivit_head.restype = C.c_int
+            L.ivit_head.argtypes = [vp, i32, i32, i32, vp, vp, i32, i32, Dyadic, vp, i32, vp, vp, vp, vp, C.c_size_t,
+                                    vp, vp]
+            L.ivit_model_workspace_bytes.restype = C.c_size_t
+            L.ivit_model_workspace_bytes.argtypes = [C.POINTER(ModelParams), i32, i32, i32]
+            L.ivit_model_forward.restype = C.c_int
+            L.ivit_model_forward.argtypes = [C.POINTER(ModelParams), vp, i32, i32, i32, vp, C.c_size_t, vp, vp]
             L.ivit_stream_status.restype = C.c_int
             L.ivit_stream_status.argtypes = [vp]
             L.ivit_launch_count.restype = C.c_uint64
@@ -283,3 +315,55 @@ def ivit_stream_status(stream=None) -> int:
 
 def ivit_launch_count() -> int:
     return int(lib().ivit_launch_count())
+
+
+def ivit_patch_embed_workspace_bytes(B: int, C_in: int, Hi: int, Wi: int, P: int, D: int) -> int:
+    return int(lib().ivit_patch_embed_workspace_bytes(int(B), int(C_in), int(Hi), int(Wi), int(P), int(D)))
+
+
+def ivit_patch_embed(img, P: int, W, bias, b, c, cls, pos, pos_add, workspace, x, stream=None):
+    """x [B*(Np+1), D] from img [B, C, Hi, Wi]: patches through W [D, C*P*P],
+    the class token first, the position embedding joined by ``pos_add``."""
+    B, C_in, Hi, Wi = img.shape
+    D = W.shape[0]
+    st = lib().ivit_patch_embed(_ptr(img, torch.int8, "img"), B, C_in, Hi, Wi, int(P), _ptr(W, torch.int8, "W"), D,
+                                _ptr(bias, torch.int32, "bias"), _ptr(b, torch.int32, "b"), _ptr(c, torch.int8, "c"),
+                                _ptr(cls, torch.int8, "cls"), _ptr(pos, torch.int8, "pos"), _res(pos_add),
+                                _ptr(workspace, torch.uint8, "workspace"), workspace.numel(), _ptr(x, torch.int8, "x"),
+                                _stream(stream))
+    _check("ivit_patch_embed", st)
+    return x
+
+
+def ivit_head_workspace_bytes(B: int, D: int) -> int:
+    return int(lib().ivit_head_workspace_bytes(int(B), int(D)))
+
+
+def ivit_head(x, B: int, Ntok: int, gamma, beta, F: int, M_ln: int, ln_out, W, bias, b, c, workspace, logits,
+              stream=None):
+    """logits [B, Ncls] from the class tokens of x [B*Ntok, D]."""
+    D = x.shape[1]
+    st = lib().ivit_head(_ptr(x, torch.int8, "x"), int(B), int(Ntok), D, _ptr(gamma, torch.int8, "gamma"),
+                         _ptr(beta, torch.int32, "beta"), int(F), int(M_ln), _dy(ln_out), _ptr(W, torch.int8, "W"),
+                         W.shape[0], _ptr(bias, torch.int32, "bias"), _ptr(b, torch.int32, "b"),
+                         _ptr(c, torch.int8, "c"), _ptr(workspace, torch.uint8, "workspace"), workspace.numel(),
+                         _ptr(logits, torch.int8, "logits"), _stream(stream))
+    _check("ivit_head", st)
+    return logits
+
+
+def ivit_model_workspace_bytes(params, B: int, Hi: int, Wi: int) -> int:
+    p = params.c if hasattr(params, "c") else params
+    return int(lib().ivit_model_workspace_bytes(C.byref(p), int(B), int(Hi), int(Wi)))
+
+
+def ivit_model_forward(params, img, workspace, logits, stream=None):
+    """logits [B, Ncls] from img [B, C, Hi, Wi]; ``params`` is a
+    :class:`ModelParams` (or an object with ``.c``)."""
+    p = params.c if hasattr(params, "c") else params
+    B, _, Hi, Wi = img.shape
+    st = lib().ivit_model_forward(C.byref(p), _ptr(img, torch.int8, "img"), B, Hi, Wi,
+                                  _ptr(workspace, torch.uint8, "workspace"), workspace.numel(),
+                                  _ptr(logits, torch.int8, "logits"), _stream(stream))
+    _check("ivit_model_forward", st)
+    return logits

@@ -252,16 +252,19 @@ size_t ivit_block_workspace_bytes(int32_t B, int32_t N, int32_t D, int32_t Dm) {
   return up(T * D) + up(T * 3 * (size_t)D) + up(T * D) + up(T * D) + up(T * (size_t)Dm);
 }
 
-ivit_status ivit_block_forward(const ivit_block_params* p, const int8_t* x, int8_t* y, void* workspace,
-                               size_t workspace_bytes, int32_t B, int32_t N, ivit_stream_t stream) {
+namespace {
+
+// Every host-side check of one block call; IVIT_OK means it may be enqueued
+// (or, with B or N zero, that there is nothing to do).
+ivit_status check_block(const ivit_block_params* p, const int8_t* x, const int8_t* y, const void* workspace,
+                        size_t workspace_bytes, int32_t B, int32_t N) {
   if (!p || !x || !y || !workspace) return IVIT_ERR_INVALID_ARG;
   if (B < 0 || N < 0 || p->H < 1 || p->D != 64 * p->H || p->Dm < 16 || p->Dm % 16 != 0 || p->D > 2048)
     return IVIT_ERR_INVALID_ARG;
   if (x == y) return IVIT_ERR_INVALID_ARG;
   if (B == 0 || N == 0) return IVIT_OK;
   if (N > 640) return IVIT_ERR_UNSUPPORTED;
-  const int32_t D = p->D, Dm = p->Dm;
-  const size_t need = ivit_block_workspace_bytes(B, N, D, Dm);
+  const size_t need = ivit_block_workspace_bytes(B, N, p->D, p->Dm);
   if (workspace_bytes < need || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return IVIT_ERR_INVALID_ARG;
   if (!p->ln1_gamma || !p->ln1_beta || !p->w_qkv || !p->b_qkv || !p->c_qkv || !p->w_o || !p->b_o || !p->c_o ||
       !p->ln2_gamma || !p->ln2_beta || !p->w1 || !p->b1 || !p->c1 || !p->w2 || !p->b2 || !p->c2)
@@ -273,9 +276,13 @@ ivit_status ivit_block_forward(const ivit_block_params* p, const int8_t* x, int8
       p->ln_F > 14 || p->ln_M < p->ln_F || p->ln_M > 23)
     return IVIT_ERR_INVALID_ARG;
   if (!attention_config_supported(N, p->k_s, p->attn_I0)) return IVIT_ERR_UNSUPPORTED;
-  DeviceCtx dc;
-  ivit_status st = device_ctx(&dc);
-  if (st != IVIT_OK) return st;
+  return IVIT_OK;
+}
+
+// Enqueues one checked block (B, N > 0).
+ivit_status enqueue_block(const DeviceCtx& dc, const ivit_block_params* p, const int8_t* x, int8_t* y,
+                          void* workspace, int32_t B, int32_t N, cudaStream_t s) {
+  const int32_t D = p->D, Dm = p->Dm;
   const int64_t T = (int64_t)B * N;
   auto up = [](size_t v) { return (v + 255) / 256 * 256; };
   int8_t* ws = static_cast<int8_t*>(workspace);
@@ -284,8 +291,8 @@ ivit_status ivit_block_forward(const ivit_block_params* p, const int8_t* x, int8
   int8_t* ctx = qkv + up((size_t)T * 3 * D);
   int8_t* xh = ctx + up((size_t)T * D);
   int8_t* g = xh + up((size_t)T * D);
-  cudaStream_t s = (cudaStream_t)stream;
   const ivit_residual none{0, 0, 0};
+  ivit_status st;
   // a1 LN1
   if ((st = launch_layernorm(dc, x, T, D, p->ln1_gamma, p->ln1_beta, p->ln_F, p->ln_M, p->ln1_out, ln, s)) != IVIT_OK)
     return st;
@@ -312,6 +319,191 @@ ivit_status ivit_block_forward(const ivit_block_params* p, const int8_t* x, int8
     return st;
   // a10 fc2 + residual 2
   return launch_gemm(dc, g, T, Dm, p->w2, D, p->bias2, p->b2, p->c2, 8, kEpiResidual, xh, p->res2, nullptr, y, s);
+}
+
+}  // namespace
+
+ivit_status ivit_block_forward(const ivit_block_params* p, const int8_t* x, int8_t* y, void* workspace,
+                               size_t workspace_bytes, int32_t B, int32_t N, ivit_stream_t stream) {
+  ivit_status st = check_block(p, x, y, workspace, workspace_bytes, B, N);
+  if (st != IVIT_OK || B == 0 || N == 0) return st;
+  DeviceCtx dc;
+  if ((st = device_ctx(&dc)) != IVIT_OK) return st;
+  return enqueue_block(dc, p, x, y, workspace, B, N, (cudaStream_t)stream);
+}
+
+// ---------------------------------------------------------------------------
+// steps either side of the blocks
+// ---------------------------------------------------------------------------
+
+size_t ivit_patch_embed_workspace_bytes(int32_t B, int32_t C, int32_t Hi, int32_t Wi, int32_t P, int32_t D) {
+  if (B < 0 || C < 1 || P < 1 || Hi < P || Wi < P || D < 0) return 0;
+  const size_t rows = (size_t)B * (size_t)(Hi / P) * (size_t)(Wi / P);
+  auto up = [](size_t v) { return (v + 255) / 256 * 256; };
+  // patch rows (rows x C P P) | embeddings (rows x D)
+  return up(rows * (size_t)C * P * P) + up(rows * (size_t)D);
+}
+
+size_t ivit_head_workspace_bytes(int32_t B, int32_t D) {
+  if (B < 0 || D < 0) return 0;
+  auto up = [](size_t v) { return (v + 255) / 256 * 256; };
+  // class tokens | their normalised copy
+  return 2 * up((size_t)B * (size_t)D);
+}
+
+namespace {
+
+ivit_status check_patch_embed(const int8_t* img, int32_t B, int32_t C, int32_t Hi, int32_t Wi, int32_t P,
+                              const int8_t* W, int32_t D, const int32_t* bias, const int32_t* b, const int8_t* c,
+                              const int8_t* cls, const int8_t* pos, ivit_residual pos_add, const void* workspace,
+                              size_t workspace_bytes, const int8_t* x) {
+  if (!img || !W || !b || !c || !cls || !pos || !x || !workspace) return IVIT_ERR_INVALID_ARG;
+  if (!aligned16(img) || !aligned16(W) || !aligned16(b) || !aligned16(c) || !aligned16(cls) || !aligned16(pos) ||
+      !aligned16(x) || (bias && !aligned16(bias)) || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+    return IVIT_ERR_INVALID_ARG;
+  if (B < 0 || C < 1 || P < 1 || Hi < P || Wi < P || Hi % P != 0 || Wi % P != 0 || D < 16 || D % 16 != 0 ||
+      !valid_residual(pos_add))
+    return IVIT_ERR_INVALID_ARG;
+  const int64_t K = (int64_t)C * P * P;
+  if (K < 16 || K % 16 != 0) return IVIT_ERR_INVALID_ARG;
+  const int64_t rows = (int64_t)B * (Hi / P) * (Wi / P);
+  if (K > 16384 || D > 16384 || rows + B > 0x7fffff00LL) return IVIT_ERR_UNSUPPORTED;
+  if (workspace_bytes < ivit_patch_embed_workspace_bytes(B, C, Hi, Wi, P, D)) return IVIT_ERR_INVALID_ARG;
+  return IVIT_OK;
+}
+
+ivit_status enqueue_patch_embed(const DeviceCtx& dc, const int8_t* img, int32_t B, int32_t C, int32_t Hi,
+                                int32_t Wi, int32_t P, const int8_t* W, int32_t D, const int32_t* bias,
+                                const int32_t* b, const int8_t* c, const int8_t* cls, const int8_t* pos,
+                                ivit_residual pos_add, void* workspace, int8_t* x, cudaStream_t s) {
+  const int32_t Np = (Hi / P) * (Wi / P), K = C * P * P;
+  const int64_t rows = (int64_t)B * Np;
+  auto up = [](size_t v) { return (v + 255) / 256 * 256; };
+  int8_t* z = static_cast<int8_t*>(workspace);
+  int8_t* e = z + up((size_t)rows * K);
+  ivit_status st;
+  if ((st = launch_im2col(dc, img, B, C, Hi, Wi, P, z, s)) != IVIT_OK) return st;
+  if ((st = launch_gemm(dc, z, rows, K, W, D, bias, b, c, 8, kEpiPlain, nullptr, ivit_residual{0, 0, 0}, nullptr, e,
+                        s)) != IVIT_OK)
+    return st;
+  return launch_tokens(dc, e, cls, pos, pos_add, B, Np, D, x, s);
+}
+
+ivit_status check_head(const int8_t* x, int32_t B, int32_t Ntok, int32_t D, const int8_t* gamma,
+                       const int32_t* beta, int32_t F, int32_t M_ln, ivit_dyadic ln_out, const int8_t* W,
+                       int32_t Ncls, const int32_t* bias, const int32_t* b, const int8_t* c, const void* workspace,
+                       size_t workspace_bytes, const int8_t* logits) {
+  if (!x || !gamma || !beta || !W || !b || !c || !logits || !workspace) return IVIT_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(gamma) || !aligned16(beta) || !aligned16(W) || !aligned16(b) || !aligned16(c) ||
+      !aligned16(logits) || (bias && !aligned16(bias)) || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+    return IVIT_ERR_INVALID_ARG;
+  if (B < 0 || Ntok < 1 || D < 16 || D > 2048 || D % 16 != 0 || Ncls < 16 || Ncls % 16 != 0 || F < 0 || F > 14 ||
+      M_ln < F || M_ln > 23 || !valid_dyadic(ln_out))
+    return IVIT_ERR_INVALID_ARG;
+  if ((int64_t)B * Ntok > 0x7fffff00LL) return IVIT_ERR_UNSUPPORTED;
+  if (workspace_bytes < ivit_head_workspace_bytes(B, D)) return IVIT_ERR_INVALID_ARG;
+  return IVIT_OK;
+}
+
+ivit_status enqueue_head(const DeviceCtx& dc, const int8_t* x, int32_t B, int32_t Ntok, int32_t D,
+                         const int8_t* gamma, const int32_t* beta, int32_t F, int32_t M_ln, ivit_dyadic ln_out,
+                         const int8_t* W, int32_t Ncls, const int32_t* bias, const int32_t* b, const int8_t* c,
+                         void* workspace, int8_t* logits, cudaStream_t s) {
+  auto up = [](size_t v) { return (v + 255) / 256 * 256; };
+  int8_t* t = static_cast<int8_t*>(workspace);
+  int8_t* n = t + up((size_t)B * D);
+  ivit_status st;
+  if ((st = launch_gather_rows(dc, x, B, Ntok, D, t, s)) != IVIT_OK) return st;
+  if ((st = launch_layernorm(dc, t, B, D, gamma, beta, F, M_ln, ln_out, n, s)) != IVIT_OK) return st;
+  return launch_gemm(dc, n, B, D, W, Ncls, bias, b, c, 8, kEpiPlain, nullptr, ivit_residual{0, 0, 0}, nullptr, logits,
+                     s);
+}
+
+}  // namespace
+
+ivit_status ivit_patch_embed(const int8_t* img, int32_t B, int32_t C, int32_t Hi, int32_t Wi, int32_t P,
+                             const int8_t* W, int32_t D, const int32_t* bias, const int32_t* b, const int8_t* c,
+                             const int8_t* cls, const int8_t* pos, ivit_residual pos_add, void* workspace,
+                             size_t workspace_bytes, int8_t* x, ivit_stream_t stream) {
+  ivit_status st = check_patch_embed(img, B, C, Hi, Wi, P, W, D, bias, b, c, cls, pos, pos_add, workspace,
+                                     workspace_bytes, x);
+  if (st != IVIT_OK || B == 0) return st;
+  DeviceCtx dc;
+  if ((st = device_ctx(&dc)) != IVIT_OK) return st;
+  return enqueue_patch_embed(dc, img, B, C, Hi, Wi, P, W, D, bias, b, c, cls, pos, pos_add, workspace, x,
+                             (cudaStream_t)stream);
+}
+
+ivit_status ivit_head(const int8_t* x, int32_t B, int32_t Ntok, int32_t D, const int8_t* gamma, const int32_t* beta,
+                      int32_t F, int32_t M_ln, ivit_dyadic ln_out, const int8_t* W, int32_t Ncls,
+                      const int32_t* bias, const int32_t* b, const int8_t* c, void* workspace,
+                      size_t workspace_bytes, int8_t* logits, ivit_stream_t stream) {
+  ivit_status st = check_head(x, B, Ntok, D, gamma, beta, F, M_ln, ln_out, W, Ncls, bias, b, c, workspace,
+                              workspace_bytes, logits);
+  if (st != IVIT_OK || B == 0) return st;
+  DeviceCtx dc;
+  if ((st = device_ctx(&dc)) != IVIT_OK) return st;
+  return enqueue_head(dc, x, B, Ntok, D, gamma, beta, F, M_ln, ln_out, W, Ncls, bias, b, c, workspace, logits,
+                      (cudaStream_t)stream);
+}
+
+size_t ivit_model_workspace_bytes(const ivit_model_params* m, int32_t B, int32_t Hi, int32_t Wi) {
+  if (!m || B < 0 || m->P < 1 || Hi < m->P || Wi < m->P || m->D < 0 || m->n_blocks < 0) return 0;
+  if (m->n_blocks > 0 && !m->blocks) return 0;
+  const int32_t Ntok = (Hi / m->P) * (Wi / m->P) + 1;
+  auto up = [](size_t v) { return (v + 255) / 256 * 256; };
+  size_t scratch = ivit_patch_embed_workspace_bytes(B, m->C, Hi, Wi, m->P, m->D);
+  for (int32_t i = 0; i < m->n_blocks; ++i) {
+    const size_t w = ivit_block_workspace_bytes(B, Ntok, m->blocks[i].D, m->blocks[i].Dm);
+    if (w > scratch) scratch = w;
+  }
+  const size_t hw = ivit_head_workspace_bytes(B, m->D);
+  if (hw > scratch) scratch = hw;
+  // two token buffers, then the scratch of whichever step runs
+  return 2 * up((size_t)B * Ntok * m->D) + scratch;
+}
+
+ivit_status ivit_model_forward(const ivit_model_params* m, const int8_t* img, int32_t B, int32_t Hi, int32_t Wi,
+                               void* workspace, size_t workspace_bytes, int8_t* logits, ivit_stream_t stream) {
+  if (!m || !img || !logits || !workspace || m->n_blocks < 0 || (m->n_blocks > 0 && !m->blocks))
+    return IVIT_ERR_INVALID_ARG;
+  if (B < 0 || m->P < 1 || Hi < m->P || Wi < m->P || m->D < 16) return IVIT_ERR_INVALID_ARG;
+  const size_t need = ivit_model_workspace_bytes(m, B, Hi, Wi);
+  if (need == 0 || workspace_bytes < need || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+    return IVIT_ERR_INVALID_ARG;
+  const int32_t Ntok = (Hi / m->P) * (Wi / m->P) + 1;
+  auto up = [](size_t v) { return (v + 255) / 256 * 256; };
+  int8_t* tok[2];
+  tok[0] = static_cast<int8_t*>(workspace);
+  tok[1] = tok[0] + up((size_t)B * Ntok * m->D);
+  void* scratch = tok[1] + up((size_t)B * Ntok * m->D);
+  const size_t scratch_bytes = workspace_bytes - 2 * up((size_t)B * Ntok * m->D);
+  // every step is checked before anything is enqueued
+  ivit_status st = check_patch_embed(img, B, m->C, Hi, Wi, m->P, m->w_pe, m->D, m->bias_pe, m->b_pe, m->c_pe,
+                                     m->cls, m->pos, m->pos_add, scratch, scratch_bytes, tok[0]);
+  if (st != IVIT_OK) return st;
+  for (int32_t i = 0; i < m->n_blocks; ++i) {
+    if (m->blocks[i].D != m->D) return IVIT_ERR_INVALID_ARG;
+    if ((st = check_block(&m->blocks[i], tok[i & 1], tok[(i + 1) & 1], scratch, scratch_bytes, B, Ntok)) != IVIT_OK)
+      return st;
+  }
+  if ((st = check_head(tok[m->n_blocks & 1], B, Ntok, m->D, m->head_gamma, m->head_beta, m->head_ln_F, m->head_ln_M,
+                       m->head_ln_out, m->w_head, m->Ncls, m->bias_head, m->b_head, m->c_head, scratch, scratch_bytes,
+                       logits)) != IVIT_OK)
+    return st;
+  if (B == 0) return IVIT_OK;
+  DeviceCtx dc;
+  if ((st = device_ctx(&dc)) != IVIT_OK) return st;
+  cudaStream_t s = (cudaStream_t)stream;
+  if ((st = enqueue_patch_embed(dc, img, B, m->C, Hi, Wi, m->P, m->w_pe, m->D, m->bias_pe, m->b_pe, m->c_pe, m->cls,
+                                m->pos, m->pos_add, scratch, tok[0], s)) != IVIT_OK)
+    return st;
+  for (int32_t i = 0; i < m->n_blocks; ++i)
+    if ((st = enqueue_block(dc, &m->blocks[i], tok[i & 1], tok[(i + 1) & 1], scratch, B, Ntok, s)) != IVIT_OK)
+      return st;
+  return enqueue_head(dc, tok[m->n_blocks & 1], B, Ntok, m->D, m->head_gamma, m->head_beta, m->head_ln_F,
+                      m->head_ln_M, m->head_ln_out, m->w_head, m->Ncls, m->bias_head, m->b_head, m->c_head, scratch,
+                      logits, s);
 }
 
 ivit_status ivit_stream_status(ivit_stream_t stream) {

@@ -67,6 +67,19 @@ ivit_status launch_attention(const DeviceCtx& dc, const int8_t* qkv, int32_t B, 
 ivit_status launch_shiftgelu(const DeviceCtx& dc, const int8_t* x, int64_t n, const GeluParams& g, int8_t* y,
                              cudaStream_t stream);
 
+// Patch rows z [B*Np x C*P*P] from img [B x C x Hi x Wi] (Hi, Wi multiples of P).
+ivit_status launch_im2col(const DeviceCtx& dc, const int8_t* img, int32_t B, int32_t C, int32_t Hi, int32_t Wi,
+                          int32_t P, int8_t* z, cudaStream_t stream);
+
+// Tokens x [B*(Np+1) x D] from the class token, the patch embeddings e
+// [B*Np x D] and the position embedding pos [(Np+1) x D] (D a multiple of 16).
+ivit_status launch_tokens(const DeviceCtx& dc, const int8_t* e, const int8_t* cls, const int8_t* pos,
+                          ivit_residual add, int32_t B, int32_t Np, int32_t D, int8_t* x, cudaStream_t stream);
+
+// t [B x D] = the first of each image's Ntok rows of x (D a multiple of 16).
+ivit_status launch_gather_rows(const DeviceCtx& dc, const int8_t* x, int32_t B, int32_t Ntok, int32_t D, int8_t* t,
+                               cudaStream_t stream);
+
 ivit_status launch_layernorm(const DeviceCtx& dc, const int8_t* x, int64_t rows, int32_t cols,
                              const int8_t* gamma, const int32_t* beta, int32_t F, int32_t M_ln, ivit_dyadic out,
                              int8_t* y, cudaStream_t stream);

@@ -15,7 +15,7 @@ from typing import Dict
 import numpy as np
 import torch
 
-from . import (BlockParams, Dyadic, Residual, ivit_dyadic_from_double, ivit_i0_from_scale,
+from . import (BlockParams, Dyadic, ModelParams, Residual, ivit_dyadic_from_double, ivit_i0_from_scale,
                ivit_residual_from_double)
 
 # method constants (readings of the pages: M = 30 for IntDiv, 8-bit Shiftmax /
@@ -102,3 +102,67 @@ def to_device(p: Dict, device="cuda") -> DeviceBlockParams:
     s.res2 = Residual(*p["res2"])
     s.ln_F, s.ln_M = p["ln_F"], p["ln_M"]
     return DeviceBlockParams(tensors=t, c=s, host=p)
+
+
+
+# ---------------------------------------------------------------------------
+# a whole model: patch embedding, blocks, classifier head
+# ---------------------------------------------------------------------------
+
+def model_integer_params(mc, **consts) -> Dict:
+    """Integer parameters of a whole model from a ``synthetic.ModelCase``-like
+    description: the patch projection and the classifier are int8 linear
+    layers (per-channel DN of S_in S_w / S_out), the position embedding joins
+    the tokens with the DN pair (S_e / S_x, S_pos / S_x), and the head's
+    I-LayerNorm output multiplier is DN(S_gamma 2^-F / S_ln)."""
+    k = dict(DEFAULTS)
+    k.update(consts)
+    S = mc.scales
+    D = mc.w_pe.shape[0]
+    m = dict(P=mc.P, C=mc.img.shape[1], D=D, Ncls_pad=mc.w_head.shape[0], ln_F=k["ln_F"], ln_M=k["ln_M"])
+    m["w_pe"], m["bias_pe"] = mc.w_pe, mc.bias_pe
+    m["b_pe"], m["c_pe"] = _per_channel(S["img"], mc.s_w_pe, np.full(D, S["e"]))
+    m["cls"], m["pos"] = mc.cls, mc.pos
+    m["pos_add"] = ivit_residual_from_double(S["e"] / S["x"], S["pos"] / S["x"])
+    m["head_gamma"], m["head_beta"] = mc.head_gamma, mc.head_beta
+    m["head_ln_out"] = ivit_dyadic_from_double(S["head_gamma"] * 2.0 ** -k["ln_F"] / S["head_ln"])
+    m["w_head"], m["bias_head"] = mc.w_head, mc.bias_head
+    m["b_head"], m["c_head"] = _per_channel(S["head_ln"], mc.s_w_head, np.full(mc.w_head.shape[0], S["logits"]))
+    m["blocks"] = [integer_params(q, **consts) for q in mc.wl.blocks]
+    return m
+
+
+_MODEL_TENSORS = {
+    "w_pe": torch.int8, "bias_pe": torch.int32, "b_pe": torch.int32, "c_pe": torch.int8, "cls": torch.int8,
+    "pos": torch.int8, "head_gamma": torch.int8, "head_beta": torch.int32, "w_head": torch.int8,
+    "bias_head": torch.int32, "b_head": torch.int32, "c_head": torch.int8,
+}
+
+
+@dataclasses.dataclass
+class DeviceModelParams:
+    """Device copies of a model's tensors, its blocks and the ``ivit_model_params`` struct."""
+    tensors: Dict[str, torch.Tensor]
+    blocks: list
+    block_array: object
+    c: ModelParams
+    host: Dict
+
+
+def model_to_device(m: Dict, device="cuda") -> DeviceModelParams:
+    t = {}
+    for name, dt in _MODEL_TENSORS.items():
+        a = np.ascontiguousarray(m[name])
+        t[name] = torch.from_numpy(a).to(device=device, dtype=dt).contiguous()
+    blocks = [to_device(p, device) for p in m["blocks"]]
+    arr = (BlockParams * max(1, len(blocks)))(*[b.c for b in blocks])
+    s = ModelParams()
+    s.C, s.P, s.D, s.n_blocks, s.Ncls = m["C"], m["P"], m["D"], len(blocks), m["Ncls_pad"]
+    for name in ("w_pe", "bias_pe", "b_pe", "c_pe", "cls", "pos", "head_gamma", "head_beta", "w_head", "bias_head",
+                 "b_head", "c_head"):
+        setattr(s, name, t[name].data_ptr())
+    s.pos_add = Residual(*m["pos_add"])
+    s.blocks = arr
+    s.head_ln_F, s.head_ln_M = m["ln_F"], m["ln_M"]
+    s.head_ln_out = Dyadic(*m["head_ln_out"])
+    return DeviceModelParams(tensors=t, blocks=blocks, block_array=arr, c=s, host=m)

@@ -375,3 +375,41 @@ def head(x, B: int, Ntok: int, gamma, beta, F: int, M_ln: int, ln_out, W, bias, 
                       out.ctypes.data) != 0:
         raise MemoryError("orc_head")
     return out
+
+
+
+def model_params(mc, **consts):
+    """The oracle's own integer parameters of a whole model (``synthetic.ModelCase``):
+    per-channel DN for the patch projection and the classifier, the DN pair
+    (S_e / S_x, S_pos / S_x) for the position term, DN(S_gamma 2^-F / S_ln) for
+    the head's I-LayerNorm; the blocks as ``block_params``."""
+    S = mc.scales
+    ln_F = consts.get("ln_F", 7)
+    ln_M = consts.get("ln_M", 23)
+    D = mc.w_pe.shape[0]
+
+    def per_channel(s_in, s_w, s_out):
+        bc = [dyadic(s_in * float(sw) / float(s_out)) for sw in s_w]
+        return (np.array([x[0] for x in bc], dtype=np.int32), np.array([x[1] for x in bc], dtype=np.int32))
+
+    m = dict(P=mc.P, ln_F=ln_F, ln_M=ln_M)
+    m["b_pe"], m["c_pe"] = per_channel(S["img"], mc.s_w_pe, S["e"])
+    m["pos_add"] = dyadic_pair(S["e"] / S["x"], S["pos"] / S["x"])
+    m["head_ln_out"] = dyadic(S["head_gamma"] * 2.0 ** -ln_F / S["head_ln"])
+    m["b_head"], m["c_head"] = per_channel(S["head_ln"], mc.s_w_head, S["logits"])
+    m["blocks"] = [block_params(q, **{k: v for k, v in consts.items() if k != "ln_M"}, ln_M=ln_M)
+                   for q in mc.wl.blocks]
+    return m
+
+
+def model_forward(m, mc, images=None):
+    """Oracle logits [len(images) x Ncls_pad] of the model on the chosen images
+    (default: all) of ``mc.img``: patch embedding, every block, the head."""
+    img = mc.img if images is None else mc.img[list(images)]
+    B = img.shape[0]
+    x = patch_embed(img, mc.P, mc.w_pe, mc.bias_pe, m["b_pe"], m["c_pe"], mc.cls, mc.pos, m["pos_add"])
+    Ntok = x.shape[0] // B
+    for p in m["blocks"]:
+        x = block_forward(p, x, B, Ntok)
+    return head(x, B, Ntok, mc.head_gamma, mc.head_beta, m["ln_F"], m["ln_M"], m["head_ln_out"], mc.w_head,
+                mc.bias_head, m["b_head"], m["c_head"])

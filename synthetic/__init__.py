@@ -40,7 +40,7 @@ CONFIG_ORDER = ["deit_t_b1", "deit_s_b64", "vit_b_b64", "vit_l_b32_x12", "vit_b3
 
 # tensor ids for independent sub-streams
 _TID = dict(x=1, chan=2, wqkv=3, bqkv=4, wo=5, bo=6, w1=7, b1=8, w2=9, b2=10, g1=11, be1=12, g2=13,
-            be2=14, rank1=15, op=16)
+            be2=14, rank1=15, op=16, img=17, wpe=18, bpe=19, cls=20, pos=21, hg=22, hbe=23, whead=24, bhead=25)
 
 
 def rng(seed: int, tensor: str, block: int = 0) -> np.random.Generator:
@@ -363,3 +363,81 @@ def layernorm_case(rows: int, cols: int, seed: int = 0, chan_std=(0.1, 10.0), F:
     yf = _layernorm_f(x[:cal] * S_x, gq * S_g, be)
     S_out = scale_of(yf)
     return LayerNormCase(x=x, gamma=gq, beta=quant_i32(be, S_g * 2.0 ** -F), out_ratio=S_g * 2.0 ** -F / S_out, F=F)
+
+
+
+# ---------------------------------------------------------------------------
+# a whole model: patch embedding, blocks, classifier head
+# ---------------------------------------------------------------------------
+
+@dataclasses.dataclass
+class ModelCase:
+    img: np.ndarray              # [B x C x Hi x Wi] int8
+    P: int
+    w_pe: np.ndarray             # [D x C*P*P] int8, per output channel
+    s_w_pe: np.ndarray
+    bias_pe: np.ndarray          # int32 at S_img * s_w_pe
+    cls: np.ndarray              # [D] int8 at the embedding scale
+    pos: np.ndarray              # [(Np+1) x D] int8
+    head_gamma: np.ndarray       # int8
+    head_beta: np.ndarray        # int32 at S_head_gamma 2^-ln_F
+    w_head: np.ndarray           # [Ncls_pad x D] int8 (rows past Ncls are zero)
+    s_w_head: np.ndarray
+    bias_head: np.ndarray        # int32 at S_head_ln * s_w_head
+    Ncls: int                    # real classes; w_head has a multiple of 16 rows
+    wl: Workload                 # the blocks (their block-0 input scale is the token scale)
+    scales: Dict[str, float]     # img, e (embeddings), pos, x (tokens), head_gamma, head_ln, logits
+
+
+def _patches_f(img, P):
+    B, Cin, Hi, Wi = img.shape
+    t = img.reshape(B, Cin, Hi // P, P, Wi // P, P).transpose(0, 2, 4, 1, 3, 5)
+    return t.reshape(B * (Hi // P) * (Wi // P), Cin * P * P)
+
+
+def model_case(B: int = 2, Hi: int = 224, Wi: int = 224, P: int = 16, C: int = 3, D: int = 192, H: int = 3,
+               Dm: int = 768, blocks: int = 2, Ncls: int = 1000, seed: int = 0, n_cal: int = 2,
+               ln_F: int = 7) -> ModelCase:
+    """Seeded synthetic ViT: an int8 image batch, patch projection, class and
+    position embeddings, ``blocks`` encoder blocks (``make_workload``) and a
+    classifier head padded to a multiple of 16 classes.  Real scales come from
+    a floating-point pass on the first ``n_cal`` images."""
+    Np = (Hi // P) * (Wi // P)
+    wl = make_workload(name="model", B=B, N=Np + 1, D=D, H=H, Dm=Dm, blocks=blocks, seed=seed, ln_F=ln_F)
+    S = {}
+    img_f = rng(seed, "img").standard_normal((B, C, Hi, Wi))
+    S["img"] = scale_of(img_f)
+    img = quant_i8(img_f, S["img"])
+    w = rng(seed, "wpe").standard_normal((D, C * P * P)) * 0.02
+    w_pe, s_w_pe = _per_channel_weights(w)
+    b_f = rng(seed, "bpe").standard_normal(D) * 0.02
+    cal = min(B, n_cal)
+    e_f = _patches_f(img[:cal].astype(np.float64) * S["img"], P) @ (w_pe * s_w_pe[:, None]).T + b_f
+    S["e"] = scale_of(e_f)
+    cls_f = rng(seed, "cls").standard_normal(D) * 0.02
+    pos_f = rng(seed, "pos").standard_normal((Np + 1, D)) * 0.02
+    S["pos"] = scale_of(pos_f)
+    S["x"] = wl.blocks[0].scales["x"]
+    # head: I-LayerNorm on the class token, then the classifier
+    hg = 1.0 + 0.1 * rng(seed, "hg").standard_normal(D)
+    hbe = 0.02 * rng(seed, "hbe").standard_normal(D)
+    S["head_gamma"] = scale_of(hg)
+    hgq = quant_i8(hg, S["head_gamma"])
+    y_last = wl.blocks[-1].scales["y"]
+    t_f = rng(seed, "hg", 1).standard_normal((max(cal, 8), D)) * 40.0 * y_last
+    ln_f = _layernorm_f(t_f, hgq * S["head_gamma"], hbe)
+    S["head_ln"] = scale_of(ln_f)
+    wh = rng(seed, "whead").standard_normal((Ncls, D)) * 0.02
+    w_head, s_w_head = _per_channel_weights(wh)
+    bh = rng(seed, "bhead").standard_normal(Ncls) * 0.02
+    S["logits"] = scale_of(ln_f @ (w_head * s_w_head[:, None]).T + bh)
+    pad = (-Ncls) % 16
+    bias_head = quant_i32(bh, S["head_ln"] * s_w_head)
+    if pad:
+        w_head = np.concatenate([w_head, np.zeros((pad, D), np.int8)])
+        s_w_head = np.concatenate([s_w_head, np.full(pad, s_w_head[0])])
+        bias_head = np.concatenate([bias_head, np.zeros(pad, np.int32)])
+    return ModelCase(img=img, P=P, w_pe=w_pe, s_w_pe=s_w_pe, bias_pe=quant_i32(b_f, S["img"] * s_w_pe),
+                     cls=quant_i8(cls_f, S["e"]), pos=quant_i8(pos_f, S["pos"]), head_gamma=hgq,
+                     head_beta=quant_i32(hbe, S["head_gamma"] * 2.0 ** -ln_F), w_head=w_head, s_w_head=s_w_head,
+                     bias_head=bias_head, Ncls=Ncls, wl=wl, scales=S)

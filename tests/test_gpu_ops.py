@@ -250,3 +250,63 @@ def test_linear_shiftgelu_parity(M, K, N):
                                dev(b_d, torch.int32), dev(c_d, torch.int8), I0_d, 30, 8, out_d, Y)
     h = oracle.linear_requant(lc.X, lc.W, lc.bias, b_o, c_o)
     np.testing.assert_array_equal(host(Y), oracle.shiftgelu(h, I0_o, 30, 8, out_o))
+
+
+# ---------------------------------------------------------------------------
+# steps either side of the blocks, and a whole model
+# ---------------------------------------------------------------------------
+
+from integer_only_quantized_int8_b200 import params as ivit_params  # noqa: E402
+
+
+def _model_case_params(mc):
+    ip = ivit_params.model_integer_params(mc)
+    om = oracle.model_params(mc)
+    # the library's host helpers and the oracle derive the same integers
+    for k in ("b_pe", "c_pe", "b_head", "c_head"):
+        np.testing.assert_array_equal(np.asarray(ip[k], np.int64), np.asarray(om[k], np.int64))
+    assert tuple(ip["pos_add"]) == tuple(om["pos_add"]) and tuple(ip["head_ln_out"]) == tuple(om["head_ln_out"])
+    return ip, om
+
+
+@pytest.mark.parametrize("Hi,Wi,P", [(64, 48, 16), (24, 40, 8), (224, 224, 16)])
+def test_patch_embed_parity(Hi, Wi, P):
+    mc = synthetic.model_case(B=2, Hi=Hi, Wi=Wi, P=P, D=192, H=3, Dm=768, blocks=1, Ncls=100, seed=Hi + Wi + P)
+    ip, om = _model_case_params(mc)
+    B, Np = 2, (Hi // P) * (Wi // P)
+    t = {k: dev(ip[k], dt) for k, dt in (("w_pe", torch.int8), ("bias_pe", torch.int32), ("b_pe", torch.int32),
+                                         ("c_pe", torch.int8), ("cls", torch.int8), ("pos", torch.int8))}
+    ws = torch.empty(ivit.ivit_patch_embed_workspace_bytes(B, 3, Hi, Wi, P, 192), dtype=torch.uint8, device="cuda")
+    x = torch.full((B * (Np + 1), 192), 99, dtype=torch.int8, device="cuda")
+    ivit.ivit_patch_embed(dev(mc.img, torch.int8), P, t["w_pe"], t["bias_pe"], t["b_pe"], t["c_pe"], t["cls"],
+                          t["pos"], ip["pos_add"], ws, x)
+    want = oracle.patch_embed(mc.img, P, mc.w_pe, mc.bias_pe, om["b_pe"], om["c_pe"], mc.cls, mc.pos, om["pos_add"])
+    np.testing.assert_array_equal(host(x), want)
+
+
+def test_head_parity():
+    mc = synthetic.model_case(B=3, Hi=32, Wi=32, P=16, D=192, H=3, Dm=768, blocks=1, Ncls=100, seed=5)
+    ip, om = _model_case_params(mc)
+    B, Ntok, D = 5, 9, 192
+    x = np.random.default_rng(6).integers(-128, 128, (B * Ntok, D), dtype=np.int8)
+    ws = torch.empty(ivit.ivit_head_workspace_bytes(B, D), dtype=torch.uint8, device="cuda")
+    logits = torch.full((B, mc.w_head.shape[0]), 99, dtype=torch.int8, device="cuda")
+    ivit.ivit_head(dev(x, torch.int8), B, Ntok, dev(mc.head_gamma, torch.int8), dev(mc.head_beta, torch.int32),
+                   7, 23, ip["head_ln_out"], dev(mc.w_head, torch.int8), dev(mc.bias_head, torch.int32),
+                   dev(ip["b_head"], torch.int32), dev(ip["c_head"], torch.int8), ws, logits)
+    want = oracle.head(x, B, Ntok, mc.head_gamma, mc.head_beta, 7, 23, om["head_ln_out"], mc.w_head, mc.bias_head,
+                       om["b_head"], om["c_head"])
+    np.testing.assert_array_equal(host(logits), want)
+
+
+def test_model_forward_parity():
+    """Patch embedding, two DeiT-Tiny-width blocks and the head through
+    ivit_model_forward, against the oracle's composition of the same steps."""
+    mc = synthetic.model_case(B=2, Hi=224, Wi=224, P=16, D=192, H=3, Dm=768, blocks=2, Ncls=1000, seed=9)
+    ip, om = _model_case_params(mc)
+    dm = ivit_params.model_to_device(ip)
+    ws = torch.empty(ivit.ivit_model_workspace_bytes(dm, 2, 224, 224), dtype=torch.uint8, device="cuda")
+    logits = torch.full((2, mc.w_head.shape[0]), 99, dtype=torch.int8, device="cuda")
+    ivit.ivit_model_forward(dm, dev(mc.img, torch.int8), ws, logits)
+    assert ivit.ivit_stream_status() == 0
+    np.testing.assert_array_equal(host(logits), oracle.model_forward(om, mc))
