@@ -163,6 +163,9 @@ IVIT_DEV void tma_store_2d(const CUtensorMap* map, int32_t x, int32_t y, const v
 IVIT_DEV void bulk_commit_group() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
 // every committed store of this thread has finished reading shared memory
 IVIT_DEV void bulk_wait_read_all() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+// every committed store group of this thread but the most recent one has
+// finished reading shared memory
+IVIT_DEV void bulk_wait_read_1() { asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory"); }
 // every committed store of this thread has completed
 IVIT_DEV void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 

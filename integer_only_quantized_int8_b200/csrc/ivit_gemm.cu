@@ -86,7 +86,12 @@ struct GemmLayout {
   static constexpr int kMaxPart = (kChunks + kEpiParts - 1) / kEpiParts;  // chunks of the largest part
   static constexpr int kOutOff = STAGES * kStageBytes;
   static constexpr int kPartSlots = kMaxPart * kSlotBytes;  // 1024-byte aligned, as the swizzle needs
-  static constexpr int kBarOff = kOutOff + kEpiParts * kPartSlots;
+  static constexpr int kSetBytes = kEpiParts * kPartSlots;    // one slot set: every part's chunks
+  // Two slot sets, used by alternate tiles, when they fit: a tile's stores
+  // then have a whole tile's time to finish reading their slots.
+  static constexpr int kFixedBytes = (2 * STAGES + 5 + kEpiParts) * 8 + 16 + 256 + 1024;
+  static constexpr int kSlotSets = (kOutOff + 2 * kSetBytes + kFixedBytes <= 227 * 1024) ? 2 : 1;
+  static constexpr int kBarOff = kOutOff + kSlotSets * kSetBytes;
   // full, empty (STAGES each), tmem full x2, tmem empty x2, drain, one skip barrier per part
   static constexpr int kNumBars = 2 * STAGES + 5 + kEpiParts;
   static constexpr int kSlotOff = kBarOff + kNumBars * 8;
@@ -457,7 +462,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     const int grp = lane >> 2;  // channel group of 4 within the warp's 32 channels
     // the part's first warp stages its skip tiles and stores its outputs
     const bool part_lead = (e & 3) == 0 && lane == 0;
-    uint8_t* slots = smem + L::kOutOff + part * L::kPartSlots;
+    uint8_t* const slots0 = smem + L::kOutOff + part * L::kPartSlots;
+    int set = 0;  // slot set of the current tile
     const uint32_t ofs_even = slot_ofs(sub, quarter, grp, 0), ofs_odd = slot_ofs(sub, quarter, grp, 1);
     uint64_t* sbar = &skip_full[part];
     const uint32_t tlane = tmem_base + ((uint32_t)(quarter * 32) << 16);
@@ -477,13 +483,24 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     int acc = 0;
     uint32_t acc_phase = 0;
     uint32_t skip_phase = 0;
+    // this lane's channel constants (multiplier, shift, bias) of a tile; the
+    // next tile's are loaded while the current one drains, so their L2
+    // latency stays off the tile's path
+    auto load_chan = [&](int t, int32_t& cb_b, int32_t& cb_c, int32_t& cb_bias) {
+      const int ch = (t % ch_tiles) * kBM + quarter * 32 + lane;
+      const bool ok = t < num_tiles && ch < N;
+      cb_b = ok ? __ldg(args.b + ch) : 0;
+      cb_c = ok ? (int32_t)__ldg(args.c + ch) : 0;
+      cb_bias = (ok && args.bias) ? __ldg(args.bias + ch) : 0;
+    };
+    int32_t nb, nc, nbias;
+    load_chan(blockIdx.x, nb, nc, nbias);
     for (int t = blockIdx.x; t < num_tiles; t += gridDim.x) {
       const int cb = t % ch_tiles, tb = t / ch_tiles;
       const int ch0 = cb * kBM + quarter * 32;  // first channel of this warp
       const int ch = ch0 + lane;                // this thread's output channel
-      const ChanConst kc = ch < N ? chan_const(__ldg(args.b + ch), (int32_t)__ldg(args.c + ch),
-                                               args.bias ? __ldg(args.bias + ch) : 0, args.K)
-                                  : chan_const(0, 0, 0, args.K);
+      const ChanConst kc = ch < N ? chan_const(nb, nc, nbias, args.K) : chan_const(0, 0, 0, args.K);
+      load_chan(t + (int)gridDim.x, nb, nc, nbias);
       // warp-uniform requant form
       const int req = __all_sync(0xffffffffu, kc.fast) ? kReqFast
                       : (__any_sync(0xffffffffu, kc.needs_clamp) ? kReqWideClamp : kReqWide);
@@ -493,9 +510,15 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       while (n > 0 && tok_base + 16 * (c_begin + n - 1) >= M) --n;
       const bool live = n > 0;  // the same for the part's four warps
       const int tile_ch = cb * kBM;
+      uint8_t* const slots = slots0 + set * L::kSetBytes;
       if (part_lead) {
-        // the slots are free again once the stores of the previous tile have read them
-        bulk_wait_read_all();
+        // the slots are free again once the stores of the tile that last used
+        // them have read them: the previous tile (one set), or the one before
+        // it (two sets; every tile commits one bulk group, possibly empty)
+        if (L::kSlotSets == 2)
+          bulk_wait_read_1();
+        else
+          bulk_wait_read_all();
         if (EPI == kEpiResidual && live) {
           mbar_arrive_expect_tx(sbar, (uint32_t)(n * kSlotBytes));
           for (int i = 0; i < n; ++i)
@@ -523,11 +546,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       // them (rows past M and channels past N are clipped)
       fence_proxy_async_smem();
       if (!part_bar_and(part, got_skip)) break;
-      if (live && part_lead) {
-        for (int i = 0; i < n; ++i)
-          tma_store_2d(&tmY, tile_ch, (int32_t)(tok_base + 16 * (c_begin + i)), slots + i * kSlotBytes);
+      if (part_lead) {
+        if (live)
+          for (int i = 0; i < n; ++i)
+            tma_store_2d(&tmY, tile_ch, (int32_t)(tok_base + 16 * (c_begin + i)), slots + i * kSlotBytes);
         bulk_commit_group();
       }
+      if (L::kSlotSets == 2) set ^= 1;
       // preload the bias of the tile that next accumulates in this buffer
       if (t + 2 * (int)gridDim.x < num_tiles) bias_fill(tbase, c_begin, c_end, next_bias);
       tmem_st_wait();
