@@ -119,6 +119,8 @@ def lib():
             L.orc_head.argtypes = [C.c_void_p, C.c_int32, C.c_int32, C.c_int32, C.c_void_p, C.c_void_p,
                                    C.c_int32, C.c_int32, C.c_int32, C.c_int32, C.c_void_p, C.c_int32,
                                    C.c_void_p, C.c_void_p, C.c_void_p, C.c_void_p]
+            L.orc_set_linear_rounding.restype = None
+            L.orc_set_linear_rounding.argtypes = [C.c_int]
             L.orc_block_forward.restype = C.c_int
             L.orc_block_forward.argtypes = [C.POINTER(BlockParamsC), C.c_void_p, C.c_void_p,
                                             C.c_int32, C.c_int32]
@@ -192,8 +194,28 @@ def shiftmax_row(L, I0: int, M: int = 30, k_out: int = 8):
     return P
 
 
-def linear_requant(X, W, bias, b, c, out_bits: int = 8, skip=None, res=(0, 0, 0)):
-    """X [M x K] int8, W [N x K] int8, bias/b/c [N] -> Y [M x N] int8."""
+class linear_rounding:
+    """Context manager: the linear layers' requant rounds half up (mode 1)
+    instead of the floor shift (mode 0) inside the block."""
+
+    def __init__(self, mode: int):
+        self.mode = int(mode)
+
+    def __enter__(self):
+        lib().orc_set_linear_rounding(self.mode)
+        return self
+
+    def __exit__(self, *exc):
+        lib().orc_set_linear_rounding(0)
+        return False
+
+
+def linear_requant(X, W, bias, b, c, out_bits: int = 8, skip=None, res=(0, 0, 0), rounding: int = 0):
+    """X [M x K] int8, W [N x K] int8, bias/b/c [N] -> Y [M x N] int8
+    (rounding 1: the requant rounds half up)."""
+    if rounding:
+        with linear_rounding(rounding):
+            return linear_requant(X, W, bias, b, c, out_bits, skip, res)
     X = np.ascontiguousarray(X, dtype=np.int8)
     W = np.ascontiguousarray(W, dtype=np.int8)
     M, K = X.shape
@@ -288,7 +310,15 @@ def block_params(q, attn_M: int = 30, attn_k_out: int = 8, k_s: int = 8,
 
 
 def block_forward(p, x, B: int, N: int):
-    """x [B*N x D] int8 -> y [B*N x D] int8 through one block."""
+    """x [B*N x D] int8 -> y [B*N x D] int8 through one block (the linear
+    layers round half up when p["linear_round"] is set)."""
+    if p.get("linear_round", 0):
+        with linear_rounding(1):
+            return _block_forward(p, x, B, N)
+    return _block_forward(p, x, B, N)
+
+
+def _block_forward(p, x, B: int, N: int):
     x = np.ascontiguousarray(x, dtype=np.int8)
     keep = []
 
@@ -404,7 +434,15 @@ def model_params(mc, **consts):
 
 def model_forward(m, mc, images=None):
     """Oracle logits [len(images) x Ncls_pad] of the model on the chosen images
-    (default: all) of ``mc.img``: patch embedding, every block, the head."""
+    (default: all) of ``mc.img``: patch embedding, every block, the head
+    (every linear layer rounds half up when m["linear_round"] is set)."""
+    if m.get("linear_round", 0):
+        with linear_rounding(1):
+            return _model_forward(m, mc, images)
+    return _model_forward(m, mc, images)
+
+
+def _model_forward(m, mc, images=None):
     img = mc.img if images is None else mc.img[list(images)]
     B = img.shape[0]
     x = patch_embed(img, mc.P, mc.w_pe, mc.bias_pe, m["b_pe"], m["c_pe"], mc.cls, mc.pos, m["pos_add"])

@@ -177,6 +177,26 @@ int64_t orc_requant(int64_t acc, int32_t b, int32_t c, int bits)
  *   Y[i, j] = sat_8((b_skip * skip[i, j] + b_branch * o_ij) >> c_res)
  * where o_ij is the requantised linear output above.
  */
+/*
+ * Rounding of the linear layers' requant.  READING (R4): the integer
+ * operation is the plain floor shift (mode 0).  Mode 1 is the variant the
+ * page's ideal form suggests, round half up: (b * acc + 2^(c - 1)) >> c
+ * (nothing is added when c = 0).  It applies to the per-channel requant of
+ * the linear layers only; the residual additions, logits, Shiftmax,
+ * ShiftGELU and I-LayerNorm keep the floor shift.
+ */
+static int g_linear_round = 0;
+
+void orc_set_linear_rounding(int mode) { g_linear_round = mode != 0; }
+
+static int64_t linear_requant_one(int64_t acc, int32_t b, int32_t c, int bits)
+{
+    if (!g_linear_round)
+        return orc_requant(acc, b, c, bits);
+    const int64_t half = c > 0 ? ((int64_t)1 << (c - 1)) : 0;
+    return sat_bits(shr_floor((int64_t)b * acc + half, c), bits);
+}
+
 void orc_linear_requant(const int8_t *X, int64_t M, int32_t K,
                         const int8_t *W, int32_t N,
                         const int32_t *bias, const int32_t *b, const int32_t *c,
@@ -191,7 +211,7 @@ void orc_linear_requant(const int8_t *X, int64_t M, int32_t K,
                 acc += (int64_t)X[i * K + k] * (int64_t)W[(int64_t)j * K + k];
             if (bias)
                 acc += bias[j];
-            int64_t o = orc_requant(acc, b[j], c[j], out_bits);
+            int64_t o = linear_requant_one(acc, b[j], c[j], out_bits);
             if (skip) {
                 int64_t s = skip[i * N + j];
                 o = sat_bits(shr_floor((int64_t)b_skip * s + (int64_t)b_branch * o,

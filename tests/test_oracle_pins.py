@@ -527,3 +527,32 @@ def test_head_takes_class_tokens_through_layernorm_and_linear():
     ln_all = oracle.layernorm(x, gamma, beta, 7, 23, (3, 12))
     want = oracle.linear_requant(ln_all[::Ntok], W, bias, b, c)
     np.testing.assert_array_equal(got, want)
+
+
+def test_linear_round_half_up_variant():
+    """Mode 1 of the linear requant rounds b acc / 2^c half up: hand-worked
+    values at b = 1 (ties go up, also for negatives: -1.5 -> -1), and over
+    random layers the result is within half an LSB of the exact quotient
+    wherever it is not saturated, and equals the floor result or one more."""
+    X = np.array([[3], [-3], [1], [-1], [5], [-5], [2], [-2]], np.int8)
+    W = np.ones((1, 1), np.int8)
+    got = oracle.linear_requant(X, W, None, np.ones(1, np.int32), np.ones(1, np.int32), rounding=1)
+    np.testing.assert_array_equal(got[:, 0], [2, -1, 1, 0, 3, -2, 1, -1])
+    got_c2 = oracle.linear_requant(X, W, None, np.ones(1, np.int32), np.full(1, 2, np.int32), rounding=1)
+    np.testing.assert_array_equal(got_c2[:, 0], [1, -1, 0, 0, 1, -1, 1, 0])   # /4: .75 -.75 .25 -.25 1.25 -1.25 .5 -.5
+    got_c0 = oracle.linear_requant(X, W, None, np.ones(1, np.int32), np.zeros(1, np.int32), rounding=1)
+    np.testing.assert_array_equal(got_c0, X)                                     # c = 0 adds nothing
+    r = np.random.default_rng(41)
+    M, K, N = 37, 96, 24
+    X = r.integers(-128, 128, (M, K), dtype=np.int8)
+    W = r.integers(-128, 128, (N, K), dtype=np.int8)
+    bias = r.integers(-2 ** 16, 2 ** 16, N).astype(np.int32)
+    b = r.integers(1, 1 << 20, N).astype(np.int32)
+    c = r.integers(14, 31, N).astype(np.int32)
+    up = oracle.linear_requant(X, W, bias, b, c, rounding=1).astype(np.int64)
+    fl = oracle.linear_requant(X, W, bias, b, c).astype(np.int64)
+    exact = (X.astype(np.int64) @ W.T.astype(np.int64) + bias) * b / 2.0 ** c
+    inside = np.abs(exact) < 126.5
+    assert inside.sum() > 100
+    assert np.all(np.abs(up[inside] - exact[inside]) <= 0.5)
+    assert np.all((up - fl >= 0) & (up - fl <= 1))
