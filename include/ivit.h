@@ -92,7 +92,8 @@ ivit_status ivit_i0_from_scale(double S, int32_t *out);
 /* INT8 linear layer with dyadic epilogue ([IVIT] 3.1-3.2; [TRIO] eqs. (1),
  * (12)), optionally followed by a residual addition:
  *   acc_ij = sum_k X[i,k] * W[j,k] + bias[j]                   (int32)
- *   o_ij   = sat_{out_bits}((b[j] * acc_ij) >> c[j])
+ *   o_ij   = sat_{out_bits}((b[j] * acc_ij) >> c[j])           rounding = 0
+ *   o_ij   = sat_{out_bits}((b[j] * acc_ij + 2^(c[j]-1)) >> c[j])   rounding = 1
  *   Y_ij   = skip ? sat_8((res.b_skip * skip[i,j] + res.b_branch * o_ij) >> res.c)
  *                 : o_ij
  * X [M x K] int8; W [N x K] int8 (one output channel per row, i.e. K-major);
@@ -100,21 +101,26 @@ ivit_status ivit_i0_from_scale(double S, int32_t *out);
  * overflow); b [N] int32 in [0, 2^31); c [N] int8 in [0, 31];
  * skip [M x N] int8 or NULL; Y [M x N] int8.
  * Constraints: M >= 1; 16 <= K <= 16384 and N >= 16, both multiples of 16;
- * 2 <= out_bits <= 8.  Runs on the tensor cores (tcgen05 kind::i8).      */
+ * 2 <= out_bits <= 8; rounding 0 (the floor shift the page's integer
+ * formula writes, the default reading) or 1 (round half up, the variant its
+ * ideal form suggests; nothing is added when c[j] = 0).  Runs on the tensor
+ * cores (tcgen05 kind::i8).                                                 */
 ivit_status ivit_linear_requant(const int8_t *X, int64_t M, int32_t K, const int8_t *W, int32_t N,
                                 const int32_t *bias, const int32_t *b, const int8_t *c, int32_t out_bits,
-                                const int8_t *skip, ivit_residual res, int8_t *Y, ivit_stream_t stream);
+                                int32_t rounding, const int8_t *skip, ivit_residual res, int8_t *Y,
+                                ivit_stream_t stream);
 
 /* fc1 of the MLP with ShiftGELU fused into the epilogue ([IVIT] 3.1, 3.2,
  * 3.4): Y = ShiftGELU(sat_8((b[j] * (X W^T + bias)_ij) >> c[j])), with the
  * ShiftGELU of ivit_shiftgelu (I0 = round(1 / S_h) of the requantised fc1
  * output, gelu_out ~ S_h 2^-(k_out-1) / S_g).  Bit-identical to
  * ivit_linear_requant followed by ivit_shiftgelu, without the intermediate
- * tensor in memory.  Same constraints as both.                              */
+ * tensor in memory.  Same constraints as both; rounding applies to the fc1
+ * requant as in ivit_linear_requant.                                        */
 ivit_status ivit_linear_shiftgelu(const int8_t *X, int64_t M, int32_t K, const int8_t *W, int32_t N,
-                                  const int32_t *bias, const int32_t *b, const int8_t *c, int32_t gelu_I0,
-                                  int32_t gelu_M, int32_t gelu_k_out, ivit_dyadic gelu_out, int8_t *Y,
-                                  ivit_stream_t stream);
+                                  const int32_t *bias, const int32_t *b, const int8_t *c, int32_t rounding,
+                                  int32_t gelu_I0, int32_t gelu_M, int32_t gelu_k_out, ivit_dyadic gelu_out,
+                                  int8_t *Y, ivit_stream_t stream);
 
 /* Multi-head attention core with Shiftmax ([IVIT] 3.1-3.3; [TRIO] eqs.
  * (1)-(3)), fused on chip (the score matrix never reaches memory):
@@ -208,6 +214,9 @@ typedef struct {
   ivit_residual res2;
   /* I-LayerNorm constants shared by both norms */
   int32_t ln_F, ln_M;
+  /* requant rounding of the four linear layers, as ivit_linear_requant's
+   * `rounding` (0 floor, 1 round half up) */
+  int32_t linear_round;
 } ivit_block_params;
 
 /* Bytes of device workspace ivit_block_forward needs for B images of N
@@ -285,8 +294,8 @@ size_t ivit_patch_embed_workspace_bytes(int32_t B, int32_t C, int32_t Hi, int32_
  * ivit_linear_requant, nothing enqueued on a failed check.                 */
 ivit_status ivit_patch_embed(const int8_t *img, int32_t B, int32_t C, int32_t Hi, int32_t Wi, int32_t P,
                              const int8_t *W, int32_t D, const int32_t *bias, const int32_t *b, const int8_t *c,
-                             const int8_t *cls, const int8_t *pos, ivit_residual pos_add, void *workspace,
-                             size_t workspace_bytes, int8_t *x, ivit_stream_t stream);
+                             int32_t rounding, const int8_t *cls, const int8_t *pos, ivit_residual pos_add,
+                             void *workspace, size_t workspace_bytes, int8_t *x, ivit_stream_t stream);
 
 /* Bytes of device workspace ivit_head needs (the class tokens, normalised). */
 size_t ivit_head_workspace_bytes(int32_t B, int32_t D);
@@ -294,11 +303,13 @@ size_t ivit_head_workspace_bytes(int32_t B, int32_t D);
 /* Classifier head: the class token of every image (row 0 of its Ntok rows
  * in x [B*Ntok x D]), I-LayerNorm (as ivit_layernorm), then an int8 linear
  * layer W [Ncls x D] to int8 logits [B x Ncls] (as ivit_linear_requant).
- * Ncls a multiple of 16 (pad a class count with zero rows of W).          */
+ * Ncls a multiple of 16 (pad a class count with zero rows of W).  rounding
+ * as in ivit_linear_requant (for the classifier; the patch embedding's
+ * `rounding` likewise applies to its projection).                          */
 ivit_status ivit_head(const int8_t *x, int32_t B, int32_t Ntok, int32_t D, const int8_t *gamma,
                       const int32_t *beta, int32_t F, int32_t M_ln, ivit_dyadic ln_out, const int8_t *W,
-                      int32_t Ncls, const int32_t *bias, const int32_t *b, const int8_t *c, void *workspace,
-                      size_t workspace_bytes, int8_t *logits, ivit_stream_t stream);
+                      int32_t Ncls, const int32_t *bias, const int32_t *b, const int8_t *c, int32_t rounding,
+                      void *workspace, size_t workspace_bytes, int8_t *logits, ivit_stream_t stream);
 
 /* A whole ViT: patch embedding, n_blocks encoder blocks, classifier head.
  * Device pointers as above; `blocks` is a host array of n_blocks entries
@@ -323,6 +334,9 @@ typedef struct {
   const int32_t *bias_head;
   const int32_t *b_head;
   const int8_t *c_head;
+  /* requant rounding of the patch projection and the classifier (the blocks
+   * carry their own) */
+  int32_t linear_round;
 } ivit_model_params;
 
 /* Bytes of device workspace ivit_model_forward needs for B images of

@@ -75,6 +75,7 @@ class BlockParams(C.Structure):
         ("w2", C.c_void_p), ("bias2", C.c_void_p), ("b2", C.c_void_p), ("c2", C.c_void_p),
         ("res2", Residual),
         ("ln_F", C.c_int32), ("ln_M", C.c_int32),
+        ("linear_round", C.c_int32),
     ]
 
 
@@ -89,6 +90,7 @@ class ModelParams(C.Structure):
         ("head_gamma", C.c_void_p), ("head_beta", C.c_void_p), ("head_ln_F", C.c_int32), ("head_ln_M", C.c_int32),
         ("head_ln_out", Dyadic),
         ("w_head", C.c_void_p), ("bias_head", C.c_void_p), ("b_head", C.c_void_p), ("c_head", C.c_void_p),
+        ("linear_round", C.c_int32),
     ]
 
 
@@ -111,9 +113,9 @@ def lib() -> C.CDLL:
             L.ivit_i0_from_scale.restype = C.c_int
             L.ivit_i0_from_scale.argtypes = [C.c_double, C.POINTER(C.c_int32)]
             L.ivit_linear_requant.restype = C.c_int
-            L.ivit_linear_requant.argtypes = [vp, i64, i32, vp, i32, vp, vp, vp, i32, vp, Residual, vp, vp]
+            L.ivit_linear_requant.argtypes = [vp, i64, i32, vp, i32, vp, vp, vp, i32, i32, vp, Residual, vp, vp]
             L.ivit_linear_shiftgelu.restype = C.c_int
-            L.ivit_linear_shiftgelu.argtypes = [vp, i64, i32, vp, i32, vp, vp, vp, i32, i32, i32, Dyadic, vp, vp]
+            L.ivit_linear_shiftgelu.argtypes = [vp, i64, i32, vp, i32, vp, vp, vp, i32, i32, i32, i32, Dyadic, vp, vp]
             L.ivit_attention.restype = C.c_int
             L.ivit_attention.argtypes = [vp, i32, i32, i32, Dyadic, i32, i32, i32, i32, Dyadic, vp, vp]
             L.ivit_shiftgelu.restype = C.c_int
@@ -129,13 +131,13 @@ def lib() -> C.CDLL:
             L.ivit_patch_embed_workspace_bytes.restype = C.c_size_t
             L.ivit_patch_embed_workspace_bytes.argtypes = [i32, i32, i32, i32, i32, i32]
             L.ivit_patch_embed.restype = C.c_int
-            L.ivit_patch_embed.argtypes = [vp, i32, i32, i32, i32, i32, vp, i32, vp, vp, vp, vp, vp, Residual, vp,
-                                           C.c_size_t, vp, vp]
+            L.ivit_patch_embed.argtypes = [vp, i32, i32, i32, i32, i32, vp, i32, vp, vp, vp, i32, vp, vp, Residual,
+                                           vp, C.c_size_t, vp, vp]
             L.ivit_head_workspace_bytes.restype = C.c_size_t
             L.ivit_head_workspace_bytes.argtypes = [i32, i32]
             L.ivit_head.restype = C.c_int
-            L.ivit_head.argtypes = [vp, i32, i32, i32, vp, vp, i32, i32, Dyadic, vp, i32, vp, vp, vp, vp, C.c_size_t,
-                                    vp, vp]
+            L.ivit_head.argtypes = [vp, i32, i32, i32, vp, vp, i32, i32, Dyadic, vp, i32, vp, vp, vp, i32, vp,
+                                    C.c_size_t, vp, vp]
             L.ivit_model_workspace_bytes.restype = C.c_size_t
             L.ivit_model_workspace_bytes.argtypes = [C.POINTER(ModelParams), i32, i32, i32]
             L.ivit_model_forward.restype = C.c_int
@@ -215,8 +217,9 @@ def ivit_i0_from_scale(S: float) -> int:
 # operators
 # ---------------------------------------------------------------------------
 
-def ivit_linear_requant(X, W, bias, b, c, Y, out_bits: int = 8, skip=None, res=None, stream=None):
-    """Y = sat((b_j (X W^T + bias)_ij) >> c_j) [+ residual]; X [M,K], W [N,K], Y [M,N] int8."""
+def ivit_linear_requant(X, W, bias, b, c, Y, out_bits: int = 8, skip=None, res=None, stream=None, rounding: int = 0):
+    """Y = sat((b_j (X W^T + bias)_ij) >> c_j) [+ residual]; X [M,K], W [N,K], Y [M,N] int8
+    (rounding 1: the requant rounds half up)."""
     M, K = X.shape
     N = W.shape[0]
     if W.shape[1] != K or tuple(Y.shape) != (M, N):
@@ -225,14 +228,14 @@ def ivit_linear_requant(X, W, bias, b, c, Y, out_bits: int = 8, skip=None, res=N
         raise ValueError("skip shape mismatch")
     st = lib().ivit_linear_requant(_ptr(X, torch.int8, "X"), M, K, _ptr(W, torch.int8, "W"), N,
                                    _ptr(bias, torch.int32, "bias"), _ptr(b, torch.int32, "b"),
-                                   _ptr(c, torch.int8, "c"), int(out_bits), _ptr(skip, torch.int8, "skip"),
+                                   _ptr(c, torch.int8, "c"), int(out_bits), int(rounding), _ptr(skip, torch.int8, "skip"),
                                    _res(res), _ptr(Y, torch.int8, "Y"), _stream(stream))
     _check("ivit_linear_requant", st)
     return Y
 
 
 def ivit_linear_shiftgelu(X, W, bias, b, c, gelu_I0: int, gelu_M: int, gelu_k_out: int, gelu_out, Y,
-                          stream=None):
+                          stream=None, rounding: int = 0):
     """Y = ShiftGELU(sat_8((b_j (X W^T + bias)_ij) >> c_j)) in one kernel."""
     M, K = X.shape
     N = W.shape[0]
@@ -240,7 +243,7 @@ def ivit_linear_shiftgelu(X, W, bias, b, c, gelu_I0: int, gelu_M: int, gelu_k_ou
         raise ValueError("shape mismatch")
     st = lib().ivit_linear_shiftgelu(_ptr(X, torch.int8, "X"), M, K, _ptr(W, torch.int8, "W"), N,
                                      _ptr(bias, torch.int32, "bias"), _ptr(b, torch.int32, "b"),
-                                     _ptr(c, torch.int8, "c"), int(gelu_I0), int(gelu_M), int(gelu_k_out),
+                                     _ptr(c, torch.int8, "c"), int(rounding), int(gelu_I0), int(gelu_M), int(gelu_k_out),
                                      _dy(gelu_out), _ptr(Y, torch.int8, "Y"), _stream(stream))
     _check("ivit_linear_shiftgelu", st)
     return Y
@@ -321,14 +324,14 @@ def ivit_patch_embed_workspace_bytes(B: int, C_in: int, Hi: int, Wi: int, P: int
     return int(lib().ivit_patch_embed_workspace_bytes(int(B), int(C_in), int(Hi), int(Wi), int(P), int(D)))
 
 
-def ivit_patch_embed(img, P: int, W, bias, b, c, cls, pos, pos_add, workspace, x, stream=None):
+def ivit_patch_embed(img, P: int, W, bias, b, c, cls, pos, pos_add, workspace, x, stream=None, rounding: int = 0):
     """x [B*(Np+1), D] from img [B, C, Hi, Wi]: patches through W [D, C*P*P],
     the class token first, the position embedding joined by ``pos_add``."""
     B, C_in, Hi, Wi = img.shape
     D = W.shape[0]
     st = lib().ivit_patch_embed(_ptr(img, torch.int8, "img"), B, C_in, Hi, Wi, int(P), _ptr(W, torch.int8, "W"), D,
                                 _ptr(bias, torch.int32, "bias"), _ptr(b, torch.int32, "b"), _ptr(c, torch.int8, "c"),
-                                _ptr(cls, torch.int8, "cls"), _ptr(pos, torch.int8, "pos"), _res(pos_add),
+                                int(rounding), _ptr(cls, torch.int8, "cls"), _ptr(pos, torch.int8, "pos"), _res(pos_add),
                                 _ptr(workspace, torch.uint8, "workspace"), workspace.numel(), _ptr(x, torch.int8, "x"),
                                 _stream(stream))
     _check("ivit_patch_embed", st)
@@ -340,13 +343,14 @@ def ivit_head_workspace_bytes(B: int, D: int) -> int:
 
 
 def ivit_head(x, B: int, Ntok: int, gamma, beta, F: int, M_ln: int, ln_out, W, bias, b, c, workspace, logits,
-              stream=None):
+              stream=None, rounding: int = 0):
     """logits [B, Ncls] from the class tokens of x [B*Ntok, D]."""
     D = x.shape[1]
     st = lib().ivit_head(_ptr(x, torch.int8, "x"), int(B), int(Ntok), D, _ptr(gamma, torch.int8, "gamma"),
                          _ptr(beta, torch.int32, "beta"), int(F), int(M_ln), _dy(ln_out), _ptr(W, torch.int8, "W"),
                          W.shape[0], _ptr(bias, torch.int32, "bias"), _ptr(b, torch.int32, "b"),
-                         _ptr(c, torch.int8, "c"), _ptr(workspace, torch.uint8, "workspace"), workspace.numel(),
+                         _ptr(c, torch.int8, "c"), int(rounding), _ptr(workspace, torch.uint8, "workspace"),
+                         workspace.numel(),
                          _ptr(logits, torch.int8, "logits"), _stream(stream))
     _check("ivit_head", st)
     return logits

@@ -166,8 +166,9 @@ ivit_status ivit_i0_from_scale(double S, int32_t* out) {
 
 ivit_status ivit_linear_requant(const int8_t* X, int64_t M, int32_t K, const int8_t* W, int32_t N,
                                 const int32_t* bias, const int32_t* b, const int8_t* c, int32_t out_bits,
-                                const int8_t* skip, ivit_residual res, int8_t* Y, ivit_stream_t stream) {
-  if (!X || !W || !b || !c || !Y) return IVIT_ERR_INVALID_ARG;
+                                int32_t rounding, const int8_t* skip, ivit_residual res, int8_t* Y,
+                                ivit_stream_t stream) {
+  if (!X || !W || !b || !c || !Y || (rounding != 0 && rounding != 1)) return IVIT_ERR_INVALID_ARG;
   if (!aligned16(X) || !aligned16(W) || !aligned16(b) || !aligned16(c) || !aligned16(Y) ||
       (bias && !aligned16(bias)) || (skip && !aligned16(skip)))
     return IVIT_ERR_INVALID_ARG;
@@ -178,15 +179,16 @@ ivit_status ivit_linear_requant(const int8_t* X, int64_t M, int32_t K, const int
   DeviceCtx dc;
   ivit_status st = device_ctx(&dc);
   if (st != IVIT_OK) return st;
-  return launch_gemm(dc, X, M, K, W, N, bias, b, c, out_bits, skip ? kEpiResidual : kEpiPlain, skip, res, nullptr, Y,
+  return launch_gemm(dc, X, M, K, W, N, bias, b, c, out_bits, rounding != 0, skip ? kEpiResidual : kEpiPlain, skip,
+                     res, nullptr, Y,
                      (cudaStream_t)stream);
 }
 
 ivit_status ivit_linear_shiftgelu(const int8_t* X, int64_t M, int32_t K, const int8_t* W, int32_t N,
-                                  const int32_t* bias, const int32_t* b, const int8_t* c, int32_t gelu_I0,
-                                  int32_t gelu_M, int32_t gelu_k_out, ivit_dyadic gelu_out, int8_t* Y,
-                                  ivit_stream_t stream) {
-  if (!X || !W || !b || !c || !Y) return IVIT_ERR_INVALID_ARG;
+                                  const int32_t* bias, const int32_t* b, const int8_t* c, int32_t rounding,
+                                  int32_t gelu_I0, int32_t gelu_M, int32_t gelu_k_out, ivit_dyadic gelu_out,
+                                  int8_t* Y, ivit_stream_t stream) {
+  if (!X || !W || !b || !c || !Y || (rounding != 0 && rounding != 1)) return IVIT_ERR_INVALID_ARG;
   if (!aligned16(X) || !aligned16(W) || !aligned16(b) || !aligned16(c) || !aligned16(Y) ||
       (bias && !aligned16(bias)))
     return IVIT_ERR_INVALID_ARG;
@@ -197,7 +199,8 @@ ivit_status ivit_linear_shiftgelu(const int8_t* X, int64_t M, int32_t K, const i
   ivit_status st = device_ctx(&dc);
   if (st != IVIT_OK) return st;
   const GeluParams gp{gelu_I0, gelu_M, gelu_k_out, gelu_out};
-  return launch_gemm(dc, X, M, K, W, N, bias, b, c, 8, kEpiGelu, nullptr, ivit_residual{0, 0, 0}, &gp, Y,
+  return launch_gemm(dc, X, M, K, W, N, bias, b, c, 8, rounding != 0, kEpiGelu, nullptr, ivit_residual{0, 0, 0}, &gp,
+                     Y,
                      (cudaStream_t)stream);
 }
 
@@ -273,7 +276,7 @@ ivit_status check_block(const ivit_block_params* p, const int8_t* x, const int8_
       !valid_shiftmax(p->gelu_I0, p->gelu_M, p->gelu_k_out) || !valid_dyadic(p->logit) ||
       !valid_dyadic(p->attn_out) || !valid_dyadic(p->gelu_out) || !valid_dyadic(p->ln1_out) ||
       !valid_dyadic(p->ln2_out) || !valid_residual(p->res1) || !valid_residual(p->res2) || p->ln_F < 0 ||
-      p->ln_F > 14 || p->ln_M < p->ln_F || p->ln_M > 23)
+      p->ln_F > 14 || p->ln_M < p->ln_F || p->ln_M > 23 || (p->linear_round != 0 && p->linear_round != 1))
     return IVIT_ERR_INVALID_ARG;
   if (!attention_config_supported(N, p->k_s, p->attn_I0)) return IVIT_ERR_UNSUPPORTED;
   return IVIT_OK;
@@ -297,7 +300,8 @@ ivit_status enqueue_block(const DeviceCtx& dc, const ivit_block_params* p, const
   if ((st = launch_layernorm(dc, x, T, D, p->ln1_gamma, p->ln1_beta, p->ln_F, p->ln_M, p->ln1_out, ln, s)) != IVIT_OK)
     return st;
   // a2 QKV
-  if ((st = launch_gemm(dc, ln, T, D, p->w_qkv, 3 * D, p->bias_qkv, p->b_qkv, p->c_qkv, 8, kEpiPlain, nullptr, none,
+  const bool rnd = p->linear_round != 0;
+  if ((st = launch_gemm(dc, ln, T, D, p->w_qkv, 3 * D, p->bias_qkv, p->b_qkv, p->c_qkv, 8, rnd, kEpiPlain, nullptr, none,
                         nullptr, qkv, s)) != IVIT_OK)
     return st;
   // a3-a5 logits, Shiftmax, A V
@@ -305,7 +309,7 @@ ivit_status enqueue_block(const DeviceCtx& dc, const ivit_block_params* p, const
                              p->attn_out, ctx, s)) != IVIT_OK)
     return st;
   // a6 W^O + residual 1
-  if ((st = launch_gemm(dc, ctx, T, D, p->w_o, D, p->bias_o, p->b_o, p->c_o, 8, kEpiResidual, x, p->res1, nullptr,
+  if ((st = launch_gemm(dc, ctx, T, D, p->w_o, D, p->bias_o, p->b_o, p->c_o, 8, rnd, kEpiResidual, x, p->res1, nullptr,
                         xh, s)) != IVIT_OK)
     return st;
   // a7 LN2
@@ -314,11 +318,12 @@ ivit_status enqueue_block(const DeviceCtx& dc, const ivit_block_params* p, const
     return st;
   // a8 + a9 fc1 with ShiftGELU in the epilogue
   const GeluParams gp{p->gelu_I0, p->gelu_M, p->gelu_k_out, p->gelu_out};
-  if ((st = launch_gemm(dc, ln, T, D, p->w1, Dm, p->bias1, p->b1, p->c1, 8, kEpiGelu, nullptr, none, &gp, g, s)) !=
+  if ((st = launch_gemm(dc, ln, T, D, p->w1, Dm, p->bias1, p->b1, p->c1, 8, rnd, kEpiGelu, nullptr, none, &gp, g, s)) !=
       IVIT_OK)
     return st;
   // a10 fc2 + residual 2
-  return launch_gemm(dc, g, T, Dm, p->w2, D, p->bias2, p->b2, p->c2, 8, kEpiResidual, xh, p->res2, nullptr, y, s);
+  return launch_gemm(dc, g, T, Dm, p->w2, D, p->bias2, p->b2, p->c2, 8, rnd, kEpiResidual, xh, p->res2, nullptr, y,
+                     s);
 }
 
 }  // namespace
@@ -355,9 +360,10 @@ namespace {
 
 ivit_status check_patch_embed(const int8_t* img, int32_t B, int32_t C, int32_t Hi, int32_t Wi, int32_t P,
                               const int8_t* W, int32_t D, const int32_t* bias, const int32_t* b, const int8_t* c,
-                              const int8_t* cls, const int8_t* pos, ivit_residual pos_add, const void* workspace,
+                              int32_t rounding, const int8_t* cls, const int8_t* pos, ivit_residual pos_add, const void* workspace,
                               size_t workspace_bytes, const int8_t* x) {
-  if (!img || !W || !b || !c || !cls || !pos || !x || !workspace) return IVIT_ERR_INVALID_ARG;
+  if (!img || !W || !b || !c || !cls || !pos || !x || !workspace || (rounding != 0 && rounding != 1))
+    return IVIT_ERR_INVALID_ARG;
   if (!aligned16(img) || !aligned16(W) || !aligned16(b) || !aligned16(c) || !aligned16(cls) || !aligned16(pos) ||
       !aligned16(x) || (bias && !aligned16(bias)) || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
     return IVIT_ERR_INVALID_ARG;
@@ -374,7 +380,7 @@ ivit_status check_patch_embed(const int8_t* img, int32_t B, int32_t C, int32_t H
 
 ivit_status enqueue_patch_embed(const DeviceCtx& dc, const int8_t* img, int32_t B, int32_t C, int32_t Hi,
                                 int32_t Wi, int32_t P, const int8_t* W, int32_t D, const int32_t* bias,
-                                const int32_t* b, const int8_t* c, const int8_t* cls, const int8_t* pos,
+                                const int32_t* b, const int8_t* c, bool round, const int8_t* cls, const int8_t* pos,
                                 ivit_residual pos_add, void* workspace, int8_t* x, cudaStream_t s) {
   const int32_t Np = (Hi / P) * (Wi / P), K = C * P * P;
   const int64_t rows = (int64_t)B * Np;
@@ -383,7 +389,7 @@ ivit_status enqueue_patch_embed(const DeviceCtx& dc, const int8_t* img, int32_t 
   int8_t* e = z + up((size_t)rows * K);
   ivit_status st;
   if ((st = launch_im2col(dc, img, B, C, Hi, Wi, P, z, s)) != IVIT_OK) return st;
-  if ((st = launch_gemm(dc, z, rows, K, W, D, bias, b, c, 8, kEpiPlain, nullptr, ivit_residual{0, 0, 0}, nullptr, e,
+  if ((st = launch_gemm(dc, z, rows, K, W, D, bias, b, c, 8, round, kEpiPlain, nullptr, ivit_residual{0, 0, 0}, nullptr, e,
                         s)) != IVIT_OK)
     return st;
   return launch_tokens(dc, e, cls, pos, pos_add, B, Np, D, x, s);
@@ -391,9 +397,10 @@ ivit_status enqueue_patch_embed(const DeviceCtx& dc, const int8_t* img, int32_t 
 
 ivit_status check_head(const int8_t* x, int32_t B, int32_t Ntok, int32_t D, const int8_t* gamma,
                        const int32_t* beta, int32_t F, int32_t M_ln, ivit_dyadic ln_out, const int8_t* W,
-                       int32_t Ncls, const int32_t* bias, const int32_t* b, const int8_t* c, const void* workspace,
-                       size_t workspace_bytes, const int8_t* logits) {
-  if (!x || !gamma || !beta || !W || !b || !c || !logits || !workspace) return IVIT_ERR_INVALID_ARG;
+                       int32_t Ncls, const int32_t* bias, const int32_t* b, const int8_t* c, int32_t rounding,
+                       const void* workspace, size_t workspace_bytes, const int8_t* logits) {
+  if (!x || !gamma || !beta || !W || !b || !c || !logits || !workspace || (rounding != 0 && rounding != 1))
+    return IVIT_ERR_INVALID_ARG;
   if (!aligned16(x) || !aligned16(gamma) || !aligned16(beta) || !aligned16(W) || !aligned16(b) || !aligned16(c) ||
       !aligned16(logits) || (bias && !aligned16(bias)) || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
     return IVIT_ERR_INVALID_ARG;
@@ -408,14 +415,15 @@ ivit_status check_head(const int8_t* x, int32_t B, int32_t Ntok, int32_t D, cons
 ivit_status enqueue_head(const DeviceCtx& dc, const int8_t* x, int32_t B, int32_t Ntok, int32_t D,
                          const int8_t* gamma, const int32_t* beta, int32_t F, int32_t M_ln, ivit_dyadic ln_out,
                          const int8_t* W, int32_t Ncls, const int32_t* bias, const int32_t* b, const int8_t* c,
-                         void* workspace, int8_t* logits, cudaStream_t s) {
+                         bool round, void* workspace, int8_t* logits, cudaStream_t s) {
   auto up = [](size_t v) { return (v + 255) / 256 * 256; };
   int8_t* t = static_cast<int8_t*>(workspace);
   int8_t* n = t + up((size_t)B * D);
   ivit_status st;
   if ((st = launch_gather_rows(dc, x, B, Ntok, D, t, s)) != IVIT_OK) return st;
   if ((st = launch_layernorm(dc, t, B, D, gamma, beta, F, M_ln, ln_out, n, s)) != IVIT_OK) return st;
-  return launch_gemm(dc, n, B, D, W, Ncls, bias, b, c, 8, kEpiPlain, nullptr, ivit_residual{0, 0, 0}, nullptr, logits,
+  return launch_gemm(dc, n, B, D, W, Ncls, bias, b, c, 8, round, kEpiPlain, nullptr, ivit_residual{0, 0, 0}, nullptr,
+                     logits,
                      s);
 }
 
@@ -423,28 +431,28 @@ ivit_status enqueue_head(const DeviceCtx& dc, const int8_t* x, int32_t B, int32_
 
 ivit_status ivit_patch_embed(const int8_t* img, int32_t B, int32_t C, int32_t Hi, int32_t Wi, int32_t P,
                              const int8_t* W, int32_t D, const int32_t* bias, const int32_t* b, const int8_t* c,
-                             const int8_t* cls, const int8_t* pos, ivit_residual pos_add, void* workspace,
-                             size_t workspace_bytes, int8_t* x, ivit_stream_t stream) {
-  ivit_status st = check_patch_embed(img, B, C, Hi, Wi, P, W, D, bias, b, c, cls, pos, pos_add, workspace,
+                             int32_t rounding, const int8_t* cls, const int8_t* pos, ivit_residual pos_add,
+                             void* workspace, size_t workspace_bytes, int8_t* x, ivit_stream_t stream) {
+  ivit_status st = check_patch_embed(img, B, C, Hi, Wi, P, W, D, bias, b, c, rounding, cls, pos, pos_add, workspace,
                                      workspace_bytes, x);
   if (st != IVIT_OK || B == 0) return st;
   DeviceCtx dc;
   if ((st = device_ctx(&dc)) != IVIT_OK) return st;
-  return enqueue_patch_embed(dc, img, B, C, Hi, Wi, P, W, D, bias, b, c, cls, pos, pos_add, workspace, x,
-                             (cudaStream_t)stream);
+  return enqueue_patch_embed(dc, img, B, C, Hi, Wi, P, W, D, bias, b, c, rounding != 0, cls, pos, pos_add,
+                             workspace, x, (cudaStream_t)stream);
 }
 
 ivit_status ivit_head(const int8_t* x, int32_t B, int32_t Ntok, int32_t D, const int8_t* gamma, const int32_t* beta,
                       int32_t F, int32_t M_ln, ivit_dyadic ln_out, const int8_t* W, int32_t Ncls,
-                      const int32_t* bias, const int32_t* b, const int8_t* c, void* workspace,
+                      const int32_t* bias, const int32_t* b, const int8_t* c, int32_t rounding, void* workspace,
                       size_t workspace_bytes, int8_t* logits, ivit_stream_t stream) {
-  ivit_status st = check_head(x, B, Ntok, D, gamma, beta, F, M_ln, ln_out, W, Ncls, bias, b, c, workspace,
+  ivit_status st = check_head(x, B, Ntok, D, gamma, beta, F, M_ln, ln_out, W, Ncls, bias, b, c, rounding, workspace,
                               workspace_bytes, logits);
   if (st != IVIT_OK || B == 0) return st;
   DeviceCtx dc;
   if ((st = device_ctx(&dc)) != IVIT_OK) return st;
-  return enqueue_head(dc, x, B, Ntok, D, gamma, beta, F, M_ln, ln_out, W, Ncls, bias, b, c, workspace, logits,
-                      (cudaStream_t)stream);
+  return enqueue_head(dc, x, B, Ntok, D, gamma, beta, F, M_ln, ln_out, W, Ncls, bias, b, c, rounding != 0, workspace,
+                      logits, (cudaStream_t)stream);
 }
 
 size_t ivit_model_workspace_bytes(const ivit_model_params* m, int32_t B, int32_t Hi, int32_t Wi) {
@@ -480,7 +488,7 @@ ivit_status ivit_model_forward(const ivit_model_params* m, const int8_t* img, in
   const size_t scratch_bytes = workspace_bytes - 2 * up((size_t)B * Ntok * m->D);
   // every step is checked before anything is enqueued
   ivit_status st = check_patch_embed(img, B, m->C, Hi, Wi, m->P, m->w_pe, m->D, m->bias_pe, m->b_pe, m->c_pe,
-                                     m->cls, m->pos, m->pos_add, scratch, scratch_bytes, tok[0]);
+                                     m->linear_round, m->cls, m->pos, m->pos_add, scratch, scratch_bytes, tok[0]);
   if (st != IVIT_OK) return st;
   for (int32_t i = 0; i < m->n_blocks; ++i) {
     if (m->blocks[i].D != m->D) return IVIT_ERR_INVALID_ARG;
@@ -488,22 +496,22 @@ ivit_status ivit_model_forward(const ivit_model_params* m, const int8_t* img, in
       return st;
   }
   if ((st = check_head(tok[m->n_blocks & 1], B, Ntok, m->D, m->head_gamma, m->head_beta, m->head_ln_F, m->head_ln_M,
-                       m->head_ln_out, m->w_head, m->Ncls, m->bias_head, m->b_head, m->c_head, scratch, scratch_bytes,
-                       logits)) != IVIT_OK)
+                       m->head_ln_out, m->w_head, m->Ncls, m->bias_head, m->b_head, m->c_head, m->linear_round,
+                       scratch, scratch_bytes, logits)) != IVIT_OK)
     return st;
   if (B == 0) return IVIT_OK;
   DeviceCtx dc;
   if ((st = device_ctx(&dc)) != IVIT_OK) return st;
   cudaStream_t s = (cudaStream_t)stream;
-  if ((st = enqueue_patch_embed(dc, img, B, m->C, Hi, Wi, m->P, m->w_pe, m->D, m->bias_pe, m->b_pe, m->c_pe, m->cls,
-                                m->pos, m->pos_add, scratch, tok[0], s)) != IVIT_OK)
+  if ((st = enqueue_patch_embed(dc, img, B, m->C, Hi, Wi, m->P, m->w_pe, m->D, m->bias_pe, m->b_pe, m->c_pe,
+                                m->linear_round != 0, m->cls, m->pos, m->pos_add, scratch, tok[0], s)) != IVIT_OK)
     return st;
   for (int32_t i = 0; i < m->n_blocks; ++i)
     if ((st = enqueue_block(dc, &m->blocks[i], tok[i & 1], tok[(i + 1) & 1], scratch, B, Ntok, s)) != IVIT_OK)
       return st;
   return enqueue_head(dc, tok[m->n_blocks & 1], B, Ntok, m->D, m->head_gamma, m->head_beta, m->head_ln_F,
-                      m->head_ln_M, m->head_ln_out, m->w_head, m->Ncls, m->bias_head, m->b_head, m->c_head, scratch,
-                      logits, s);
+                      m->head_ln_M, m->head_ln_out, m->w_head, m->Ncls, m->bias_head, m->b_head, m->c_head,
+                      m->linear_round != 0, scratch, logits, s);
 }
 
 ivit_status ivit_stream_status(ivit_stream_t stream) {

@@ -70,6 +70,7 @@ struct GemmArgs {
   const int32_t* b;
   const int8_t* c;
   int32_t lo, hi;  // saturation range of the requantised output
+  int32_t round;   // 1: the requant rounds half up (else the floor shift)
   ivit_residual res;
   GeluParams gelu;
   int* status;
@@ -147,16 +148,36 @@ IVIT_DEV ChanConst chan_const(int32_t b, int32_t c, int32_t bias, int32_t K) {
 }
 
 // Requant forms, chosen per warp and tile: every channel of the warp fast, or
-// the 64-bit product with or without the accumulator clamp.
-enum ReqForm : int { kReqFast = 0, kReqWide = 1, kReqWideClamp = 2 };
+// the 64-bit product with or without the accumulator clamp; each with the
+// floor shift or, in the round-half-up variant of the linear layers, with
+// 2^(c - 1) added before it.
+enum ReqForm : int {
+  kReqFast = 0,
+  kReqWide = 1,
+  kReqWideClamp = 2,
+  kReqRound = 3,  // added to a form: round half up
+};
 
-// floor(b acc / 2^c); in the wide forms the result fits int32 (see above), so
-// the low word of the 64-bit shift is one funnel shift (c <= 31)
+// floor(b acc / 2^c) (ROUND: floor(b acc / 2^c + 1/2)).  In the wide forms
+// the result fits int32 (see above; adding half an LSB changes nothing
+// there), so the low word of the 64-bit shift is one funnel shift (c <= 31).
+// The fast form with rounding: b acc / 2^c = bq acc / 2^32 exactly, and
+// floor((bq acc + 2^31) / 2^32) is the high word plus the top bit of the low
+// word.  The clamp keeps the saturation direction: acc = +-u still gives a
+// result of magnitude >= 128 after rounding.
 template <int REQ>
 IVIT_DEV int32_t requant_acc(int32_t acc, const ChanConst& k) {
-  if (REQ == kReqFast) return __mulhi(k.bq, acc);
-  const int32_t a = REQ == kReqWideClamp ? min(max(acc, -k.lim), k.lim) : acc;
-  const int64_t v = (int64_t)k.b * a;
+  constexpr int form = REQ % kReqRound;
+  constexpr bool round = REQ >= kReqRound;
+  if (form == kReqFast) {
+    const int32_t hi = __mulhi(k.bq, acc);
+    if (!round) return hi;
+    const uint32_t lo = (uint32_t)k.bq * (uint32_t)acc;
+    return hi + (int32_t)(lo >> 31);
+  }
+  const int32_t a = form == kReqWideClamp ? min(max(acc, -k.lim), k.lim) : acc;
+  int64_t v = (int64_t)k.b * a;
+  if (round && k.c > 0) v += (int64_t)1 << (k.c - 1);
   return (int32_t)__funnelshift_r((uint32_t)v, (uint32_t)(v >> 32), (uint32_t)k.c);
 }
 
@@ -535,13 +556,24 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       }
       tc_fence_after();
       const uint32_t tbase = tlane + (uint32_t)(acc * BN);
-      if (req == kReqFast)
-        epi_tile<EPI, NARROW, kReqFast>(tbase, c_begin, n, kc, args, gelu_tab, slots, ofs_even, ofs_odd, sel2, sel1);
-      else if (req == kReqWide)
-        epi_tile<EPI, NARROW, kReqWide>(tbase, c_begin, n, kc, args, gelu_tab, slots, ofs_even, ofs_odd, sel2, sel1);
-      else
-        epi_tile<EPI, NARROW, kReqWideClamp>(tbase, c_begin, n, kc, args, gelu_tab, slots, ofs_even, ofs_odd, sel2,
-                                             sel1);
+#define IVIT_EPI_TILE(R) \
+  epi_tile<EPI, NARROW, R>(tbase, c_begin, n, kc, args, gelu_tab, slots, ofs_even, ofs_odd, sel2, sel1)
+      if (!args.round) {
+        if (req == kReqFast)
+          IVIT_EPI_TILE(kReqFast);
+        else if (req == kReqWide)
+          IVIT_EPI_TILE(kReqWide);
+        else
+          IVIT_EPI_TILE(kReqWideClamp);
+      } else {
+        if (req == kReqFast)
+          IVIT_EPI_TILE(kReqFast + kReqRound);
+        else if (req == kReqWide)
+          IVIT_EPI_TILE(kReqWide + kReqRound);
+        else
+          IVIT_EPI_TILE(kReqWideClamp + kReqRound);
+      }
+#undef IVIT_EPI_TILE
       // staged words -> global by TMA once the part's four warps have written
       // them (rows past M and channels past N are clipped)
       fence_proxy_async_smem();
@@ -650,10 +682,11 @@ ivit_status dispatch_bn(const DeviceCtx& dc, const int8_t* X, const int8_t* W, c
 }  // namespace
 
 ivit_status launch_gemm(const DeviceCtx& dc, const int8_t* X, int64_t M, int32_t K, const int8_t* W, int32_t N,
-                        const int32_t* bias, const int32_t* b, const int8_t* c, int32_t out_bits, EpiMode mode,
-                        const int8_t* skip, ivit_residual res, const GeluParams* gelu, int8_t* Y,
+                        const int32_t* bias, const int32_t* b, const int8_t* c, int32_t out_bits, bool round,
+                        EpiMode mode, const int8_t* skip, ivit_residual res, const GeluParams* gelu, int8_t* Y,
                         cudaStream_t stream) {
   GemmArgs a;
+  a.round = round ? 1 : 0;
   a.M = M;
   a.N = N;
   a.K = K;

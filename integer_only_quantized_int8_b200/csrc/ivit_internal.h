@@ -51,8 +51,8 @@ ivit_status encode_tmap_2d_u8(CUtensorMap* map, const void* base, uint64_t inner
                               CUtensorMapSwizzle swizzle);
 
 ivit_status launch_gemm(const DeviceCtx& dc, const int8_t* X, int64_t M, int32_t K, const int8_t* W, int32_t N,
-                        const int32_t* bias, const int32_t* b, const int8_t* c, int32_t out_bits, EpiMode mode,
-                        const int8_t* skip, ivit_residual res, const GeluParams* gelu, int8_t* Y,
+                        const int32_t* bias, const int32_t* b, const int8_t* c, int32_t out_bits, bool round,
+                        EpiMode mode, const int8_t* skip, ivit_residual res, const GeluParams* gelu, int8_t* Y,
                         cudaStream_t stream);
 
 // Whether the attention kernels take (N, k_s, I0): up to 640 keys; logits

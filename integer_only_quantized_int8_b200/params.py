@@ -101,6 +101,7 @@ def to_device(p: Dict, device="cuda") -> DeviceBlockParams:
     s.res1 = Residual(*p["res1"])
     s.res2 = Residual(*p["res2"])
     s.ln_F, s.ln_M = p["ln_F"], p["ln_M"]
+    s.linear_round = int(p.get("linear_round", 0))
     return DeviceBlockParams(tensors=t, c=s, host=p)
 
 
@@ -165,4 +166,5 @@ def model_to_device(m: Dict, device="cuda") -> DeviceModelParams:
     s.blocks = arr
     s.head_ln_F, s.head_ln_M = m["ln_F"], m["ln_M"]
     s.head_ln_out = Dyadic(*m["head_ln_out"])
+    s.linear_round = int(m.get("linear_round", 0))
     return DeviceModelParams(tensors=t, blocks=blocks, block_array=arr, c=s, host=m)

@@ -73,22 +73,23 @@ def test_validation_rejects_before_launch():
     L = ivit.lib()
     none = ivit.Residual(0, 0, 0)
     # null pointers
-    assert L.ivit_linear_requant(None, 16, 16, None, 16, None, None, None, 8, None, none, None, None) == 1
+    assert L.ivit_linear_requant(None, 16, 16, None, 16, None, None, None, 8, 0, None, none, None, None) == 1
     # misaligned pointer (odd address) and bad shapes; no device pointer is touched
     p = 0x1000
-    assert L.ivit_linear_requant(p + 1, 16, 16, p, 16, None, p, p, 8, None, none, p, None) == 1
-    assert L.ivit_linear_requant(p, 16, 24, p, 16, None, p, p, 8, None, none, p, None) == 1   # K % 16
-    assert L.ivit_linear_requant(p, 16, 16, p, 16, None, p, p, 9, None, none, p, None) == 1   # out_bits
+    assert L.ivit_linear_requant(p + 1, 16, 16, p, 16, None, p, p, 8, 0, None, none, p, None) == 1
+    assert L.ivit_linear_requant(p, 16, 24, p, 16, None, p, p, 8, 0, None, none, p, None) == 1   # K % 16
+    assert L.ivit_linear_requant(p, 16, 16, p, 16, None, p, p, 9, 0, None, none, p, None) == 1   # out_bits
+    assert L.ivit_linear_requant(p, 16, 16, p, 16, None, p, p, 8, 2, None, none, p, None) == 1   # rounding mode
     d = ivit.Dyadic(1, 0)
     assert L.ivit_attention(p, 1, 8, 1, d, 17, 4, 30, 8, d, p, None) == 1     # k_s > 16
     # patch embedding: null image, patch size not dividing the image, C P P not a multiple of 16
-    assert L.ivit_patch_embed(None, 1, 3, 32, 32, 16, p, 64, None, p, p, p, p, none, p, 1 << 20, p, None) == 1
-    assert L.ivit_patch_embed(p, 1, 3, 40, 32, 16, p, 64, None, p, p, p, p, none, p, 1 << 20, p, None) == 1
-    assert L.ivit_patch_embed(p, 1, 3, 28, 28, 14, p, 64, None, p, p, p, p, none, p, 1 << 20, p, None) == 1
-    assert L.ivit_patch_embed(p, 1, 3, 32, 32, 16, p, 64, None, p, p, p, p, none, p, 16, p, None) == 1  # workspace
+    assert L.ivit_patch_embed(None, 1, 3, 32, 32, 16, p, 64, None, p, p, 0, p, p, none, p, 1 << 20, p, None) == 1
+    assert L.ivit_patch_embed(p, 1, 3, 40, 32, 16, p, 64, None, p, p, 0, p, p, none, p, 1 << 20, p, None) == 1
+    assert L.ivit_patch_embed(p, 1, 3, 28, 28, 14, p, 64, None, p, p, 0, p, p, none, p, 1 << 20, p, None) == 1
+    assert L.ivit_patch_embed(p, 1, 3, 32, 32, 16, p, 64, None, p, p, 0, p, p, none, p, 16, p, None) == 1  # workspace
     # head: class count not a multiple of 16, width past 2048
-    assert L.ivit_head(p, 1, 3, 64, p, p, 7, 23, d, p, 1000, None, p, p, p, 1 << 20, p, None) == 1
-    assert L.ivit_head(p, 1, 3, 4096, p, p, 7, 23, d, p, 1008, None, p, p, p, 1 << 20, p, None) == 1
+    assert L.ivit_head(p, 1, 3, 64, p, p, 7, 23, d, p, 1000, None, p, p, 0, p, 1 << 20, p, None) == 1
+    assert L.ivit_head(p, 1, 3, 4096, p, p, 7, 23, d, p, 1008, None, p, p, 0, p, 1 << 20, p, None) == 1
     assert L.ivit_attention(p, 1, 300, 1, d, 12, 4, 30, 8, d, p, None) == 2   # wide logits past 256 keys
     assert L.ivit_attention(p, 1, 8, 1, d, 16, 50000, 30, 8, d, p, None) == 2  # n_max * I0 >= 2^32
     assert L.ivit_attention(p, 1, 8, 1, d, 8, 0, 30, 8, d, p, None) == 1      # I0 < 1

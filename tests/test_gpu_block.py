@@ -84,3 +84,22 @@ def test_block_parity_full_size(name):
         np.testing.assert_array_equal(got[b * wl.N:(b + 1) * wl.N], want[b], err_msg=f"{name} image {b}")
     # the block is not degenerate at this size: the output uses the int8 range
     assert np.unique(got).size > 100
+
+
+def test_block_parity_linear_round_half_up():
+    """A block whose four linear layers round half up, against the oracle's
+    block with the same reading."""
+    wl = synthetic.make_workload(seed=11, n_cal=2, B=2, N=61, D=192, H=3, Dm=768)
+    ip = ivit_params.integer_params(wl.blocks[0])
+    ip["linear_round"] = 1
+    dp = ivit_params.to_device(ip)
+    ws = torch.empty(ivit.ivit_block_workspace_bytes(wl.B, wl.N, wl.D, wl.Dm), dtype=torch.uint8, device="cuda")
+    x = torch.from_numpy(wl.x).cuda()
+    y = torch.empty_like(x)
+    ivit.ivit_block_forward(dp, x, y, ws, wl.B, wl.N)
+    op = oracle.block_params(wl.blocks[0])
+    op["linear_round"] = 1
+    want = oracle.block_forward(op, wl.x, wl.B, wl.N)
+    np.testing.assert_array_equal(y.cpu().numpy(), want)
+    op["linear_round"] = 0
+    assert not np.array_equal(want, oracle.block_forward(op, wl.x, wl.B, wl.N))

@@ -86,6 +86,53 @@ def test_linear_saturation_and_extremes():
     np.testing.assert_array_equal(host(Y), oracle.linear_requant(X, W, bias, b, c))
 
 
+@pytest.mark.parametrize("M,K,N", [(197, 192, 576), (300, 768, 3072), (129, 64, 272)])
+def test_linear_round_half_up_parity(M, K, N):
+    """The round-half-up variant of the linear requant: plain, residual and
+    narrow outputs, and the fused fc1 + ShiftGELU."""
+    lc = synthetic.linear_case(M, K, N, seed=3 * M + N, with_skip=True)
+    bq = [ivit.ivit_dyadic_from_double(r) for r in lc.ratio]
+    b = np.array([x[0] for x in bq], np.int32)
+    c = np.array([x[1] for x in bq], np.int32)
+    X, W = dev(lc.X, torch.int8), dev(lc.W, torch.int8)
+    bd, cd, biasd = dev(b, torch.int32), dev(c, torch.int8), dev(lc.bias, torch.int32)
+    Y = torch.empty((M, N), dtype=torch.int8, device="cuda")
+    ivit.ivit_linear_requant(X, W, biasd, bd, cd, Y, rounding=1)
+    want = oracle.linear_requant(lc.X, lc.W, lc.bias, b, c, rounding=1)
+    np.testing.assert_array_equal(host(Y), want)
+    assert not np.array_equal(want, oracle.linear_requant(lc.X, lc.W, lc.bias, b, c))  # the variant differs
+    res = ivit.ivit_residual_from_double(*lc.res_ratio)
+    ivit.ivit_linear_requant(X, W, biasd, bd, cd, Y, skip=dev(lc.skip, torch.int8), res=res, rounding=1)
+    np.testing.assert_array_equal(host(Y), oracle.linear_requant(lc.X, lc.W, lc.bias, b, c, skip=lc.skip, res=res,
+                                                                 rounding=1))
+    ivit.ivit_linear_requant(X, W, biasd, bd, cd, Y, out_bits=4, rounding=1)
+    np.testing.assert_array_equal(host(Y), oracle.linear_requant(lc.X, lc.W, lc.bias, b, c, out_bits=4, rounding=1))
+    gc = synthetic.gelu_case(1024, seed=M)
+    I0 = ivit.ivit_i0_from_scale(gc.S_h)
+    go = ivit.ivit_dyadic_from_double(gc.out_ratio)
+    ivit.ivit_linear_shiftgelu(X, W, biasd, bd, cd, I0, 30, 8, go, Y, rounding=1)
+    h = oracle.linear_requant(lc.X, lc.W, lc.bias, b, c, rounding=1)
+    np.testing.assert_array_equal(host(Y), oracle.shiftgelu(h, I0, 30, 8, go))
+
+
+def test_linear_round_half_up_extremes():
+    """Wide and clamped requant forms (b = 2^31 - 1, every shift 0..31) with
+    rounding, at K = 4096 with saturating inputs."""
+    r = np.random.default_rng(31)
+    M, K, N = 64, 4096, 32
+    X = r.integers(-128, 128, (M, K), dtype=np.int8)
+    X[::3] = -128
+    W = r.choice(np.array([-128, 127, 1, -1], np.int8), size=(N, K))
+    b = np.full(N, 2 ** 31 - 1, np.int32)
+    b[::2] = r.integers(1, 1 << 12, N // 2)
+    c = (np.arange(N) % 32).astype(np.int32)
+    bias = r.integers(-2 ** 20, 2 ** 20, size=N).astype(np.int32)
+    Y = torch.empty((M, N), dtype=torch.int8, device="cuda")
+    ivit.ivit_linear_requant(dev(X, torch.int8), dev(W, torch.int8), dev(bias, torch.int32), dev(b, torch.int32),
+                             dev(c, torch.int8), Y, rounding=1)
+    np.testing.assert_array_equal(host(Y), oracle.linear_requant(X, W, bias, b, c, rounding=1))
+
+
 # ---------------------------------------------------------------------------
 # fused attention with Shiftmax
 # ---------------------------------------------------------------------------
