@@ -629,6 +629,9 @@ def kernel_breakdown(ivit, wl, dp, ws, xs, reps, dev):
     add("attention_logits16", lambda i: ivit.ivit_attention(qkv, B, N, H, logit16, 16, I0_16, p["attn_M"],
                                                             p["attn_k_out"], p["attn_out"], ctx_o),
         "alu", SHIFTMAX_OPS_PER_SCORE * B * H * N * N, in_block=False)
+    add("gemm_qkv_round_half_up", lambda i: ivit.ivit_linear_requant(ln, t["w_qkv"], t["bias_qkv"], t["b_qkv"],
+                                                                     t["c_qkv"], qkv_o, rounding=1),
+        "tensor", gemm(T, D, 3 * D), in_block=False)
     add("gemm_o_residual", lambda i: ivit.ivit_linear_requant(ctx, t["w_o"], t["bias_o"], t["b_o"], t["c_o"], y,
                                                               skip=xs[i % R], res=p["res1"]),
         "tensor", gemm(T, D, D))

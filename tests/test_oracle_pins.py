@@ -556,3 +556,24 @@ def test_linear_round_half_up_variant():
     assert inside.sum() > 100
     assert np.all(np.abs(up[inside] - exact[inside]) <= 0.5)
     assert np.all((up - fl >= 0) & (up - fl <= 1))
+
+
+def test_linear_rounding_error_report():
+    """What the two readings of the requant cost in accuracy: against the
+    exact quotient b acc / 2^c, the floor shift is biased by -1/2 LSB on
+    average and round half up is unbiased; both stay within one LSB (floor)
+    or half an LSB (round) on every unsaturated output."""
+    r = np.random.default_rng(42)
+    M, K, N = 256, 192, 64
+    X = r.integers(-128, 128, (M, K), dtype=np.int8)
+    W = r.integers(-128, 128, (N, K), dtype=np.int8)
+    bias = r.integers(-2 ** 14, 2 ** 14, N).astype(np.int32)
+    b = r.integers(1 << 19, 1 << 20, N).astype(np.int32)
+    c = np.full(N, 31, np.int32)   # b / 2^c in [2^-12, 2^-11): outputs spread over tens of LSB
+    exact = (X.astype(np.int64) @ W.T.astype(np.int64) + bias) * b / 2.0 ** c
+    inside = np.abs(exact) < 126
+    assert inside.mean() > 0.9
+    e_floor = oracle.linear_requant(X, W, bias, b, c)[inside] - exact[inside]
+    e_round = oracle.linear_requant(X, W, bias, b, c, rounding=1)[inside] - exact[inside]
+    assert abs(e_floor.mean() + 0.5) < 0.02 and abs(e_round.mean()) < 0.02
+    assert np.all((e_floor <= 0) & (e_floor > -1)) and np.all(np.abs(e_round) <= 0.5)
