@@ -504,29 +504,50 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     int acc = 0;
     uint32_t acc_phase = 0;
     uint32_t skip_phase = 0;
-    // this lane's channel constants (multiplier, shift, bias) of a tile; the
-    // next tile's are loaded while the current one drains, so their L2
-    // latency stays off the tile's path
-    auto load_chan = [&](int t, int32_t& cb_b, int32_t& cb_c, int32_t& cb_bias) {
-      const int ch = (t % ch_tiles) * kBM + quarter * 32 + lane;
-      const bool ok = t < num_tiles && ch < N;
-      cb_b = ok ? __ldg(args.b + ch) : 0;
-      cb_c = ok ? (int32_t)__ldg(args.c + ch) : 0;
-      cb_bias = (ok && args.bias) ? __ldg(args.bias + ch) : 0;
+    // Tile coordinates advance by gridDim.x tiles without divisions: (cb, tb)
+    // of the current tile, cb1 / cb2 the channel blocks one and two tiles on.
+    const int step_cb = (int)gridDim.x % ch_tiles, step_tb = (int)gridDim.x / ch_tiles;
+    auto advance = [&](int& cbx, int& tbx) {
+      cbx += step_cb;
+      tbx += step_tb;
+      if (cbx >= ch_tiles) {
+        cbx -= ch_tiles;
+        ++tbx;
+      }
+    };
+    int cb = (int)blockIdx.x % ch_tiles, tb = (int)blockIdx.x / ch_tiles;
+    int cb1 = cb, tb1 = tb;
+    advance(cb1, tb1);
+    int cb2 = cb1, tb2 = tb1;
+    advance(cb2, tb2);
+    // This lane's channel constants (multiplier, shift, bias) are loaded one
+    // tile ahead and turned into the requant form at the end of the tile
+    // before, so neither their L2 latency nor their derivation sits on a
+    // tile's path.
+    auto load_chan = [&](int t, int cbx, int32_t& cb_b, int32_t& cb_c, int32_t& cb_bias) {
+      const int chx = cbx * kBM + quarter * 32 + lane;
+      const bool ok = t < num_tiles && chx < N;
+      cb_b = ok ? __ldg(args.b + chx) : 0;
+      cb_c = ok ? (int32_t)__ldg(args.c + chx) : 0;
+      cb_bias = (ok && args.bias) ? __ldg(args.bias + chx) : 0;
+    };
+    auto derive = [&](int cbx, int32_t vb, int32_t vc, int32_t vbias, ChanConst& kx, int& reqx) {
+      kx = cbx * kBM + quarter * 32 + lane < N ? chan_const(vb, vc, vbias, args.K) : chan_const(0, 0, 0, args.K);
+      // warp-uniform requant form
+      reqx = __all_sync(0xffffffffu, kx.fast) ? kReqFast
+                                               : (__any_sync(0xffffffffu, kx.needs_clamp) ? kReqWideClamp : kReqWide);
     };
     int32_t nb, nc, nbias;
-    load_chan(blockIdx.x, nb, nc, nbias);
+    load_chan(blockIdx.x, cb, nb, nc, nbias);
+    ChanConst kc;
+    int req;
+    derive(cb, nb, nc, nbias, kc, req);
     for (int t = blockIdx.x; t < num_tiles; t += gridDim.x) {
-      const int cb = t % ch_tiles, tb = t / ch_tiles;
-      const int ch0 = cb * kBM + quarter * 32;  // first channel of this warp
-      const int ch = ch0 + lane;                // this thread's output channel
-      const ChanConst kc = ch < N ? chan_const(nb, nc, nbias, args.K) : chan_const(0, 0, 0, args.K);
-      load_chan(t + (int)gridDim.x, nb, nc, nbias);
-      // warp-uniform requant form
-      const int req = __all_sync(0xffffffffu, kc.fast) ? kReqFast
-                      : (__any_sync(0xffffffffu, kc.needs_clamp) ? kReqWideClamp : kReqWide);
+      load_chan(t + (int)gridDim.x, cb1, nb, nc, nbias);
       const int64_t tok_base = (int64_t)tb * BN;
-      const int32_t next_bias = bias_of(t + 2 * (int)gridDim.x);
+      const int ch_next2 = cb2 * kBM + quarter * 32 + lane;
+      const int32_t next_bias =
+          (args.bias && ch_next2 < N && t + 2 * (int)gridDim.x < num_tiles) ? __ldg(args.bias + ch_next2) : 0;
       int n = c_end - c_begin;  // chunks that hold at least one real token
       while (n > 0 && tok_base + 16 * (c_begin + n - 1) >= M) --n;
       const bool live = n > 0;  // the same for the part's four warps
@@ -593,6 +614,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       if (lane == 0) mbar_arrive(&tempty[acc]);
       acc ^= 1;
       if (acc == 0) acc_phase ^= 1;
+      // the next tile's requant form, from constants loaded during this one
+      derive(cb1, nb, nc, nbias, kc, req);
+      cb = cb1;
+      tb = tb1;
+      cb1 = cb2;
+      tb1 = tb2;
+      advance(cb2, tb2);
     }
     if (part_lead) bulk_wait_all();
     __syncwarp();
