@@ -626,9 +626,10 @@ def kernel_breakdown(ivit, wl, dp, ws, xs, reps, dev):
     S_l16 = (1.0 / p["attn_I0"]) * 255.0 / 65535.0
     logit16 = ivit.ivit_dyadic_from_double(p["logit"][0] / 2.0 ** p["logit"][1] * 65535.0 / 255.0)
     I0_16 = ivit.ivit_i0_from_scale(S_l16)
-    add("attention_logits16", lambda i: ivit.ivit_attention(qkv, B, N, H, logit16, 16, I0_16, p["attn_M"],
-                                                            p["attn_k_out"], p["attn_out"], ctx_o),
-        "alu", SHIFTMAX_OPS_PER_SCORE * B * H * N * N, in_block=False)
+    if N <= 256:  # 16-bit logits run on the short-sequence kernel only
+        add("attention_logits16", lambda i: ivit.ivit_attention(qkv, B, N, H, logit16, 16, I0_16, p["attn_M"],
+                                                                p["attn_k_out"], p["attn_out"], ctx_o),
+            "alu", SHIFTMAX_OPS_PER_SCORE * B * H * N * N, in_block=False)
     add("gemm_qkv_round_half_up", lambda i: ivit.ivit_linear_requant(ln, t["w_qkv"], t["bias_qkv"], t["b_qkv"],
                                                                      t["c_qkv"], qkv_o, rounding=1),
         "tensor", gemm(T, D, 3 * D), in_block=False)

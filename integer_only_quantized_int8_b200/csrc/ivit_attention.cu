@@ -1,6 +1,6 @@
 // ivit_attention.cu -- fused integer attention with Shiftmax on sm_100a.
 //
-// Per (128-query tile, head, image) one CTA of 4 warps computes
+// Per (128-query tile, head, image) one CTA of 16 warps computes
 //   S = Q K^T                 tcgen05.mma kind::i8 (s8 x s8 -> s32) into TMEM
 //   L = sat_ks((b_s S) >> c_s)  dyadic logit requant, row max     (CUDA cores)
 //   P = Shiftmax(L)           ShiftExp table + IntDiv, u8 probabilities
@@ -9,14 +9,17 @@
 // following "I-ViT: Integer-only Quantization for Efficient Vision Transformer
 // Inference", sections 3.2-3.3, and the Trio-ViT article, eqs. (1)-(3).  The
 // score matrix stays on chip: S in TMEM, k_s-bit logits and u8 P in shared
-// memory.  Thread t owns query row t of the tile (TMEM lane t), so the row
-// reductions need no shuffles.
+// memory.  The four warps w, w + 4, w + 8, w + 12 share TMEM lane quarter
+// w & 3 (query rows 32 (w & 3) .. + 31) and split every row's keys: each
+// reads a quarter of the score columns, keeps a partial row maximum and sum,
+// and the four partials of a row meet in shared memory.
 //
 // Shared memory (runtime N, keys padded to 64 for loads and 32 for the MMAs):
 //   R0  Q (128 x 64 B) and K (N64 x 64 B), 64B swizzle; later reused for P
 //       (128 x N32 u8, K-major, 128B swizzle, 16 KB per 128 keys)
 //   V   (N64 x 64 B), 64B swizzle, read MN-major by the P V MMA
-//   logits (128 rows x lstride B), exp table (2^k_s int32), barriers
+//   logits (128 rows x lstride B), exp table (2^k_s int32), the row
+//   partials (4 x 128 maxima, 4 x 128 sums), barriers
 #include <climits>
 
 #include "ivit_common.cuh"
@@ -25,7 +28,8 @@
 namespace ivit {
 namespace {
 
-constexpr int kAttnThreads = 128;
+constexpr int kAttnSplit = 4;                   // threads (warps of one lane quarter) per query row
+constexpr int kAttnThreads = 128 * kAttnSplit;  // 16 warps
 constexpr int kQTile = 128;
 constexpr int kHeadDim = 64;
 constexpr int kMaxKeys = 640;
@@ -46,7 +50,7 @@ struct AttnArgs {
 
 struct AttnLayout {
   int n64, n32, kblocks, lstride;
-  int r0_bytes, v_off, logit_off, tab_off, bar_off, total;
+  int r0_bytes, v_off, logit_off, tab_off, part_off, bar_off, total;
 };
 
 __host__ __device__ inline AttnLayout attn_layout(int N) {
@@ -64,7 +68,8 @@ __host__ __device__ inline AttnLayout attn_layout(int N) {
   L.v_off = L.r0_bytes;
   L.logit_off = L.v_off + (L.n64 * kHeadDim + 1023) / 1024 * 1024;
   L.tab_off = L.logit_off + kQTile * L.lstride;
-  L.bar_off = (L.tab_off + 256 * 4 + 15) / 16 * 16;
+  L.part_off = (L.tab_off + 256 * 4 + 15) / 16 * 16;
+  L.bar_off = L.part_off + 2 * kAttnSplit * kQTile * 4;
   L.total = L.bar_off + 64;
   return L;
 }
@@ -130,11 +135,17 @@ __global__ void __launch_bounds__(kAttnThreads)
   }
 
   bool ok = true;
+  const int quarter = warp & 3;           // TMEM lane quarter: query rows 32 quarter .. + 31
+  const int slice = warp >> 2;            // which quarter of every row's keys this thread takes
+  const int row = quarter * 32 + (tid & 31);
   int32_t mx = a.ks_lo;
-  int8_t* my_log = slog + tid * L.lstride;
-  const uint32_t t_lane = tmem + ((uint32_t)(warp * 32) << 16);
+  int8_t* my_log = slog + row * L.lstride;
+  const uint32_t t_lane = tmem + ((uint32_t)(quarter * 32) << 16);
+  int32_t* part_max = reinterpret_cast<int32_t*>(smem + L.part_off);  // [slice][row]
+  uint32_t* part_sum = reinterpret_cast<uint32_t*>(part_max + kAttnSplit * kQTile);
 
-  // ---- S = Q K^T in chunks of up to 256 keys, requantised to k_s-bit logits
+  // ---- S = Q K^T in chunks of up to 256 keys, requantised to k_s-bit logits;
+  // the chunk's 32-column groups go round-robin to the four slices
   const int nchunks = (L.n32 + 255) / 256;
   for (int c = 0; c < nchunks; ++c) {
     const int w = (L.n32 - c * 256) < 256 ? (L.n32 - c * 256) : 256;
@@ -156,7 +167,7 @@ __global__ void __launch_bounds__(kAttnThreads)
     ok = __all_sync(0xffffffffu, ok);  // warp-uniform: guards a warp-collective TMEM load
     tc_fence_after();
     if (ok) {
-      for (int cc = 0; cc < w / 32; ++cc) {
+      for (int cc = slice; cc < w / 32; cc += kAttnSplit) {
         uint32_t r[32];
         tmem_ld32(t_lane + (uint32_t)(cc * 32), r);
         tmem_ld_wait();
@@ -184,29 +195,38 @@ __global__ void __launch_bounds__(kAttnThreads)
     tc_fence_before();
     __syncthreads();
   }
+  // the row maximum from the four slices' partial maxima
+  part_max[slice * kQTile + row] = mx;
+  __syncthreads();
+  mx = max(max(part_max[row], part_max[kQTile + row]), max(part_max[2 * kQTile + row], part_max[3 * kQTile + row]));
 
-  // ---- Shiftmax row sum: e_j = ShiftExp(L_j - max) by table
+  // ---- Shiftmax row sum: e_j = ShiftExp(L_j - max) by table, over this
+  // slice's 16-key units u = slice, slice + 4, ...
   // (after a timed-out wait the logits are not written: skip to zero P)
   uint32_t sum = 0;
   const int nfull = ok ? N / 16 : 0;
-  for (int cidx = 0; cidx < nfull; ++cidx) {
-    const int4 v = *reinterpret_cast<const int4*>(my_log + cidx * 16);
+  for (int u = slice; u < nfull; u += kAttnSplit) {
+    const int4 v = *reinterpret_cast<const int4*>(my_log + u * 16);
     const int8_t* lb = reinterpret_cast<const int8_t*>(&v);
 #pragma unroll
     for (int e = 0; e < 16; ++e) sum += (uint32_t)tab[mx - (int32_t)lb[e]];
   }
-  if (ok)
+  if (ok && (nfull % kAttnSplit) == slice)  // the ragged last unit
     for (int j = nfull * 16; j < N; ++j) sum += (uint32_t)tab[mx - (int32_t)my_log[j]];
+  part_sum[slice * kQTile + row] = sum;
+  __syncthreads();
+  sum = (part_sum[row] + part_sum[kQTile + row]) + (part_sum[2 * kQTile + row] + part_sum[3 * kQTile + row]);
   if (sum == 0) sum = 1;
   const uint32_t dv = (1u << a.M) / sum;
   const int pshift = a.M - (a.k_out - 1);
 
-  // ---- P = (Dv e_j) >> (M - k_out + 1) as u8, into the K-major 128B-swizzled operand
+  // ---- P = (Dv e_j) >> (M - k_out + 1) as u8, into the K-major 128B-swizzled
+  // operand; this slice's 16-key units (zero past the last key)
   fence_proxy_async_smem();
-  const int rlo = tid & 7;
-  uint8_t* prow = sP + (tid >> 3) * 1024 + rlo * 128;
-  for (int cidx = 0; cidx < L.n32 / 16; ++cidx) {
-    const int j0 = cidx * 16;
+  const int rlo = row & 7;
+  uint8_t* prow = sP + (row >> 3) * 1024 + rlo * 128;
+  for (int u = slice; u < L.n32 / 16; u += kAttnSplit) {
+    const int j0 = u * 16;
     uint32_t packed[4] = {0, 0, 0, 0};
     if (ok && j0 < N) {
       const int4 v = *reinterpret_cast<const int4*>(my_log + j0);
@@ -246,31 +266,24 @@ __global__ void __launch_bounds__(kAttnThreads)
   ok = __all_sync(0xffffffffu, ok);
   tc_fence_after();
 
-  // ---- ctx = sat_8((b_o O) >> c_o)
+  // ---- ctx = sat_8((b_o O) >> c_o); slice s writes columns [16 s, 16 s + 16)
   {
-    uint32_t r0v[32], r1v[32];
-    tmem_ld32(t_lane, r0v);
-    tmem_ld32(t_lane + 32, r1v);
+    uint32_t r[16];
+    tmem_ld16(t_lane + (uint32_t)(slice * 16), r);
     tmem_ld_wait();
-    const int q = q0 + tid;
+    const int q = q0 + row;
     if (ok && q < N) {
-      int8_t* dst = a.ctx + (int64_t)(row0 + q) * D + h * kHeadDim;
-      uint32_t packed[16];
+      int8_t* dst = a.ctx + (int64_t)(row0 + q) * D + h * kHeadDim + slice * 16;
+      uint32_t packed[4];
 #pragma unroll
-      for (int wd = 0; wd < 16; ++wd) {
+      for (int wd = 0; wd < 4; ++wd) {
         uint32_t word = 0;
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const int i = wd * 4 + e;
-          const int32_t acc = (int32_t)(i < 32 ? r0v[i] : r1v[i - 32]);
-          word |= ((uint32_t)requant8(acc, a.out_b, a.out_c) & 0xFFu) << (8 * e);
-        }
+        for (int e = 0; e < 4; ++e)
+          word |= ((uint32_t)requant8((int32_t)r[wd * 4 + e], a.out_b, a.out_c) & 0xFFu) << (8 * e);
         packed[wd] = word;
       }
-#pragma unroll
-      for (int v = 0; v < 4; ++v)
-        reinterpret_cast<int4*>(dst)[v] =
-            make_int4(packed[4 * v], packed[4 * v + 1], packed[4 * v + 2], packed[4 * v + 3]);
+      *reinterpret_cast<int4*>(dst) = make_int4(packed[0], packed[1], packed[2], packed[3]);
     }
   }
 
