@@ -74,8 +74,11 @@ __host__ __device__ inline AttnLayout attn_layout(int N) {
   return L;
 }
 
+// FASTQ: the logit requant is one mul.hi by bq = b_s 2^(32 - c_s), exact
+// when b_s < 2^(c_s - 1), then the k_s-bit saturation.
+template <bool FASTQ>
 __global__ void __launch_bounds__(kAttnThreads)
-    attention_shiftmax_kernel(const __grid_constant__ CUtensorMap tm, const AttnArgs a) {
+    attention_shiftmax_kernel(const __grid_constant__ CUtensorMap tm, const AttnArgs a, const int32_t bq) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align_smem_1024(smem_raw);
   const int N = a.N;
@@ -179,7 +182,9 @@ __global__ void __launch_bounds__(kAttnThreads)
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
             const int i = wd * 4 + e;
-            const int32_t l = requant_bits((int32_t)r[i], a.logit_b, a.logit_c, a.ks_lo, a.ks_hi);
+            const int32_t l =
+                FASTQ ? min(max(__mulhi(bq, (int32_t)r[i]), a.ks_lo), a.ks_hi)
+                      : requant_bits((int32_t)r[i], a.logit_b, a.logit_c, a.ks_lo, a.ks_hi);
             if (j0 + i < N) mx = l > mx ? l : mx;
             word |= ((uint32_t)l & 0xFFu) << (8 * e);
           }
@@ -886,12 +891,20 @@ ivit_status launch_attention(const DeviceCtx& dc, const int8_t* qkv, int32_t B, 
   if (smem < 80 * 1024) smem = 80 * 1024;
   static int attr_bytes = 0;
   if (smem > attr_bytes) {
-    if (cudaFuncSetAttribute(attention_shiftmax_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024) !=
-        cudaSuccess)
+    if (cudaFuncSetAttribute(attention_shiftmax_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             227 * 1024) != cudaSuccess ||
+        cudaFuncSetAttribute(attention_shiftmax_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             227 * 1024) != cudaSuccess)
       return IVIT_ERR_CUDA;
     attr_bytes = 227 * 1024;
   }
-  const cudaError_t e = launch_pdl(attention_shiftmax_kernel, grid, dim3(kAttnThreads), smem, stream, tm, a);
+  // bq = b 2^(32 - c) when it fits a positive int32: the logit requant is then one mul.hi
+  const bool fastq_long = logit.c >= 1 && (int64_t)logit.b < ((int64_t)1 << (logit.c - 1));
+  const int32_t bq_long = fastq_long ? (int32_t)((int64_t)logit.b << (32 - logit.c)) : 0;
+  const cudaError_t e =
+      fastq_long
+          ? launch_pdl(attention_shiftmax_kernel<true>, grid, dim3(kAttnThreads), smem, stream, tm, a, bq_long)
+          : launch_pdl(attention_shiftmax_kernel<false>, grid, dim3(kAttnThreads), smem, stream, tm, a, bq_long);
   note_launch();
   return e == cudaSuccess ? IVIT_OK : IVIT_ERR_CUDA;
 }
