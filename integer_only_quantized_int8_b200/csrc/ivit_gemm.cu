@@ -14,13 +14,16 @@
 // (tcgen05.st) before the MMAs accumulate onto it.  When b_j < 2^(c_j - 1) (a
 // requant scale below one half, the usual case) the requant
 // floor(b acc / 2^c) is then one mul.hi by b 2^(32 - c); the saturating byte
-// pack clips.  A 4 x 4 byte transpose across lanes turns channel-major bytes
-// into token-major 4-byte words.  The four warps that cover the tile's 128
-// channels for the same tokens (one per TMEM lane quarter: a "part") fill one
-// 16-token x 128-channel staging slot per chunk, 128B-swizzled, and one thread
-// of the part sends it out with a single TMA store: 16 rows of 128 bytes
-// instead of four boxes of 16 rows of 32 bytes, which the TMA unit drains four
-// times faster.  The residual's skip tile arrives the same way.
+// pack clips (a round-half-up variant adds half an LSB first).  A 4 x 4 byte
+// transpose across lanes turns channel-major bytes into token-major 4-byte
+// words.  The four warps that cover the tile's 128 channels for the same
+// tokens (one per TMEM lane quarter: a "part") fill one 16-token x
+// 128-channel staging slot per chunk, 128B-swizzled, and one thread of the
+// part sends it out with a single TMA store of 16 rows of 128 bytes (a
+// quarter as many stores as one per warp).  Where shared memory allows, two
+// slot sets serve alternate tiles.  The residual's skip tile arrives the
+// same way.  Each tile's channel constants are loaded and turned into its
+// requant form one tile ahead.
 //
 // Roles (one CTA per SM, persistent over 128 x BN tiles):
 //   warp 0      TMA producer: W and X k-slices of 128 bytes, 128B swizzle,
