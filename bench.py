@@ -326,6 +326,7 @@ def run_ours(args):
     c0 = ivit.ivit_launch_count()
     out = step(0)
     torch.cuda.synchronize()
+    out = out.clone()  # the intermediates are reused by every later step
     launches_per_step = ivit.ivit_launch_count() - c0
     assert ivit.ivit_stream_status() == 0
 
@@ -626,7 +627,15 @@ def kernel_breakdown(ivit, wl, dp, ws, xs, reps, dev):
     S_l16 = (1.0 / p["attn_I0"]) * 255.0 / 65535.0
     logit16 = ivit.ivit_dyadic_from_double(p["logit"][0] / 2.0 ** p["logit"][1] * 65535.0 / 255.0)
     I0_16 = ivit.ivit_i0_from_scale(S_l16)
-    if N <= 256:  # 16-bit logits run on the short-sequence kernel only
+    # 16-bit logits run on the short-sequence kernel only, and only where the
+    # re-derived I0 keeps the per-score division exact (the library refuses
+    # the others before enqueueing anything)
+    try:
+        ivit.ivit_attention(qkv, B, N, H, logit16, 16, I0_16, p["attn_M"], p["attn_k_out"], p["attn_out"], ctx_o)
+        wide_ok = True
+    except ivit.IvitError:
+        wide_ok = False
+    if wide_ok:
         add("attention_logits16", lambda i: ivit.ivit_attention(qkv, B, N, H, logit16, 16, I0_16, p["attn_M"],
                                                                 p["attn_k_out"], p["attn_out"], ctx_o),
             "alu", SHIFTMAX_OPS_PER_SCORE * B * H * N * N, in_block=False)
