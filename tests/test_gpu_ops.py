@@ -71,6 +71,28 @@ def test_linear_requant_parity(M, K, N):
     np.testing.assert_array_equal(host(Y), oracle.linear_requant(lc.X, lc.W, lc.bias, b_o, c_o, out_bits=4))
 
 
+# shapes whose token-tile width (chosen for the fewest rounds of tiles over
+# 148 SMs) is 256 (three-stage ring, one MMA issuer), 224, 192 and 160 (two
+# issuers), each with a ragged last token tile, and odd and even k-slice counts
+TILE_WIDTH_SHAPES = [(5421, 384, 768), (4655, 768, 768), (3890, 384, 768), (3121, 768, 768)]
+
+
+@pytest.mark.parametrize("M,K,N", TILE_WIDTH_SHAPES)
+def test_linear_parity_every_tile_width(M, K, N):
+    lc = synthetic.linear_case(M, K, N, seed=M + 2 * K + N, with_skip=True)
+    bq = [ivit.ivit_dyadic_from_double(r) for r in lc.ratio]
+    b = np.array([x[0] for x in bq], np.int32)
+    c = np.array([x[1] for x in bq], np.int32)
+    X, W = dev(lc.X, torch.int8), dev(lc.W, torch.int8)
+    bd, cd, biasd = dev(b, torch.int32), dev(c, torch.int8), dev(lc.bias, torch.int32)
+    Y = torch.empty((M, N), dtype=torch.int8, device="cuda")
+    ivit.ivit_linear_requant(X, W, biasd, bd, cd, Y)
+    np.testing.assert_array_equal(host(Y), oracle.linear_requant(lc.X, lc.W, lc.bias, b, c))
+    res = ivit.ivit_residual_from_double(*lc.res_ratio)
+    ivit.ivit_linear_requant(X, W, biasd, bd, cd, Y, skip=dev(lc.skip, torch.int8), res=res)
+    np.testing.assert_array_equal(host(Y), oracle.linear_requant(lc.X, lc.W, lc.bias, b, c, skip=lc.skip, res=res))
+
+
 def test_linear_saturation_and_extremes():
     r = np.random.default_rng(30)
     M, K, N = 64, 4096, 32
