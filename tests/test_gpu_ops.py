@@ -65,10 +65,14 @@ def test_linear_requant_parity(M, K, N):
                              skip=dev(lc.skip, torch.int8), res=res_d)
     want = oracle.linear_requant(lc.X, lc.W, lc.bias, b_o, c_o, skip=lc.skip, res=res_o)
     np.testing.assert_array_equal(host(Y), want)
-    # a narrower output width
+    # a narrower output width, alone and before the residual addition
     ivit.ivit_linear_requant(X, W, dev(lc.bias, torch.int32), dev(b_d, torch.int32), dev(c_d, torch.int8), Y,
                              out_bits=4)
     np.testing.assert_array_equal(host(Y), oracle.linear_requant(lc.X, lc.W, lc.bias, b_o, c_o, out_bits=4))
+    ivit.ivit_linear_requant(X, W, dev(lc.bias, torch.int32), dev(b_d, torch.int32), dev(c_d, torch.int8), Y,
+                             out_bits=5, skip=dev(lc.skip, torch.int8), res=res_d)
+    np.testing.assert_array_equal(host(Y), oracle.linear_requant(lc.X, lc.W, lc.bias, b_o, c_o, out_bits=5,
+                                                                 skip=lc.skip, res=res_o))
 
 
 # shapes whose token-tile width (chosen for the fewest rounds of tiles over
