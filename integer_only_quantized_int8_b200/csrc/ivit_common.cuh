@@ -86,20 +86,6 @@ IVIT_DEV bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
-// Non-blocking test of phase completion (never suspends the thread), for a
-// thread that polls several barriers in turn.
-IVIT_DEV bool mbar_test(uint64_t* bar, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(ok)
-      : "r"(smem_u32(bar)), "r"(parity)
-      : "memory");
-  return ok != 0;
-}
-
 // As mbar_try_wait, but the thread may be suspended in hardware for up to
 // kSuspendHintNs while the phase is incomplete (it resumes as soon as the
 // phase completes), so a waiting warp does not spin on the issue slots.
@@ -323,13 +309,6 @@ IVIT_DEV int32_t requant8(int32_t v, int32_t b, int32_t c) {
 IVIT_DEV int32_t requant_bits(int32_t v, int32_t b, int32_t c, int32_t lo, int32_t hi) {
   const int64_t q = ((int64_t)b * (int64_t)v) >> c;
   return (int32_t)(q < lo ? lo : (q > hi ? hi : q));
-}
-
-// Residual addition of two int8 tensors on a common shift:
-// sat_8((b_skip * skip + b_branch * branch) >> c)
-IVIT_DEV int32_t residual8(int32_t skip, int32_t branch, int32_t b_skip, int32_t b_branch, int32_t c) {
-  const int64_t q = ((int64_t)b_skip * skip + (int64_t)b_branch * branch) >> c;
-  return (int32_t)(q < -128 ? -128 : (q > 127 ? 127 : q));
 }
 
 // Shift-exponential of d <= 0 at scale 1/I0 (I-ViT section 3.3):
