@@ -255,10 +255,23 @@ def source_hash(paths):
     return h.hexdigest()[:16]
 
 
-def kernel_source_hash():
-    csrc = os.path.join(ROOT, "integer_only_quantized_int8_b200", "csrc")
-    return source_hash(glob.glob(os.path.join(csrc, "*.cu")) + glob.glob(os.path.join(csrc, "*.cuh")) +
-                       glob.glob(os.path.join(csrc, "*.h")))
+# the source file that holds each timed kernel's device code and launcher
+KERNEL_FILES = {"gemm": "ivit_gemm.cu", "attention": "ivit_attention.cu", "layernorm": "ivit_elementwise.cu",
+                "shiftgelu": "ivit_elementwise.cu"}
+
+
+def kernel_sources(kernel, csrc):
+    """Files whose change can change `kernel`: its own file plus every csrc
+    file that holds no other kernel family (shared headers, the C ABI)."""
+    own = {v for v in KERNEL_FILES.values()} | {"ivit_model.cu"}
+    mine = next(v for k, v in KERNEL_FILES.items() if kernel.startswith(k))
+    files = [p for p in glob.glob(os.path.join(csrc, "*")) if p.endswith((".cu", ".cuh", ".h"))]
+    return [p for p in files if os.path.basename(p) not in own or os.path.basename(p) == mine]
+
+
+def kernel_source_hash(kernel, csrc=None):
+    csrc = csrc or os.path.join(ROOT, "integer_only_quantized_int8_b200", "csrc")
+    return source_hash(kernel_sources(kernel, csrc))
 
 
 def load_traffic(kernel, workload):
@@ -268,7 +281,7 @@ def load_traffic(kernel, workload):
         with open(path) as f:
             tab = json.load(f)
         ent = tab.get(f"{kernel}@{workload}")
-        if ent and ent.get("source_hash") == kernel_source_hash():
+        if ent and ent.get("source_hash") == kernel_source_hash(kernel):
             return float(ent["dram_bytes_per_launch"])
     except Exception:
         pass

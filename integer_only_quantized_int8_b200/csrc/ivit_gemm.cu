@@ -102,7 +102,10 @@ struct GemmLayout {
   static constexpr int kGeluOff = kSlotOff + 16;
   static constexpr int kBytes = kGeluOff + 256;
   static constexpr int kAlloc = kBytes + 1024;  // slack to align the base to 1024 bytes
-  static constexpr int kTmemCols = (2 * BN <= 256) ? 256 : 512;
+  // TMEM columns per accumulator buffer: BN rounded up to 32, so the second
+  // buffer starts on a 32-column boundary whatever the tile width
+  static constexpr int kAccCols = (BN + 31) / 32 * 32;
+  static constexpr int kTmemCols = (2 * kAccCols <= 256) ? 256 : 512;
 };
 
 IVIT_DEV int32_t sat_i32(int64_t v) {
@@ -441,7 +444,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         // the buffer holds this tile's bias once the epilogue has drained it
         if (!mbar_wait(&tempty[acc], acc_phase, args.status)) break;
         tc_fence_after();
-        const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BN);
+        const uint32_t d_tmem = tmem_base + (uint32_t)(acc * L::kAccCols);
         int kb = kb0;
         for (; kb < num_kb; kb += kStep) {
           if (!mbar_wait(&full[stage], phase, args.status)) {
@@ -498,7 +501,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     // both accumulator buffers start out holding the bias of their first tile
     for (int a = 0; a < 2; ++a) {
       const int t = (int)blockIdx.x + a * (int)gridDim.x;
-      if (t < num_tiles) bias_fill(tlane + (uint32_t)(a * BN), c_begin, c_end, bias_of(t));
+      if (t < num_tiles) bias_fill(tlane + (uint32_t)(a * L::kAccCols), c_begin, c_end, bias_of(t));
       tmem_st_wait();
       tc_fence_before();
       __syncwarp();
@@ -579,7 +582,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         skip_phase ^= 1;
       }
       tc_fence_after();
-      const uint32_t tbase = tlane + (uint32_t)(acc * BN);
+      const uint32_t tbase = tlane + (uint32_t)(acc * L::kAccCols);
 #define IVIT_EPI_TILE(R) \
   epi_tile<EPI, NARROW, R>(tbase, c_begin, n, kc, args, gelu_tab, slots, ofs_even, ofs_odd, sel2, sel1)
       if (!args.round) {
@@ -673,18 +676,24 @@ ivit_status run_gemm(const DeviceCtx& dc, const int8_t* X, const int8_t* W, cons
   return e == cudaSuccess ? IVIT_OK : IVIT_ERR_CUDA;
 }
 
-// Token-tile width: fewest rounds of tiles over the SMs, weighted by the tile
-// width plus a fixed per-tile cost, so narrower tiles win only when they save
-// a round.
+// Token-tile width: the fewest rounds of tiles over the SMs, each round
+// costing the tile width plus a fixed per-tile cost of about 112 token
+// columns (channel constants, bias preload, accumulator hand-off, ring
+// ramp), and 20 more at BN = 256, whose three-stage ring has one MMA issuer.
+// Among widths with the same number of rounds the narrowest wins; a narrower
+// width that needs one more round wins only when it is much narrower.  The
+// two constants are fitted to per-kernel timings of the ViT-B, ViT-L,
+// DeiT-S and ViT-B/384 layers on a B200 (148 SMs), where they reproduce
+// every measured preference between widths.
 int pick_bn(int64_t M, int N, int num_sms) {
-  static const int cands[] = {256, 224, 192, 160, 128};
+  static const int cands[] = {256, 224, 192, 176, 160, 128};
   const int ch_tiles = (N + kBM - 1) / kBM;
   int best = 256;
   int64_t best_cost = INT64_MAX;
   for (int bn : cands) {
     const int64_t tiles = (int64_t)ch_tiles * ((M + bn - 1) / bn);
     const int64_t rounds = (tiles + num_sms - 1) / num_sms;
-    const int64_t cost = rounds * (bn + 32);
+    const int64_t cost = rounds * (bn + 112 + (bn == 256 ? 20 : 0));
     if (cost < best_cost) {
       best_cost = cost;
       best = bn;
@@ -703,6 +712,8 @@ ivit_status dispatch_bn(const DeviceCtx& dc, const int8_t* X, const int8_t* W, c
       return run_gemm<224, 4, EPI, NARROW>(dc, X, W, skip, Y, a, stream);
     case 192:
       return run_gemm<192, 4, EPI, NARROW>(dc, X, W, skip, Y, a, stream);
+    case 176:
+      return run_gemm<176, 4, EPI, NARROW>(dc, X, W, skip, Y, a, stream);
     case 160:
       return run_gemm<160, 4, EPI, NARROW>(dc, X, W, skip, Y, a, stream);
     default:

@@ -75,10 +75,20 @@ def test_linear_requant_parity(M, K, N):
                                                                  skip=lc.skip, res=res_o))
 
 
-# shapes whose token-tile width (chosen for the fewest rounds of tiles over
-# 148 SMs) is 256 (three-stage ring, one MMA issuer), 224, 192 and 160 (two
-# issuers), each with a ragged last token tile, and odd and even k-slice counts
-TILE_WIDTH_SHAPES = [(5421, 384, 768), (4655, 768, 768), (3890, 384, 768), (3121, 768, 768)]
+# Shapes whose token-tile width (chosen for the fewest rounds of tiles over
+# 148 SMs) is, in order, 256 (three-stage ring, one MMA issuer), 224, 192,
+# 176 (twice, the second with a ragged channel tile), 160 and 128 (two
+# issuers).  Every M leaves a ragged last token tile, and the k-slice counts
+# are odd and even.
+TILE_WIDTH_SHAPES = [
+    (5421, 384, 768),
+    (4655, 768, 768),
+    (4226, 384, 768),
+    (3890, 384, 768),
+    (2881, 768, 1008),
+    (3121, 768, 768),
+    (1013, 384, 768),
+]
 
 
 @pytest.mark.parametrize("M,K,N", TILE_WIDTH_SHAPES)
