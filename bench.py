@@ -248,8 +248,10 @@ class ClockSampler:
 # ---------------------------------------------------------------------------
 
 def source_hash(paths):
+    """Hash of the files' contents in file-name order (so it does not depend
+    on where the tree sits)."""
     h = hashlib.sha256()
-    for p in sorted(paths):
+    for p in sorted(paths, key=os.path.basename):
         with open(p, "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]
@@ -260,18 +262,20 @@ KERNEL_FILES = {"gemm": "ivit_gemm.cu", "attention": "ivit_attention.cu", "layer
                 "shiftgelu": "ivit_elementwise.cu"}
 
 
-def kernel_sources(kernel, csrc):
-    """Files whose change can change `kernel`: its own file plus every csrc
-    file that holds no other kernel family (shared headers, the C ABI)."""
-    own = {v for v in KERNEL_FILES.values()} | {"ivit_model.cu"}
+def kernel_sources(kernel, csrc, include):
+    """The translation unit that builds `kernel`: its own .cu file (device
+    code, launcher, tile dispatch) and the headers that file includes.  The C
+    ABI's host-side checks live elsewhere and cannot change what the kernel
+    reads or writes."""
     mine = next(v for k, v in KERNEL_FILES.items() if kernel.startswith(k))
-    files = [p for p in glob.glob(os.path.join(csrc, "*")) if p.endswith((".cu", ".cuh", ".h"))]
-    return [p for p in files if os.path.basename(p) not in own or os.path.basename(p) == mine]
+    return [os.path.join(csrc, mine), os.path.join(csrc, "ivit_common.cuh"), os.path.join(csrc, "ivit_internal.h"),
+            os.path.join(include, "ivit.h")]
 
 
-def kernel_source_hash(kernel, csrc=None):
+def kernel_source_hash(kernel, csrc=None, include=None):
     csrc = csrc or os.path.join(ROOT, "integer_only_quantized_int8_b200", "csrc")
-    return source_hash(kernel_sources(kernel, csrc))
+    include = include or os.path.join(ROOT, "include")
+    return source_hash(kernel_sources(kernel, csrc, include))
 
 
 def load_traffic(kernel, workload):

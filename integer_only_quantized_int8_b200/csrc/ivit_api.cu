@@ -278,6 +278,15 @@ ivit_status check_block(const ivit_block_params* p, const int8_t* x, const int8_
       !valid_dyadic(p->ln2_out) || !valid_residual(p->res1) || !valid_residual(p->res2) || p->ln_F < 0 ||
       p->ln_F > 14 || p->ln_M < p->ln_F || p->ln_M > 23 || (p->linear_round != 0 && p->linear_round != 1))
     return IVIT_ERR_INVALID_ARG;
+  // the kernels read and write all of these by 16-byte vector accesses or TMA
+  const void* const need16[] = {x,         y,        p->ln1_gamma, p->ln1_beta, p->w_qkv, p->b_qkv,
+                                p->c_qkv,  p->w_o,   p->b_o,       p->c_o,      p->ln2_gamma, p->ln2_beta,
+                                p->w1,     p->b1,    p->c1,        p->w2,       p->b2,    p->c2};
+  for (const void* q : need16)
+    if (!aligned16(q)) return IVIT_ERR_INVALID_ARG;
+  const void* const bias16[] = {p->bias_qkv, p->bias_o, p->bias1, p->bias2};  // optional
+  for (const void* q : bias16)
+    if (q && !aligned16(q)) return IVIT_ERR_INVALID_ARG;
   if (!attention_config_supported(N, p->k_s, p->attn_I0)) return IVIT_ERR_UNSUPPORTED;
   return IVIT_OK;
 }

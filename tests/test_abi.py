@@ -104,6 +104,49 @@ def test_validation_rejects_before_launch():
     assert L.ivit_layernorm(None, 0, 32, None, None, 7, 23, d, None, None) == 0
 
 
+def test_block_checks_every_pointer_before_launch():
+    """ivit_block_forward refuses a misaligned activation or parameter pointer
+    with nothing enqueued.  The baseline call is valid except that it asks for
+    12-bit logits over 300 keys, which the host refuses as unsupported after
+    every pointer check, so no call here reaches a launch on any machine."""
+    import ctypes as C
+    L = ivit.lib()
+    ptr_fields = [name for name, t in ivit.BlockParams._fields_ if t is C.c_void_p]
+    base = 0x100000
+
+    def params(**over):
+        p = ivit.BlockParams()
+        p.D, p.H, p.Dm = 64, 1, 256
+        for i, f in enumerate(ptr_fields):
+            setattr(p, f, base + 0x1000 * (i + 1))
+        p.ln1_out = p.ln2_out = p.logit = p.attn_out = p.gelu_out = ivit.Dyadic(1, 0)
+        p.k_s, p.attn_I0, p.attn_M, p.attn_k_out = 12, 4, 30, 8
+        p.gelu_I0, p.gelu_M, p.gelu_k_out = 4, 30, 8
+        p.res1 = p.res2 = ivit.Residual(1, 1, 1)
+        p.ln_F, p.ln_M, p.linear_round = 7, 23, 0
+        for k, v in over.items():
+            setattr(p, k, v)
+        return p
+
+    B, N = 1, 300
+    x, y, ws = 0x1000000, 0x2000000, 0x3000000
+    ws_bytes = ivit.ivit_block_workspace_bytes(B, N, 64, 256)
+
+    def call(p, xx=x, yy=y):
+        return L.ivit_block_forward(C.byref(p), xx, yy, ws, ws_bytes, B, N, None)
+
+    assert call(params()) == 2                      # every pointer passes; the attention shape does not
+    assert call(params(), xx=x + 8) == 1            # misaligned input
+    assert call(params(), yy=y + 4) == 1            # misaligned output
+    for f in ptr_fields:
+        good = getattr(params(), f)
+        assert call(params(**{f: good + 1})) == 1, f  # misaligned parameter
+        if f.startswith("bias"):
+            assert call(params(**{f: None})) == 2, f  # the biases are optional
+        else:
+            assert call(params(**{f: None})) == 1, f  # the rest are not
+
+
 def test_workspace_bytes():
     assert ivit.ivit_block_workspace_bytes(0, 197, 768, 3072) == 0
     T, D, Dm = 64 * 197, 768, 3072
