@@ -177,6 +177,14 @@ def _ptr(t, dtype, name):
     return t.data_ptr()
 
 
+def _holds(n: int, **tensors):
+    """Each given tensor must hold at least n elements: the library reads or
+    writes that many through its pointer."""
+    for name, t in tensors.items():
+        if t is not None and t.numel() < n:
+            raise ValueError(f"{name} holds {t.numel()} elements, needs {n}")
+
+
 def _dy(d) -> Dyadic:
     return d if isinstance(d, Dyadic) else Dyadic(int(d[0]), int(d[1]))
 
@@ -226,6 +234,7 @@ def ivit_linear_requant(X, W, bias, b, c, Y, out_bits: int = 8, skip=None, res=N
         raise ValueError("shape mismatch")
     if skip is not None and tuple(skip.shape) != (M, N):
         raise ValueError("skip shape mismatch")
+    _holds(N, bias=bias, b=b, c=c)
     st = lib().ivit_linear_requant(_ptr(X, torch.int8, "X"), M, K, _ptr(W, torch.int8, "W"), N,
                                    _ptr(bias, torch.int32, "bias"), _ptr(b, torch.int32, "b"),
                                    _ptr(c, torch.int8, "c"), int(out_bits), int(rounding), _ptr(skip, torch.int8, "skip"),
@@ -241,6 +250,7 @@ def ivit_linear_shiftgelu(X, W, bias, b, c, gelu_I0: int, gelu_M: int, gelu_k_ou
     N = W.shape[0]
     if W.shape[1] != K or tuple(Y.shape) != (M, N):
         raise ValueError("shape mismatch")
+    _holds(N, bias=bias, b=b, c=c)
     st = lib().ivit_linear_shiftgelu(_ptr(X, torch.int8, "X"), M, K, _ptr(W, torch.int8, "W"), N,
                                      _ptr(bias, torch.int32, "bias"), _ptr(b, torch.int32, "b"),
                                      _ptr(c, torch.int8, "c"), int(rounding), int(gelu_I0), int(gelu_M), int(gelu_k_out),
@@ -287,6 +297,7 @@ def ivit_block_workspace_bytes(B: int, N: int, D: int, Dm: int) -> int:
 def ivit_block_forward(params, x, y, workspace, B: int, N: int, stream=None):
     """One encoder block; ``params`` is a :class:`BlockParams` (or an object with ``.c``)."""
     p = params.c if hasattr(params, "c") else params
+    _holds(int(B) * int(N) * p.D, x=x, y=y)
     st = lib().ivit_block_forward(C.byref(p), _ptr(x, torch.int8, "x"), _ptr(y, torch.int8, "y"),
                                   _ptr(workspace, torch.uint8, "workspace"), workspace.numel(), int(B), int(N),
                                   _stream(stream))
@@ -306,6 +317,7 @@ def ivit_block_forward_static(params, x, y, B: int, N: int, stream=None):
     calls on a device: calls that overlap on the GPU race.  Larger batches
     raise IvitError (IVIT_ERR_UNSUPPORTED)."""
     p = params.c if hasattr(params, "c") else params
+    _holds(int(B) * int(N) * p.D, x=x, y=y)
     st = lib().ivit_block_forward_static(C.byref(p), _ptr(x, torch.int8, "x"), _ptr(y, torch.int8, "y"), int(B),
                                          int(N), _stream(stream))
     _check("ivit_block_forward_static", st)
@@ -329,6 +341,12 @@ def ivit_patch_embed(img, P: int, W, bias, b, c, cls, pos, pos_add, workspace, x
     the class token first, the position embedding joined by ``pos_add``."""
     B, C_in, Hi, Wi = img.shape
     D = W.shape[0]
+    if W.numel() != D * C_in * P * P:
+        raise ValueError(f"W must be [D, C*P*P] = [{D}, {C_in * P * P}]")
+    Ntok = (Hi // P) * (Wi // P) + 1
+    _holds(D, bias=bias, b=b, c=c, cls=cls)
+    _holds(Ntok * D, pos=pos)
+    _holds(B * Ntok * D, x=x)
     st = lib().ivit_patch_embed(_ptr(img, torch.int8, "img"), B, C_in, Hi, Wi, int(P), _ptr(W, torch.int8, "W"), D,
                                 _ptr(bias, torch.int32, "bias"), _ptr(b, torch.int32, "b"), _ptr(c, torch.int8, "c"),
                                 int(rounding), _ptr(cls, torch.int8, "cls"), _ptr(pos, torch.int8, "pos"), _res(pos_add),
@@ -346,6 +364,13 @@ def ivit_head(x, B: int, Ntok: int, gamma, beta, F: int, M_ln: int, ln_out, W, b
               stream=None, rounding: int = 0):
     """logits [B, Ncls] from the class tokens of x [B*Ntok, D]."""
     D = x.shape[1]
+    Ncls = W.shape[0]
+    if W.shape[1] != D:
+        raise ValueError(f"W must be [Ncls, D] with D = {D}")
+    _holds(int(B) * int(Ntok) * D, x=x)
+    _holds(D, gamma=gamma, beta=beta)
+    _holds(Ncls, bias=bias, b=b, c=c)
+    _holds(int(B) * Ncls, logits=logits)
     st = lib().ivit_head(_ptr(x, torch.int8, "x"), int(B), int(Ntok), D, _ptr(gamma, torch.int8, "gamma"),
                          _ptr(beta, torch.int32, "beta"), int(F), int(M_ln), _dy(ln_out), _ptr(W, torch.int8, "W"),
                          W.shape[0], _ptr(bias, torch.int32, "bias"), _ptr(b, torch.int32, "b"),
@@ -365,7 +390,10 @@ def ivit_model_forward(params, img, workspace, logits, stream=None):
     """logits [B, Ncls] from img [B, C, Hi, Wi]; ``params`` is a
     :class:`ModelParams` (or an object with ``.c``)."""
     p = params.c if hasattr(params, "c") else params
-    B, _, Hi, Wi = img.shape
+    B, C_in, Hi, Wi = img.shape
+    if C_in != p.C:
+        raise ValueError(f"img has {C_in} channels, the model {p.C}")
+    _holds(B * p.Ncls, logits=logits)
     st = lib().ivit_model_forward(C.byref(p), _ptr(img, torch.int8, "img"), B, Hi, Wi,
                                   _ptr(workspace, torch.uint8, "workspace"), workspace.numel(),
                                   _ptr(logits, torch.int8, "logits"), _stream(stream))
