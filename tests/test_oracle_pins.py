@@ -419,6 +419,48 @@ def test_attention_hardmax_reduces_to_argmax():
                     np.testing.assert_array_equal(ctx[b * N + i, h * 64:(h + 1) * 64], want)
 
 
+def test_attention_logit_requant_floors_worked_example():
+    """Worked by hand from the definitions (I_0 = 1 makes Shiftmax a hard max).
+    One image, two tokens, one head.  Query 0 has q = e_0 and the keys have
+    k_0 = -3 e_0, k_1 = -2 e_0, so S = [-3, -2]; with (b_s, c_s) = (1, 1) the
+    floor shift gives L = [-2, -1], a single max at key 1, P = [0, 128] and
+    ctx = (128 v_1) >> 7 = v_1.  (A truncating shift would give [-1, -1], a
+    tie, P = [64, 64] and ctx = 15 in the first column.)  Query 1 has q = 0:
+    S = [0, 0], P = [64, 64], ctx = (64 v_0 + 64 v_1) >> 7."""
+    qkv = np.zeros((2, 3 * 64), np.int8)
+    qkv[0, 0] = 1                      # q_0 = e_0, q_1 = 0
+    qkv[0, 64], qkv[1, 64] = -3, -2    # k_0, k_1
+    qkv[0, 128], qkv[1, 128] = 10, 20  # v_0, v_1 (first column)
+    qkv[0, 129], qkv[1, 129] = -7, 5   # second column: floors below zero
+    ctx = oracle.attention(qkv, 1, 2, 1, (1, 1), 8, 1, 30, 8, (1, 7))
+    assert ctx[0, 0] == 20 and ctx[0, 1] == 5
+    assert ctx[1, 0] == 15                       # (640 + 1280) >> 7
+    assert ctx[1, 1] == -1                       # (-448 + 320) >> 7 = floor(-1)
+    assert not ctx[:, 2:].any()
+
+
+def test_attention_dyadic_multipliers_are_exact_scalings():
+    """b / 2^c is a number, not a pair: (2^c, c) must act as (1, 0), and
+    (2 b, c + 1) as (b, c), for the logits and for the output alike; and an
+    output multiplier b_o scales the single-key context exactly."""
+    r = np.random.default_rng(13)
+    B, N, H = 2, 11, 2
+    qkv = _qkv(r, B, N, H, -4, 5)
+    base = oracle.attention(qkv, B, N, H, (1, 0), 8, 3, 30, 8, (1, 4))
+    for c in (1, 7, 19, 30):
+        np.testing.assert_array_equal(oracle.attention(qkv, B, N, H, (2 ** c, c), 8, 3, 30, 8, (1, 4)), base)
+        np.testing.assert_array_equal(oracle.attention(qkv, B, N, H, (1, 0), 8, 3, 30, 8, (2 ** c, c + 4)), base)
+    for b, c in ((3, 9), (12345, 20), (2 ** 29 + 1, 30)):
+        lo = oracle.attention(qkv, B, N, H, (b, c), 8, 5, 30, 8, (7, 9))
+        np.testing.assert_array_equal(oracle.attention(qkv, B, N, H, (2 * b, c + 1), 8, 5, 30, 8, (7, 9)), lo)
+        np.testing.assert_array_equal(oracle.attention(qkv, B, N, H, (b, c), 8, 5, 30, 8, (14, 10)), lo)
+    # one key: P = 128 (I_0 = 16 divides 2^30), ctx = sat_8((3 * 128 v) >> 9)
+    qkv1 = _qkv(r, 3, 1, 2)
+    ctx = oracle.attention(qkv1, 3, 1, 2, (5, 3), 8, 16, 30, 8, (3, 9))
+    v = qkv1[:, 2 * 128:].astype(np.int64)
+    np.testing.assert_array_equal(ctx, np.clip(np.floor_divide(3 * 128 * v, 2 ** 9), -128, 127))
+
+
 # --------------------------------------------------------------------------
 # block (section 3.1)
 # --------------------------------------------------------------------------
