@@ -28,12 +28,18 @@ _lock = threading.Lock()
 _lib = None
 
 
+def compile_source(src: str, out: str) -> str:
+    """Compile one C source of the oracle into the shared library `out`."""
+    tmp = out + f".tmp{os.getpid()}"
+    subprocess.check_call(["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-o", tmp, src, "-lm"])
+    os.replace(tmp, out)
+    return out
+
+
 def build(force: bool = False) -> str:
     """Compile ivit_oracle.c into a shared library next to it."""
     if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
-        tmp = _LIB + f".tmp{os.getpid()}"
-        subprocess.check_call(["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-o", tmp, _SRC, "-lm"])
-        os.replace(tmp, _LIB)
+        compile_source(_SRC, _LIB)
     return _LIB
 
 
@@ -68,64 +74,76 @@ class BlockParamsC(C.Structure):
     ]]
 
 
+def use_library(path: str):
+    """Bind the oracle's functions to another build of its C source from now
+    on (the planted-mistake test uses this on copies it has altered)."""
+    global _lib
+    with _lock:
+        _lib = _bind(C.CDLL(path))
+
+
 def lib():
     global _lib
     with _lock:
         if _lib is None:
-            L = C.CDLL(build())
-            L.orc_quantize.restype = C.c_int32
-            L.orc_quantize.argtypes = [C.c_double, C.c_double, C.c_int]
-            L.orc_dyadic.restype = C.c_int
-            L.orc_dyadic.argtypes = [C.c_double, C.POINTER(C.c_int32), C.POINTER(C.c_int32)]
-            L.orc_dyadic_pair.restype = C.c_int
-            L.orc_dyadic_pair.argtypes = [C.c_double, C.c_double, C.POINTER(C.c_int32),
-                                          C.POINTER(C.c_int32), C.POINTER(C.c_int32)]
-            L.orc_recip_i0.restype = C.c_int32
-            L.orc_recip_i0.argtypes = [C.c_double]
-            L.orc_requant.restype = C.c_int64
-            L.orc_requant.argtypes = [C.c_int64, C.c_int32, C.c_int32, C.c_int]
-            L.orc_linear_requant.restype = None
-            L.orc_linear_requant.argtypes = [C.c_void_p, C.c_int64, C.c_int32, C.c_void_p, C.c_int32,
-                                             C.c_void_p, C.c_void_p, C.c_void_p, C.c_int,
-                                             C.c_void_p, C.c_int32, C.c_int32, C.c_int32, C.c_void_p]
-            L.orc_shift_exp.restype = C.c_int64
-            L.orc_shift_exp.argtypes = [C.c_int64, C.c_int64]
-            L.orc_int_div.restype = C.c_int64
-            L.orc_int_div.argtypes = [C.c_int64, C.c_int64, C.c_int, C.c_int]
-            L.orc_shiftmax_row.restype = None
-            L.orc_shiftmax_row.argtypes = [C.c_void_p, C.c_int, C.c_int32, C.c_int, C.c_int, C.c_void_p]
-            L.orc_attention.restype = None
-            L.orc_attention.argtypes = [C.c_void_p, C.c_int32, C.c_int32, C.c_int32,
-                                        C.c_int32, C.c_int32, C.c_int32, C.c_int32,
-                                        C.c_int32, C.c_int32, C.c_int32, C.c_int32, C.c_void_p]
-            L.orc_shift_sigmoid.restype = C.c_int64
-            L.orc_shift_sigmoid.argtypes = [C.c_int64, C.c_int64, C.c_int32, C.c_int32]
-            L.orc_shiftgelu_one.restype = C.c_int32
-            L.orc_shiftgelu_one.argtypes = [C.c_int32, C.c_int32, C.c_int32, C.c_int32, C.c_int32,
-                                            C.c_int32, C.POINTER(C.c_int32)]
-            L.orc_shiftgelu.restype = None
-            L.orc_shiftgelu.argtypes = [C.c_void_p, C.c_int64, C.c_int32, C.c_int32, C.c_int32,
-                                        C.c_int32, C.c_int32, C.c_void_p]
-            L.orc_isqrt_newton.restype = C.c_int64
-            L.orc_isqrt_newton.argtypes = [C.c_int64]
-            L.orc_layernorm.restype = None
-            L.orc_layernorm.argtypes = [C.c_void_p, C.c_int64, C.c_int32, C.c_void_p, C.c_void_p,
-                                        C.c_int32, C.c_int32, C.c_int32, C.c_int32, C.c_void_p]
-            L.orc_patch_embed.restype = C.c_int
-            L.orc_patch_embed.argtypes = [C.c_void_p, C.c_int32, C.c_int32, C.c_int32, C.c_int32, C.c_int32,
-                                          C.c_void_p, C.c_void_p, C.c_void_p, C.c_void_p, C.c_int32,
-                                          C.c_void_p, C.c_void_p, C.c_int32, C.c_int32, C.c_int32, C.c_void_p]
-            L.orc_head.restype = C.c_int
-            L.orc_head.argtypes = [C.c_void_p, C.c_int32, C.c_int32, C.c_int32, C.c_void_p, C.c_void_p,
-                                   C.c_int32, C.c_int32, C.c_int32, C.c_int32, C.c_void_p, C.c_int32,
-                                   C.c_void_p, C.c_void_p, C.c_void_p, C.c_void_p]
-            L.orc_set_linear_rounding.restype = None
-            L.orc_set_linear_rounding.argtypes = [C.c_int]
-            L.orc_block_forward.restype = C.c_int
-            L.orc_block_forward.argtypes = [C.POINTER(BlockParamsC), C.c_void_p, C.c_void_p,
-                                            C.c_int32, C.c_int32]
-            _lib = L
+            _lib = _bind(C.CDLL(build()))
     return _lib
+
+
+def _bind(L):
+    """Declare the argument and result types of every exported function."""
+    L.orc_quantize.restype = C.c_int32
+    L.orc_quantize.argtypes = [C.c_double, C.c_double, C.c_int]
+    L.orc_dyadic.restype = C.c_int
+    L.orc_dyadic.argtypes = [C.c_double, C.POINTER(C.c_int32), C.POINTER(C.c_int32)]
+    L.orc_dyadic_pair.restype = C.c_int
+    L.orc_dyadic_pair.argtypes = [C.c_double, C.c_double, C.POINTER(C.c_int32),
+                                  C.POINTER(C.c_int32), C.POINTER(C.c_int32)]
+    L.orc_recip_i0.restype = C.c_int32
+    L.orc_recip_i0.argtypes = [C.c_double]
+    L.orc_requant.restype = C.c_int64
+    L.orc_requant.argtypes = [C.c_int64, C.c_int32, C.c_int32, C.c_int]
+    L.orc_linear_requant.restype = None
+    L.orc_linear_requant.argtypes = [C.c_void_p, C.c_int64, C.c_int32, C.c_void_p, C.c_int32,
+                                     C.c_void_p, C.c_void_p, C.c_void_p, C.c_int,
+                                     C.c_void_p, C.c_int32, C.c_int32, C.c_int32, C.c_void_p]
+    L.orc_shift_exp.restype = C.c_int64
+    L.orc_shift_exp.argtypes = [C.c_int64, C.c_int64]
+    L.orc_int_div.restype = C.c_int64
+    L.orc_int_div.argtypes = [C.c_int64, C.c_int64, C.c_int, C.c_int]
+    L.orc_shiftmax_row.restype = None
+    L.orc_shiftmax_row.argtypes = [C.c_void_p, C.c_int, C.c_int32, C.c_int, C.c_int, C.c_void_p]
+    L.orc_attention.restype = None
+    L.orc_attention.argtypes = [C.c_void_p, C.c_int32, C.c_int32, C.c_int32,
+                                C.c_int32, C.c_int32, C.c_int32, C.c_int32,
+                                C.c_int32, C.c_int32, C.c_int32, C.c_int32, C.c_void_p]
+    L.orc_shift_sigmoid.restype = C.c_int64
+    L.orc_shift_sigmoid.argtypes = [C.c_int64, C.c_int64, C.c_int32, C.c_int32]
+    L.orc_shiftgelu_one.restype = C.c_int32
+    L.orc_shiftgelu_one.argtypes = [C.c_int32, C.c_int32, C.c_int32, C.c_int32, C.c_int32,
+                                    C.c_int32, C.POINTER(C.c_int32)]
+    L.orc_shiftgelu.restype = None
+    L.orc_shiftgelu.argtypes = [C.c_void_p, C.c_int64, C.c_int32, C.c_int32, C.c_int32,
+                                C.c_int32, C.c_int32, C.c_void_p]
+    L.orc_isqrt_newton.restype = C.c_int64
+    L.orc_isqrt_newton.argtypes = [C.c_int64]
+    L.orc_layernorm.restype = None
+    L.orc_layernorm.argtypes = [C.c_void_p, C.c_int64, C.c_int32, C.c_void_p, C.c_void_p,
+                                C.c_int32, C.c_int32, C.c_int32, C.c_int32, C.c_void_p]
+    L.orc_patch_embed.restype = C.c_int
+    L.orc_patch_embed.argtypes = [C.c_void_p, C.c_int32, C.c_int32, C.c_int32, C.c_int32, C.c_int32,
+                                  C.c_void_p, C.c_void_p, C.c_void_p, C.c_void_p, C.c_int32,
+                                  C.c_void_p, C.c_void_p, C.c_int32, C.c_int32, C.c_int32, C.c_void_p]
+    L.orc_head.restype = C.c_int
+    L.orc_head.argtypes = [C.c_void_p, C.c_int32, C.c_int32, C.c_int32, C.c_void_p, C.c_void_p,
+                           C.c_int32, C.c_int32, C.c_int32, C.c_int32, C.c_void_p, C.c_int32,
+                           C.c_void_p, C.c_void_p, C.c_void_p, C.c_void_p]
+    L.orc_set_linear_rounding.restype = None
+    L.orc_set_linear_rounding.argtypes = [C.c_int]
+    L.orc_block_forward.restype = C.c_int
+    L.orc_block_forward.argtypes = [C.POINTER(BlockParamsC), C.c_void_p, C.c_void_p,
+                                    C.c_int32, C.c_int32]
+    return L
 
 
 # ---------------------------------------------------------------------------

@@ -45,6 +45,13 @@ def test_quantizer_endpoints_and_grid():
         assert oracle.quantize(k * S, m) == k      # exact grid points
     assert oracle.quantize(2.5 * S, m) == 3        # half away from zero
     assert oracle.quantize(-2.5 * S, m) == -3
+    # off the grid the step S = 2m / (2^k - 1) shows: 63.4 S -> 63 and 126.6 S
+    # -> 127 (a step of 2m / 2^k would give 64 and 127; 2m / (2^k - 2) 63, 126)
+    assert oracle.quantize(63.4 * S, m) == 63
+    assert oracle.quantize(-63.4 * S, m) == -63
+    assert oracle.quantize(126.6 * S, m) == 127
+    assert oracle.quantize(1.0, 127.5) == 1         # m = 127.5: S = 1 exactly
+    assert oracle.quantize(100.49, 127.5) == 100
 
 
 # --------------------------------------------------------------------------
@@ -349,6 +356,12 @@ def test_layernorm_hand_cases():
     y = oracle.layernorm(np.array([[-4, 4, -4, 4]], np.int8), np.ones(4, np.int8), np.zeros(4, np.int32), 7, 23,
                          (1, 1))
     assert list(y[0]) == [-64, 64, -64, 64]
+    # population variance (LayerNorm divides by n): [-3, 3] -> V = 18 / 2 = 9,
+    # sigma = 3, f = floor(2^23 / 3) = 2796202, d f >> 16 = +-8388606 / 2^16,
+    # which floors to 127 and -128.  Dividing by n - 1 would give V = 18,
+    # sigma = 4 and [-96, 96]; a truncating shift would give -127.
+    y = oracle.layernorm(np.array([[-3, 3]], np.int8), np.ones(2, np.int8), np.zeros(2, np.int32), 7, 23, (1, 0))
+    assert list(y[0]) == [-128, 127]
 
 
 def test_layernorm_close_to_float():
