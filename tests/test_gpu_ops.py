@@ -79,7 +79,8 @@ def test_linear_requant_parity(M, K, N):
 # 148 SMs) is, in order, 256 (three-stage ring, one MMA issuer), 224, 192,
 # 176 (twice, the second with a ragged channel tile), 160 and 128 (two
 # issuers).  Every M leaves a ragged last token tile, and the k-slice counts
-# are odd and even.
+# are odd and even.  Each shape runs the plain, residual, narrow-output and
+# fused ShiftGELU epilogues.
 TILE_WIDTH_SHAPES = [
     (5421, 384, 768),
     (4655, 768, 768),
@@ -101,10 +102,23 @@ def test_linear_parity_every_tile_width(M, K, N):
     bd, cd, biasd = dev(b, torch.int32), dev(c, torch.int8), dev(lc.bias, torch.int32)
     Y = torch.empty((M, N), dtype=torch.int8, device="cuda")
     ivit.ivit_linear_requant(X, W, biasd, bd, cd, Y)
-    np.testing.assert_array_equal(host(Y), oracle.linear_requant(lc.X, lc.W, lc.bias, b, c))
+    plain = oracle.linear_requant(lc.X, lc.W, lc.bias, b, c)
+    np.testing.assert_array_equal(host(Y), plain)
     res = ivit.ivit_residual_from_double(*lc.res_ratio)
-    ivit.ivit_linear_requant(X, W, biasd, bd, cd, Y, skip=dev(lc.skip, torch.int8), res=res)
+    skip = dev(lc.skip, torch.int8)
+    ivit.ivit_linear_requant(X, W, biasd, bd, cd, Y, skip=skip, res=res)
     np.testing.assert_array_equal(host(Y), oracle.linear_requant(lc.X, lc.W, lc.bias, b, c, skip=lc.skip, res=res))
+    # the narrow-output and fused ShiftGELU epilogues at the same tile width
+    ivit.ivit_linear_requant(X, W, biasd, bd, cd, Y, out_bits=4)
+    np.testing.assert_array_equal(host(Y), oracle.linear_requant(lc.X, lc.W, lc.bias, b, c, out_bits=4))
+    ivit.ivit_linear_requant(X, W, biasd, bd, cd, Y, out_bits=6, skip=skip, res=res)
+    np.testing.assert_array_equal(host(Y), oracle.linear_requant(lc.X, lc.W, lc.bias, b, c, out_bits=6,
+                                                                 skip=lc.skip, res=res))
+    gc = synthetic.gelu_case(1024, seed=M)
+    I0 = ivit.ivit_i0_from_scale(gc.S_h)
+    go = ivit.ivit_dyadic_from_double(gc.out_ratio)
+    ivit.ivit_linear_shiftgelu(X, W, biasd, bd, cd, I0, 30, 8, go, Y)
+    np.testing.assert_array_equal(host(Y), oracle.shiftgelu(plain, I0, 30, 8, go))
 
 
 def test_linear_saturation_and_extremes():
