@@ -104,6 +104,26 @@ def test_validation_rejects_before_launch():
     assert L.ivit_layernorm(None, 0, 32, None, None, 7, 23, d, None, None) == 0
 
 
+def test_product_model_params_equal_oracle_model_params():
+    """Patch embedding, position add, head and every block: the library's host
+    helpers and the oracle derive the same integers (no GPU involved)."""
+    mc = synthetic.model_case(B=2, Hi=32, Wi=48, P=16, D=192, H=3, Dm=768, blocks=2, Ncls=100, seed=4)
+    a = ivit_params.model_integer_params(mc)
+    b = oracle.model_params(mc)
+    for k in ("b_pe", "c_pe", "b_head", "c_head"):
+        np.testing.assert_array_equal(np.asarray(a[k], np.int64), np.asarray(b[k], np.int64), err_msg=k)
+    assert tuple(a["pos_add"]) == tuple(b["pos_add"])
+    assert tuple(a["head_ln_out"]) == tuple(b["head_ln_out"])
+    assert (a["ln_F"], a["ln_M"], a["P"]) == (b["ln_F"], b["ln_M"], b["P"])
+    assert len(a["blocks"]) == len(b["blocks"]) == 2
+    for qa, qb in zip(a["blocks"], b["blocks"]):
+        for k, v in qb.items():
+            if isinstance(v, np.ndarray):
+                np.testing.assert_array_equal(np.asarray(qa[k]).astype(np.int64), v.astype(np.int64), err_msg=k)
+            else:
+                assert tuple(np.atleast_1d(qa[k])) == tuple(np.atleast_1d(v)), k
+
+
 def test_block_checks_every_pointer_before_launch():
     """ivit_block_forward refuses a misaligned activation or parameter pointer
     with nothing enqueued.  The baseline call is valid except that it asks for
