@@ -301,6 +301,30 @@ def test_shiftgelu_exhaustive_properties():
     assert sig == 0
 
 
+def test_rowmax_shiftgelu_reading_divides_zero_by_zero(capsys):
+    """Evidence for the per-element reading of ShiftGELU's I_max (section 3.4,
+    where the derivation stops before defining it).  Read instead as the row
+    maximum of I_p over a token's fc1 channels, as Shiftmax does over keys,
+    both exponentials ShiftExp(I_p - I_max) and ShiftExp(-I_max) floor to 0
+    for nearly every element of an fc1-like row at int8 resolution, leaving
+    sigma = 0 / 0.  Reported, and required to hold for most elements."""
+    import synthetic
+    gc = synthetic.gelu_case(768 * 64, seed=0)
+    I0 = oracle.recip_i0(gc.S_h)
+    x = gc.x.reshape(64, 768).astype(np.int64)
+    Ip = x + (x >> 1) + (x >> 3) + (x >> 4)       # 1.702 x ~ 1.1011b x, floor shifts
+    Imax = Ip.max(1, keepdims=True)
+    exp = {d: oracle.shift_exp(d, I0) for d in range(int(min((Ip - Imax).min(), -Imax.max())), 1)}
+    e1 = np.vectorize(exp.get)(Ip - Imax)
+    e2 = np.vectorize(exp.get)(-Imax)
+    frac = float(((e1 + e2) == 0).mean())
+    with capsys.disabled():
+        print(f"\n[reading report] row-max ShiftGELU: {100 * frac:.1f} % of elements are 0/0 (I0 = {I0})")
+    assert frac > 0.5
+    # the per-element reading never divides by zero: e1 + e2 >= I0 >= 1
+    assert all(oracle.shift_sigmoid(int(v), I0) >= 0 for v in np.unique(Ip))
+
+
 def test_shiftgelu_close_to_gelu():
     """Reported FP check over all 256 inputs against x * Phi(x)."""
     for S in (8 / 127, 4 / 127, 12 / 127):
