@@ -57,7 +57,7 @@ def parse_args():
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=synthetic.CONFIG_ORDER)
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--no-graph", action="store_true", help="launch eagerly instead of replaying CUDA graphs")
-    ap.add_argument("--cpu-units", type=int, default=10,
+    ap.add_argument("--cpu-units", type=int, default=24,
                     help="CPU-baseline sample: (image, block) units the oracle runs")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--kernel-reps", type=int, default=50)
