@@ -32,7 +32,7 @@ def sources():
 
 def deps():
     return sources() + sorted(glob.glob(os.path.join(PKG, "csrc", "*.cuh"))) + \
-        sorted(glob.glob(os.path.join(PKG, "csrc", "*.h"))) + [os.path.join(ROOT, "include", "ivit.h")]
+        sorted(glob.glob(os.path.join(PKG, "csrc", "*.h"))) + sorted(glob.glob(os.path.join(ROOT, "include", "*.h")))
 
 
 def up_to_date() -> bool:

@@ -27,7 +27,8 @@ def built():
 
 
 def _declared():
-    src = open(os.path.join(ROOT, "include", "ivit.h")).read()
+    src = "".join(open(os.path.join(ROOT, "include", h)).read()
+                  for h in sorted(os.listdir(os.path.join(ROOT, "include"))) if h.endswith(".h"))
     src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
     return sorted(set(re.findall(r"\b(ivit_[a-z0-9_]+)\s*\(", src)))
 
