@@ -33,6 +33,25 @@ def host(t):
     return t.cpu().numpy()
 
 
+GUARD = 4096   # canary bytes on each side of a guarded output (keeps 16-byte alignment)
+CANARY = 0x5A
+
+
+def guarded(shape):
+    """An int8 output inside a larger buffer whose canary bytes on both sides
+    must survive the call: a check for writes past either end of the output
+    (they land in the test's own memory, so they cannot fault)."""
+    n = int(np.prod(shape))
+    buf = torch.full((n + 2 * GUARD,), CANARY, dtype=torch.uint8, device="cuda")
+    view = buf[GUARD:GUARD + n].view(torch.int8).view(shape)
+
+    def untouched():
+        h = host(buf)
+        return bool((h[:GUARD] == CANARY).all() and (h[GUARD + n:] == CANARY).all())
+
+    return view, untouched
+
+
 # ---------------------------------------------------------------------------
 # INT8 linear + dyadic requant (tcgen05 GEMM)
 # ---------------------------------------------------------------------------
@@ -51,7 +70,7 @@ def test_linear_requant_parity(M, K, N):
     b_d, c_d = np.array([x[0] for x in bq], np.int32), np.array([x[1] for x in bq], np.int8)
     b_o, c_o = np.array([x[0] for x in bo], np.int32), np.array([x[1] for x in bo], np.int32)
     X, W = dev(lc.X, torch.int8), dev(lc.W, torch.int8)
-    Y = torch.empty((M, N), dtype=torch.int8, device="cuda")
+    Y, untouched = guarded((M, N))
     for use_bias in (True, False):
         bias = lc.bias if use_bias else None
         ivit.ivit_linear_requant(X, W, None if bias is None else dev(bias, torch.int32), dev(b_d, torch.int32),
@@ -73,6 +92,7 @@ def test_linear_requant_parity(M, K, N):
                              out_bits=5, skip=dev(lc.skip, torch.int8), res=res_d)
     np.testing.assert_array_equal(host(Y), oracle.linear_requant(lc.X, lc.W, lc.bias, b_o, c_o, out_bits=5,
                                                                  skip=lc.skip, res=res_o))
+    assert untouched()
 
 
 # Shapes whose token-tile width (chosen for the fewest rounds of tiles over
@@ -100,7 +120,7 @@ def test_linear_parity_every_tile_width(M, K, N):
     c = np.array([x[1] for x in bq], np.int32)
     X, W = dev(lc.X, torch.int8), dev(lc.W, torch.int8)
     bd, cd, biasd = dev(b, torch.int32), dev(c, torch.int8), dev(lc.bias, torch.int32)
-    Y = torch.empty((M, N), dtype=torch.int8, device="cuda")
+    Y, untouched = guarded((M, N))
     ivit.ivit_linear_requant(X, W, biasd, bd, cd, Y)
     plain = oracle.linear_requant(lc.X, lc.W, lc.bias, b, c)
     np.testing.assert_array_equal(host(Y), plain)
@@ -119,6 +139,7 @@ def test_linear_parity_every_tile_width(M, K, N):
     go = ivit.ivit_dyadic_from_double(gc.out_ratio)
     ivit.ivit_linear_shiftgelu(X, W, biasd, bd, cd, I0, 30, 8, go, Y)
     np.testing.assert_array_equal(host(Y), oracle.shiftgelu(plain, I0, 30, 8, go))
+    assert untouched()
 
 
 def test_linear_saturation_and_extremes():
@@ -204,10 +225,11 @@ def test_attention_parity(B, N, H, tails, k_s):
     out_d, out_o = ivit.ivit_dyadic_from_double(ac.out_ratio), oracle.dyadic(ac.out_ratio)
     I0_d, I0_o = ivit.ivit_i0_from_scale(ac.S_logit), oracle.recip_i0(ac.S_logit)
     qkv = dev(ac.qkv, torch.int8)
-    ctx = torch.full((B * N, H * 64), 99, dtype=torch.int8, device="cuda")
+    ctx, untouched = guarded((B * N, H * 64))
     ivit.ivit_attention(qkv, B, N, H, logit_d, k_s, I0_d, 30, 8, out_d, ctx)
     want = oracle.attention(ac.qkv, B, N, H, logit_o, k_s, I0_o, 30, 8, out_o)
     np.testing.assert_array_equal(host(ctx), want)
+    assert untouched()
 
 
 @pytest.mark.parametrize("k_s", [8, 12, 16])
@@ -245,9 +267,10 @@ def test_shiftgelu_parity(n):
     I0_d, out_d = ivit.ivit_i0_from_scale(gc.S_h), ivit.ivit_dyadic_from_double(gc.out_ratio)
     I0_o, out_o = oracle.recip_i0(gc.S_h), oracle.dyadic(gc.out_ratio)
     xd = dev(x, torch.int8) if n else torch.empty(0, dtype=torch.int8, device="cuda")
-    y = torch.empty_like(xd)
+    y, untouched = guarded((n,))
     ivit.ivit_shiftgelu(xd, I0_d, 30, 8, out_d, y)
     np.testing.assert_array_equal(host(y), oracle.shiftgelu(x, I0_o, 30, 8, out_o))
+    assert untouched()
 
 
 @pytest.mark.parametrize("I0", [1, 2, 5, 16, 25, 64, 1000])
@@ -270,9 +293,10 @@ def test_layernorm_parity(rows, cols):
     x = nc.x.copy()
     x[0] = 17                                    # a constant row (variance 0)
     out_d, out_o = ivit.ivit_dyadic_from_double(nc.out_ratio), oracle.dyadic(nc.out_ratio)
-    y = torch.empty((rows, cols), dtype=torch.int8, device="cuda")
+    y, untouched = guarded((rows, cols))
     ivit.ivit_layernorm(dev(x, torch.int8), dev(nc.gamma, torch.int8), dev(nc.beta, torch.int32), 7, 23, out_d, y)
     np.testing.assert_array_equal(host(y), oracle.layernorm(x, nc.gamma, nc.beta, 7, 23, out_o))
+    assert untouched()
 
 
 def test_layernorm_extreme_rows():
