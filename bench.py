@@ -18,7 +18,6 @@ sample of the same workload instead.
 from __future__ import annotations
 
 import argparse
-import glob
 import hashlib
 import json
 import math
