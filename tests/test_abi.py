@@ -11,6 +11,7 @@ import re
 
 import numpy as np
 import pytest
+import torch
 
 import integer_only_quantized_int8_b200 as ivit
 import oracle
@@ -123,6 +124,49 @@ def test_product_model_params_equal_oracle_model_params():
                 np.testing.assert_array_equal(np.asarray(qa[k]).astype(np.int64), v.astype(np.int64), err_msg=k)
             else:
                 assert tuple(np.atleast_1d(qa[k])) == tuple(np.atleast_1d(v)), k
+
+
+def _read(ptr, like):
+    """The bytes at a host address, as an array shaped like `like`."""
+    import ctypes as C
+    a = np.asarray(like)
+    raw = (C.c_char * a.nbytes).from_address(ptr)
+    return np.frombuffer(bytes(raw), dtype=a.dtype).reshape(a.shape)
+
+
+def test_parameter_structs_point_at_the_right_tables():
+    """params.to_device / model_to_device on host memory: every pointer of the
+    C structs reads back its own table, and every scalar is the dict's."""
+    mc = synthetic.model_case(B=2, Hi=32, Wi=32, P=16, D=128, H=2, Dm=256, blocks=2, Ncls=40, seed=6)
+    m = ivit_params.model_integer_params(mc)
+    m["linear_round"] = 1
+    for blk in m["blocks"]:
+        blk["linear_round"] = 1
+    dm = ivit_params.model_to_device(m, "cpu")
+    s = dm.c
+    assert (s.C, s.P, s.D, s.n_blocks, s.Ncls) == (m["C"], m["P"], m["D"], 2, m["Ncls_pad"])
+    assert (s.pos_add.b_skip, s.pos_add.b_branch, s.pos_add.c) == tuple(m["pos_add"])
+    assert (s.head_ln_out.b, s.head_ln_out.c) == tuple(m["head_ln_out"])
+    assert (s.head_ln_F, s.head_ln_M, s.linear_round) == (m["ln_F"], m["ln_M"], 1)
+    for name, dt in (("w_pe", np.int8), ("bias_pe", np.int32), ("b_pe", np.int32), ("c_pe", np.int8),
+                     ("cls", np.int8), ("pos", np.int8), ("head_gamma", np.int8), ("head_beta", np.int32),
+                     ("w_head", np.int8), ("bias_head", np.int32), ("b_head", np.int32), ("c_head", np.int8)):
+        want = np.asarray(m[name]).astype(dt)
+        np.testing.assert_array_equal(_read(getattr(s, name), want), want, err_msg=name)
+    for i, p in enumerate(m["blocks"]):
+        bs = s.blocks[i]
+        assert (bs.D, bs.H, bs.Dm) == (p["D"], p["H"], p["Dm"])
+        for f in ("ln1_out", "ln2_out", "logit", "attn_out", "gelu_out"):
+            assert (getattr(bs, f).b, getattr(bs, f).c) == tuple(p[f]), f
+        for f in ("res1", "res2"):
+            r = getattr(bs, f)
+            assert (r.b_skip, r.b_branch, r.c) == tuple(p[f]), f
+        for f in ("k_s", "attn_I0", "attn_M", "attn_k_out", "gelu_I0", "gelu_M", "gelu_k_out", "ln_F", "ln_M",
+                  "linear_round"):
+            assert getattr(bs, f) == p[f], f
+        for name, dt in ivit_params._TENSORS.items():
+            want = np.asarray(p[name]).astype({torch.int8: np.int8, torch.int32: np.int32}[dt])
+            np.testing.assert_array_equal(_read(getattr(bs, name), want), want, err_msg=f"block {i} {name}")
 
 
 def test_block_checks_every_pointer_before_launch():
