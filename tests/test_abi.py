@@ -212,6 +212,28 @@ def test_block_checks_every_pointer_before_launch():
             assert call(params(**{f: None})) == 1, f  # the rest are not
 
 
+def test_empty_batches_are_no_ops_on_every_entry_point():
+    """B = 0 (or N = 0) returns IVIT_OK after the argument checks, touches no
+    memory and needs no device, for the block, attention, patch embedding
+    and head as for the elementwise operators."""
+    import ctypes as C
+    L = ivit.lib()
+    p = 0x100000
+    d = ivit.Dyadic(1, 0)
+    none = ivit.Residual(0, 0, 0)
+    blk = ivit.BlockParams()
+    blk.D, blk.H, blk.Dm = 64, 1, 256
+    assert L.ivit_block_forward(C.byref(blk), p, p + 0x1000, p + 0x2000, 0, 0, 197, None) == 0
+    assert L.ivit_block_forward(C.byref(blk), p, p + 0x1000, p + 0x2000, 0, 4, 0, None) == 0
+    assert L.ivit_attention(p, 0, 197, 12, d, 8, 4, 30, 8, d, p, None) == 0
+    assert L.ivit_attention(p, 3, 0, 12, d, 8, 4, 30, 8, d, p, None) == 0
+    assert L.ivit_patch_embed(p, 0, 3, 32, 32, 16, p, 64, None, p, p, 0, p, p, none, p, 1 << 20, p, None) == 0
+    assert L.ivit_head(p, 0, 5, 64, p, p, 7, 23, d, p, 32, None, p, p, 0, p, 1 << 20, p, None) == 0
+    # an empty batch still gets its arguments checked
+    assert L.ivit_block_forward(C.byref(blk), p, p, p + 0x2000, 0, 0, 197, None) == 1     # x aliases y
+    assert L.ivit_attention(p, 0, 197, 12, d, 17, 4, 30, 8, d, p, None) == 1              # k_s > 16
+
+
 def test_workspace_bytes():
     assert ivit.ivit_block_workspace_bytes(0, 197, 768, 3072) == 0
     T, D, Dm = 64 * 197, 768, 3072

@@ -142,19 +142,27 @@ def test_linear_parity_every_tile_width(M, K, N):
     assert untouched()
 
 
-def test_linear_saturation_and_extremes():
+@pytest.mark.parametrize("K", [4096, 16384])
+def test_linear_saturation_and_extremes(K):
+    """Saturating operands with b = 2^31 - 1 and every shift 0..31 (the wide
+    and clamped requant forms).  K = 16384 is the largest reduction the ABI
+    accepts; with |bias| up to 2^30 the accumulator reaches 2^28 + 2^30, the
+    int32 range the ABI guarantees."""
     r = np.random.default_rng(30)
-    M, K, N = 64, 4096, 32
+    M, N = 64, 32
     X = np.full((M, K), -128, np.int8)
     X[1::2] = 127
     W = r.choice(np.array([-128, 127], np.int8), size=(N, K))
+    W[0] = -128                                  # row 0 of X times W[0]: 2^14 K = 2^28 at K = 16384
     b = np.zeros(N, np.int32); b[:] = 2 ** 31 - 1
     c = (np.arange(N) % 32).astype(np.int32)
     bias = r.integers(-2 ** 20, 2 ** 20, size=N).astype(np.int32)
-    Y = torch.empty((M, N), dtype=torch.int8, device="cuda")
+    bias[0], bias[1] = 2 ** 30, -2 ** 30
+    Y, untouched = guarded((M, N))
     ivit.ivit_linear_requant(dev(X, torch.int8), dev(W, torch.int8), dev(bias, torch.int32), dev(b, torch.int32),
                              dev(c, torch.int8), Y)
     np.testing.assert_array_equal(host(Y), oracle.linear_requant(X, W, bias, b, c))
+    assert untouched()
 
 
 @pytest.mark.parametrize("M,K,N", [(197, 192, 576), (300, 768, 3072), (129, 64, 272)])
