@@ -14,8 +14,14 @@ import torch
 import integer_only_quantized_int8_b200 as ivit
 import oracle
 import synthetic
+from integer_only_quantized_int8_b200 import build as ivit_build
 
 pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def built():
+    ivit_build.build()
 
 
 def test_wait_that_runs_out_reports_timeout_and_context_stays_usable():
