@@ -318,8 +318,10 @@ def ivit_block_forward_static(params, x, y, B: int, N: int, stream=None):
     has reserved the whole device, loops that cannot afford cudaMalloc).  The
     intermediates live in the library's own 32 MiB device array, shared by all
     calls on a device: calls that overlap on the GPU race.  Larger batches
-    raise IvitError (IVIT_ERR_UNSUPPORTED)."""
+    raise IvitError (IVIT_ERR_UNSUPPORTED) before any tensor is looked at."""
     p = params.c if hasattr(params, "c") else params
+    if ivit_block_workspace_bytes(B, N, p.D, p.Dm) > STATIC_SCRATCH_BYTES:
+        raise IvitError("ivit_block_forward_static", 2)
     _holds(int(B) * int(N) * p.D, x=x, y=y)
     st = lib().ivit_block_forward_static(C.byref(p), _ptr(x, torch.int8, "x"), _ptr(y, torch.int8, "y"), int(B),
                                          int(N), _stream(stream))

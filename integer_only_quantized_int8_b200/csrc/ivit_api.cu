@@ -255,20 +255,19 @@ size_t ivit_block_workspace_bytes(int32_t B, int32_t N, int32_t D, int32_t Dm) {
   return up(T * D) + up(T * 3 * (size_t)D) + up(T * D) + up(T * D) + up(T * (size_t)Dm);
 }
 
-namespace {
+}  // extern "C"
 
-// Every host-side check of one block call; IVIT_OK means it may be enqueued
-// (or, with B or N zero, that there is nothing to do).
-ivit_status check_block(const ivit_block_params* p, const int8_t* x, const int8_t* y, const void* workspace,
-                        size_t workspace_bytes, int32_t B, int32_t N) {
-  if (!p || !x || !y || !workspace) return IVIT_ERR_INVALID_ARG;
+// Every host-side check of one block call except those of the workspace;
+// IVIT_OK means the arguments may be enqueued (or, with B or N zero, that
+// there is nothing to do).
+ivit_status ivit::check_block_args(const ivit_block_params* p, const int8_t* x, const int8_t* y, int32_t B,
+                                   int32_t N) {
+  if (!p || !x || !y) return IVIT_ERR_INVALID_ARG;
   if (B < 0 || N < 0 || p->H < 1 || p->D != 64 * p->H || p->Dm < 16 || p->Dm % 16 != 0 || p->D > 2048)
     return IVIT_ERR_INVALID_ARG;
   if (x == y) return IVIT_ERR_INVALID_ARG;
   if (B == 0 || N == 0) return IVIT_OK;
   if (N > 640) return IVIT_ERR_UNSUPPORTED;
-  const size_t need = ivit_block_workspace_bytes(B, N, p->D, p->Dm);
-  if (workspace_bytes < need || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return IVIT_ERR_INVALID_ARG;
   if (!p->ln1_gamma || !p->ln1_beta || !p->w_qkv || !p->b_qkv || !p->c_qkv || !p->w_o || !p->b_o || !p->c_o ||
       !p->ln2_gamma || !p->ln2_beta || !p->w1 || !p->b1 || !p->c1 || !p->w2 || !p->b2 || !p->c2)
     return IVIT_ERR_INVALID_ARG;
@@ -288,6 +287,22 @@ ivit_status check_block(const ivit_block_params* p, const int8_t* x, const int8_
   for (const void* q : bias16)
     if (q && !aligned16(q)) return IVIT_ERR_INVALID_ARG;
   if (!attention_config_supported(N, p->k_s, p->attn_I0)) return IVIT_ERR_UNSUPPORTED;
+  return IVIT_OK;
+}
+
+extern "C" {
+
+namespace {
+
+// Every host-side check of one block call; IVIT_OK means it may be enqueued
+// (or, with B or N zero, that there is nothing to do).
+ivit_status check_block(const ivit_block_params* p, const int8_t* x, const int8_t* y, const void* workspace,
+                        size_t workspace_bytes, int32_t B, int32_t N) {
+  if (!workspace) return IVIT_ERR_INVALID_ARG;
+  const ivit_status st = check_block_args(p, x, y, B, N);
+  if (st != IVIT_OK || B == 0 || N == 0) return st;
+  const size_t need = ivit_block_workspace_bytes(B, N, p->D, p->Dm);
+  if (workspace_bytes < need || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return IVIT_ERR_INVALID_ARG;
   return IVIT_OK;
 }
 

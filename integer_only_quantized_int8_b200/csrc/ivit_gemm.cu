@@ -575,7 +575,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       }
       const bool got = mbar_wait(&tfull[acc], acc_phase, args.status);
       // the whole part has its accumulator and free slots, or gives up together
-      if (!part_bar_and(part, got)) break;
+      if (!part_bar_and(part, got)) {
+        // the skip loads issued above still write into the slots: let them
+        // land (a bounded wait) before the CTA can release its shared memory
+        if (EPI == kEpiResidual && live && part_lead) mbar_wait(sbar, skip_phase, args.status);
+        break;
+      }
       bool got_skip = true;
       if (EPI == kEpiResidual && live) {
         got_skip = mbar_wait(sbar, skip_phase, args.status);

@@ -50,6 +50,10 @@ ivit_status encode_tmap_2d_u8(CUtensorMap* map, const void* base, uint64_t inner
                               uint64_t row_stride_bytes, uint32_t box_inner, uint32_t box_outer,
                               CUtensorMapSwizzle swizzle);
 
+// The host-side checks of one encoder-block call other than those of its
+// workspace (parameters, alignment, sizes, attention configuration).
+ivit_status check_block_args(const ivit_block_params* p, const int8_t* x, const int8_t* y, int32_t B, int32_t N);
+
 ivit_status launch_gemm(const DeviceCtx& dc, const int8_t* X, int64_t M, int32_t K, const int8_t* W, int32_t N,
                         const int32_t* bias, const int32_t* b, const int8_t* c, int32_t out_bits, bool round,
                         EpiMode mode, const int8_t* skip, ivit_residual res, const GeluParams* gelu, int8_t* Y,

@@ -31,13 +31,15 @@ std::mutex g_scratch_mu;
 void* g_scratch_ptr[kMaxScratchDevices] = {};
 
 // Device address of g_block_scratch on the current device (set up once).
-ivit_status scratch_address(void** out) {
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxScratchDevices) return IVIT_ERR_CUDA;
+ivit_status scratch_address(int dev, void** out) {
+  if (dev < 0 || dev >= kMaxScratchDevices) return IVIT_ERR_CUDA;
   std::lock_guard<std::mutex> lk(g_scratch_mu);
   if (!g_scratch_ptr[dev]) {
     void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_block_scratch) != cudaSuccess || !p) return IVIT_ERR_CUDA;
+    if (cudaGetSymbolAddress(&p, g_block_scratch) != cudaSuccess || !p) {
+      (void)cudaGetLastError();  // leave no error behind for the next launch check
+      return IVIT_ERR_CUDA;
+    }
     g_scratch_ptr[dev] = p;
   }
   *out = g_scratch_ptr[dev];
@@ -48,12 +50,14 @@ ivit_status scratch_address(void** out) {
 
 extern "C" ivit_status ivit_block_forward_static(const ivit_block_params* p, const int8_t* x, int8_t* y,
                                                  int32_t B, int32_t N, ivit_stream_t stream) {
-  if (!p || B < 0 || N < 0 || p->D < 0 || p->Dm < 0) return IVIT_ERR_INVALID_ARG;
-  // Refuse work whose intermediates do not fit the fixed array.
+  // the checks of ivit_block_forward, in its order, then the array's capacity
+  ivit_status st = ivit::check_block_args(p, x, y, B, N);
+  if (st != IVIT_OK || B == 0 || N == 0) return st;
   if (ivit_block_workspace_bytes(B, N, p->D, p->Dm) > kScratchBytes) return IVIT_ERR_UNSUPPORTED;
+  ivit::DeviceCtx dc;
+  if ((st = ivit::device_ctx(&dc)) != IVIT_OK) return st;  // not an sm_100 device: UNSUPPORTED
   void* scratch = nullptr;
-  const ivit_status st = scratch_address(&scratch);
-  if (st != IVIT_OK) return st;
+  if ((st = scratch_address(dc.device, &scratch)) != IVIT_OK) return st;
   // Every intermediate is written in full before it is read, so nothing in the
   // array has to start at zero and nothing is cleared between calls.
   return ivit_block_forward(p, x, y, scratch, kScratchBytes, B, N, stream);
