@@ -59,6 +59,8 @@ def parse_args():
     ap.add_argument("--cpu-units", type=int, default=24,
                     help="CPU-baseline sample: (image, block) units the oracle runs")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-workloads", action="store_true",
+                    help="skip the other four workloads (measured after the headline one by default)")
     ap.add_argument("--kernel-reps", type=int, default=50)
     ap.add_argument("--model-blocks", type=int, default=12,
                     help="blocks of the whole-model timing (ViT-B workload only; 0 skips it)")
@@ -111,13 +113,40 @@ def load_peaks():
 
 
 def peak_for(bound, peaks, num_sms):
-    """(peak, unit, note) of a roofline bound."""
+    """(peak, unit, note) of a roofline bound.  The integer (ALU) roof is the
+    rate the library's integer-mix probe measured in this run when there is
+    one, else the nominal issue rate (SMs x 128 lanes x maximum SM clock)."""
     if bound == "tensor":
         return peaks["bf16_tflops"] * INT8_PER_BF16, "TOP/s", f"INT8 dense = {INT8_PER_BF16:g} x bf16 burst"
     if bound == "alu":
+        if peaks.get("alu_tops"):
+            return peaks["alu_tops"], "TOP/s", peaks["alu_note"]
         pk = num_sms * INT_LANES_PER_SM * peaks["sm_max_mhz"] * 1e6 / 1e12
-        return pk, "TOP/s", f"{num_sms} SMs x {INT_LANES_PER_SM} integer lanes x {peaks['sm_max_mhz']:.0f} MHz"
+        return pk, "TOP/s", f"nominal: {num_sms} SMs x {INT_LANES_PER_SM} lanes x {peaks['sm_max_mhz']:.0f} MHz"
     return peaks["hbm_gbs"], "GB/s", "HBM copy"
+
+
+def measure_int_rate(ivit, dev, iters=8192, reps=5):
+    """Integer operations per second of the Shiftmax instruction mix (the
+    library's probe: 8 independent chains of requant mul.hi, two clamps, an
+    offset, a table index and shared-memory table load, a row-sum add, a
+    shift and two adds), best of ``reps`` launches timed with CUDA events."""
+    import torch
+    num_sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    sink = torch.zeros(4 * num_sms, dtype=torch.int32, device=dev)
+    ivit.ivit_selftest_int_rate(64, sink)
+    torch.cuda.synchronize()
+    best = None
+    ops = 0
+    for _ in range(reps):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        ops = ivit.ivit_selftest_int_rate(iters, sink)
+        b.record()
+        torch.cuda.synchronize()
+        ms = a.elapsed_time(b)
+        best = ms if best is None else min(best, ms)
+    return ops / (best / 1e3) / 1e12, best
 
 
 # ---------------------------------------------------------------------------
@@ -125,7 +154,7 @@ def peak_for(bound, peaks, num_sms):
 # ---------------------------------------------------------------------------
 
 def oracle_units(wl, units):
-    """Time the oracle on ``units`` (image, block) pairs; returns (seconds, images/s)."""
+    """Time the oracle on ``units`` (image, block) pairs on one core; returns (seconds, images/s)."""
     import oracle
     ps = [oracle.block_params(q) for q in wl.blocks]
     N, nb = wl.N, len(wl.blocks)
@@ -140,46 +169,68 @@ def oracle_units(wl, units):
     return t, units / (t * nb)
 
 
+def oracle_all_cores(wl, block, images, threads=0):
+    """Time one block of the oracle over ``images`` images of the batch, one
+    image per task on every host core (thread per image); returns (seconds,
+    threads)."""
+    import oracle
+    p = oracle.block_params(wl.blocks[block])
+    N = wl.N
+    n = min(images, wl.B)
+    t0 = time.perf_counter()
+    _, used = oracle.block_forward_images(p, wl.x[:n * N], n, N, threads=threads)
+    return time.perf_counter() - t0, used
+
+
 def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return 0
     wl = synthetic.workload(args.workload, seed=args.seed)
     import oracle
-    ps = [oracle.block_params(q) for q in wl.blocks]
-    N, nb = wl.N, len(wl.blocks)
+    cores = oracle.host_cores()
+    per_step = min(cores, wl.B)
+    nb = len(wl.blocks)
     times = []
     for step in range(args.warmup + args.steps):
-        b = step % nb
-        img = (step // nb) % wl.B
-        xin = wl.x[img * N:(img + 1) * N]
-        t0 = time.perf_counter()
-        oracle.block_forward(ps[b], xin, 1, N)
-        dt = time.perf_counter() - t0
+        dt, used = oracle_all_cores(wl, step % nb, per_step, threads=cores)
         if step >= args.warmup:
             times.append(dt)
     step_s = sum(times) / len(times)
-    value = 1.0 / (step_s * nb)
-    sample = (f"each step: 1 image x 1 block of {args.workload} (block cycles over the {nb} block(s)); "
-              f"images/s = 1 / (step time x {nb} blocks)")
+    value = per_step / (step_s * nb)
+    sample = (f"each step: {per_step} images of {args.workload} through 1 block (block cycles over the {nb} "
+              f"block(s)), one image per thread on {used} host threads; images/s = images / (step time x {nb} "
+              f"blocks)")
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "images/s", "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_s * 1e3, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "int64", "data": "synthetic",
         "config": workload_config(wl, args),
-        "cpu_baseline": {"value": value, "unit": "images/s", "cores": 1, "kind": "oracle", "sample": sample},
+        "cpu_baseline": {"value": value, "unit": "images/s", "cores": used, "kind": "oracle", "sample": sample},
         "e2e": {"value": value, "unit": "images/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
     return 0
 
 
-def workload_config(wl, args, extra=None):
-    cfg = {"workload": wl.name, "B": wl.B, "N": wl.N, "D": wl.D, "H": wl.H, "Dm": wl.Dm,
-           "blocks": len(wl.blocks), "seed": args.seed}
-    if extra:
-        cfg.update(extra)
-    return cfg
+L2_NOMINAL = 126_000_000  # bytes; the input copies of a step rotate over at least twice this
+
+
+def input_copies(xbytes: int) -> int:
+    """Copies of the batch the timed steps rotate over: together more than
+    twice the L2, so every step reads its input from HBM."""
+    return max(2, min(64, math.ceil(2 * L2_NOMINAL / max(1, xbytes)) + 1))
+
+
+def workload_config(wl, args):
+    """The workload, identical in both arms (sizes, seed, parallelism and how
+    the timed steps keep their inputs out of the L2)."""
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    R = input_copies(wl.B * wl.N * wl.D)
+    return {"workload": wl.name, "B": wl.B, "N": wl.N, "D": wl.D, "H": wl.H, "Dm": wl.Dm,
+            "blocks": len(wl.blocks), "seed": args.seed,
+            "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+            "l2": l2_note(R, wl.B * wl.N * wl.D, L2_NOMINAL)}
 
 
 # ---------------------------------------------------------------------------
@@ -250,7 +301,8 @@ class ClockSampler:
             bits |= s[2]
         return {"sm_mhz": statistics.median(s[1] for s in busy), "sm_max_mhz": self.max_mhz,
                 "reasons": [n for b, n in _REASONS if bits & b and n != "gpu_idle"], "samples": len(busy),
-                "source": "nvml, every 10 ms over warm-up + timed steps"}
+                "source": f"nvml, every {self.period * 1e3:.0f} ms over a soak of the same steps and the timed steps",
+                "window_s": round(t1 - t0, 3)}
 
 
 # ---------------------------------------------------------------------------
@@ -302,6 +354,168 @@ def load_traffic(kernel, workload):
     return None
 
 
+class BlockRunner:
+    """Every block of a workload over one batch, replayed from CUDA graphs:
+    the input rotates over enough copies that they exceed twice the L2."""
+
+    def __init__(self, ivit, ivit_params, wl, dev, use_graph=True):
+        import torch
+        self.torch, self.ivit, self.wl, self.dev = torch, ivit, wl, dev
+        B, N, D, Dm = wl.B, wl.N, wl.D, wl.Dm
+        T = B * N
+        self.dps = [ivit_params.to_device(ivit_params.integer_params(q), dev) for q in wl.blocks]
+        self.ws = torch.empty(ivit.ivit_block_workspace_bytes(B, N, D, Dm), dtype=torch.uint8, device=dev)
+        self.R = input_copies(T * D)
+        x0 = torch.from_numpy(wl.x).to(dev)
+        self.xs = [x0.clone() for _ in range(self.R)]
+        self.ya = torch.empty((T, D), dtype=torch.int8, device=dev)
+        self.yb = torch.empty((T, D), dtype=torch.int8, device=dev)
+        # eager first pass (sets kernel attributes), launch accounting
+        c0 = ivit.ivit_launch_count()
+        self.out = self.step(0)
+        torch.cuda.synchronize()
+        self.out = self.out.clone()  # the intermediates are reused by every later step
+        self.launches_per_step = ivit.ivit_launch_count() - c0
+        if ivit.ivit_stream_status() != 0:
+            raise SystemExit("a kernel reported a timed-out wait")
+        self.use_graph = use_graph
+        self.graphs = []
+        if use_graph:
+            s = torch.cuda.Stream(device=dev)
+            s.wait_stream(torch.cuda.current_stream())
+            with torch.cuda.stream(s):
+                for r in range(self.R):
+                    g = torch.cuda.CUDAGraph()
+                    with torch.cuda.graph(g, stream=s):
+                        self.step(r)
+                    self.graphs.append(g)
+            torch.cuda.current_stream().wait_stream(s)
+            torch.cuda.synchronize()
+
+    def step(self, r, inp=None, out=None):
+        """All blocks over one batch: inp (default copy r) -> out (default the
+        last of the alternating intermediates)."""
+        cur = self.xs[r] if inp is None else inp
+        n = len(self.dps)
+        for i, dp in enumerate(self.dps):
+            nxt = self.ya if i % 2 == 0 else self.yb
+            if out is not None and i == n - 1:
+                nxt = out
+            self.ivit.ivit_block_forward(dp, cur, nxt, self.ws, self.wl.B, self.wl.N)
+            cur = nxt
+        return cur
+
+    def run(self, i):
+        if self.use_graph:
+            self.graphs[i % self.R].replay()
+        else:
+            self.step(i % self.R)
+
+    def timed(self, warmup, steps, barrier=lambda: None, soak_s=0.0):
+        """(device ms of `steps` steps after `warmup` untimed ones, wall-clock
+        window (t0, t1) that covers a soak of at least soak_s seconds of steps
+        just before the timed ones, and the timed steps)."""
+        torch = self.torch
+        for i in range(warmup):
+            self.run(i)
+        torch.cuda.synchronize()
+        t0 = time.perf_counter()
+        i = warmup
+        while time.perf_counter() - t0 < soak_s:
+            for _ in range(64):
+                self.run(i)
+                i += 1
+            torch.cuda.synchronize()
+        barrier()
+        torch.cuda.synchronize()
+        ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        ev0.record()
+        for k in range(steps):
+            self.run(i + k)
+        ev1.record()
+        torch.cuda.synchronize()
+        t1 = time.perf_counter()
+        barrier()
+        if self.ivit.ivit_stream_status() != 0:
+            raise SystemExit("a kernel reported a timed-out wait")
+        return ev0.elapsed_time(ev1), (t0, t1)
+
+    def release(self):
+        self.graphs.clear()
+
+
+def attention_launch_ms(ivit, wl, dp, ws, reps, dev):
+    """Device time of one attention launch on the workload's own QKV (from a
+    block forward), averaged over ``reps`` launches replayed from one graph."""
+    import torch
+    B, N, D, H = wl.B, wl.N, wl.D, wl.H
+    T = B * N
+    p = dp.host
+    up = lambda v: (v + 255) // 256 * 256
+    w8 = ws.view(torch.int8)
+    x = torch.from_numpy(wl.x).to(dev)
+    y = torch.empty_like(x)
+    ivit.ivit_block_forward(dp, x, y, ws, B, N)
+    torch.cuda.synchronize()
+    o_qkv = up(T * D)
+    qkv = w8[o_qkv:o_qkv + T * 3 * D].view(T, 3 * D).clone()
+    ctx = torch.empty((T, D), dtype=torch.int8, device=dev)
+    fn = lambda: ivit.ivit_attention(qkv, B, N, H, p["logit"], p["k_s"], p["attn_I0"], p["attn_M"],
+                                     p["attn_k_out"], p["attn_out"], ctx)
+    return graph_time_ms(fn, reps, dev)
+
+
+def graph_time_ms(fn, reps, dev):
+    """Average device ms of fn() over ``reps`` calls captured in one CUDA graph."""
+    import torch
+    for _ in range(3):
+        fn()
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    s = torch.cuda.Stream(device=dev)
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        with torch.cuda.graph(g, stream=s):
+            for _ in range(reps):
+                fn()
+    torch.cuda.current_stream().wait_stream(s)
+    g.replay()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    g.replay()
+    b.record()
+    torch.cuda.synchronize()
+    del g
+    return a.elapsed_time(b) / reps
+
+
+def other_workload(ivit, ivit_params, name, args, dev, peaks, num_sms):
+    """Images/s, effective TOP/s, fraction of the INT8 peak and the attention
+    roofline fraction of one more workload, measured the same way as the
+    headline one (graph replay, rotating inputs, CUDA events)."""
+    t0 = time.perf_counter()
+    wl = synthetic.workload(name, seed=args.seed)
+    gen_s = time.perf_counter() - t0
+    runner = BlockRunner(ivit, ivit_params, wl, dev, use_graph=not args.no_graph)
+    steps = max(10, min(args.steps, 50))
+    ms, _ = runner.timed(max(3, args.warmup), steps)
+    ms_step = ms / steps
+    nb = len(wl.blocks)
+    ops = wl.B * nb * ops_per_image_block(wl.N, wl.D)
+    eff = ops / (ms_step / 1e3) / 1e12
+    attn_ms = attention_launch_ms(ivit, wl, runner.dps[0], runner.ws, max(5, args.kernel_reps // 2), dev)
+    alu_peak, _, _ = peak_for("alu", peaks, num_sms)
+    attn_ops = SHIFTMAX_OPS_PER_SCORE * wl.B * wl.H * wl.N * wl.N
+    out = {"images_per_s": wl.B / (ms_step / 1e3), "ms_per_step": ms_step, "steps": steps,
+           "effective_tops": eff, "frac_int8_peak": eff / (peaks["bf16_tflops"] * INT8_PER_BF16),
+           "attention_ms": attn_ms, "attention_roofline_frac": attn_ops / (attn_ms / 1e3) / 1e12 / alu_peak,
+           "gpu_launches_per_step": int(runner.launches_per_step), "config": workload_config(wl, args),
+           "setup_s": round(gen_s, 1)}
+    runner.release()
+    return out
+
+
 def run_ours(args):
     import torch
     import torch.distributed as dist
@@ -324,85 +538,34 @@ def run_ours(args):
             dist.barrier()
 
     wl = synthetic.workload(args.workload, seed=args.seed + rank)
-    B, N, D, Dm = wl.B, wl.N, wl.D, wl.Dm
+    B, N, D = wl.B, wl.N, wl.D
     T = B * N
     nblk = len(wl.blocks)
-    dps = [ivit_params.to_device(ivit_params.integer_params(q), dev) for q in wl.blocks]
-    ws = torch.empty(ivit.ivit_block_workspace_bytes(B, N, D, Dm), dtype=torch.uint8, device=dev)
-    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
-    xbytes = T * D
-    R = max(2, min(64, math.ceil(2 * l2 / xbytes)))
-    x0 = torch.from_numpy(wl.x).to(dev)
-    xs = [x0.clone() for _ in range(R)]
-    ya = torch.empty((T, D), dtype=torch.int8, device=dev)
-    yb = torch.empty((T, D), dtype=torch.int8, device=dev)
+    runner = BlockRunner(ivit, ivit_params, wl, dev, use_graph=not args.no_graph)
+    use_graph = runner.use_graph
+    out = runner.out
 
-    def step(r, inp=None, out=None):
-        """All blocks over one batch: inp (default xs[r]) -> out (default the
-        last of the alternating intermediates)."""
-        cur = xs[r] if inp is None else inp
-        for i, dp in enumerate(dps):
-            nxt = ya if i % 2 == 0 else yb
-            if out is not None and i == nblk - 1:
-                nxt = out
-            ivit.ivit_block_forward(dp, cur, nxt, ws, B, N)
-            cur = nxt
-        return cur
-
-    # eager warm-up (sets kernel attributes), launch accounting
-    c0 = ivit.ivit_launch_count()
-    out = step(0)
-    torch.cuda.synchronize()
-    out = out.clone()  # the intermediates are reused by every later step
-    launches_per_step = ivit.ivit_launch_count() - c0
-    assert ivit.ivit_stream_status() == 0
-
-    use_graph = not args.no_graph
-    graphs = []
-    if use_graph:
-        s = torch.cuda.Stream(device=dev)
-        s.wait_stream(torch.cuda.current_stream())
-        with torch.cuda.stream(s):
-            for r in range(R):
-                g = torch.cuda.CUDAGraph()
-                with torch.cuda.graph(g, stream=s):
-                    step(r)
-                graphs.append(g)
-        torch.cuda.current_stream().wait_stream(s)
-        torch.cuda.synchronize()
-
-    def run(i):
-        if use_graph:
-            graphs[i % R].replay()
-        else:
-            step(i % R)
-
-    sampler = ClockSampler(local)
+    # Clocks are sampled every 5 ms from the start of a soak of at least half a
+    # second of the same steps, run right before the timed ones, to the end of
+    # the timed steps (the timed region alone lasts only a few ms at K = 20).
+    sampler = ClockSampler(local, period_s=0.005)
     sampler.start()
-    t_w0 = time.perf_counter()
-    for i in range(args.warmup):
-        run(i)
-    torch.cuda.synchronize()
-    barrier()
-    torch.cuda.synchronize()
-    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    ev0.record()
-    for i in range(args.steps):
-        run(args.warmup + i)
-    ev1.record()
-    torch.cuda.synchronize()
-    t_w1 = time.perf_counter()
-    barrier()
-    elapsed_ms = max_over_ranks(ev0.elapsed_time(ev1), world, dev)
+    elapsed_ms, (t_w0, t_w1) = runner.timed(args.warmup, args.steps, barrier, soak_s=0.6)
+    elapsed_ms = max_over_ranks(elapsed_ms, world, dev)
     sampler.stop()
     clocks = sampler.summary(t_w0, t_w1)
-    if ivit.ivit_stream_status() != 0:
-        raise SystemExit("a kernel reported a timed-out wait")
     ms_per_step = elapsed_ms / args.steps
     images_per_s = whole_job_images_per_s(world, B, args.steps, elapsed_ms)
 
+    # ---------------- the integer roof of the attention kernels, measured on this GPU
+    peaks, peak_src = load_peaks()
+    alu_tops, alu_ms = measure_int_rate(ivit, dev)
+    peaks["alu_tops"] = alu_tops
+    peaks["alu_note"] = (f"measured: integer Shiftmax-mix probe, {alu_tops:.2f} TOP/s "
+                         f"(best of 5 launches of {alu_ms:.2f} ms)")
+
     # ---------------- per-kernel breakdown of block 0 (CUDA events, same stream)
-    kern = kernel_breakdown(ivit, wl, dps[0], ws, xs, args.kernel_reps, dev)
+    kern = kernel_breakdown(ivit, wl, runner.dps[0], runner.ws, runner.xs, args.kernel_reps, dev, peaks)
 
     # ---------------- a whole model on synthetic weights (rank 0, not part of the metric)
     model = None
@@ -429,7 +592,7 @@ def run_ours(args):
             for j in range(2):
                 g = torch.cuda.CUDAGraph()
                 with torch.cuda.graph(g, stream=s_comp):
-                    step(0, e_in[j], e_out[j])
+                    runner.step(0, e_in[j], e_out[j])
                 e_graphs.append(g)
         torch.cuda.synchronize()
     k_e2e = max(1, min(args.steps, 50))
@@ -454,7 +617,7 @@ def run_ours(args):
                 if use_graph:
                     e_graphs[j].replay()
                 else:
-                    step(0, e_in[j], e_out[j])
+                    runner.step(0, e_in[j], e_out[j])
                 comp_done[j] = ev()
                 comp_done[j].record(s_comp)
             with torch.cuda.stream(s_out):
@@ -479,15 +642,24 @@ def run_ours(args):
     if not np.array_equal(y_host[(k_e2e - 1) % 2].numpy(), out.cpu().numpy()):
         raise SystemExit("end-to-end output differs from the device-resident run")
     e_graphs.clear()
+    launches_per_step = runner.launches_per_step
+    runner.release()
+
+    num_sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    # ---------------- the other workloads, each measured the same way (rank 0 at N = 1 only)
+    others = None
+    if world == 1 and not args.no_workloads and args.workload == DEFAULT_WORKLOAD:
+        others = {}
+        for name in synthetic.CONFIG_ORDER:
+            if name != wl.name:
+                others[name] = other_workload(ivit, ivit_params, name, args, dev, peaks, num_sms)
 
     # release graphs before the process group goes away
-    graphs.clear()
     if world > 1:
         dist.destroy_process_group()
     if rank != 0:
         return 0
 
-    peaks, peak_src = load_peaks()
     ops_step = world * B * nblk * ops_per_image_block(N, D)
     eff_tops = ops_step / (ms_per_step / 1e3) / 1e12
     int8_peak_burst = peaks["bf16_tflops"] * INT8_PER_BF16
@@ -498,24 +670,33 @@ def run_ours(args):
     traffic = load_traffic(dom["name"], wl.name)
     roofline = {"kernel": dom["name"], "bound": dom["bound"], "achieved": dom["achieved"], "peak": dom["peak"],
                 "unit": dom["unit"], "frac": dom["frac"], "traffic": traffic,
-                "peak_source": f"{dom['peak_note']} ({peak_src})", "launch_ms": dom["ms"],
+                "peak_source": dom["peak_note"] if dom["bound"] == "alu" else f"{dom['peak_note']} ({peak_src})",
+                "launch_ms": dom["ms"],
                 "algorithmic_per_launch": dom["amount"], "algorithmic_unit": dom["amount_unit"]}
+    for k in kern:
+        k["traffic"] = load_traffic(k["name"], wl.name)
 
     cpu = None
     if world == 1 and not args.no_cpu_baseline:
-        secs, ips = oracle_units(wl, args.cpu_units)
-        cpu = {"value": ips, "unit": "images/s", "cores": 1, "kind": "oracle",
-               "sample": f"{args.cpu_units} (image, block) units of {wl.name} through the single-threaded C "
-                         f"oracle ({secs:.1f} s); images/s = units / (time x {nblk} blocks)"}
+        secs1, ips1 = oracle_units(wl, args.cpu_units)
+        import oracle
+        n_all = min(wl.B, 2 * oracle.host_cores())
+        secs_all, used = oracle_all_cores(wl, 0, n_all)
+        ips_all = n_all / (secs_all * nblk)
+        cpu = {"value": ips_all, "unit": "images/s", "cores": used, "kind": "oracle",
+               "sample": f"{n_all} images of {wl.name} through block 0 of the C oracle, one image per thread on "
+                         f"{used} host threads ({secs_all:.1f} s); images/s = images / (time x {nblk} blocks)",
+               "single_core": {"value": ips1, "unit": "images/s", "cores": 1,
+                               "sample": f"{args.cpu_units} (image, block) units of {wl.name} through the "
+                                         f"single-threaded C oracle ({secs1:.1f} s); images/s = units / "
+                                         f"(time x {nblk} blocks)"}}
 
     line = {
         "metric": METRIC, "value": images_per_s, "unit": "images/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "int8", "data": "synthetic",
-        "config": workload_config(wl, args, {
-            "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
-            "l2": l2_note(R, xbytes, l2),
-            "graph": use_graph}),
+        "config": workload_config(wl, args),
+        "launch": "CUDA graph replay" if use_graph else "eager launches",
         "effective_tops": eff_tops,
         "frac_int8_peak_e2e": {"burst": eff_tops / int8_peak_burst, "sustained": eff_tops / int8_peak_sust,
                                "peak_source": f"{INT8_PER_BF16:g} x bf16 ({peak_src})"},
@@ -528,6 +709,8 @@ def run_ours(args):
         "clocks": clocks,
         "gpu_launches": int(launches_per_step * args.steps),
     }
+    if others is not None:
+        line["workloads"] = others
     if model is not None:
         line["model"] = model
     print(json.dumps(line), flush=True)
@@ -581,7 +764,7 @@ def model_forward_timing(ivit, n_blocks, B, dev, reps=10):
             "setup_s": setup_s}
 
 
-def kernel_breakdown(ivit, wl, dp, ws, xs, reps, dev):
+def kernel_breakdown(ivit, wl, dp, ws, xs, reps, dev, peaks):
     """Average device time per launch of every kernel of one block, each timed
     alone over ``reps`` back-to-back launches with CUDA events.  Inputs are the
     block's own intermediates (left in the workspace by a block forward)."""
@@ -682,7 +865,6 @@ def kernel_breakdown(ivit, wl, dp, ws, xs, reps, dev):
     add("shiftgelu_standalone", lambda i: ivit.ivit_shiftgelu(hs[i % len(hs)], p["gelu_I0"], p["gelu_M"],
                                                               p["gelu_k_out"], p["gelu_out"], h_o),
         "hbm", 2 * T * Dm, in_block=False)
-    peaks, src = load_peaks()
     num_sms = torch.cuda.get_device_properties(dev).multi_processor_count
     for k in out:
         k["peak"], k["unit"], k["peak_note"] = peak_for(k["bound"], peaks, num_sms)

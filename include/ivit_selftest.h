@@ -1,7 +1,8 @@
 /*
  * ivit_selftest.h -- diagnostic entry points of the integer-only ViT library.
  *
- * These exercise the library's failure path without a GPU fault.  Every wait
+ * The first exercises the library's failure path without a GPU fault; the
+ * second measures the integer throughput that bounds the attention kernels.  Every wait
  * inside the library's kernels (an mbarrier spin) is bounded by a budget of
  * one second of %globaltimer; a wait that runs out records IVIT_ERR_TIMEOUT
  * in the per-device status word, and the kernel returns instead of hanging.
@@ -25,6 +26,23 @@ extern "C" {
  * IVIT_ERR_UNSUPPORTED without an sm_100 device, IVIT_ERR_CUDA if the launch
  * failed.  Takes about one second of GPU time.                               */
 ivit_status ivit_selftest_wait_timeout(ivit_stream_t stream);
+
+/* Integer throughput probe: the roof of the attention kernels' Shiftmax
+ * passes ("I-ViT", section 3.3), whose per-score work runs on the CUDA cores.
+ * Enqueues one kernel of 4 x (SM count) blocks of 256 threads; every thread
+ * runs `iters` iterations over 8 independent chains of the per-score integer
+ * mix (requant mul.hi, two clamps, offset from the row maximum, table index,
+ * ShiftExp table load from shared memory, row-sum add, a shift and two adds
+ * that feed the next step: 10 operations).  *ops receives the operations one
+ * launch executes (blocks x 256 x iters x 8 x 10); the caller times the
+ * launch (CUDA events on `stream`) and divides.  sink: device int32 array of
+ * at least sink_len >= 4 x (SM count) elements, owned by the caller, which
+ * receives one checksum per block (read-modify-write: its contents are not
+ * meaningful).  Returns IVIT_ERR_INVALID_ARG for iters < 1, a NULL pointer or
+ * a short sink, IVIT_ERR_UNSUPPORTED without an sm_100 device, IVIT_ERR_CUDA
+ * if the launch failed.                                                      */
+ivit_status ivit_selftest_int_rate(int32_t iters, int32_t *sink, int32_t sink_len, int64_t *ops,
+                                   ivit_stream_t stream);
 
 #ifdef __cplusplus
 }

@@ -23,7 +23,7 @@ __all__ = [
     "ivit_block_workspace_bytes", "ivit_block_forward", "ivit_stream_status", "ivit_launch_count",
     "ivit_block_forward_static", "STATIC_SCRATCH_BYTES", "EXPORTED_SYMBOLS",
     "ModelParams", "ivit_patch_embed_workspace_bytes", "ivit_patch_embed", "ivit_head_workspace_bytes", "ivit_head",
-    "ivit_model_workspace_bytes", "ivit_model_forward", "ivit_selftest_wait_timeout",
+    "ivit_model_workspace_bytes", "ivit_model_forward", "ivit_selftest_wait_timeout", "ivit_selftest_int_rate",
 ]
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
@@ -39,7 +39,7 @@ EXPORTED_SYMBOLS = (
     "ivit_block_forward_static",
     "ivit_patch_embed_workspace_bytes", "ivit_patch_embed", "ivit_head_workspace_bytes", "ivit_head",
     "ivit_model_workspace_bytes", "ivit_model_forward",
-    "ivit_selftest_wait_timeout",
+    "ivit_selftest_wait_timeout", "ivit_selftest_int_rate",
 )
 
 _STATUS = {0: "IVIT_OK", 1: "IVIT_ERR_INVALID_ARG", 2: "IVIT_ERR_UNSUPPORTED", 3: "IVIT_ERR_CUDA",
@@ -149,6 +149,8 @@ def lib() -> C.CDLL:
             L.ivit_launch_count.argtypes = []
             L.ivit_selftest_wait_timeout.restype = C.c_int
             L.ivit_selftest_wait_timeout.argtypes = [vp]
+            L.ivit_selftest_int_rate.restype = C.c_int
+            L.ivit_selftest_int_rate.argtypes = [i32, vp, i32, C.POINTER(C.c_int64), vp]
             _lib = L
     return _lib
 
@@ -341,6 +343,15 @@ def ivit_selftest_wait_timeout(stream=None):
     """Enqueue the diagnostic kernel whose bounded wait runs out (about one
     second); ivit_stream_status() then reports IVIT_ERR_TIMEOUT once."""
     _check("ivit_selftest_wait_timeout", lib().ivit_selftest_wait_timeout(_stream(stream)))
+
+
+def ivit_selftest_int_rate(iters: int, sink, stream=None) -> int:
+    """Enqueue the integer-throughput probe; returns the integer operations
+    the launch executes (time it on the stream to get a rate)."""
+    ops = C.c_int64(0)
+    _check("ivit_selftest_int_rate", lib().ivit_selftest_int_rate(int(iters), _ptr(sink, torch.int32, "sink"),
+                                                                  sink.numel(), C.byref(ops), _stream(stream)))
+    return int(ops.value)
 
 
 def ivit_patch_embed_workspace_bytes(B: int, C_in: int, Hi: int, Wi: int, P: int, D: int) -> int:

@@ -338,6 +338,56 @@ def block_forward(p, x, B: int, N: int):
 
 def _block_forward(p, x, B: int, N: int):
     x = np.ascontiguousarray(x, dtype=np.int8)
+    s, keep = _block_struct(p)
+    y = np.zeros_like(x)
+    rc = lib().orc_block_forward(C.byref(s), x.ctypes.data, y.ctypes.data, int(B), int(N))
+    if rc != 0:
+        raise MemoryError("oracle block forward could not allocate scratch")
+    return y
+
+
+def host_cores() -> int:
+    """Host cores this process may run on."""
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:  # pragma: no cover - non-Linux
+        return os.cpu_count() or 1
+
+
+def block_forward_images(p, x, B: int, N: int, threads: int = 0):
+    """The same result as ``block_forward(p, x, B, N)``, computed one image per
+    task on ``threads`` host threads (default: every core this process may
+    use).  Images never interact in the block, and each task is one call of
+    the single-threaded C oracle on its own image (ctypes releases the
+    interpreter lock for the call), so the output is identical to the
+    single-call one.  Returns (y, threads used)."""
+    from concurrent.futures import ThreadPoolExecutor
+    x = np.ascontiguousarray(x, dtype=np.int8)
+    threads = max(1, min(int(threads) or host_cores(), max(1, int(B))))
+    if p.get("linear_round", 0):
+        lib().orc_set_linear_rounding(1)
+    try:
+        s, keep = _block_struct(p)
+        y = np.zeros_like(x)
+        D = int(p["D"])
+        row = N * D
+
+        def one(img):
+            off = img * row
+            return lib().orc_block_forward(C.byref(s), x.ctypes.data + off, y.ctypes.data + off, 1, int(N))
+
+        with ThreadPoolExecutor(max_workers=threads) as ex:
+            rcs = list(ex.map(one, range(int(B))))
+    finally:
+        if p.get("linear_round", 0):
+            lib().orc_set_linear_rounding(0)
+    if any(rcs):
+        raise MemoryError("oracle block forward could not allocate scratch")
+    return y, threads
+
+
+def _block_struct(p):
+    """The C parameter struct of a block, and the arrays it points into."""
     keep = []
 
     def arr(a, dt):
@@ -367,11 +417,7 @@ def _block_forward(p, x, B: int, N: int):
     s.b2, s.c2 = arr(p["b2"], np.int32), arr(p["c2"], np.int32)
     s.res2_b_skip, s.res2_b_branch, s.res2_c = p["res2"]
     s.ln_F, s.ln_M = p["ln_F"], p["ln_M"]
-    y = np.zeros_like(x)
-    rc = lib().orc_block_forward(C.byref(s), x.ctypes.data, y.ctypes.data, int(B), int(N))
-    if rc != 0:
-        raise MemoryError("oracle block forward could not allocate scratch")
-    return y
+    return s, keep
 
 
 # ---------------------------------------------------------------------------
