@@ -240,6 +240,43 @@ def test_attention_parity(B, N, H, tails, k_s):
     assert untouched()
 
 
+# Short sequences with 8-bit logits: key counts that change how the 16-key
+# chunks split over the two half rows (a ragged last chunk or none, chunks
+# that stop short of the 32-key MMA step), both tails, and enough heads and
+# images that every CTA takes many items through both softmax groups
+SHORT_CASES = [(3, 1, 2, "normal"), (2, 17, 3, "laplace"), (4, 64, 2, "normal"), (2, 100, 3, "laplace"),
+                 (1, 129, 2, "normal"), (2, 160, 3, "normal"), (2, 176, 2, "laplace"), (3, 193, 4, "normal"),
+                 (64, 197, 12, "normal"), (5, 197, 3, "laplace"), (2, 200, 5, "laplace"), (3, 208, 4, "normal"),
+                 (2, 209, 3, "laplace"), (4, 224, 4, "normal"), (1, 197, 1, "normal")]
+
+
+@pytest.mark.parametrize("B,N,H,tails", SHORT_CASES)
+def test_attention_short_parity(B, N, H, tails):
+    ac = synthetic.attention_case(B, N, H, seed=7 * N + H, tails=tails, k_s=8)
+    I0 = oracle.recip_i0(ac.S_logit)
+    logit, out = oracle.dyadic(ac.logit_ratio), oracle.dyadic(ac.out_ratio)
+    qkv = dev(ac.qkv, torch.int8)
+    ctx, untouched = guarded((B * N, H * 64))
+    ivit.ivit_attention(qkv, B, N, H, logit, 8, I0, 30, 8, out, ctx)
+    np.testing.assert_array_equal(host(ctx), oracle.attention(ac.qkv, B, N, H, logit, 8, I0, 30, 8, out))
+    assert untouched()
+
+
+@pytest.mark.parametrize("I0,M,k_out", [(1, 30, 8), (2, 20, 8), (255, 30, 8), (97, 30, 5), (40, 12, 8),
+                                        (256, 30, 8), (4096, 30, 8)])
+def test_attention_short_shiftmax_parameters(I0, M, k_out):
+    """N = 197 at I0 = 1 (a hard maximum), I0 at and past one byte, large I0,
+    a small IntDiv M (the exact 32-bit product path instead of mul.hi) and
+    k_out < 8."""
+    ac = synthetic.attention_case(3, 197, 2, seed=300 + I0, tails="laplace")
+    qkv = dev(ac.qkv, torch.int8)
+    ctx = torch.empty((3 * 197, 128), dtype=torch.int8, device="cuda")
+    logit = oracle.dyadic(ac.logit_ratio)
+    out = oracle.dyadic(ac.out_ratio * 2 ** (8 - k_out))
+    ivit.ivit_attention(qkv, 3, 197, 2, logit, 8, I0, M, k_out, out, ctx)
+    np.testing.assert_array_equal(host(ctx), oracle.attention(ac.qkv, 3, 197, 2, logit, 8, I0, M, k_out, out))
+
+
 @pytest.mark.parametrize("k_s", [8, 12, 16])
 def test_attention_hardmax_wide_logits(k_s):
     """I_0 = 1 (the division by I_0 is the identity) and (b_s, c_s) = (1, 0):
