@@ -130,6 +130,19 @@ def _bind(L):
     L.orc_layernorm.restype = None
     L.orc_layernorm.argtypes = [C.c_void_p, C.c_int64, C.c_int32, C.c_void_p, C.c_void_p,
                                 C.c_int32, C.c_int32, C.c_int32, C.c_int32, C.c_void_p]
+    L.orc_shiftgelu_rowmax.restype = None
+    L.orc_shiftgelu_rowmax.argtypes = [C.c_void_p, C.c_int64, C.c_int32, C.c_int32, C.c_int32, C.c_int32,
+                                       C.c_int32, C.c_int32, C.c_void_p]
+    L.orc_log2_code.restype = C.c_int32
+    L.orc_log2_code.argtypes = [C.c_int64]
+    L.orc_lis_row.restype = None
+    L.orc_lis_row.argtypes = [C.c_void_p, C.c_int, C.c_int32, C.c_int, C.c_void_p]
+    L.orc_attention_lis.restype = None
+    L.orc_attention_lis.argtypes = [C.c_void_p, C.c_int32, C.c_int32, C.c_int32, C.c_int32, C.c_int32, C.c_int32,
+                                    C.c_int32, C.c_int32, C.c_int32, C.c_int32, C.c_void_p]
+    L.orc_layernorm_ptf.restype = None
+    L.orc_layernorm_ptf.argtypes = [C.c_void_p, C.c_int64, C.c_int32, C.c_void_p, C.c_void_p, C.c_void_p,
+                                    C.c_int32, C.c_int32, C.c_int32, C.c_int32, C.c_void_p]
     L.orc_patch_embed.restype = C.c_int
     L.orc_patch_embed.argtypes = [C.c_void_p, C.c_int32, C.c_int32, C.c_int32, C.c_int32, C.c_int32,
                                   C.c_void_p, C.c_void_p, C.c_void_p, C.c_void_p, C.c_int32,
@@ -280,6 +293,56 @@ def layernorm(x, gamma, beta, F: int, M_ln: int, out):
     y = np.zeros_like(x)
     lib().orc_layernorm(x.ctypes.data, rows, cols, gamma.ctypes.data, beta.ctypes.data,
                         int(F), int(M_ln), int(out[0]), int(out[1]), y.ctypes.data)
+    return y
+
+
+# ---------------------------------------------------------------------------
+# variants: row-max ShiftGELU, Log-Int-Softmax attention, PTF I-LayerNorm
+# ---------------------------------------------------------------------------
+
+def shiftgelu_rowmax(x, I0: int, M: int, k_out: int, out):
+    """x [rows x cols] int8 -> ShiftGELU with I_max the row's largest exponent."""
+    x = np.ascontiguousarray(x, dtype=np.int8)
+    rows, cols = x.shape
+    y = np.zeros_like(x)
+    lib().orc_shiftgelu_rowmax(x.ctypes.data, rows, cols, int(I0), int(M), int(k_out), int(out[0]), int(out[1]),
+                               y.ctypes.data)
+    return y
+
+
+def log2_code(P16: int) -> int:
+    return int(lib().orc_log2_code(int(P16)))
+
+
+def lis_row(L, I0: int, M: int = 30):
+    """4-bit log2 codes of one row of integer logits (Log-Int-Softmax)."""
+    L = np.ascontiguousarray(L, dtype=np.int32)
+    codes = np.zeros(L.size, dtype=np.int32)
+    lib().orc_lis_row(L.ctypes.data, L.size, int(I0), int(M), codes.ctypes.data)
+    return codes
+
+
+def attention_lis(qkv, B: int, N: int, H: int, logit, k_s: int, I0: int, M: int, out):
+    """qkv [B*N x 3*H*64] int8 -> ctx [B*N x H*64] int8 with Log-Int-Softmax."""
+    qkv = np.ascontiguousarray(qkv, dtype=np.int8)
+    assert qkv.shape == (B * N, 3 * H * 64)
+    ctx = np.zeros((B * N, H * 64), dtype=np.int8)
+    lib().orc_attention_lis(qkv.ctypes.data, B, N, H, int(logit[0]), int(logit[1]), int(k_s), int(I0), int(M),
+                            int(out[0]), int(out[1]), ctx.ctypes.data)
+    return ctx
+
+
+def layernorm_ptf(x, alpha, gamma, beta, F: int, M_ln: int, out):
+    """I-LayerNorm of x [rows x cols] whose channel i carries the power-of-two factor 2^alpha[i]."""
+    x = np.ascontiguousarray(x, dtype=np.int8)
+    rows, cols = x.shape
+    alpha = np.ascontiguousarray(alpha, dtype=np.uint8)
+    gamma = np.ascontiguousarray(gamma, dtype=np.int8)
+    beta = np.ascontiguousarray(beta, dtype=np.int32)
+    assert alpha.size == cols and int(alpha.max(initial=0)) <= 3
+    y = np.zeros_like(x)
+    lib().orc_layernorm_ptf(x.ctypes.data, rows, cols, alpha.ctypes.data, gamma.ctypes.data, beta.ctypes.data,
+                            int(F), int(M_ln), int(out[0]), int(out[1]), y.ctypes.data)
     return y
 
 

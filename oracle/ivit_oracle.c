@@ -428,6 +428,165 @@ void orc_layernorm(const int8_t *x, int64_t rows, int32_t cols,
 }
 
 /* ------------------------------------------------------------------------ */
+/* variants of the steps above (readings the pages leave open)              */
+/* ------------------------------------------------------------------------ */
+
+/*
+ * ShiftGELU with a row maximum, [IVIT] 3.4.  The page multiplies the
+ * sigmoid's numerator and denominator by e^(-S I_max) and stops before it
+ * defines I_max.  READING (variant of the per-element one above): I_max is
+ * the largest exponent over the whole row, max(0, max_i I_p,i), as Shiftmax
+ * subtracts its row maximum; the 0 keeps both exponents I_p - I_max and
+ * -I_max <= 0, which the shift-exponential requires.  Each element takes
+ * e1 = ShiftExp(I_p - I_max), e2 = ShiftExp(-I_max), sigma = IntDiv(e1, e1 + e2).
+ * READING: when both exponentials floor to 0 the IntDiv divisor is taken as
+ * 1 (no division by zero), so sigma = 0.  x: rows x cols int8.
+ */
+void orc_shiftgelu_rowmax(const int8_t *x, int64_t rows, int32_t cols, int32_t I0,
+                          int32_t M, int32_t k_out, int32_t b_g, int32_t c_g,
+                          int8_t *y)
+{
+    for (int64_t r = 0; r < rows; ++r) {
+        const int8_t *xr = x + r * cols;
+        int64_t I_max = 0;
+        for (int32_t i = 0; i < cols; ++i) {
+            int64_t v = xr[i];
+            int64_t I_p = v + shr_floor(v, 1) + shr_floor(v, 3) + shr_floor(v, 4);
+            if (I_p > I_max)
+                I_max = I_p;
+        }
+        int64_t e2 = orc_shift_exp(-I_max, I0);
+        for (int32_t i = 0; i < cols; ++i) {
+            int64_t v = xr[i];
+            int64_t I_p = v + shr_floor(v, 1) + shr_floor(v, 3) + shr_floor(v, 4);
+            int64_t e1 = orc_shift_exp(I_p - I_max, I0);
+            int64_t sum = e1 + e2;
+            int64_t sigma = orc_int_div(e1, sum > 0 ? sum : 1, M, k_out);
+            y[r * cols + i] = (int8_t)orc_requant(v * sigma, b_g, c_g, 8);
+        }
+    }
+}
+
+/*
+ * 4-bit log2 code of a 16-bit attention probability P16 (scale 2^-15):
+ * k = clip(15 - round(log2 P16), 0, 15), P16 = 0 giving 15, so that the
+ * probability is about 2^-k.  After the log2 quantiser of the Trio-ViT
+ * article, section IV-D (clip(round(log2(.)), -a, b)).  round(log2 P) of an
+ * integer P >= 1 is floor(log2 P) + 1 exactly when P >= 2^floor(log2 P) sqrt 2,
+ * i.e. when P^2 >= 2^(2 floor(log2 P) + 1): integer arithmetic only.
+ */
+int32_t orc_log2_code(int64_t P16)
+{
+    if (P16 <= 0)
+        return 15;
+    int fl = bit_length(P16) - 1;
+    int r = fl + ((P16 * P16 >= ((int64_t)1 << (2 * fl + 1))) ? 1 : 0);
+    int k = 15 - r;
+    return k < 0 ? 0 : (k > 15 ? 15 : k);
+}
+
+/*
+ * Log-Int-Softmax of one row of n logits (the FQ-ViT record, abstract: the
+ * attention map quantised to 4 bits on a log2 grid, multiplied with V by
+ * BitShift).  READING: the integer Shiftmax of [IVIT] 3.3 up to its row sum,
+ * then the IntDiv taken to 16 bits, P16 = IntDiv(e, sum, M, 16) in [0, 2^15]
+ * (M >= 15), then its 4-bit code (orc_log2_code).  codes: n entries in [0, 15].
+ */
+void orc_lis_row(const int32_t *L, int n, int32_t I0, int M, int32_t *codes)
+{
+    int32_t mx = L[0];
+    for (int j = 1; j < n; ++j)
+        if (L[j] > mx) mx = L[j];
+    int64_t sum = 0;
+    for (int j = 0; j < n; ++j)
+        sum += orc_shift_exp((int64_t)L[j] - mx, I0);
+    for (int j = 0; j < n; ++j)
+        codes[j] = orc_log2_code(orc_int_div(orc_shift_exp((int64_t)L[j] - mx, I0), sum, M, 16));
+}
+
+/*
+ * Attention with Log-Int-Softmax: as orc_attention, with the attention map of
+ * each row the 4-bit codes k_j of orc_lis_row and the product with V the bit
+ * shift acc_d = sum_j V_jd << (15 - k_j) (2^-k_j at scale 2^-15: exact),
+ * requantised with (b_o, c_o), b_o / 2^c_o ~ S_v 2^-15 / S_ctx.  READING: the
+ * left shift at scale 2^-15 (a right shift of the int8 V by k would drop all
+ * of V at k >= 8).
+ */
+void orc_attention_lis(const int8_t *QKV, int32_t B, int32_t N, int32_t H,
+                       int32_t b_s, int32_t c_s, int32_t k_s, int32_t I0,
+                       int32_t M, int32_t b_o, int32_t c_o, int8_t *ctx)
+{
+    const int64_t D = (int64_t)H * 64;
+    const int64_t ld = 3 * D;
+    int32_t *L = (int32_t *)malloc(sizeof(int32_t) * (size_t)N);
+    int32_t *K = (int32_t *)malloc(sizeof(int32_t) * (size_t)N);
+    for (int32_t bi = 0; bi < B; ++bi) {
+        const int8_t *base = QKV + (int64_t)bi * N * ld;
+        for (int32_t h = 0; h < H; ++h) {
+            for (int32_t i = 0; i < N; ++i) {
+                const int8_t *q = base + (int64_t)i * ld + h * 64;
+                for (int32_t j = 0; j < N; ++j) {
+                    const int8_t *k = base + (int64_t)j * ld + D + h * 64;
+                    int64_t s = 0;
+                    for (int d = 0; d < 64; ++d)
+                        s += (int64_t)q[d] * (int64_t)k[d];
+                    L[j] = (int32_t)orc_requant(s, b_s, c_s, k_s);
+                }
+                orc_lis_row(L, N, I0, M, K);
+                int8_t *out = ctx + ((int64_t)bi * N + i) * D + h * 64;
+                for (int d = 0; d < 64; ++d) {
+                    int64_t acc = 0;
+                    for (int32_t j = 0; j < N; ++j)
+                        acc += (int64_t)base[(int64_t)j * ld + 2 * D + h * 64 + d] * ((int64_t)1 << (15 - K[j]));
+                    out[d] = (int8_t)orc_requant(acc, b_o, c_o, 8);
+                }
+            }
+        }
+    }
+    free(L);
+    free(K);
+}
+
+/*
+ * I-LayerNorm of an input quantised with power-of-two factors (the FQ-ViT
+ * record, abstract: the Power-of-Two Factor against the inter-channel
+ * variation of LayerNorm inputs).  READING: channel i of the int8 input
+ * carries the scale S 2^alpha_i, with one layer-wise S and alpha_i in
+ * {0, 1, 2, 3}; the LayerNorm input at the common scale S is the bit shift
+ * x_i << alpha_i, and I-LayerNorm ([IVIT] 3.5, as orc_layernorm) runs on it
+ * unchanged.  alpha: cols entries.
+ */
+void orc_layernorm_ptf(const int8_t *x, int64_t rows, int32_t cols,
+                       const uint8_t *alpha, const int8_t *gamma,
+                       const int32_t *beta, int32_t F, int32_t M_ln, int32_t b,
+                       int32_t c, int8_t *y)
+{
+    for (int64_t r = 0; r < rows; ++r) {
+        const int8_t *xr = x + r * cols;
+        int64_t sx = 0;
+        for (int32_t i = 0; i < cols; ++i)
+            sx += (int64_t)xr[i] * ((int64_t)1 << alpha[i]);
+        int64_t mu = floor_div(sx, cols);
+        int64_t sd2 = 0;
+        for (int32_t i = 0; i < cols; ++i) {
+            int64_t d = (int64_t)xr[i] * ((int64_t)1 << alpha[i]) - mu;
+            sd2 += d * d;
+        }
+        int64_t V = floor_div(sd2, cols);
+        int64_t sigma = orc_isqrt_newton(V);
+        if (sigma < 1)
+            sigma = 1;
+        int64_t f = floor_div((int64_t)1 << M_ln, sigma);
+        for (int32_t i = 0; i < cols; ++i) {
+            int64_t d = (int64_t)xr[i] * ((int64_t)1 << alpha[i]) - mu;
+            int64_t nv = shr_floor(d * f, M_ln - F);
+            int64_t acc = nv * gamma[i] + beta[i];
+            y[r * cols + i] = (int8_t)orc_requant(acc, b, c, 8);
+        }
+    }
+}
+
+/* ------------------------------------------------------------------------ */
 /* the encoder block, [IVIT] 3.1 (pre-LN, two residuals), [TRIO] eqs (1)-(3)*/
 /* ------------------------------------------------------------------------ */
 

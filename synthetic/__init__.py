@@ -365,6 +365,43 @@ def layernorm_case(rows: int, cols: int, seed: int = 0, chan_std=(0.1, 10.0), F:
     return LayerNormCase(x=x, gamma=gq, beta=quant_i32(be, S_g * 2.0 ** -F), out_ratio=S_g * 2.0 ** -F / S_out, F=F)
 
 
+@dataclasses.dataclass
+class PtfCase:
+    x_ptf: np.ndarray            # int8, channel i at scale s 2^alpha_i
+    alpha: np.ndarray            # uint8 power-of-two factors in [0, 3]
+    x_tensor: np.ndarray         # int8, one per-tensor scale (= s 2^3)
+    gamma: np.ndarray
+    beta: np.ndarray
+    out_ratio: float             # S_gamma 2^-F / S_out
+    S_out: float
+    ln_float: np.ndarray         # floating-point LayerNorm of the unquantised rows
+    F: int = 7
+
+
+def ptf_case(rows: int, cols: int, seed: int = 0, chan_std=(0.1, 20.0), K: int = 3, F: int = 7) -> PtfCase:
+    """LayerNorm inputs with inter-channel variation (per-channel std
+    log-uniform on chan_std, as the ViT-B workload), quantised two ways: one
+    per-tensor scale S, and power-of-two factors on a layer-wise s = S / 2^K,
+    where channel i takes the smallest alpha_i in [0, K] whose range
+    s 2^alpha_i 127.5 covers the channel (off-line calibration)."""
+    r = rng(seed, "op", 5)
+    sig = np.exp(r.uniform(math.log(chan_std[0]), math.log(chan_std[1]), size=cols))
+    xf = r.standard_normal((rows, cols)) * sig[None, :]
+    S = scale_of(xf)
+    s = S / 2.0 ** K
+    m = np.max(np.abs(xf), axis=0)
+    alpha = np.clip(np.ceil(np.log2(np.maximum(m / (127.5 * s), 1e-30))), 0, K).astype(np.uint8)
+    x_ptf = quant_i8(xf, s * 2.0 ** alpha.astype(np.float64)[None, :])
+    x_tensor = quant_i8(xf, S)
+    g = 1.0 + 0.1 * r.standard_normal(cols)
+    be = 0.02 * r.standard_normal(cols)
+    S_g = scale_of(g)
+    gq = quant_i8(g, S_g)
+    ln_f = _layernorm_f(xf, gq * S_g, be)
+    S_out = scale_of(ln_f)
+    return PtfCase(x_ptf=x_ptf, alpha=alpha, x_tensor=x_tensor, gamma=gq, beta=quant_i32(be, S_g * 2.0 ** -F),
+                   out_ratio=S_g * 2.0 ** -F / S_out, S_out=S_out, ln_float=ln_f, F=F)
+
 
 # ---------------------------------------------------------------------------
 # a whole model: patch embedding, blocks, classifier head

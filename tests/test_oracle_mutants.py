@@ -4,8 +4,9 @@ The oracle is test infrastructure, and its pins are meant to fail on any
 plausible mistake in it: a dropped term, a wrong sign, shift or index, a
 transposed operand, truncation where the method floors.  This test plants
 one such mistake at a time in a copy of the oracle's C source (on the CPU),
-builds the copy, and runs the pins of test_oracle_pins.py against it in a
-separate process, which stops at the first failing pin.  A copy that passes
+builds the copy, and runs the pins of test_oracle_pins.py and
+test_oracle_next.py against it in a separate process, which stops at the
+first failing pin.  A copy that passes
 every pin is a slip the pins miss, and fails this test.
 
 Deliberately absent: removing the quantiser's clip to [-m, m].  The clamp to
@@ -98,6 +99,30 @@ MUTANTS = [
     ("head reads the last token", "x[(int64_t)bi * Ntok * D + j]", "x[((int64_t)bi * Ntok + Ntok - 1) * D + j]"),
     ("head LayerNorm shift off by one", "orc_layernorm(t, B, D, gamma, beta, F, M_ln, ln_b, ln_c, n);",
      "orc_layernorm(t, B, D, gamma, beta, F, M_ln, ln_b, ln_c + 1, n);"),
+    # ShiftGELU with a row maximum
+    ("row-max ShiftGELU takes the row minimum", "if (I_p > I_max)\n                I_max = I_p;",
+     "if (I_p < I_max)\n                I_max = I_p;"),
+    ("row maximum without the floor at 0", "int64_t I_max = 0;\n        for (int32_t i = 0; i < cols; ++i) {\n            int64_t v",
+     "int64_t I_max = -300;\n        for (int32_t i = 0; i < cols; ++i) {\n            int64_t v"),
+    ("second exponential at 0", "int64_t e2 = orc_shift_exp(-I_max, I0);\n        for",
+     "int64_t e2 = orc_shift_exp(0, I0);\n        for"),
+    ("0 / 0 read as one half", "int64_t sigma = orc_int_div(e1, sum > 0 ? sum : 1, M, k_out);",
+     "int64_t sigma = sum > 0 ? orc_int_div(e1, sum, M, k_out) : ((int64_t)1 << (k_out - 2));"),
+    # Log-Int-Softmax
+    ("log2 rounded at 2 instead of sqrt 2", "((int64_t)1 << (2 * fl + 1))", "((int64_t)1 << (2 * fl + 2))"),
+    ("zero probability coded 0", "if (P16 <= 0)\n        return 15;", "if (P16 <= 0)\n        return 0;"),
+    ("LIS probability to 15 bits", "sum, M, 16));", "sum, M, 15));"),
+    ("BitShift one place short", "((int64_t)1 << (15 - K[j]))", "((int64_t)1 << (14 - K[j]))"),
+    ("LIS reads V from the K columns", "base[(int64_t)j * ld + 2 * D + h * 64 + d] * ((int64_t)1",
+     "base[(int64_t)j * ld + D + h * 64 + d] * ((int64_t)1"),
+    # I-LayerNorm with power-of-two factors
+    ("PTF mean without the factors", "sx += (int64_t)xr[i] * ((int64_t)1 << alpha[i]);", "sx += (int64_t)xr[i];"),
+    ("PTF variance without the factors",
+     "int64_t d = (int64_t)xr[i] * ((int64_t)1 << alpha[i]) - mu;\n            sd2",
+     "int64_t d = (int64_t)xr[i] - mu;\n            sd2"),
+    ("PTF normalises the unshifted input",
+     "int64_t d = (int64_t)xr[i] * ((int64_t)1 << alpha[i]) - mu;\n            int64_t nv",
+     "int64_t d = (int64_t)xr[i] - mu;\n            int64_t nv"),
 ]
 
 # Runs the pins against one build, stopping at the first failure: exit 1 if
@@ -107,13 +132,14 @@ import inspect, sys
 sys.path[:0] = [sys.argv[2], sys.argv[3]]
 import oracle
 oracle.use_library(sys.argv[1])
-import test_oracle_pins as pins
-for name, fn in inspect.getmembers(pins, inspect.isfunction):
-    if name.startswith("test_") and not inspect.signature(fn).parameters:
-        try:
-            fn()
-        except Exception:
-            sys.exit(1)
+import test_oracle_pins, test_oracle_next
+for pins in (test_oracle_pins, test_oracle_next):
+    for name, fn in inspect.getmembers(pins, inspect.isfunction):
+        if name.startswith("test_") and not inspect.signature(fn).parameters:
+            try:
+                fn()
+            except Exception:
+                sys.exit(1)
 sys.exit(0)
 """
 
