@@ -6,7 +6,12 @@
  * ShiftGELU and I-LayerNorm.  Sources, cited per entry point below:
  *   [IVIT] "I-ViT: Integer-only Quantization for Efficient Vision Transformer
  *          Inference" (mer.run notes), sections 3.1-3.5.
- *   [TRIO] "Trio-ViT" article (cloud.tencent.com), eqs. (1)-(3) and (12).
+ *   [TRIO] "Trio-ViT" article (cloud.tencent.com), eqs. (1)-(3) and (12);
+ *          section IV-D (log2 quantisation).
+ *   [FQ]   "FQ-ViT: Post-Training Quantization for Fully Quantized Vision
+ *          Transformer" (ijcai.org record), abstract: Power-of-Two Factor
+ *          (PTF) for LayerNorm inputs, Log-Int-Softmax (LIS) with 4-bit
+ *          attention maps and the BitShift operator.
  *
  * Conventions for every entry point:
  *   - Tensors are device pointers, row-major and contiguous, each 16-byte
@@ -164,6 +169,55 @@ ivit_status ivit_shiftgelu(const int8_t *x, int64_t n, int32_t I0, int32_t M, in
 ivit_status ivit_layernorm(const int8_t *x, int64_t rows, int32_t cols, const int8_t *gamma,
                            const int32_t *beta, int32_t F, int32_t M_ln, ivit_dyadic out, int8_t *y,
                            ivit_stream_t stream);
+
+/* ---------------------------------------------------------------------------
+ * Variants where the pages leave a step open or name an alternative
+ * ------------------------------------------------------------------------- */
+
+/* ShiftGELU with a row maximum ([IVIT] 3.4, which multiplies the sigmoid's
+ * numerator and denominator by e^(-S I_max) and stops before defining I_max).
+ * READING: I_max is the largest exponent of the row, max(0, max_i I_p,i), as
+ * Shiftmax subtracts its row maximum (ivit_shiftgelu takes max(I_p, 0) per
+ * element instead):
+ *   e1 = ShiftExp(I_p - I_max); e2 = ShiftExp(-I_max)
+ *   sigma = IntDiv(e1, e1 + e2), and sigma = 0 when e1 + e2 = 0 (both
+ *           exponentials underflow: the divisor is taken as 1)
+ *   y = sat_8((out.b * x * sigma) >> out.c)
+ * x, y [rows x cols] int8, one row per token (e.g. cols = Dm channels of fc1's
+ * output).  Constraints: rows >= 0; 16 <= cols <= 16384, multiple of 16;
+ * I0 >= 1; k_out - 1 <= M <= 30; 1 <= k_out <= 8.                          */
+ivit_status ivit_shiftgelu_rowmax(const int8_t *x, int64_t rows, int32_t cols, int32_t I0, int32_t M,
+                                  int32_t k_out, ivit_dyadic out, int8_t *y, ivit_stream_t stream);
+
+/* Attention with Log-Int-Softmax ([FQ] abstract: the attention map quantised
+ * to 4 bits on a log2 grid and multiplied with V by BitShift; the log2
+ * quantiser clip(round(log2(.)), -a, b) of [TRIO] IV-D).  S and the logits
+ * as in ivit_attention; then, READING, per query row:
+ *   e = ShiftExp(L - max L), Dv = floor(2^M / sum e)          ([IVIT] 3.3)
+ *   P16 = (Dv * e) >> (M - 15)             (16-bit probability, scale 2^-15)
+ *   k = clip(15 - round(log2 P16), 0, 15), k = 15 when P16 = 0 (4-bit code;
+ *       round(log2 P) rounds up exactly when P^2 >= 2^(2 floor(log2 P) + 1))
+ *   ctx_id = sat_8((out.b * sum_j (V_jd << (15 - k_j))) >> out.c)
+ *            out ~ S_v 2^-15 / S_ctx
+ * (the bit shift at scale 2^-15 is exact; it runs on the tensor cores as two
+ * u8 x s8 products over the power-of-two planes 2^(7-k), k <= 7, and
+ * 2^(15-k), k >= 8).  Layouts as ivit_attention.  Constraints: B, H >= 1;
+ * 1 <= N <= 640; 2 <= k_s <= 8; I0 >= 1; 15 <= M <= 30.                    */
+ivit_status ivit_attention_lis(const int8_t *qkv, int32_t B, int32_t N, int32_t H, ivit_dyadic logit,
+                               int32_t k_s, int32_t I0, int32_t M, ivit_dyadic out, int8_t *ctx,
+                               ivit_stream_t stream);
+
+/* I-LayerNorm of an input quantised with power-of-two factors ([FQ] abstract:
+ * PTF against the inter-channel variation of LayerNorm inputs).  READING:
+ * channel i of x carries the scale S 2^alpha_i (one layer-wise S, alpha_i in
+ * {0, 1, 2, 3}, chosen off-line per channel); the LayerNorm input at the
+ * common scale S is x_i << alpha_i, and ivit_layernorm's steps ([IVIT] 3.5)
+ * run on it unchanged.  alpha [cols] uint8 (device; only its two low bits are
+ * read).  Constraints as ivit_layernorm, with M_ln <= 20 (|x << alpha - mu|
+ * < 2^11 keeps (x - mu) * floor(2^M_ln / sigma) below 2^31).               */
+ivit_status ivit_layernorm_ptf(const int8_t *x, int64_t rows, int32_t cols, const uint8_t *alpha,
+                               const int8_t *gamma, const int32_t *beta, int32_t F, int32_t M_ln,
+                               ivit_dyadic out, int8_t *y, ivit_stream_t stream);
 
 /* ---------------------------------------------------------------------------
  * The encoder block ([IVIT] 3.1): X^ = MSA(LN1(X)) + X; Y = MLP(LN2(X^)) + X^

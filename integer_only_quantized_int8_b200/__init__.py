@@ -24,6 +24,7 @@ __all__ = [
     "ivit_block_forward_static", "STATIC_SCRATCH_BYTES", "EXPORTED_SYMBOLS",
     "ModelParams", "ivit_patch_embed_workspace_bytes", "ivit_patch_embed", "ivit_head_workspace_bytes", "ivit_head",
     "ivit_model_workspace_bytes", "ivit_model_forward", "ivit_selftest_wait_timeout", "ivit_selftest_int_rate",
+    "ivit_shiftgelu_rowmax", "ivit_attention_lis", "ivit_layernorm_ptf",
 ]
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
@@ -40,6 +41,7 @@ EXPORTED_SYMBOLS = (
     "ivit_patch_embed_workspace_bytes", "ivit_patch_embed", "ivit_head_workspace_bytes", "ivit_head",
     "ivit_model_workspace_bytes", "ivit_model_forward",
     "ivit_selftest_wait_timeout", "ivit_selftest_int_rate",
+    "ivit_shiftgelu_rowmax", "ivit_attention_lis", "ivit_layernorm_ptf",
 )
 
 _STATUS = {0: "IVIT_OK", 1: "IVIT_ERR_INVALID_ARG", 2: "IVIT_ERR_UNSUPPORTED", 3: "IVIT_ERR_CUDA",
@@ -149,6 +151,12 @@ def lib() -> C.CDLL:
             L.ivit_launch_count.argtypes = []
             L.ivit_selftest_wait_timeout.restype = C.c_int
             L.ivit_selftest_wait_timeout.argtypes = [vp]
+            L.ivit_shiftgelu_rowmax.restype = C.c_int
+            L.ivit_shiftgelu_rowmax.argtypes = [vp, i64, i32, i32, i32, i32, Dyadic, vp, vp]
+            L.ivit_attention_lis.restype = C.c_int
+            L.ivit_attention_lis.argtypes = [vp, i32, i32, i32, Dyadic, i32, i32, i32, Dyadic, vp, vp]
+            L.ivit_layernorm_ptf.restype = C.c_int
+            L.ivit_layernorm_ptf.argtypes = [vp, i64, i32, vp, vp, vp, i32, i32, Dyadic, vp, vp]
             L.ivit_selftest_int_rate.restype = C.c_int
             L.ivit_selftest_int_rate.argtypes = [i32, vp, i32, C.POINTER(C.c_int64), vp]
             _lib = L
@@ -292,6 +300,39 @@ def ivit_layernorm(x, gamma, beta, F: int, M_ln: int, out, y, stream=None):
                               _ptr(beta, torch.int32, "beta"), int(F), int(M_ln), _dy(out),
                               _ptr(y, torch.int8, "y"), _stream(stream))
     _check("ivit_layernorm", st)
+    return y
+
+
+def ivit_shiftgelu_rowmax(x, I0: int, M: int, k_out: int, out, y, stream=None):
+    """ShiftGELU of x [rows, cols] with I_max the row's largest exponent."""
+    rows, cols = x.shape
+    if tuple(y.shape) != (rows, cols):
+        raise ValueError("shape mismatch")
+    st = lib().ivit_shiftgelu_rowmax(_ptr(x, torch.int8, "x"), rows, cols, int(I0), int(M), int(k_out), _dy(out),
+                                     _ptr(y, torch.int8, "y"), _stream(stream))
+    _check("ivit_shiftgelu_rowmax", st)
+    return y
+
+
+def ivit_attention_lis(qkv, B: int, N: int, H: int, logit, k_s: int, I0: int, M: int, out, ctx, stream=None):
+    """Attention with Log-Int-Softmax (4-bit log2 attention map, A V by bit shifts)."""
+    _holds(int(B) * int(N) * 3 * int(H) * 64, qkv=qkv)
+    _holds(int(B) * int(N) * int(H) * 64, ctx=ctx)
+    st = lib().ivit_attention_lis(_ptr(qkv, torch.int8, "qkv"), int(B), int(N), int(H), _dy(logit), int(k_s),
+                                  int(I0), int(M), _dy(out), _ptr(ctx, torch.int8, "ctx"), _stream(stream))
+    _check("ivit_attention_lis", st)
+    return ctx
+
+
+def ivit_layernorm_ptf(x, alpha, gamma, beta, F: int, M_ln: int, out, y, stream=None):
+    """I-LayerNorm of x [rows, cols] whose channel i carries the factor 2^alpha[i]."""
+    rows, cols = x.shape
+    if tuple(y.shape) != (rows, cols) or gamma.numel() != cols or beta.numel() != cols or alpha.numel() != cols:
+        raise ValueError("shape mismatch")
+    st = lib().ivit_layernorm_ptf(_ptr(x, torch.int8, "x"), rows, cols, _ptr(alpha, torch.uint8, "alpha"),
+                                  _ptr(gamma, torch.int8, "gamma"), _ptr(beta, torch.int32, "beta"), int(F),
+                                  int(M_ln), _dy(out), _ptr(y, torch.int8, "y"), _stream(stream))
+    _check("ivit_layernorm_ptf", st)
     return y
 
 

@@ -247,6 +247,50 @@ ivit_status ivit_layernorm(const int8_t* x, int64_t rows, int32_t cols, const in
   return launch_layernorm(dc, x, rows, cols, gamma, beta, F, M_ln, out, y, (cudaStream_t)stream);
 }
 
+ivit_status ivit_shiftgelu_rowmax(const int8_t* x, int64_t rows, int32_t cols, int32_t I0, int32_t M,
+                                  int32_t k_out, ivit_dyadic out, int8_t* y, ivit_stream_t stream) {
+  if (rows < 0 || cols < 16 || cols > 16384 || cols % 16 != 0 || !valid_shiftmax(I0, M, k_out) ||
+      !valid_dyadic(out))
+    return IVIT_ERR_INVALID_ARG;
+  if (rows == 0) return IVIT_OK;
+  if (!x || !y || !aligned16(x) || !aligned16(y)) return IVIT_ERR_INVALID_ARG;
+  DeviceCtx dc;
+  ivit_status st = device_ctx(&dc);
+  if (st != IVIT_OK) return st;
+  const GeluParams g{I0, M, k_out, out};
+  return launch_shiftgelu_rowmax(dc, x, rows, cols, g, y, (cudaStream_t)stream);
+}
+
+ivit_status ivit_attention_lis(const int8_t* qkv, int32_t B, int32_t N, int32_t H, ivit_dyadic logit, int32_t k_s,
+                               int32_t I0, int32_t M, ivit_dyadic out, int8_t* ctx, ivit_stream_t stream) {
+  if (!qkv || !ctx || !aligned16(qkv) || !aligned16(ctx)) return IVIT_ERR_INVALID_ARG;
+  if (B < 0 || N < 0 || H < 1 || k_s < 2 || k_s > 8 || I0 < 1 || I0 > (1 << 22) || M < 15 || M > 30 ||
+      !valid_dyadic(logit) || !valid_dyadic(out))
+    return IVIT_ERR_INVALID_ARG;
+  if (N > 640 || (int64_t)B * N > 0x7fffff00LL || H > 4096) return IVIT_ERR_UNSUPPORTED;
+  if (B == 0 || N == 0) return IVIT_OK;
+  DeviceCtx dc;
+  ivit_status st = device_ctx(&dc);
+  if (st != IVIT_OK) return st;
+  return launch_attention(dc, qkv, B, N, H, logit, k_s, I0, M, 8, out, ctx, (cudaStream_t)stream, true);
+}
+
+ivit_status ivit_layernorm_ptf(const int8_t* x, int64_t rows, int32_t cols, const uint8_t* alpha,
+                               const int8_t* gamma, const int32_t* beta, int32_t F, int32_t M_ln, ivit_dyadic out,
+                               int8_t* y, ivit_stream_t stream) {
+  if (rows < 0 || cols < 16 || cols > 2048 || cols % 16 != 0 || F < 0 || F > 14 || M_ln < F || M_ln > 20 ||
+      !valid_dyadic(out))
+    return IVIT_ERR_INVALID_ARG;
+  if (rows == 0) return IVIT_OK;
+  if (!x || !y || !alpha || !gamma || !beta || !aligned16(x) || !aligned16(y) || !aligned16(alpha) ||
+      !aligned16(gamma) || !aligned16(beta))
+    return IVIT_ERR_INVALID_ARG;
+  DeviceCtx dc;
+  ivit_status st = device_ctx(&dc);
+  if (st != IVIT_OK) return st;
+  return launch_layernorm_ptf(dc, x, rows, cols, alpha, gamma, beta, F, M_ln, out, y, (cudaStream_t)stream);
+}
+
 size_t ivit_block_workspace_bytes(int32_t B, int32_t N, int32_t D, int32_t Dm) {
   if (B < 0 || N < 0 || D < 0 || Dm < 0) return 0;
   const size_t T = (size_t)B * (size_t)N;

@@ -74,9 +74,23 @@ __host__ __device__ inline AttnLayout attn_layout(int N) {
   return L;
 }
 
+// 4-bit log2 code of a 16-bit probability P16 (scale 2^-15): 15 -
+// round(log2 P16), clipped to [0, 15]; P16 = 0 gives 15.  round(log2 P) of an
+// integer P >= 1 is floor(log2 P) + 1 exactly when P^2 >= 2^(2 floor(log2 P) + 1).
+IVIT_DEV uint32_t lis_code(uint32_t p16) {
+  if (p16 == 0u) return 15u;
+  const uint32_t fl = 31u - (uint32_t)__clz((int)p16);
+  const uint32_t r = fl + ((p16 * p16 >= (1u << (2 * fl + 1))) ? 1u : 0u);  // p16 <= 2^15: no overflow
+  return r >= 15u ? 0u : 15u - r;
+}
+
 // FASTQ: the logit requant is one mul.hi by bq = b_s 2^(32 - c_s), exact
 // when b_s < 2^(c_s - 1), then the k_s-bit saturation.
-template <bool FASTQ>
+// LIS: Log-Int-Softmax instead of Shiftmax (see ivit_attention_lis): the row's
+// 16-bit probabilities become 4-bit log2 codes k, and P V is the bit shift
+// sum_j V_j 2^(15 - k_j), computed as two u8 x s8 MMAs over the planes
+// 2^(7 - k) (k <= 7) and 2^(15 - k) (k >= 8), combined as 256 hi + lo.
+template <bool FASTQ, bool LIS>
 __global__ void __launch_bounds__(kAttnThreads)
     attention_shiftmax_kernel(const __grid_constant__ CUtensorMap tm, const AttnArgs a, const int32_t bq) {
   extern __shared__ uint8_t smem_raw[];
@@ -225,57 +239,84 @@ __global__ void __launch_bounds__(kAttnThreads)
   const uint32_t dv = (1u << a.M) / sum;
   const int pshift = a.M - (a.k_out - 1);
 
-  // ---- P = (Dv e_j) >> (M - k_out + 1) as u8, into the K-major 128B-swizzled
-  // operand; this slice's 16-key units (zero past the last key)
-  fence_proxy_async_smem();
+  // ---- P as u8 into the K-major 128B-swizzled operand; this slice's 16-key
+  // units (zero past the last key).  Shiftmax: P = (Dv e_j) >> (M - k_out + 1).
+  // LIS: plane `plane` of the code k_j of P16 = (Dv e_j) >> (M - 15).
   const int rlo = row & 7;
   uint8_t* prow = sP + (row >> 3) * 1024 + rlo * 128;
-  for (int u = slice; u < L.n32 / 16; u += kAttnSplit) {
-    const int j0 = u * 16;
-    uint32_t packed[4] = {0, 0, 0, 0};
-    if (ok && j0 < N) {
-      const int4 v = *reinterpret_cast<const int4*>(my_log + j0);
-      const int8_t* lb = reinterpret_cast<const int8_t*>(&v);
+  auto write_p = [&](int plane) {
+    fence_proxy_async_smem();
+    for (int u = slice; u < L.n32 / 16; u += kAttnSplit) {
+      const int j0 = u * 16;
+      uint32_t packed[4] = {0, 0, 0, 0};
+      if (ok && j0 < N) {
+        const int4 v = *reinterpret_cast<const int4*>(my_log + j0);
+        const int8_t* lb = reinterpret_cast<const int8_t*>(&v);
 #pragma unroll
-      for (int e = 0; e < 16; ++e) {
-        const uint32_t p = (j0 + e < N) ? (dv * (uint32_t)tab[mx - (int32_t)lb[e]]) >> pshift : 0u;
-        packed[e >> 2] |= p << (8 * (e & 3));
+        for (int e = 0; e < 16; ++e) {
+          uint32_t p = 0u;
+          if (j0 + e < N) {
+            const uint32_t ev = (uint32_t)tab[mx - (int32_t)lb[e]];
+            if (!LIS) {
+              p = (dv * ev) >> pshift;
+            } else {
+              const uint32_t k = lis_code((dv * ev) >> (a.M - 15));
+              p = plane == 0 ? (k <= 7u ? 1u << (7u - k) : 0u) : (k >= 8u ? 1u << (15u - k) : 0u);
+            }
+          }
+          packed[e >> 2] |= p << (8 * (e & 3));
+        }
       }
+      const int kb = j0 >> 7;
+      const int ch = (j0 & 127) >> 4;
+      *reinterpret_cast<int4*>(prow + kb * 16384 + ((ch ^ rlo) << 4)) =
+          make_int4(packed[0], packed[1], packed[2], packed[3]);
     }
-    const int kb = j0 >> 7;
-    const int ch = (j0 & 127) >> 4;
-    *reinterpret_cast<int4*>(prow + kb * 16384 + ((ch ^ rlo) << 4)) =
-        make_int4(packed[0], packed[1], packed[2], packed[3]);
-  }
-  fence_proxy_async_smem();
-  tc_fence_before();
-  __syncthreads();
-
-  // ---- O = P V
-  if (tid == 0 && ok) {
-    if (!mbar_wait(bar_v, 0, a.status)) ok = false;
-    if (ok) {
-      tc_fence_after();
-      const uint32_t idesc = idesc_i8(kQTile, kHeadDim, false, true, true);
-      const uint32_t pa = smem_u32(sP);
-      const uint32_t va = smem_u32(sV);
-      for (int k = 0; k < L.n32 / 32; ++k) {
-        const uint64_t da = smem_desc(pa + (k >> 2) * 16384 + (k & 3) * 32, 16, 1024, kSwizzle128B);
-        const uint64_t db = smem_desc(va + k * 32 * kHeadDim, 512, 512, kSwizzle64B);
-        umma_i8(tmem, da, db, idesc, k != 0);
+    fence_proxy_async_smem();
+    tc_fence_before();
+    __syncthreads();
+  };
+  // ---- O = P V (one commit phase of bar_o per product)
+  auto pv = [&](int phase) {
+    if (tid == 0 && ok) {
+      if (phase == 0 && !mbar_wait(bar_v, 0, a.status)) ok = false;
+      if (ok) {
+        tc_fence_after();
+        const uint32_t idesc = idesc_i8(kQTile, kHeadDim, false, true, true);
+        const uint32_t pa = smem_u32(sP);
+        const uint32_t va = smem_u32(sV);
+        for (int k = 0; k < L.n32 / 32; ++k) {
+          const uint64_t da = smem_desc(pa + (k >> 2) * 16384 + (k & 3) * 32, 16, 1024, kSwizzle128B);
+          const uint64_t db = smem_desc(va + k * 32 * kHeadDim, 512, 512, kSwizzle64B);
+          umma_i8(tmem, da, db, idesc, k != 0);
+        }
       }
+      umma_commit(bar_o);
     }
-    umma_commit(bar_o);
+    if (!mbar_wait(bar_o, (uint32_t)phase, a.status)) ok = false;
+    ok = __all_sync(0xffffffffu, ok);
+    tc_fence_after();
+  };
+  write_p(0);
+  pv(0);
+  // slice s reads columns [16 s, 16 s + 16) of O
+  uint32_t r[16];
+  tmem_ld16(t_lane + (uint32_t)(slice * 16), r);
+  tmem_ld_wait_regs(r);
+  uint32_t rlo16[16];
+  if (LIS) {
+    // the low plane's product replaces the high one's in the same columns,
+    // once every thread has read the high one
+    tc_fence_before();
+    __syncthreads();
+    write_p(1);
+    pv(1);
+    tmem_ld16(t_lane + (uint32_t)(slice * 16), rlo16);
+    tmem_ld_wait_regs(rlo16);
   }
-  if (!mbar_wait(bar_o, 0, a.status)) ok = false;
-  ok = __all_sync(0xffffffffu, ok);
-  tc_fence_after();
 
   // ---- ctx = sat_8((b_o O) >> c_o); slice s writes columns [16 s, 16 s + 16)
   {
-    uint32_t r[16];
-    tmem_ld16(t_lane + (uint32_t)(slice * 16), r);
-    tmem_ld_wait();
     const int q = q0 + row;
     if (ok && q < N) {
       int8_t* dst = a.ctx + (int64_t)(row0 + q) * D + h * kHeadDim + slice * 16;
@@ -284,8 +325,18 @@ __global__ void __launch_bounds__(kAttnThreads)
       for (int wd = 0; wd < 4; ++wd) {
         uint32_t word = 0;
 #pragma unroll
-        for (int e = 0; e < 4; ++e)
-          word |= ((uint32_t)requant8((int32_t)r[wd * 4 + e], a.out_b, a.out_c) & 0xFFu) << (8 * e);
+        for (int e = 0; e < 4; ++e) {
+          int32_t y;
+          if (!LIS) {
+            y = requant8((int32_t)r[wd * 4 + e], a.out_b, a.out_c);
+          } else {
+            // acc = sum_j V_j 2^(15 - k_j) = 256 hi + lo, |acc| < 2^32; (b_o acc) >> c_o in 64 bits
+            const int64_t acc = 256 * (int64_t)(int32_t)r[wd * 4 + e] + (int64_t)(int32_t)rlo16[wd * 4 + e];
+            const int64_t v = ((int64_t)a.out_b * acc) >> a.out_c;
+            y = (int32_t)(v < -128 ? -128 : (v > 127 ? 127 : v));
+          }
+          word |= ((uint32_t)y & 0xFFu) << (8 * e);
+        }
         packed[wd] = word;
       }
       *reinterpret_cast<int4*>(dst) = make_int4(packed[0], packed[1], packed[2], packed[3]);
@@ -809,7 +860,7 @@ bool attention_config_supported(int32_t N, int32_t k_s, int32_t I0) {
 
 ivit_status launch_attention(const DeviceCtx& dc, const int8_t* qkv, int32_t B, int32_t N, int32_t H,
                              ivit_dyadic logit, int32_t k_s, int32_t I0, int32_t M, int32_t k_out,
-                             ivit_dyadic out, int8_t* ctx, cudaStream_t stream) {
+                             ivit_dyadic out, int8_t* ctx, cudaStream_t stream, bool lis) {
   if (B == 0 || N == 0) return IVIT_OK;
   if (N > kMaxKeys) return IVIT_ERR_UNSUPPORTED;
   const int64_t T = (int64_t)B * N;
@@ -857,7 +908,7 @@ ivit_status launch_attention(const DeviceCtx& dc, const int8_t* qkv, int32_t B, 
   a.ctx = ctx;
   a.status = dc.status;
   dim3 grid((unsigned)((N + kQTile - 1) / kQTile), (unsigned)H, (unsigned)B);
-  if (N <= kShortMaxKeys) {
+  if (N <= kShortMaxKeys && !lis) {
     const PersistLayout P = persist_layout(N);
     const int smem = P.total + 1024;
     // bq = b 2^(32 - c) when it fits a positive int32: the logit requant is then one mul.hi
@@ -891,9 +942,13 @@ ivit_status launch_attention(const DeviceCtx& dc, const int8_t* qkv, int32_t B, 
   if (smem < 80 * 1024) smem = 80 * 1024;
   static int attr_bytes = 0;
   if (smem > attr_bytes) {
-    if (cudaFuncSetAttribute(attention_shiftmax_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    if (cudaFuncSetAttribute(attention_shiftmax_kernel<true, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              227 * 1024) != cudaSuccess ||
-        cudaFuncSetAttribute(attention_shiftmax_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        cudaFuncSetAttribute(attention_shiftmax_kernel<false, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             227 * 1024) != cudaSuccess ||
+        cudaFuncSetAttribute(attention_shiftmax_kernel<true, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             227 * 1024) != cudaSuccess ||
+        cudaFuncSetAttribute(attention_shiftmax_kernel<false, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              227 * 1024) != cudaSuccess)
       return IVIT_ERR_CUDA;
     attr_bytes = 227 * 1024;
@@ -901,10 +956,9 @@ ivit_status launch_attention(const DeviceCtx& dc, const int8_t* qkv, int32_t B, 
   // bq = b 2^(32 - c) when it fits a positive int32: the logit requant is then one mul.hi
   const bool fastq_long = logit.c >= 1 && (int64_t)logit.b < ((int64_t)1 << (logit.c - 1));
   const int32_t bq_long = fastq_long ? (int32_t)((int64_t)logit.b << (32 - logit.c)) : 0;
-  const cudaError_t e =
-      fastq_long
-          ? launch_pdl(attention_shiftmax_kernel<true>, grid, dim3(kAttnThreads), smem, stream, tm, a, bq_long)
-          : launch_pdl(attention_shiftmax_kernel<false>, grid, dim3(kAttnThreads), smem, stream, tm, a, bq_long);
+  auto kern = fastq_long ? (lis ? attention_shiftmax_kernel<true, true> : attention_shiftmax_kernel<true, false>)
+                         : (lis ? attention_shiftmax_kernel<false, true> : attention_shiftmax_kernel<false, false>);
+  const cudaError_t e = launch_pdl(kern, grid, dim3(kAttnThreads), smem, stream, tm, a, bq_long);
   note_launch();
   return e == cudaSuccess ? IVIT_OK : IVIT_ERR_CUDA;
 }

@@ -244,7 +244,188 @@ __global__ void __launch_bounds__(kLnThreads)
   }
 }
 
+// ---------------------------------------------------------------------------
+// ShiftGELU with a row maximum (I-ViT section 3.4, I_max read as the row's
+// largest exponent; see include/ivit.h): one CTA per row.  I_p is
+// non-decreasing in x, so the row's largest exponent is I_p of the row's
+// largest byte; given it, the output is a function of the int8 input alone,
+// which the CTA tabulates (256 entries) and streams the row through.
+// ---------------------------------------------------------------------------
+constexpr int kRowGeluThreads = 256;
+
+__global__ void __launch_bounds__(kRowGeluThreads)
+    shiftgelu_rowmax_kernel(const int8_t* __restrict__ x, int64_t rows, int32_t cols, GeluParams g,
+                            int8_t* __restrict__ y) {
+  __shared__ int8_t tab[256];
+  __shared__ int32_t wmax[kRowGeluThreads / 32];
+  pdl_wait();  // x comes from an earlier kernel
+  pdl_launch_dependents();
+  const int nvec = cols >> 4;
+  for (int64_t row = blockIdx.x; row < rows; row += gridDim.x) {
+    const int4* xv = reinterpret_cast<const int4*>(x + row * cols);
+    int32_t m = -128;
+    for (int v = threadIdx.x; v < nvec; v += blockDim.x) {
+      const int4 in = __ldg(xv + v);
+      const uint32_t w[4] = {(uint32_t)in.x, (uint32_t)in.y, (uint32_t)in.z, (uint32_t)in.w};
+#pragma unroll
+      for (int k = 0; k < 4; ++k)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) m = max(m, (int32_t)(int8_t)(w[k] >> (8 * e)));
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(0xffffffffu, m, o));
+    if ((threadIdx.x & 31) == 0) wmax[threadIdx.x >> 5] = m;
+    __syncthreads();
+    int32_t xm = wmax[0];
+#pragma unroll
+    for (int i = 1; i < kRowGeluThreads / 32; ++i) xm = max(xm, wmax[i]);
+    // I_max = max(0, I_p(largest x)); e2 = ShiftExp(-I_max)
+    const int32_t ipm = xm + (xm >> 1) + (xm >> 3) + (xm >> 4);
+    const int32_t I_max = ipm > 0 ? ipm : 0;
+    {
+      const int32_t xi = (int32_t)threadIdx.x - 128;  // one table entry per thread
+      const int32_t ip = xi + (xi >> 1) + (xi >> 3) + (xi >> 4);
+      const int32_t e1 = shift_exp(ip - I_max, g.I0);
+      const int32_t e2 = shift_exp(-I_max, g.I0);
+      const uint32_t sum = (uint32_t)(e1 + e2);
+      const uint32_t dv = (1u << g.M) / (sum > 0u ? sum : 1u);  // both exponentials 0: sigma = 0
+      const int32_t sig = (int32_t)((dv * (uint32_t)e1) >> (g.M - (g.k_out - 1)));
+      tab[threadIdx.x] = (int8_t)requant8(xi * sig, g.out.b, g.out.c);
+    }
+    __syncthreads();
+    int4* yv = reinterpret_cast<int4*>(y + row * cols);
+    for (int v = threadIdx.x; v < nvec; v += blockDim.x) {
+      const int4 in = __ldg(xv + v);
+      const uint32_t w[4] = {(uint32_t)in.x, (uint32_t)in.y, (uint32_t)in.z, (uint32_t)in.w};
+      uint32_t o[4];
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        uint32_t r = 0;
+#pragma unroll
+        for (int e = 0; e < 4; ++e) r |= ((uint32_t)(uint8_t)tab[((w[k] >> (8 * e)) & 0xFFu) ^ 0x80u]) << (8 * e);
+        o[k] = r;
+      }
+      __stcs(yv + v, make_int4((int)o[0], (int)o[1], (int)o[2], (int)o[3]));
+    }
+    __syncthreads();  // the table and the maxima are rewritten for the next row
+  }
+}
+
+// ---------------------------------------------------------------------------
+// I-LayerNorm of an input with power-of-two channel factors (the FQ-ViT
+// record's Power-of-Two Factor; see include/ivit.h): one warp per row; the
+// LayerNorm input is x_i << alpha_i (|x << alpha| <= 1024).  Sums are exact
+// in 32 bits for cols <= 2048 (2048 * 1024^2 < 2^31); (x - mu) f stays below
+// 2^31 because the host requires M_ln <= 23 - max alpha.
+// ---------------------------------------------------------------------------
+constexpr int kPtfThreads = 256;
+
+template <bool FASTQ>
+__global__ void __launch_bounds__(kPtfThreads)
+    layernorm_ptf_kernel(const int8_t* __restrict__ x, int64_t rows, int32_t cols, const uint8_t* __restrict__ alpha,
+                         const int8_t* __restrict__ gamma, const int32_t* __restrict__ beta, int32_t F, int32_t M_ln,
+                         ivit_dyadic out, int32_t out_bq, int8_t* __restrict__ y) {
+  pdl_wait();  // x comes from an earlier kernel
+  pdl_launch_dependents();
+  const int lane = threadIdx.x & 31;
+  const int nchunk = cols >> 4;
+  for (int64_t row = (int64_t)blockIdx.x * (kPtfThreads / 32) + (threadIdx.x >> 5); row < rows;
+       row += (int64_t)gridDim.x * (kPtfThreads / 32)) {
+    const int4* xr = reinterpret_cast<const int4*>(x + row * cols);
+    int32_t s1 = 0, s2 = 0;
+    for (int ci = lane; ci < nchunk; ci += 32) {
+      const int4 xv = __ldg(xr + ci);
+      const int4 av = __ldg(reinterpret_cast<const int4*>(alpha) + ci);
+      const uint32_t xw[4] = {(uint32_t)xv.x, (uint32_t)xv.y, (uint32_t)xv.z, (uint32_t)xv.w};
+      const uint32_t aw[4] = {(uint32_t)av.x, (uint32_t)av.y, (uint32_t)av.z, (uint32_t)av.w};
+#pragma unroll
+      for (int q = 0; q < 4; ++q)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int32_t v = sext_byte(xw[q], e) << ((aw[q] >> (8 * e)) & 3u);
+          s1 += v;
+          s2 += v * v;
+        }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      s1 += __shfl_xor_sync(0xffffffffu, s1, o);
+      s2 += __shfl_xor_sync(0xffffffffu, s2, o);
+    }
+    // mu = floor(sum / n); V = floor(sum (v - mu)^2 / n) = floor((s2 - 2 mu s1 + n mu^2) / n), in 64 bits
+    const int64_t mu = s1 >= 0 ? (int64_t)s1 / cols : -((-(int64_t)s1 + cols - 1) / cols);
+    const int64_t sd2 = (int64_t)s2 - 2 * mu * s1 + (int64_t)cols * mu * mu;
+    const int32_t V = (int32_t)(sd2 / cols);  // sd2 >= 0
+    int32_t sigma = isqrt_newton10(V);
+    if (sigma < 1) sigma = 1;
+    const int32_t f = (int32_t)((1u << M_ln) / (uint32_t)sigma);
+    const int sh = M_ln - F;
+    int8_t* yr = y + row * cols;
+    for (int ci = lane; ci < nchunk; ci += 32) {
+      const int c0 = ci * 16;
+      const int4 xv = __ldg(xr + ci);
+      const int4 av = __ldg(reinterpret_cast<const int4*>(alpha) + ci);
+      const int4 gv = __ldg(reinterpret_cast<const int4*>(gamma + c0));
+      const uint32_t xw[4] = {(uint32_t)xv.x, (uint32_t)xv.y, (uint32_t)xv.z, (uint32_t)xv.w};
+      const uint32_t aw[4] = {(uint32_t)av.x, (uint32_t)av.y, (uint32_t)av.z, (uint32_t)av.w};
+      const uint32_t gw[4] = {(uint32_t)gv.x, (uint32_t)gv.y, (uint32_t)gv.z, (uint32_t)gv.w};
+      uint32_t o[4];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const int4 bt = __ldg(reinterpret_cast<const int4*>(beta + c0) + q);
+        const int32_t bb[4] = {bt.x, bt.y, bt.z, bt.w};
+        int32_t r[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int32_t v = sext_byte(xw[q], e) << ((aw[q] >> (8 * e)) & 3u);
+          const int32_t nv = ((v - (int32_t)mu) * f) >> sh;
+          const int32_t acc = nv * sext_byte(gw[q], e) + bb[e];
+          if (FASTQ) {
+            r[e] = __mulhi(out_bq, acc);
+          } else {
+            const int64_t q64 = ((int64_t)out.b * acc) >> out.c;
+            r[e] = (int32_t)(q64 < -128 ? -128 : (q64 > 127 ? 127 : q64));
+          }
+        }
+        o[q] = pack_sat4_ln(r[0], r[1], r[2], r[3]);
+      }
+      __stcs(reinterpret_cast<int4*>(yr) + ci, make_int4((int)o[0], (int)o[1], (int)o[2], (int)o[3]));
+    }
+  }
+}
+
 }  // namespace
+
+ivit_status launch_shiftgelu_rowmax(const DeviceCtx& dc, const int8_t* x, int64_t rows, int32_t cols,
+                                    const GeluParams& g, int8_t* y, cudaStream_t stream) {
+  if (rows == 0) return IVIT_OK;
+  const int64_t cap = (int64_t)dc.num_sms * 8;
+  const unsigned grid = (unsigned)(rows < cap ? rows : cap);
+  const cudaError_t e =
+      launch_pdl(shiftgelu_rowmax_kernel, dim3(grid), dim3(kRowGeluThreads), 0, stream, x, rows, cols, g, y);
+  note_launch();
+  return e == cudaSuccess ? IVIT_OK : IVIT_ERR_CUDA;
+}
+
+ivit_status launch_layernorm_ptf(const DeviceCtx& dc, const int8_t* x, int64_t rows, int32_t cols,
+                                 const uint8_t* alpha, const int8_t* gamma, const int32_t* beta, int32_t F,
+                                 int32_t M_ln, ivit_dyadic out, int8_t* y, cudaStream_t stream) {
+  if (rows == 0) return IVIT_OK;
+  const int64_t rows_per_cta = kPtfThreads / 32;
+  int64_t blocks = (rows + rows_per_cta - 1) / rows_per_cta;
+  const int64_t cap = (int64_t)dc.num_sms * 16;
+  if (blocks > cap) blocks = cap;
+  // the output requant is one mul.hi by b 2^(32 - c) when that fits a positive int32
+  const bool fastq = out.c >= 1 && (int64_t)out.b < ((int64_t)1 << (out.c - 1));
+  const int32_t bq = fastq ? (int32_t)((int64_t)out.b << (32 - out.c)) : 0;
+  const cudaError_t e =
+      fastq ? launch_pdl(layernorm_ptf_kernel<true>, dim3((unsigned)blocks), dim3(kPtfThreads), 0, stream, x, rows,
+                         cols, alpha, gamma, beta, F, M_ln, out, bq, y)
+            : launch_pdl(layernorm_ptf_kernel<false>, dim3((unsigned)blocks), dim3(kPtfThreads), 0, stream, x, rows,
+                         cols, alpha, gamma, beta, F, M_ln, out, bq, y);
+  note_launch();
+  return e == cudaSuccess ? IVIT_OK : IVIT_ERR_CUDA;
+}
 
 ivit_status launch_shiftgelu(const DeviceCtx& dc, const int8_t* x, int64_t n, const GeluParams& g, int8_t* y,
                              cudaStream_t stream) {

@@ -64,12 +64,25 @@ ivit_status launch_gemm(const DeviceCtx& dc, const int8_t* X, int64_t M, int32_t
 // with (largest -I_p) * I0 < 2^32.
 bool attention_config_supported(int32_t N, int32_t k_s, int32_t I0);
 
+// lis: Log-Int-Softmax instead of Shiftmax (logits of at most 8 bits, M >= 15;
+// k_out is then unused)
 ivit_status launch_attention(const DeviceCtx& dc, const int8_t* qkv, int32_t B, int32_t N, int32_t H,
                              ivit_dyadic logit, int32_t k_s, int32_t I0, int32_t M, int32_t k_out,
-                             ivit_dyadic out, int8_t* ctx, cudaStream_t stream);
+                             ivit_dyadic out, int8_t* ctx, cudaStream_t stream, bool lis = false);
 
 ivit_status launch_shiftgelu(const DeviceCtx& dc, const int8_t* x, int64_t n, const GeluParams& g, int8_t* y,
                              cudaStream_t stream);
+
+// ShiftGELU with the row's largest exponent as I_max, x [rows x cols]
+// (cols a multiple of 16).
+ivit_status launch_shiftgelu_rowmax(const DeviceCtx& dc, const int8_t* x, int64_t rows, int32_t cols,
+                                    const GeluParams& g, int8_t* y, cudaStream_t stream);
+
+// I-LayerNorm of x << alpha (alpha [cols], values 0 .. 3; cols a multiple of
+// 16, at most 2048; M_ln <= 20).
+ivit_status launch_layernorm_ptf(const DeviceCtx& dc, const int8_t* x, int64_t rows, int32_t cols,
+                                 const uint8_t* alpha, const int8_t* gamma, const int32_t* beta, int32_t F,
+                                 int32_t M_ln, ivit_dyadic out, int8_t* y, cudaStream_t stream);
 
 // Patch rows z [B*Np x C*P*P] from img [B x C x Hi x Wi] (Hi, Wi multiples of P).
 ivit_status launch_im2col(const DeviceCtx& dc, const int8_t* img, int32_t B, int32_t C, int32_t Hi, int32_t Wi,
