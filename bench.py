@@ -44,6 +44,10 @@ INT8_PER_BF16 = 2.0  # nominal dense tensor-core ratio on B200 (4.5 vs 2.25 PFLO
 # division, one multiply and one subtraction (3), (I_0 + ((-r) >> 1)) >> q (3), row sum (1),
 # P = (Dv e) >> (M - k_out + 1) (2).
 SHIFTMAX_OPS_PER_SCORE = 19
+# Log-Int-Softmax (the FQ-ViT record's 4-bit log2 attention map): the Shiftmax steps up to the
+# row sum (17), the 16-bit IntDiv (2), the 4-bit log2 code (bit length, square, compare, add,
+# subtract and clip: 6) and the power-of-two plane of the code (2).
+LIS_OPS_PER_SCORE = 27
 INT_LANES_PER_SM = 128  # 4 sub-partitions x 32 lanes, one integer instruction per lane per clock
 
 
@@ -865,6 +869,20 @@ def kernel_breakdown(ivit, wl, dp, ws, xs, reps, dev, peaks):
     add("shiftgelu_standalone", lambda i: ivit.ivit_shiftgelu(hs[i % len(hs)], p["gelu_I0"], p["gelu_M"],
                                                               p["gelu_k_out"], p["gelu_out"], h_o),
         "hbm", 2 * T * Dm, in_block=False)
+    # the variants (not on the block's path): ShiftGELU with a row maximum over
+    # each token's Dm channels, Log-Int-Softmax attention, PTF I-LayerNorm
+    add("shiftgelu_rowmax", lambda i: ivit.ivit_shiftgelu_rowmax(hs[i % len(hs)], p["gelu_I0"], p["gelu_M"],
+                                                                 p["gelu_k_out"], p["gelu_out"], h_o),
+        "hbm", 2 * T * Dm, in_block=False)
+    ob, oc = p["attn_out"]
+    lis_out = ivit.ivit_dyadic_from_double(ob / 2.0 ** oc / 256.0)   # scale 2^-15 instead of 2^-7
+    add("attention_lis", lambda i: ivit.ivit_attention_lis(qkv, B, N, H, p["logit"], p["k_s"], p["attn_I0"],
+                                                           p["attn_M"], lis_out, ctx_o),
+        "alu", LIS_OPS_PER_SCORE * B * H * N * N, in_block=False)
+    alpha = torch.from_numpy(np.random.default_rng(0).integers(0, 4, size=D).astype(np.uint8)).to(dev)
+    add("layernorm_ptf", lambda i: ivit.ivit_layernorm_ptf(xs[i % R], alpha, t["ln1_gamma"], t["ln1_beta"],
+                                                           p["ln_F"], 20, p["ln1_out"], y),
+        "hbm", 2 * T * D, in_block=False)
     num_sms = torch.cuda.get_device_properties(dev).multi_processor_count
     for k in out:
         k["peak"], k["unit"], k["peak_note"] = peak_for(k["bound"], peaks, num_sms)
@@ -872,7 +890,8 @@ def kernel_breakdown(ivit, wl, dp, ws, xs, reps, dev, peaks):
         k["achieved"] = k["amount"] / (k["ms"] / 1e3) / scale
         k["frac"] = k["achieved"] / k["peak"]
         k["amount_unit"] = {"hbm": "bytes", "tensor": "int8 ops (2 x MAC)",
-                            "alu": "Shiftmax integer ops (19 per score)"}[k["bound"]]
+                            "alu": ("Log-Int-Softmax integer ops (27 per score)" if k["name"] == "attention_lis"
+                                    else "Shiftmax integer ops (19 per score)")}[k["bound"]]
     return out
 
 

@@ -1,8 +1,9 @@
 /*
  * ivit_selftest.h -- diagnostic entry points of the integer-only ViT library.
  *
- * The first exercises the library's failure path without a GPU fault; the
- * second measures the integer throughput that bounds the attention kernels.  Every wait
+ * They exercise the library's failure paths without a GPU fault (a wait that
+ * nothing completes; a producer told to stop early) and measure the integer
+ * throughput that bounds the attention kernels.  Every wait
  * inside the library's kernels (an mbarrier spin) is bounded by a budget of
  * one second of %globaltimer; a wait that runs out records IVIT_ERR_TIMEOUT
  * in the per-device status word, and the kernel returns instead of hanging.
@@ -43,6 +44,22 @@ ivit_status ivit_selftest_wait_timeout(ivit_stream_t stream);
  * if the launch failed.                                                      */
 ivit_status ivit_selftest_int_rate(int32_t iters, int32_t *sink, int32_t sink_len, int64_t *ops,
                                    ivit_stream_t stream);
+
+/* Failure path of the production kernels, without a fault.  After this call
+ * the next launch of the named kernel -- 1: the INT8 GEMM of every linear
+ * layer (ivit_linear_requant, ivit_linear_shiftgelu and the linear layers of
+ * ivit_block_forward); 2: the short-sequence attention kernel (ivit_attention
+ * with N <= 256) -- has the TMA producer of its first CTA stop before its
+ * `index`-th load (a k-slice of the GEMM, an item of the attention), so the
+ * tensor-core issuer's bounded wait for that load runs out after one second.
+ * The kernel then records IVIT_ERR_TIMEOUT in the device status word, every
+ * role gives up its waits, the issued MMAs and copies drain, the tensor
+ * memory is released and the kernel returns; its output is incomplete.
+ * ivit_stream_status() then returns IVIT_ERR_TIMEOUT once.  The request is
+ * taken by that one launch (a later call replaces a pending one).  index
+ * beyond the CTA's loads leaves that launch untouched.  Returns
+ * IVIT_ERR_INVALID_ARG for another kernel number or a negative index.      */
+ivit_status ivit_selftest_withhold(int32_t kernel, int32_t index);
 
 #ifdef __cplusplus
 }

@@ -24,7 +24,7 @@ __all__ = [
     "ivit_block_forward_static", "STATIC_SCRATCH_BYTES", "EXPORTED_SYMBOLS",
     "ModelParams", "ivit_patch_embed_workspace_bytes", "ivit_patch_embed", "ivit_head_workspace_bytes", "ivit_head",
     "ivit_model_workspace_bytes", "ivit_model_forward", "ivit_selftest_wait_timeout", "ivit_selftest_int_rate",
-    "ivit_shiftgelu_rowmax", "ivit_attention_lis", "ivit_layernorm_ptf",
+    "ivit_shiftgelu_rowmax", "ivit_attention_lis", "ivit_layernorm_ptf", "ivit_selftest_withhold",
 ]
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
@@ -41,7 +41,7 @@ EXPORTED_SYMBOLS = (
     "ivit_patch_embed_workspace_bytes", "ivit_patch_embed", "ivit_head_workspace_bytes", "ivit_head",
     "ivit_model_workspace_bytes", "ivit_model_forward",
     "ivit_selftest_wait_timeout", "ivit_selftest_int_rate",
-    "ivit_shiftgelu_rowmax", "ivit_attention_lis", "ivit_layernorm_ptf",
+    "ivit_shiftgelu_rowmax", "ivit_attention_lis", "ivit_layernorm_ptf", "ivit_selftest_withhold",
 )
 
 _STATUS = {0: "IVIT_OK", 1: "IVIT_ERR_INVALID_ARG", 2: "IVIT_ERR_UNSUPPORTED", 3: "IVIT_ERR_CUDA",
@@ -157,6 +157,8 @@ def lib() -> C.CDLL:
             L.ivit_attention_lis.argtypes = [vp, i32, i32, i32, Dyadic, i32, i32, i32, Dyadic, vp, vp]
             L.ivit_layernorm_ptf.restype = C.c_int
             L.ivit_layernorm_ptf.argtypes = [vp, i64, i32, vp, vp, vp, i32, i32, Dyadic, vp, vp]
+            L.ivit_selftest_withhold.restype = C.c_int
+            L.ivit_selftest_withhold.argtypes = [i32, i32]
             L.ivit_selftest_int_rate.restype = C.c_int
             L.ivit_selftest_int_rate.argtypes = [i32, vp, i32, C.POINTER(C.c_int64), vp]
             _lib = L
@@ -384,6 +386,18 @@ def ivit_selftest_wait_timeout(stream=None):
     """Enqueue the diagnostic kernel whose bounded wait runs out (about one
     second); ivit_stream_status() then reports IVIT_ERR_TIMEOUT once."""
     _check("ivit_selftest_wait_timeout", lib().ivit_selftest_wait_timeout(_stream(stream)))
+
+
+SELFTEST_GEMM = 1
+SELFTEST_ATTENTION = 2
+
+
+def ivit_selftest_withhold(kernel: int, index: int):
+    """Make the next launch of a production kernel (SELFTEST_GEMM or
+    SELFTEST_ATTENTION) have its first CTA's TMA producer stop before its
+    index-th load, so a bounded wait in that kernel runs out (about one
+    second): ivit_stream_status() then reports IVIT_ERR_TIMEOUT once."""
+    _check("ivit_selftest_withhold", lib().ivit_selftest_withhold(int(kernel), int(index)))
 
 
 def ivit_selftest_int_rate(iters: int, sink, stream=None) -> int:

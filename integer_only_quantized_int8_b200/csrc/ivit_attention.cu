@@ -46,6 +46,7 @@ struct AttnArgs {
   uint32_t exp_magic;  // ceil(2^32 / I0) for the arithmetic ShiftExp of logits wider than 8 bits (0 when I0 = 1)
   int8_t* ctx;
   int* status;
+  int32_t withhold;  // diagnostic: CTA 0's producer stops before this local item (-1: never)
 };
 
 struct AttnLayout {
@@ -628,6 +629,9 @@ __global__ void __launch_bounds__(kPersistThreads, 1)
         const int s = j % kLoadStages;
         const uint32_t ph = (uint32_t)((j / kLoadStages) & 1);
         if (!wait_or_abort(&stage_empty[s], ph ^ 1, a.status, abort_flag)) break;
+        // diagnostic (ivit_selftest_withhold): the item's loads are never issued,
+        // so the S issuer's bounded wait for them runs out
+        if (j == a.withhold && blockIdx.x == 0) break;
         const int qt = item % qtiles, h = (item / qtiles) % a.H, img = item / (qtiles * a.H);
         const int row0 = img * N;
         uint8_t* st = smem + s * L.stage_bytes;
@@ -907,6 +911,7 @@ ivit_status launch_attention(const DeviceCtx& dc, const int8_t* qkv, int32_t B, 
   a.exp_magic = I0 > 1 ? (uint32_t)((((uint64_t)1 << 32) + (uint64_t)I0 - 1) / (uint64_t)I0) : 0u;
   a.ctx = ctx;
   a.status = dc.status;
+  a.withhold = N <= kShortMaxKeys && !lis ? take_withhold(kWithholdAttention) : -1;
   dim3 grid((unsigned)((N + kQTile - 1) / kQTile), (unsigned)H, (unsigned)B);
   if (N <= kShortMaxKeys && !lis) {
     const PersistLayout P = persist_layout(N);

@@ -77,6 +77,7 @@ struct GemmArgs {
   ivit_residual res;
   GeluParams gelu;
   int* status;
+  int32_t withhold;  // diagnostic: CTA 0's producer stops before this k-slice of its sequence (-1: never)
 };
 
 template <int BN, int STAGES>
@@ -403,10 +404,17 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       int stage = 0;
       uint32_t phase = 0;
       bool ok = true;
+      int issued = 0;  // k-slices loaded so far by this CTA
       for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
         const int cb = t % ch_tiles, tb = t / ch_tiles;
-        for (int kb = 0; kb < num_kb; ++kb) {
+        for (int kb = 0; kb < num_kb; ++kb, ++issued) {
           if (!mbar_wait(&empty[stage], phase ^ 1, args.status)) {
+            ok = false;
+            break;
+          }
+          // diagnostic (ivit_selftest_withhold): this k-slice is never loaded, so
+          // the MMA issuer's bounded wait for it runs out
+          if (issued == args.withhold && blockIdx.x == 0) {
             ok = false;
             break;
           }
@@ -745,6 +753,7 @@ ivit_status launch_gemm(const DeviceCtx& dc, const int8_t* X, int64_t M, int32_t
   a.res = res;
   a.gelu = gelu ? *gelu : GeluParams{1, 30, 8, {0, 0}};
   a.status = dc.status;
+  a.withhold = take_withhold(kWithholdGemm);
   const bool narrow = out_bits < 8;
   switch (mode) {
     case kEpiPlain:

@@ -27,6 +27,11 @@ ivit_status device_ctx(DeviceCtx* out);
 // Count a kernel launch (for ivit_launch_count).
 void note_launch(int n = 1);
 
+// Diagnostics (ivit_selftest_withhold): the index at which the next launch of
+// the given kernel has its producer stop, or -1; taking it clears it.
+enum WithholdKernel : int { kWithholdGemm = 1, kWithholdAttention = 2 };
+int32_t take_withhold(int kernel);
+
 // Launch with programmatic stream serialization: the kernel may start while
 // the previous kernel of the stream finishes; it must call pdl_wait() before
 // touching that kernel's outputs or writing global memory.

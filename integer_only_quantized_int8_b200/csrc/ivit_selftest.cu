@@ -3,9 +3,26 @@
 // afterwards) can be tested without faulting or hanging a GPU; and a probe of
 // the integer throughput of the instruction mix the Shiftmax passes issue,
 // which gives the attention kernels their measured roof.
+#include <atomic>
+
 #include "ivit_common.cuh"
 #include "ivit_internal.h"
 #include "../../include/ivit_selftest.h"
+
+namespace ivit {
+namespace {
+// (kernel << 32) | index of the pending withhold request, 0 when none
+std::atomic<uint64_t> g_withhold{0};
+}  // namespace
+
+int32_t take_withhold(int kernel) {
+  uint64_t cur = g_withhold.load(std::memory_order_relaxed);
+  while (cur != 0 && (int)(cur >> 32) == kernel) {
+    if (g_withhold.compare_exchange_weak(cur, 0, std::memory_order_acq_rel)) return (int32_t)(uint32_t)cur;
+  }
+  return -1;
+}
+}  // namespace ivit
 
 namespace ivit {
 namespace {
@@ -86,4 +103,10 @@ extern "C" ivit_status ivit_selftest_int_rate(int32_t iters, int32_t* sink, int3
   ivit::int_rate_kernel<<<grid, ivit::kIntThreads, 0, (cudaStream_t)stream>>>(iters, 0x2b8e5f31, sink);
   ivit::note_launch();
   return cudaGetLastError() == cudaSuccess ? IVIT_OK : IVIT_ERR_CUDA;
+}
+
+extern "C" ivit_status ivit_selftest_withhold(int32_t kernel, int32_t index) {
+  if ((kernel != ivit::kWithholdGemm && kernel != ivit::kWithholdAttention) || index < 0) return IVIT_ERR_INVALID_ARG;
+  ivit::g_withhold.store(((uint64_t)(uint32_t)kernel << 32) | (uint32_t)index, std::memory_order_release);
+  return IVIT_OK;
 }
