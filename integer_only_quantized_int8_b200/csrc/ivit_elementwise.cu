@@ -6,9 +6,10 @@
 // with the integer formula and streams 16-byte vectors through the table.
 //
 // I-LayerNorm (same page, section 3.5): one half-warp per row, so a whole
-// activation tensor is in flight in one wave; sums of x and x^2 with dp4a,
-// exact integer variance, 10 Newton steps of the integer square root, then the
-// per-element normalisation, affine and dyadic requant.
+// activation tensor is in flight in one wave; gamma and beta staged in shared
+// memory; sums of x and x^2 with dp4a, exact integer variance, 10 Newton steps
+// of the integer square root, then the per-element normalisation, affine and
+// dyadic requant.
 #include <climits>
 #include <cmath>
 
@@ -160,26 +161,48 @@ __device__ __forceinline__ int32_t sext_byte(uint32_t w, int i) {
   return r;
 }
 
-// One row of `cols` int8 values per half-warp; lane l of the half-warp holds
-// the 16-byte chunks l, l + 16, ... (CPL of them).  CLAMP = false when the host
-// has shown that (b acc) >> c fits int32 for every reachable acc.
-template <int CPL, bool CLAMP, bool FASTQ>
+// I-LayerNorm with gamma and beta staged in shared memory: LPR lanes per row,
+// lane l of a row holding its 16-byte chunks l, l + LPR, ... (at most CPL).
+// gamma (sign-extended to 32 bits) and beta are parameters, not outputs of an
+// earlier kernel, so every CTA stages them before the dependent-launch wait,
+// while the previous kernel of the stream finishes.  Sums of x and x^2 come
+// from dp4a; the mean and variance divisions and 2^M / sigma use an exact
+// fp32 reciprocal quotient with one integer correction (udiv_fast); the root
+// is isqrt_newton10; then the per-element normalisation, affine and dyadic
+// requant.  CLAMP = false when the host has shown that (b acc) >> c fits
+// int32 for every reachable acc; FASTQ: the requant is one mul.hi.
+constexpr int kLnLanes = 16;  // a half-warp per row
+template <int LPR, int CPL, bool CLAMP, bool FASTQ>
 __global__ void __launch_bounds__(kLnThreads)
-    layernorm_kernel(const int8_t* __restrict__ x, int64_t rows, int32_t cols, const int8_t* __restrict__ gamma,
-                     const int32_t* __restrict__ beta, int32_t F, int32_t M_ln, ivit_dyadic out, int32_t out_bq,
-                     int8_t* __restrict__ y) {
+    layernorm_staged_kernel(const int8_t* __restrict__ x, int64_t rows, int32_t cols,
+                            const int8_t* __restrict__ gamma, const int32_t* __restrict__ beta, int32_t F,
+                            int32_t M_ln, ivit_dyadic out, int32_t out_bq, int8_t* __restrict__ y) {
+  // gamma (sign-extended) and beta as 16-byte groups of four channels, stored
+  // [q][chunk]: group q of 16-channel chunk ci at q * nchunk + ci, so the
+  // lanes of a row, which hold consecutive chunks, read consecutive 16-byte
+  // slots (no bank conflicts)
+  extern __shared__ int4 ln_smem[];
+  const int nchunk = cols >> 4;
+  int4* gs = ln_smem;                 // [4][nchunk]
+  int4* bs = ln_smem + 4 * nchunk;    // [4][nchunk]
+  for (int i = threadIdx.x; i < cols / 4; i += blockDim.x) {
+    const int ci = i >> 2, q = i & 3;
+    const uint32_t g4 = __ldg(reinterpret_cast<const uint32_t*>(gamma) + i);
+    gs[q * nchunk + ci] = make_int4(sext_byte(g4, 0), sext_byte(g4, 1), sext_byte(g4, 2), sext_byte(g4, 3));
+    bs[q * nchunk + ci] = __ldg(reinterpret_cast<const int4*>(beta) + i);
+  }
+  __syncthreads();
   pdl_wait();  // x comes from an earlier kernel
   pdl_launch_dependents();
-  const int hl = threadIdx.x & 15;
-  const int64_t row = (int64_t)blockIdx.x * (kLnThreads / 16) + (threadIdx.x >> 4);
+  const int hl = threadIdx.x % LPR;
+  const int64_t row = (int64_t)blockIdx.x * (kLnThreads / LPR) + (threadIdx.x / LPR);
   const bool active = row < rows;
-  const int nchunk = cols >> 4;
   const int8_t* xr = x + (active ? row : 0) * cols;
   int4 v[CPL];
   int32_t s1 = 0, s2 = 0;
 #pragma unroll
   for (int k = 0; k < CPL; ++k) {
-    const int ci = hl + 16 * k;
+    const int ci = hl + LPR * k;
     if (active && ci < nchunk) {
       v[k] = __ldcs(reinterpret_cast<const int4*>(xr) + ci);
       const int w[4] = {v[k].x, v[k].y, v[k].z, v[k].w};
@@ -191,49 +214,46 @@ __global__ void __launch_bounds__(kLnThreads)
     }
   }
 #pragma unroll
-  for (int o = 8; o > 0; o >>= 1) {  // reduce within each half-warp
+  for (int o = LPR / 2; o > 0; o >>= 1) {  // reduce within each row's lanes
     s1 += __shfl_xor_sync(0xffffffffu, s1, o);
     s2 += __shfl_xor_sync(0xffffffffu, s2, o);
   }
   if (!active) return;
-  // mu = floor(sum x / n) (|sum x| <= 2^18); sum (x - mu)^2 = sum x^2 - 2 mu sum x + n mu^2,
-  // all within int32 (at most 2^27)
   const int32_t as1 = s1 < 0 ? -s1 : s1;
   const int32_t q1 = udiv_fast(as1, cols);
   const int32_t mu = s1 >= 0 ? q1 : -q1 - (as1 - q1 * cols != 0 ? 1 : 0);
   const int32_t sd2 = s2 - 2 * mu * s1 + cols * mu * mu;
-  const int32_t V = udiv_fast(sd2, cols);  // sd2 >= 0, quotient <= 16256
+  const int32_t V = udiv_fast(sd2, cols);
   int32_t sigma = isqrt_newton10(V);
   if (sigma < 1) sigma = 1;
-  const int32_t f = udiv_fast(1 << M_ln, sigma);  // M_ln <= 23: quotient 2^M_ln exact for sigma = 1
+  const int32_t f = udiv_fast(1 << M_ln, sigma);
   const int sh = M_ln - F;
-  const int32_t muf = mu * f;  // (x - mu) f = x f - mu f, exact in 32-bit arithmetic (|(x - mu) f| < 2^31)
+  const int32_t muf = mu * f;
   int32_t lo = INT_MIN, hi = INT_MAX;
   if (CLAMP) out_bounds(out.b, out.c, lo, hi);
   int8_t* yr = y + row * cols;
 #pragma unroll
   for (int k = 0; k < CPL; ++k) {
-    const int ci = hl + 16 * k;
+    const int ci = hl + LPR * k;
     if (ci < nchunk) {
-      const int c0 = ci * 16;
-      const int4 gv = __ldg(reinterpret_cast<const int4*>(gamma + c0));
-      const uint32_t gw[4] = {(uint32_t)gv.x, (uint32_t)gv.y, (uint32_t)gv.z, (uint32_t)gv.w};
       const uint32_t xw[4] = {(uint32_t)v[k].x, (uint32_t)v[k].y, (uint32_t)v[k].z, (uint32_t)v[k].w};
       uint32_t o[4];
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
-        const int4 bt = __ldg(reinterpret_cast<const int4*>(beta + c0) + q);
-        const int32_t bb[4] = {bt.x, bt.y, bt.z, bt.w};
+        const int4 g4 = gs[q * nchunk + ci];
+        const int4 b4 = bs[q * nchunk + ci];
+        const int32_t gg[4] = {g4.x, g4.y, g4.z, g4.w};
+        const int32_t bb[4] = {b4.x, b4.y, b4.z, b4.w};
         int32_t r[4];
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
           const int32_t nv = (sext_byte(xw[q], e) * f - muf) >> sh;
-          int32_t acc = nv * sext_byte(gw[q], e) + bb[e];
+          int32_t acc = nv * gg[e] + bb[e];
           if (FASTQ) {
-            r[e] = __mulhi(out_bq, acc);  // floor(b acc / 2^c) with bq = b 2^(32 - c), exact
+            r[e] = __mulhi(out_bq, acc);
           } else {
             if (CLAMP) acc = min(max(acc, lo), hi);
-            const int64_t pr = (int64_t)out.b * acc;  // (b acc) >> c fits int32: one funnel shift
+            const int64_t pr = (int64_t)out.b * acc;
             r[e] = (int32_t)__funnelshift_r((uint32_t)pr, (uint32_t)(pr >> 32), (uint32_t)out.c);
           }
         }
@@ -246,55 +266,57 @@ __global__ void __launch_bounds__(kLnThreads)
 
 // ---------------------------------------------------------------------------
 // ShiftGELU with a row maximum (I-ViT section 3.4, I_max read as the row's
-// largest exponent; see include/ivit.h): one CTA per row.  I_p is
+// largest exponent; see include/ivit.h): one warp per row.  I_p is
 // non-decreasing in x, so the row's largest exponent is I_p of the row's
 // largest byte; given it, the output is a function of the int8 input alone,
-// which the CTA tabulates (256 entries) and streams the row through.
+// which the warp tabulates (256 entries) and streams the row through.  The
+// table is kept while consecutive rows of the warp share their I_max (rows
+// that reach x = 127 all do).
 // ---------------------------------------------------------------------------
 constexpr int kRowGeluThreads = 256;
 
 __global__ void __launch_bounds__(kRowGeluThreads)
     shiftgelu_rowmax_kernel(const int8_t* __restrict__ x, int64_t rows, int32_t cols, GeluParams g,
                             int8_t* __restrict__ y) {
-  __shared__ int8_t tab[256];
-  __shared__ int32_t wmax[kRowGeluThreads / 32];
+  __shared__ int8_t tabs[kRowGeluThreads / 32][256];
   pdl_wait();  // x comes from an earlier kernel
   pdl_launch_dependents();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  int8_t* tab = tabs[warp];
   const int nvec = cols >> 4;
-  for (int64_t row = blockIdx.x; row < rows; row += gridDim.x) {
+  int32_t tab_imax = -1;  // the I_max the warp's table holds (none yet)
+  for (int64_t row = (int64_t)blockIdx.x * (kRowGeluThreads / 32) + warp; row < rows;
+       row += (int64_t)gridDim.x * (kRowGeluThreads / 32)) {
     const int4* xv = reinterpret_cast<const int4*>(x + row * cols);
-    int32_t m = -128;
-    for (int v = threadIdx.x; v < nvec; v += blockDim.x) {
+    uint32_t m4 = 0x80808080u;  // four running maxima of signed bytes
+    for (int v = lane; v < nvec; v += 32) {
       const int4 in = __ldg(xv + v);
-      const uint32_t w[4] = {(uint32_t)in.x, (uint32_t)in.y, (uint32_t)in.z, (uint32_t)in.w};
-#pragma unroll
-      for (int k = 0; k < 4; ++k)
-#pragma unroll
-        for (int e = 0; e < 4; ++e) m = max(m, (int32_t)(int8_t)(w[k] >> (8 * e)));
+      m4 = __vmaxs4(m4, __vmaxs4(__vmaxs4((uint32_t)in.x, (uint32_t)in.y), __vmaxs4((uint32_t)in.z, (uint32_t)in.w)));
     }
+    int32_t m = max(max((int32_t)(int8_t)m4, (int32_t)(int8_t)(m4 >> 8)),
+                    max((int32_t)(int8_t)(m4 >> 16), (int32_t)(int8_t)(m4 >> 24)));
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(0xffffffffu, m, o));
-    if ((threadIdx.x & 31) == 0) wmax[threadIdx.x >> 5] = m;
-    __syncthreads();
-    int32_t xm = wmax[0];
-#pragma unroll
-    for (int i = 1; i < kRowGeluThreads / 32; ++i) xm = max(xm, wmax[i]);
-    // I_max = max(0, I_p(largest x)); e2 = ShiftExp(-I_max)
-    const int32_t ipm = xm + (xm >> 1) + (xm >> 3) + (xm >> 4);
+    // I_max = max(0, I_p(largest x)), warp-uniform
+    const int32_t ipm = m + (m >> 1) + (m >> 3) + (m >> 4);
     const int32_t I_max = ipm > 0 ? ipm : 0;
-    {
-      const int32_t xi = (int32_t)threadIdx.x - 128;  // one table entry per thread
-      const int32_t ip = xi + (xi >> 1) + (xi >> 3) + (xi >> 4);
-      const int32_t e1 = shift_exp(ip - I_max, g.I0);
+    if (I_max != tab_imax) {
+      __syncwarp();  // every lane is done with the previous table
       const int32_t e2 = shift_exp(-I_max, g.I0);
-      const uint32_t sum = (uint32_t)(e1 + e2);
-      const uint32_t dv = (1u << g.M) / (sum > 0u ? sum : 1u);  // both exponentials 0: sigma = 0
-      const int32_t sig = (int32_t)((dv * (uint32_t)e1) >> (g.M - (g.k_out - 1)));
-      tab[threadIdx.x] = (int8_t)requant8(xi * sig, g.out.b, g.out.c);
+      for (int i = lane; i < 256; i += 32) {
+        const int32_t xi = i - 128;
+        const int32_t ip = xi + (xi >> 1) + (xi >> 3) + (xi >> 4);
+        const int32_t e1 = shift_exp(ip - I_max, g.I0);
+        const uint32_t sum = (uint32_t)(e1 + e2);
+        const uint32_t dv = (1u << g.M) / (sum > 0u ? sum : 1u);  // both exponentials 0: sigma = 0
+        const int32_t sig = (int32_t)((dv * (uint32_t)e1) >> (g.M - (g.k_out - 1)));
+        tab[i] = (int8_t)requant8(xi * sig, g.out.b, g.out.c);
+      }
+      __syncwarp();
+      tab_imax = I_max;
     }
-    __syncthreads();
     int4* yv = reinterpret_cast<int4*>(y + row * cols);
-    for (int v = threadIdx.x; v < nvec; v += blockDim.x) {
+    for (int v = lane; v < nvec; v += 32) {
       const int4 in = __ldg(xv + v);
       const uint32_t w[4] = {(uint32_t)in.x, (uint32_t)in.y, (uint32_t)in.z, (uint32_t)in.w};
       uint32_t o[4];
@@ -307,7 +329,6 @@ __global__ void __launch_bounds__(kRowGeluThreads)
       }
       __stcs(yv + v, make_int4((int)o[0], (int)o[1], (int)o[2], (int)o[3]));
     }
-    __syncthreads();  // the table and the maxima are rewritten for the next row
   }
 }
 
@@ -399,10 +420,12 @@ __global__ void __launch_bounds__(kPtfThreads)
 ivit_status launch_shiftgelu_rowmax(const DeviceCtx& dc, const int8_t* x, int64_t rows, int32_t cols,
                                     const GeluParams& g, int8_t* y, cudaStream_t stream) {
   if (rows == 0) return IVIT_OK;
+  const int64_t rows_per_cta = kRowGeluThreads / 32;
+  int64_t blocks = (rows + rows_per_cta - 1) / rows_per_cta;
   const int64_t cap = (int64_t)dc.num_sms * 8;
-  const unsigned grid = (unsigned)(rows < cap ? rows : cap);
-  const cudaError_t e =
-      launch_pdl(shiftgelu_rowmax_kernel, dim3(grid), dim3(kRowGeluThreads), 0, stream, x, rows, cols, g, y);
+  if (blocks > cap) blocks = cap;
+  const cudaError_t e = launch_pdl(shiftgelu_rowmax_kernel, dim3((unsigned)blocks), dim3(kRowGeluThreads), 0, stream,
+                                   x, rows, cols, g, y);
   note_launch();
   return e == cudaSuccess ? IVIT_OK : IVIT_ERR_CUDA;
 }
@@ -445,8 +468,10 @@ ivit_status launch_layernorm(const DeviceCtx& dc, const int8_t* x, int64_t rows,
                              int8_t* y, cudaStream_t stream) {
   (void)dc;
   if (rows == 0) return IVIT_OK;
-  const int64_t blocks = (rows + kLnThreads / 16 - 1) / (kLnThreads / 16);
+  const int64_t rows_per_cta = kLnThreads / kLnLanes;
+  const int64_t blocks = (rows + rows_per_cta - 1) / rows_per_cta;
   if (blocks > 0x7fffffff) return IVIT_ERR_UNSUPPORTED;
+  const size_t smem = (size_t)cols * 8;  // gamma and beta as int32
   const unsigned g = (unsigned)blocks;
   const int nchunk = cols / 16;
   // |n| <= 255 2^F, |gamma| <= 128, |beta| <= 2^30: when b times that bound stays
@@ -456,22 +481,27 @@ ivit_status launch_layernorm(const DeviceCtx& dc, const int8_t* x, int64_t rows,
   // the output requant is one mul.hi by b 2^(32 - c) when that fits a positive int32
   const bool fastq = out.c >= 1 && (int64_t)out.b < ((int64_t)1 << (out.c - 1));
   const int32_t bq = fastq ? (int32_t)((int64_t)out.b << (32 - out.c)) : 0;
-#define IVIT_LN_LAUNCH(CPL)                                                                                \
-  launch_pdl(fastq   ? layernorm_kernel<CPL, false, true>                                                      \
-             : clamp ? layernorm_kernel<CPL, true, false>                                                      \
-                     : layernorm_kernel<CPL, false, false>,                                                    \
-             dim3(g), dim3(kLnThreads), 0, stream, x, rows, cols, gamma, beta, F, M_ln, out, bq, y)
+#define IVIT_LN_LAUNCH(CPL)                                                                                  \
+  launch_pdl(fastq   ? layernorm_staged_kernel<kLnLanes, CPL, false, true>                                      \
+             : clamp ? layernorm_staged_kernel<kLnLanes, CPL, true, false>                                      \
+                     : layernorm_staged_kernel<kLnLanes, CPL, false, false>,                                    \
+             dim3(g), dim3(kLnThreads), smem, stream, x, rows, cols, gamma, beta, F, M_ln, out, bq, y)
   cudaError_t e;
-  if (nchunk <= 16)
+  const int cpl = (nchunk + kLnLanes - 1) / kLnLanes;
+  if (cpl <= 1)
     e = IVIT_LN_LAUNCH(1);
-  else if (nchunk <= 32)
+  else if (cpl <= 2)
     e = IVIT_LN_LAUNCH(2);
-  else if (nchunk <= 48)
+  else if (cpl <= 3)
     e = IVIT_LN_LAUNCH(3);
-  else if (nchunk <= 64)
+  else if (cpl <= 4)
     e = IVIT_LN_LAUNCH(4);
-  else
+  else if (cpl <= 6)
+    e = IVIT_LN_LAUNCH(6);
+  else if (cpl <= 8)
     e = IVIT_LN_LAUNCH(8);
+  else
+    e = IVIT_LN_LAUNCH(16);
 #undef IVIT_LN_LAUNCH
   note_launch();
   return e == cudaSuccess ? IVIT_OK : IVIT_ERR_CUDA;
