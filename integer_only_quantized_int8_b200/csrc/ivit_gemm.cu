@@ -654,6 +654,330 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   }
 }
 
+// ---------------------------------------------------------------------------
+// Own-tile variant: three TMEM accumulators (tile widths up to 160 tokens),
+// and each of the three epilogue parts drains whole tiles -- part p takes the
+// CTA's tiles p, p + 3, ... -- instead of all three parts sharing every tile.
+// A tile's epilogue carries a fixed latency (the wait for the accumulator,
+// the part barriers, the stores and the bias refill) besides its arithmetic;
+// with three tiles draining at once those latencies overlap.  Producer and
+// MMA issuers are those of gemm_i8_requant_kernel with the accumulator index
+// cycling over three buffers.
+// ---------------------------------------------------------------------------
+constexpr int kOwnAcc = 3;
+
+template <int BN, int STAGES>
+struct OwnLayout {
+  static constexpr int kIssuers = (STAGES % 2 == 0) ? 2 : 1;
+  static constexpr int kABytes = kBM * kBK;
+  static constexpr int kBBytes = BN * kBK;
+  static constexpr int kStageBytes = kABytes + kBBytes;
+  static constexpr int kChunks = BN / 16;
+  static constexpr int kOutOff = STAGES * kStageBytes;
+  static constexpr int kPartSlots = kChunks * kSlotBytes;  // a whole tile per part
+  static constexpr int kBarOff = kOutOff + kEpiParts * kPartSlots;
+  // full, empty (STAGES each), tmem full / empty (three each), drain, one skip barrier per part
+  static constexpr int kNumBars = 2 * STAGES + 2 * kOwnAcc + 1 + kEpiParts;
+  static constexpr int kSlotOff = kBarOff + kNumBars * 8;
+  static constexpr int kGeluOff = kSlotOff + 16;
+  static constexpr int kBytes = kGeluOff + 256;
+  static constexpr int kAlloc = kBytes + 1024;
+  static constexpr int kAccCols = (BN + 31) / 32 * 32;
+  static_assert(kOwnAcc * kAccCols <= 512, "three accumulators must fit the TMEM columns");
+  static_assert(kAlloc <= 227 * 1024, "shared memory budget");
+};
+
+template <int BN, int STAGES, int EPI, bool NARROW>
+__global__ void __launch_bounds__(kGemmThreads, 1)
+    gemm_own_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX,
+                    const __grid_constant__ CUtensorMap tmY, const __grid_constant__ CUtensorMap tmS,
+                    const GemmArgs args) {
+  using L = OwnLayout<BN, STAGES>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = align_smem_1024(smem_raw);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + L::kBarOff);
+  uint64_t* empty = full + STAGES;
+  uint64_t* tfull = empty + STAGES;      // [3]
+  uint64_t* tempty = tfull + kOwnAcc;    // [3]
+  uint64_t* drain = tempty + kOwnAcc;
+  uint64_t* skip_full = drain + 1;       // [kEpiParts]
+  uint32_t* tslot = reinterpret_cast<uint32_t*>(smem + L::kSlotOff);
+  int8_t* gelu_tab = reinterpret_cast<int8_t*>(smem + L::kGeluOff);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int64_t M = args.M;
+  const int N = args.N;
+  const int ch_tiles = (N + kBM - 1) / kBM;
+  const int tok_tiles = (int)((M + BN - 1) / BN);
+  const int num_tiles = ch_tiles * tok_tiles;
+  const int num_kb = (args.K + kBK - 1) / kBK;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int a = 0; a < kOwnAcc; ++a) {
+      mbar_init(&tfull[a], L::kIssuers);  // one commit per issuing thread
+      mbar_init(&tempty[a], 4);           // the four warps of the part that owns the buffer
+    }
+    mbar_init(drain, L::kIssuers);
+    for (int e = 0; e < kEpiParts; ++e) mbar_init(&skip_full[e], 1);
+    fence_barrier_init();
+    prefetch_tensormap(&tmW);
+    prefetch_tensormap(&tmX);
+    prefetch_tensormap(&tmY);
+    if (EPI == kEpiResidual) prefetch_tensormap(&tmS);
+  }
+  if (EPI == kEpiGelu) {
+    for (int i = threadIdx.x; i < 256; i += blockDim.x)
+      gelu_tab[i] = (int8_t)shiftgelu8(i - 128, args.gelu.I0, args.gelu.M, args.gelu.k_out, args.gelu.out.b,
+                                       args.gelu.out.c);
+  }
+  if (warp == 1) {
+    __syncwarp();
+    tmem_alloc(tslot, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tslot;
+  pdl_wait();  // X and the skip tensor come from earlier kernels
+  pdl_launch_dependents();
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      int issued = 0;
+      for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
+        const int cb = t % ch_tiles, tb = t / ch_tiles;
+        for (int kb = 0; kb < num_kb; ++kb, ++issued) {
+          if (!mbar_wait(&empty[stage], phase ^ 1, args.status)) {
+            ok = false;
+            break;
+          }
+          if (issued == args.withhold && blockIdx.x == 0) {  // diagnostic (ivit_selftest_withhold)
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(&full[stage], L::kStageBytes);
+          uint8_t* sa = smem + stage * L::kStageBytes;
+          tma_load_2d(sa, &tmW, kb * kBK, cb * kBM, &full[stage]);
+          tma_load_2d(sa + L::kABytes, &tmX, kb * kBK, tb * BN, &full[stage]);
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+      }
+    }
+  } else if (warp <= 2) {
+    // ------------------------------------------------------------ MMA issuers
+    if (lane == 0 && warp <= L::kIssuers) {
+      constexpr int kStep = L::kIssuers;
+      const uint32_t idesc = idesc_i8(kBM, BN, true, true, false);
+      const uint64_t d0 = smem_desc(smem_u32(smem), 16, 1024, kSwizzle128B);
+      const uint32_t d_lo0 = (uint32_t)d0, d_hi = (uint32_t)(d0 >> 32);
+      int stage = warp - 1;
+      uint32_t phase = 0;
+      int kb0 = warp - 1;
+      int acc = 0;
+      uint32_t acc_phase = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
+        if (!mbar_wait(&tempty[acc], acc_phase, args.status)) break;
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + (uint32_t)(acc * L::kAccCols);
+        int kb = kb0;
+        for (; kb < num_kb; kb += kStep) {
+          if (!mbar_wait(&full[stage], phase, args.status)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a_lo = d_lo0 + (uint32_t)(stage * (L::kStageBytes >> 4));
+          const uint32_t b_lo = a_lo + (uint32_t)(L::kABytes >> 4);
+#pragma unroll
+          for (int k = 0; k < kBK / 32; ++k) umma_i8_acc(d_tmem, a_lo + 2 * k, d_hi, b_lo + 2 * k, d_hi, idesc);
+          umma_commit(&empty[stage]);
+          stage += kStep;
+          if (stage >= STAGES) {
+            stage -= STAGES;
+            phase ^= 1;
+          }
+        }
+        if (!ok) break;
+        kb0 = kb - num_kb;
+        umma_commit(&tfull[acc]);
+        if (++acc == kOwnAcc) {
+          acc = 0;
+          acc_phase ^= 1;
+        }
+      }
+      umma_commit(drain);
+      mbar_wait(drain, 0, args.status);
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue
+    constexpr int kChunks = L::kChunks;
+    const int e = warp - 3;
+    const int quarter = warp & 3;
+    const int part = e >> 2;  // owns accumulator `part` and the CTA's tiles part, part + 3, ...
+    const uint32_t sel2 = (lane & 2) ? 0x3276u : 0x5410u;
+    const uint32_t sel1 = (lane & 1) ? 0x3715u : 0x6240u;
+    const int sub = lane & 3;
+    const int grp = lane >> 2;
+    const bool part_lead = (e & 3) == 0 && lane == 0;
+    uint8_t* const slots = smem + L::kOutOff + part * L::kPartSlots;
+    const uint32_t ofs_even = slot_ofs(sub, quarter, grp, 0), ofs_odd = slot_ofs(sub, quarter, grp, 1);
+    uint64_t* sbar = &skip_full[part];
+    const uint32_t tbase = tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(part * L::kAccCols);
+    const int tstep = kOwnAcc * (int)gridDim.x;  // tiles between two of this part's tiles
+    auto chan_of = [&](int t) { return (t % ch_tiles) * kBM + quarter * 32 + lane; };
+    // the buffer starts out holding the bias of the part's first tile
+    int t = (int)blockIdx.x + part * (int)gridDim.x;
+    if (t < num_tiles) {
+      const int ch = chan_of(t);
+      bias_fill(tbase, 0, kChunks, (args.bias && ch < N) ? __ldg(args.bias + ch) : 0);
+    }
+    tmem_st_wait();
+    tc_fence_before();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&tempty[part]);
+    uint32_t acc_phase = 0;
+    uint32_t skip_phase = 0;
+    // this lane's channel constants, loaded one own tile ahead
+    auto load_chan = [&](int tt, int32_t& vb, int32_t& vc, int32_t& vbias) {
+      const int ch = chan_of(tt);
+      const bool okc = tt < num_tiles && ch < N;
+      vb = okc ? __ldg(args.b + ch) : 0;
+      vc = okc ? (int32_t)__ldg(args.c + ch) : 0;
+      vbias = (okc && args.bias) ? __ldg(args.bias + ch) : 0;
+    };
+    auto derive = [&](int tt, int32_t vb, int32_t vc, int32_t vbias, ChanConst& kx, int& reqx) {
+      kx = chan_of(tt) < N ? chan_const(vb, vc, vbias, args.K) : chan_const(0, 0, 0, args.K);
+      reqx = __all_sync(0xffffffffu, kx.fast) ? kReqFast
+                                              : (__any_sync(0xffffffffu, kx.needs_clamp) ? kReqWideClamp : kReqWide);
+    };
+    int32_t nb, nc, nbias;
+    load_chan(t, nb, nc, nbias);
+    ChanConst kc;
+    int req;
+    derive(t, nb, nc, nbias, kc, req);
+    for (; t < num_tiles; t += tstep) {
+      const int tn = t + tstep;  // this part's next tile
+      load_chan(tn, nb, nc, nbias);
+      const int cb = t % ch_tiles, tb = t / ch_tiles;
+      const int64_t tok_base = (int64_t)tb * BN;
+      int n = kChunks;  // chunks that hold at least one real token
+      while (n > 0 && tok_base + 16 * (n - 1) >= M) --n;
+      const bool live = n > 0;
+      const int tile_ch = cb * kBM;
+      if (part_lead) {
+        bulk_wait_read_all();  // the part's previous stores have read its slots
+        if (EPI == kEpiResidual && live) {
+          mbar_arrive_expect_tx(sbar, (uint32_t)(n * kSlotBytes));
+          for (int i = 0; i < n; ++i)
+            tma_load_2d(slots + i * kSlotBytes, &tmS, tile_ch, (int32_t)(tok_base + 16 * i), sbar);
+        }
+      }
+      const bool got = mbar_wait(&tfull[part], acc_phase, args.status);
+      if (!part_bar_and(part, got)) {
+        if (EPI == kEpiResidual && live && part_lead) mbar_wait(sbar, skip_phase, args.status);
+        break;
+      }
+      bool got_skip = true;
+      if (EPI == kEpiResidual && live) {
+        got_skip = mbar_wait(sbar, skip_phase, args.status);
+        skip_phase ^= 1;
+      }
+      tc_fence_after();
+#define IVIT_OWN_TILE(R) \
+  epi_tile<EPI, NARROW, R>(tbase, 0, n, kc, args, gelu_tab, slots, ofs_even, ofs_odd, sel2, sel1)
+      if (!args.round) {
+        if (req == kReqFast)
+          IVIT_OWN_TILE(kReqFast);
+        else if (req == kReqWide)
+          IVIT_OWN_TILE(kReqWide);
+        else
+          IVIT_OWN_TILE(kReqWideClamp);
+      } else {
+        if (req == kReqFast)
+          IVIT_OWN_TILE(kReqFast + kReqRound);
+        else if (req == kReqWide)
+          IVIT_OWN_TILE(kReqWide + kReqRound);
+        else
+          IVIT_OWN_TILE(kReqWideClamp + kReqRound);
+      }
+#undef IVIT_OWN_TILE
+      fence_proxy_async_smem();
+      if (!part_bar_and(part, got_skip)) break;
+      if (part_lead) {
+        if (live)
+          for (int i = 0; i < n; ++i)
+            tma_store_2d(&tmY, tile_ch, (int32_t)(tok_base + 16 * i), slots + i * kSlotBytes);
+        bulk_commit_group();
+      }
+      // the buffer takes the bias of the part's next tile
+      if (tn < num_tiles) bias_fill(tbase, 0, kChunks, nbias);
+      tmem_st_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&tempty[part]);
+      acc_phase ^= 1;
+      derive(tn, nb, nc, nbias, kc, req);
+    }
+    if (part_lead) bulk_wait_all();
+    __syncwarp();
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem_base, 512);
+  }
+}
+
+template <int BN, int STAGES, int EPI, bool NARROW>
+ivit_status run_gemm_own(const DeviceCtx& dc, const int8_t* X, const int8_t* W, const int8_t* skip, int8_t* Y,
+                         const GemmArgs& a, cudaStream_t stream) {
+  using L = OwnLayout<BN, STAGES>;
+  CUtensorMap tmW, tmX, tmY, tmS;
+  ivit_status st = encode_tmap_2d_u8(&tmW, W, (uint64_t)a.K, (uint64_t)a.N, (uint64_t)a.K, kBK, kBM,
+                                     CU_TENSOR_MAP_SWIZZLE_128B);
+  if (st != IVIT_OK) return st;
+  st = encode_tmap_2d_u8(&tmX, X, (uint64_t)a.K, (uint64_t)a.M, (uint64_t)a.K, kBK, BN, CU_TENSOR_MAP_SWIZZLE_128B);
+  if (st != IVIT_OK) return st;
+  st = encode_tmap_2d_u8(&tmY, Y, (uint64_t)a.N, (uint64_t)a.M, (uint64_t)a.N, kBM, 16, CU_TENSOR_MAP_SWIZZLE_128B);
+  if (st != IVIT_OK) return st;
+  if (EPI == kEpiResidual) {
+    st = encode_tmap_2d_u8(&tmS, skip, (uint64_t)a.N, (uint64_t)a.M, (uint64_t)a.N, kBM, 16,
+                           CU_TENSOR_MAP_SWIZZLE_128B);
+    if (st != IVIT_OK) return st;
+  } else {
+    tmS = tmY;  // unused
+  }
+  auto kern = gemm_own_kernel<BN, STAGES, EPI, NARROW>;
+  static bool attr_done = false;  // benign race: the attribute value is the same
+  if (!attr_done) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAlloc) != cudaSuccess)
+      return IVIT_ERR_CUDA;
+    attr_done = true;
+  }
+  const int tiles = ((a.N + kBM - 1) / kBM) * (int)((a.M + BN - 1) / BN);
+  const int grid = tiles < dc.num_sms ? tiles : dc.num_sms;
+  const cudaError_t e = launch_pdl(kern, dim3(grid), dim3(kGemmThreads), L::kAlloc, stream, tmW, tmX, tmY, tmS, a);
+  note_launch();
+  return e == cudaSuccess ? IVIT_OK : IVIT_ERR_CUDA;
+}
+
 template <int BN, int STAGES, int EPI, bool NARROW>
 ivit_status run_gemm(const DeviceCtx& dc, const int8_t* X, const int8_t* W, const int8_t* skip, int8_t* Y,
                      const GemmArgs& a, cudaStream_t stream) {
@@ -715,9 +1039,50 @@ int pick_bn(int64_t M, int N, int num_sms) {
   return best;
 }
 
+// Token-tile width of the own-tile variant (three accumulators: at most 160
+// tokens), by the same cost model.
+int pick_bn_own(int64_t M, int N, int num_sms) {
+  static const int cands[] = {160, 144, 128};
+  const int ch_tiles = (N + kBM - 1) / kBM;
+  int best = 160;
+  int64_t best_cost = INT64_MAX;
+  for (int bn : cands) {
+    const int64_t tiles = (int64_t)ch_tiles * ((M + bn - 1) / bn);
+    const int64_t rounds = (tiles + num_sms - 1) / num_sms;
+    const int64_t cost = rounds * (bn + 112);
+    if (cost < best_cost) {
+      best_cost = cost;
+      best = bn;
+    }
+  }
+  return best;
+}
+
+// Whether the own-tile variant takes a GEMM: where the epilogue outweighs
+// the MMAs of a tile -- a short reduction (K <= 512), or the ShiftGELU
+// epilogue at K <= 768.  Same-box timings of the ViT-B, ViT-L and DeiT-S
+// layers (us, shared-tile / own-tile): DeiT-S (K = 384) QKV 11.1 / 9.0,
+// W^O 8.9 / 7.8, fc1 16.0 / 14.0; ViT-B fc1 30.1 / 27.5; but ViT-B QKV
+// 18.8 / 20.3, W^O 13.0 / 13.5, fc2 25.9 / 29.9 and every ViT-L layer were
+// slower (tiles of at most 160 tokens take an extra round of tiles there).
+template <int EPI>
+bool use_own_tiles(int K) {
+  return K <= 512 || (EPI == kEpiGelu && K <= 768);
+}
+
 template <int EPI, bool NARROW>
 ivit_status dispatch_bn(const DeviceCtx& dc, const int8_t* X, const int8_t* W, const int8_t* skip, int8_t* Y,
                         const GemmArgs& a, cudaStream_t stream) {
+  if (use_own_tiles<EPI>(a.K)) {
+    switch (pick_bn_own(a.M, a.N, dc.num_sms)) {
+      case 160:
+        return run_gemm_own<160, 4, EPI, NARROW>(dc, X, W, skip, Y, a, stream);
+      case 144:
+        return run_gemm_own<144, 4, EPI, NARROW>(dc, X, W, skip, Y, a, stream);
+      default:
+        return run_gemm_own<128, 4, EPI, NARROW>(dc, X, W, skip, Y, a, stream);
+    }
+  }
   switch (pick_bn(a.M, a.N, dc.num_sms)) {
     case 256:
       return run_gemm<256, 3, EPI, NARROW>(dc, X, W, skip, Y, a, stream);

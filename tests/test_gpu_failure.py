@@ -53,9 +53,10 @@ def _timeout_then_exact(run, want):
     np.testing.assert_array_equal(got, want)
 
 
-@pytest.mark.parametrize("residual", [False, True])
-def test_gemm_producer_stops_and_the_gemm_reports_timeout(residual):
-    lc = synthetic.linear_case(1000, 1024, 512, seed=31, with_skip=residual)
+# K = 1024 takes the shared-tile GEMM kernel, K = 384 the own-tile one
+@pytest.mark.parametrize("K,residual", [(1024, False), (1024, True), (384, False), (384, True)])
+def test_gemm_producer_stops_and_the_gemm_reports_timeout(K, residual):
+    lc = synthetic.linear_case(1000, K, 512, seed=31, with_skip=residual)
     b, c = zip(*[ivit.ivit_dyadic_from_double(r) for r in lc.ratio])
     b = np.array(b, dtype=np.int32)
     c = np.array(c, dtype=np.int8)
@@ -68,7 +69,7 @@ def test_gemm_producer_stops_and_the_gemm_reports_timeout(residual):
 
     def run():
         if state.pop("first", False):
-            ivit.ivit_selftest_withhold(ivit.SELFTEST_GEMM, 3)   # the fourth k-slice of CTA 0
+            ivit.ivit_selftest_withhold(ivit.SELFTEST_GEMM, 2)   # the third k-slice of CTA 0
         Y.fill_(0)
         ivit.ivit_linear_requant(X, W, bias, bd, cd, Y, skip=skip, res=res)
         torch.cuda.synchronize()

@@ -96,18 +96,27 @@ def test_linear_requant_parity(M, K, N):
 
 
 # Shapes whose token-tile width (chosen for the fewest rounds of tiles over
-# 148 SMs) is, in order, 256 (three-stage ring, one MMA issuer), 224, 192,
-# 176 (twice, the second with a ragged channel tile), 160 and 128 (two
-# issuers).  Every M leaves a ragged last token tile, and the k-slice counts
-# are odd and even.  Each shape runs the plain, residual, narrow-output and
-# fused ShiftGELU epilogues.
+# 148 SMs) covers every width of both GEMM kernels: the shared-tile kernel
+# at 256 (three-stage ring, one MMA issuer), 224, 192, 176 (twice, the second
+# with a ragged channel tile), 160 and 128 (two issuers), and the own-tile
+# kernel (three accumulators, K <= 512) at 160, 144 and 128.  Every M leaves
+# a ragged last token tile, and the k-slice counts are odd and even.  Each
+# shape runs the plain, residual, narrow-output and fused ShiftGELU
+# epilogues (the ShiftGELU one takes the own-tile kernel up to K = 768).
 TILE_WIDTH_SHAPES = [
-    (5421, 384, 768),
-    (4655, 768, 768),
-    (4226, 384, 768),
-    (3890, 384, 768),
-    (2881, 768, 1008),
-    (3121, 768, 768),
+    # shared-tile kernel (K > 512; the ShiftGELU epilogue at K > 768)
+    (5421, 1024, 768),    # 256 tokens
+    (4655, 896, 768),     # 224
+    (4226, 1024, 768),    # 192
+    (3890, 640, 768),     # 176
+    (2881, 1152, 1008),   # 176, ragged channel tile
+    (3121, 896, 768),     # 160
+    (1013, 1024, 768),    # 128
+    # own-tile kernel (K <= 512): 160, 144 and 128 tokens
+    (3461, 384, 768),
+    (3076, 512, 768),
+    (2593, 384, 1008),    # ragged channel tile
+    (2306, 256, 1008),
     (1013, 384, 768),
 ]
 
