@@ -392,7 +392,8 @@ inline bool shift_exp_alu_exact(int32_t k_s, int32_t I0) {
   const int64_t nmax = m + (m + 1) / 2 - (m + 15) / 16;
   return nmax * (int64_t)I0 < ((int64_t)1 << 32);
 }
-constexpr int kSoftWarps = 8;    // per softmax group
+constexpr int kRowSplit = 2;     // warps (per lane quarter) that split a query row's keys (3 measured slower)
+constexpr int kSoftWarps = 4 * kRowSplit;  // per softmax group
 constexpr int kSoftGroups = 2;   // groups take alternate items, one TMEM buffer each
 constexpr int kLoadStages = 3;
 constexpr int kPersistThreads = 96 + 32 * kSoftWarps * kSoftGroups;
@@ -425,7 +426,7 @@ __host__ __device__ inline PersistLayout persist_layout(int N) {
   L.p_bytes = L.kblocks * 128 * 128;       // 16 KB per 128 keys
   L.tab_off = L.p_off + kSoftGroups * L.p_bytes;
   L.part_off = L.tab_off + 256 * 32 * 4;
-  L.bar_off = L.part_off + kSoftGroups * 2 * 2 * kQTile * 4;
+  L.bar_off = L.part_off + kSoftGroups * kRowSplit * 2 * kQTile * 4;
   L.total = L.bar_off + 24 * 8;
   return L;
 }
@@ -693,14 +694,16 @@ __global__ void __launch_bounds__(kPersistThreads, 1)
     const int sw = warp - 3;
     const int group = sw / kSoftWarps;   // handles local items j with j % 2 == group
     const int quarter = warp & 3;
-    const int half = (sw >> 2) & 1;
+    const int half = (sw >> 2) % kRowSplit;  // which slice of the row's key chunks
     const int row = quarter * 32 + lane;  // query row of the tile = TMEM lane
-    const int hcols = L.n32 / 2;          // key columns per half (a multiple of 16)
-    const int cbase = half * hcols;
-    const int nch = hcols / 16;
+    const int nc32 = L.n32 / 16;          // 16-key chunks of the MMA-padded row
+    const int c_lo = (nc32 * half) / kRowSplit, c_hi = (nc32 * (half + 1)) / kRowSplit;
+    const int cbase = 16 * c_lo;
+    const int nch = c_hi - c_lo;
     int nvalid = 0;  // chunks of this half that hold at least one real key
     while (nvalid < nch && cbase + 16 * nvalid < N) ++nvalid;
-    int32_t* part = reinterpret_cast<int32_t*>(smem + L.part_off) + group * 512;  // [half][max, sum][128 rows]
+    // [slice][max, sum][128 rows]
+    int32_t* part = reinterpret_cast<int32_t*>(smem + L.part_off) + group * (kRowSplit * 2 * kQTile);
     const int rlo = row & 7;
     uint8_t* prow = smem + L.p_off + group * L.p_bytes + (row >> 3) * 1024 + rlo * 128;
     const uint32_t t_row = tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(group * L.sbuf);
@@ -738,9 +741,11 @@ __global__ void __launch_bounds__(kPersistThreads, 1)
         });
       }
       int32_t smax = max(max(m4[0], m4[1]), max(m4[2], m4[3]));
-      part[half * 256 + row] = smax;
+      part[half * 2 * kQTile + row] = smax;
       softmax_bar(group);
-      smax = max(part[row], part[256 + row]);
+      smax = part[row];
+#pragma unroll
+      for (int sl = 1; sl < kRowSplit; ++sl) smax = max(smax, part[sl * 2 * kQTile + row]);
       const int32_t vmax = logit_unclamped<FASTQ>(smax, bq, a.logit_b, a.logit_c);
       const int32_t lmax = min(max(vmax, a.ks_lo), a.ks_hi);
 
@@ -753,9 +758,11 @@ __global__ void __launch_bounds__(kPersistThreads, 1)
         else
           sum = shiftmax_pass2<FASTQ, false, ALU>(t_row, cbase, nvalid, N, tb, lmax, bq, a);
       }
-      part[half * 256 + 128 + row] = (int32_t)sum;
+      part[half * 2 * kQTile + kQTile + row] = (int32_t)sum;
       softmax_bar(group);
-      sum = (uint32_t)part[128 + row] + (uint32_t)part[256 + 128 + row];
+      sum = 0;
+#pragma unroll
+      for (int sl = 0; sl < kRowSplit; ++sl) sum += (uint32_t)part[sl * 2 * kQTile + kQTile + row];
       if (sum == 0) sum = 1;  // rows that skipped the passes
       const uint32_t dv = (1u << a.M) / sum;
 
@@ -798,11 +805,11 @@ __global__ void __launch_bounds__(kPersistThreads, 1)
         if (sep_o) mbar_arrive(&tmem_empty[group]);  // S is consumed: the next S may land
       }
 
-      // ---- ctx = sat_8((b_o O) >> c_o); half h writes columns [32 h, 32 h + 32)
+      // ---- ctx = sat_8((b_o O) >> c_o); slices 0 and 1 write columns [32 h, 32 h + 32)
       if (ok) ok = wait_or_abort(&o_full[group], ph, a.status, abort_flag);
       ok = __all_sync(0xffffffffu, ok);
       tc_fence_after();
-      if (ok && work) {
+      if (ok && work && half < 2) {  // the output's 64 columns: two slices of 32
         uint32_t r[32];
         tmem_ld32(t_out + (uint32_t)(half * 32), r);
         tmem_ld_wait();
