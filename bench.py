@@ -66,6 +66,10 @@ def parse_args():
     ap.add_argument("--no-workloads", action="store_true",
                     help="skip the other four workloads (measured after the headline one by default)")
     ap.add_argument("--kernel-reps", type=int, default=50)
+    ap.add_argument("--profile-op", default=None, metavar="KERNEL",
+                    help="for profilers: one block forward, then only this kernel of the per-kernel table "
+                         "(e.g. gemm_o_residual), once untimed and --kernel-reps times between "
+                         "cudaProfilerStart and cudaProfilerStop; prints a status line, no benchmark")
     ap.add_argument("--model-blocks", type=int, default=12,
                     help="blocks of the whole-model timing (ViT-B workload only; 0 skips it)")
     return ap.parse_args()
@@ -768,10 +772,11 @@ def model_forward_timing(ivit, n_blocks, B, dev, reps=10):
             "setup_s": setup_s}
 
 
-def kernel_breakdown(ivit, wl, dp, ws, xs, reps, dev, peaks):
-    """Average device time per launch of every kernel of one block, each timed
-    alone over ``reps`` back-to-back launches with CUDA events.  Inputs are the
-    block's own intermediates (left in the workspace by a block forward)."""
+def block_kernels(ivit, wl, dp, ws, xs, dev):
+    """Every kernel of one block (and the variants beside it) as a launch
+    function of the repetition index, with its roofline bound and algorithmic
+    amount per launch.  Runs one block forward first: the kernels' inputs are
+    the block's own intermediates, left in the workspace."""
     import torch
     B, N, D, Dm, H = wl.B, wl.N, wl.D, wl.Dm, wl.H
     T = B * N
@@ -797,36 +802,11 @@ def kernel_breakdown(ivit, wl, dp, ws, xs, reps, dev, peaks):
     h_o = torch.empty_like(g)
     R = len(xs)
     hs = [g.clone() for _ in range(max(2, math.ceil(2 * 126e6 / (2 * T * Dm))))]
-
-    def timed(fn):
-        # reps launches captured in one CUDA graph and replayed, so host launch
-        # overhead does not enter the per-launch device time
-        for i in range(3):
-            fn(i)
-        torch.cuda.synchronize()
-        g = torch.cuda.CUDAGraph()
-        s = torch.cuda.Stream(device=dev)
-        s.wait_stream(torch.cuda.current_stream())
-        with torch.cuda.stream(s):
-            with torch.cuda.graph(g, stream=s):
-                for i in range(reps):
-                    fn(i)
-        torch.cuda.current_stream().wait_stream(s)
-        g.replay()
-        torch.cuda.synchronize()
-        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        a.record()
-        g.replay()
-        b.record()
-        torch.cuda.synchronize()
-        del g
-        return a.elapsed_time(b) / reps
-
     gemm = lambda M, K, Nn: 2 * M * K * Nn
     out = []
 
     def add(name, fn, bound, amount, in_block=True, per_block=1):
-        out.append({"name": name, "ms": timed(fn), "bound": bound, "amount": amount, "in_block": in_block,
+        out.append({"name": name, "fn": fn, "bound": bound, "amount": amount, "in_block": in_block,
                     "per_block": per_block})
 
     add("layernorm", lambda i: ivit.ivit_layernorm(xs[i % R], t["ln1_gamma"], t["ln1_beta"], p["ln_F"], p["ln_M"],
@@ -883,6 +863,44 @@ def kernel_breakdown(ivit, wl, dp, ws, xs, reps, dev, peaks):
     add("layernorm_ptf", lambda i: ivit.ivit_layernorm_ptf(xs[i % R], alpha, t["ln1_gamma"], t["ln1_beta"],
                                                            p["ln_F"], 20, p["ln1_out"], y),
         "hbm", 2 * T * D, in_block=False)
+    return out
+
+
+def kernel_breakdown(ivit, wl, dp, ws, xs, reps, dev, peaks):
+    """Average device time per launch of every kernel of one block, each timed
+    alone over ``reps`` back-to-back launches with CUDA events.  Inputs are the
+    block's own intermediates (left in the workspace by a block forward)."""
+    import torch
+
+    def timed(fn):
+        # reps launches captured in one CUDA graph and replayed, so host launch
+        # overhead does not enter the per-launch device time
+        for i in range(3):
+            fn(i)
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        s = torch.cuda.Stream(device=dev)
+        s.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(s):
+            with torch.cuda.graph(g, stream=s):
+                for i in range(reps):
+                    fn(i)
+        torch.cuda.current_stream().wait_stream(s)
+        g.replay()
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        g.replay()
+        b.record()
+        torch.cuda.synchronize()
+        del g
+        return a.elapsed_time(b) / reps
+
+    out = []
+    for k in block_kernels(ivit, wl, dp, ws, xs, dev):
+        fn = k.pop("fn")
+        k["ms"] = timed(fn)
+        out.append(k)
     num_sms = torch.cuda.get_device_properties(dev).multi_processor_count
     for k in out:
         k["peak"], k["unit"], k["peak_note"] = peak_for(k["bound"], peaks, num_sms)
@@ -895,10 +913,47 @@ def kernel_breakdown(ivit, wl, dp, ws, xs, reps, dev, peaks):
     return out
 
 
+def run_profile_op(args):
+    """One kernel of the block on the block's own intermediates, for a
+    profiler: ``ncu --profile-from-start off`` captures only the launches
+    between cudaProfilerStart and cudaProfilerStop."""
+    import torch
+    import integer_only_quantized_int8_b200 as ivit
+    from integer_only_quantized_int8_b200 import params as ivit_params
+
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device (there is no CPU fallback)")
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    wl = synthetic.workload(args.workload, seed=args.seed)
+    B, N, D, Dm = wl.B, wl.N, wl.D, wl.Dm
+    dp = ivit_params.to_device(ivit_params.integer_params(wl.blocks[0]), dev)
+    ws = torch.empty(ivit.ivit_block_workspace_bytes(B, N, D, Dm), dtype=torch.uint8, device=dev)
+    x0 = torch.from_numpy(wl.x).to(dev)
+    xs = [x0.clone() for _ in range(input_copies(B * N * D))]
+    kernels = {k["name"]: k for k in block_kernels(ivit, wl, dp, ws, xs, dev)}
+    if args.profile_op not in kernels:
+        raise SystemExit(f"unknown kernel {args.profile_op!r}; one of {', '.join(kernels)}")
+    fn = kernels[args.profile_op]["fn"]
+    fn(0)
+    torch.cuda.synchronize()
+    torch.cuda.profiler.start()
+    for i in range(args.kernel_reps):
+        fn(i + 1)
+    torch.cuda.synchronize()
+    torch.cuda.profiler.stop()
+    status = ivit.ivit_stream_status()
+    print(json.dumps({"profile_op": args.profile_op, "workload": wl.name, "launches": args.kernel_reps,
+                      "status": ivit.ivit_status_string(status)}))
+    return 0 if status == 0 else 1
+
+
 def main():
     args = parse_args()
     if args.impl == "reference":
         return run_reference(args)
+    if args.profile_op:
+        return run_profile_op(args)
     return run_ours(args)
 
 
