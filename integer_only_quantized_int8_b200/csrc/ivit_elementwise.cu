@@ -268,66 +268,119 @@ __global__ void __launch_bounds__(kLnThreads)
 // ShiftGELU with a row maximum (I-ViT section 3.4, I_max read as the row's
 // largest exponent; see include/ivit.h): one warp per row.  I_p is
 // non-decreasing in x, so the row's largest exponent is I_p of the row's
-// largest byte; given it, the output is a function of the int8 input alone,
-// which the warp tabulates (256 entries) and streams the row through.  The
-// table is kept while consecutive rows of the warp share their I_max (rows
-// that reach x = 127 all do).
+// largest byte; given it, the output is a function of the int8 input alone:
+// a 256-entry table, which the warp builds when its row's I_max differs
+// from its previous row's (rows of a real activation rarely share one).  A
+// table entry takes its two exponentials from a per-CTA ShiftExp table over
+// every reachable exponent offset (built before the dependent-launch wait:
+// it depends on I0 only) and one integer division.  Tables are indexed by the
+// raw byte and sit on 256-byte boundaries, so a lookup address is one
+// bitwise merge of the byte and the table base.  With VPL > 0 a row of at
+// most 32 VPL 16-byte vectors stays in registers between the maximum and the
+// lookups; VPL = 0 reads a row twice.
 // ---------------------------------------------------------------------------
 constexpr int kRowGeluThreads = 256;
+constexpr int kRowGeluWarps = kRowGeluThreads / 32;
+// I_max - I_p(x) over int8 x: I_max <= I_p(127) = 212 and I_p(-128) = -216
+constexpr int kRowGeluExpSpan = 432;
 
+__device__ __forceinline__ int32_t gelu_ip(int32_t x) { return x + (x >> 1) + (x >> 3) + (x >> 4); }
+
+// the four signed-byte maxima of v folded into m4
+__device__ __forceinline__ uint32_t vmax_int4(uint32_t m4, const int4& v) {
+  return __vmaxs4(m4, __vmaxs4(__vmaxs4((uint32_t)v.x, (uint32_t)v.y), __vmaxs4((uint32_t)v.z, (uint32_t)v.w)));
+}
+
+__device__ __forceinline__ uint32_t lds_u8(uint32_t addr) {
+  uint32_t v;
+  asm volatile("ld.shared.u8 %0, [%1];" : "=r"(v) : "r"(addr));
+  return v;
+}
+
+// 16 table lookups, one per byte; tbase is the table's shared-memory address
+// (a multiple of 256)
+__device__ __forceinline__ int4 gelu_lookup16(uint32_t tbase, const int4& in) {
+  const uint32_t w[4] = {(uint32_t)in.x, (uint32_t)in.y, (uint32_t)in.z, (uint32_t)in.w};
+  uint32_t o[4];
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const uint32_t v0 = lds_u8(tbase | (w[k] & 0xFFu));
+    const uint32_t v1 = lds_u8(tbase | ((w[k] >> 8) & 0xFFu));
+    const uint32_t v2 = lds_u8(tbase | ((w[k] >> 16) & 0xFFu));
+    const uint32_t v3 = lds_u8(tbase | (w[k] >> 24));
+    o[k] = __byte_perm(__byte_perm(v0, v1, 0x0040u), __byte_perm(v2, v3, 0x0040u), 0x5410u);
+  }
+  return make_int4((int)o[0], (int)o[1], (int)o[2], (int)o[3]);
+}
+
+template <int VPL>
 __global__ void __launch_bounds__(kRowGeluThreads)
     shiftgelu_rowmax_kernel(const int8_t* __restrict__ x, int64_t rows, int32_t cols, GeluParams g,
                             int8_t* __restrict__ y) {
-  __shared__ int8_t tabs[kRowGeluThreads / 32][256];
+  __shared__ __align__(256) uint8_t tabs[kRowGeluWarps][256];
+  __shared__ int32_t expt[kRowGeluExpSpan];  // expt[d] = ShiftExp(-d)
+  for (int d = threadIdx.x; d < kRowGeluExpSpan; d += blockDim.x) expt[d] = shift_exp(-d, g.I0);
+  __syncthreads();
   pdl_wait();  // x comes from an earlier kernel
   pdl_launch_dependents();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  int8_t* tab = tabs[warp];
+  uint8_t* own = tabs[warp];
+  const uint32_t tbase = smem_u32(own);
   const int nvec = cols >> 4;
-  int32_t tab_imax = -1;  // the I_max the warp's table holds (none yet)
-  for (int64_t row = (int64_t)blockIdx.x * (kRowGeluThreads / 32) + warp; row < rows;
-       row += (int64_t)gridDim.x * (kRowGeluThreads / 32)) {
-    const int4* xv = reinterpret_cast<const int4*>(x + row * cols);
-    uint32_t m4 = 0x80808080u;  // four running maxima of signed bytes
-    for (int v = lane; v < nvec; v += 32) {
-      const int4 in = __ldg(xv + v);
-      m4 = __vmaxs4(m4, __vmaxs4(__vmaxs4((uint32_t)in.x, (uint32_t)in.y), __vmaxs4((uint32_t)in.z, (uint32_t)in.w)));
+  const int sh = g.M - (g.k_out - 1);
+  int32_t own_imax = -1;  // the I_max the warp's table holds (none yet)
+  // the table of a row with largest byte m (warp-uniform)
+  auto make_table = [&](int32_t m) {
+    const int32_t ipm = gelu_ip(m);
+    const int32_t I_max = ipm > 0 ? ipm : 0;
+    if (I_max == own_imax) return;
+    __syncwarp();  // every lane is done with the previous table
+    const uint32_t e2 = (uint32_t)expt[I_max];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const int32_t xi = (int32_t)(int8_t)(uint8_t)(lane + 32 * j);  // entry (uint8_t) xi
+      // bytes above the row's maximum never occur in the row: their entries
+      // are unused, and the offset is clamped only to stay inside the table
+      const uint32_t e1 = (uint32_t)expt[max(I_max - gelu_ip(xi), 0)];
+      const uint32_t sum = e1 + e2;
+      const uint32_t dv = (1u << g.M) / (sum > 0u ? sum : 1u);  // both exponentials 0: sigma = 0
+      const int32_t sig = (int32_t)((dv * e1) >> sh);
+      own[lane + 32 * j] = (uint8_t)(int8_t)requant8(xi * sig, g.out.b, g.out.c);
     }
+    __syncwarp();
+    own_imax = I_max;
+  };
+  auto warp_max = [&](uint32_t m4) {
     int32_t m = max(max((int32_t)(int8_t)m4, (int32_t)(int8_t)(m4 >> 8)),
                     max((int32_t)(int8_t)(m4 >> 16), (int32_t)(int8_t)(m4 >> 24)));
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(0xffffffffu, m, o));
-    // I_max = max(0, I_p(largest x)), warp-uniform
-    const int32_t ipm = m + (m >> 1) + (m >> 3) + (m >> 4);
-    const int32_t I_max = ipm > 0 ? ipm : 0;
-    if (I_max != tab_imax) {
-      __syncwarp();  // every lane is done with the previous table
-      const int32_t e2 = shift_exp(-I_max, g.I0);
-      for (int i = lane; i < 256; i += 32) {
-        const int32_t xi = i - 128;
-        const int32_t ip = xi + (xi >> 1) + (xi >> 3) + (xi >> 4);
-        const int32_t e1 = shift_exp(ip - I_max, g.I0);
-        const uint32_t sum = (uint32_t)(e1 + e2);
-        const uint32_t dv = (1u << g.M) / (sum > 0u ? sum : 1u);  // both exponentials 0: sigma = 0
-        const int32_t sig = (int32_t)((dv * (uint32_t)e1) >> (g.M - (g.k_out - 1)));
-        tab[i] = (int8_t)requant8(xi * sig, g.out.b, g.out.c);
-      }
-      __syncwarp();
-      tab_imax = I_max;
-    }
+    return m;
+  };
+  const int64_t rstep = (int64_t)gridDim.x * kRowGeluWarps;
+  for (int64_t row = (int64_t)blockIdx.x * kRowGeluWarps + warp; row < rows; row += rstep) {
+    const int4* xv = reinterpret_cast<const int4*>(x + row * cols);
     int4* yv = reinterpret_cast<int4*>(y + row * cols);
-    for (int v = lane; v < nvec; v += 32) {
-      const int4 in = __ldg(xv + v);
-      const uint32_t w[4] = {(uint32_t)in.x, (uint32_t)in.y, (uint32_t)in.z, (uint32_t)in.w};
-      uint32_t o[4];
+    if (VPL > 0) {
+      int4 v[VPL > 0 ? VPL : 1];
+      uint32_t m4 = 0x80808080u;  // padding vectors hold -128, which never raises the maximum
 #pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        uint32_t r = 0;
-#pragma unroll
-        for (int e = 0; e < 4; ++e) r |= ((uint32_t)(uint8_t)tab[((w[k] >> (8 * e)) & 0xFFu) ^ 0x80u]) << (8 * e);
-        o[k] = r;
+      for (int k = 0; k < VPL; ++k) {
+        const int c = lane + 32 * k;
+        v[k] = c < nvec ? __ldcs(xv + c) : make_int4((int)0x80808080, (int)0x80808080, (int)0x80808080, (int)0x80808080);
+        m4 = vmax_int4(m4, v[k]);
       }
-      __stcs(yv + v, make_int4((int)o[0], (int)o[1], (int)o[2], (int)o[3]));
+      make_table(warp_max(m4));
+#pragma unroll
+      for (int k = 0; k < VPL; ++k) {
+        const int c = lane + 32 * k;
+        if (c < nvec) __stcs(yv + c, gelu_lookup16(tbase, v[k]));
+      }
+    } else {
+      uint32_t m4 = 0x80808080u;
+      for (int c = lane; c < nvec; c += 32) m4 = vmax_int4(m4, __ldg(xv + c));
+      make_table(warp_max(m4));
+      for (int c = lane; c < nvec; c += 32) __stcs(yv + c, gelu_lookup16(tbase, __ldg(xv + c)));
     }
   }
 }
@@ -420,12 +473,33 @@ __global__ void __launch_bounds__(kPtfThreads)
 ivit_status launch_shiftgelu_rowmax(const DeviceCtx& dc, const int8_t* x, int64_t rows, int32_t cols,
                                     const GeluParams& g, int8_t* y, cudaStream_t stream) {
   if (rows == 0) return IVIT_OK;
-  const int64_t rows_per_cta = kRowGeluThreads / 32;
-  int64_t blocks = (rows + rows_per_cta - 1) / rows_per_cta;
-  const int64_t cap = (int64_t)dc.num_sms * 8;
-  if (blocks > cap) blocks = cap;
-  const cudaError_t e = launch_pdl(shiftgelu_rowmax_kernel, dim3((unsigned)blocks), dim3(kRowGeluThreads), 0, stream,
-                                   x, rows, cols, g, y);
+  // rows in registers up to 32 x 8 vectors (4096 columns); one wave of
+  // resident CTAs, so that each warp takes several rows and the next row's
+  // load overlaps the current lookups
+  const int vpl = (cols / 16 + 31) / 32;
+  static int per_sm_of[6] = {0, 0, 0, 0, 0, 0};  // resident CTAs per SM of each instance (benign race: same value)
+  auto run = [&](int id, void (*kernel)(const int8_t*, int64_t, int32_t, GeluParams, int8_t*)) -> cudaError_t {
+    int& per_sm = per_sm_of[id];
+    if (per_sm == 0 && cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, kRowGeluThreads, 0) != cudaSuccess)
+      return cudaErrorUnknown;
+    int64_t blocks = (rows + kRowGeluWarps - 1) / kRowGeluWarps;
+    const int64_t cap = (int64_t)dc.num_sms * (per_sm > 0 ? per_sm : 1);
+    if (blocks > cap) blocks = cap;
+    return launch_pdl(kernel, dim3((unsigned)blocks), dim3(kRowGeluThreads), 0, stream, x, rows, cols, g, y);
+  };
+  cudaError_t e;
+  if (vpl <= 1)
+    e = run(0, shiftgelu_rowmax_kernel<1>);
+  else if (vpl <= 2)
+    e = run(1, shiftgelu_rowmax_kernel<2>);
+  else if (vpl <= 4)
+    e = run(2, shiftgelu_rowmax_kernel<4>);
+  else if (vpl <= 6)
+    e = run(3, shiftgelu_rowmax_kernel<6>);
+  else if (vpl <= 8)
+    e = run(4, shiftgelu_rowmax_kernel<8>);
+  else
+    e = run(5, shiftgelu_rowmax_kernel<0>);
   note_launch();
   return e == cudaSuccess ? IVIT_OK : IVIT_ERR_CUDA;
 }

@@ -60,6 +60,26 @@ def test_shiftgelu_rowmax_parity(rows, cols):
     assert untouched()
 
 
+@pytest.mark.parametrize("rows,cols", [(20000, 256), (12000, 592), (6000, 1536), (4000, 2560), (3000, 4096),
+                                       (600, 4112)])
+def test_shiftgelu_rowmax_many_rows(rows, cols):
+    """More rows than the kernel's warps, so that warps take several rows
+    (the next row loads while the current one is looked up), at row lengths
+    that cover every register-resident width and the two-pass fallback; row
+    maxima vary at random, so a warp's rows switch between the shared table
+    of rows that reach 127 and its own tables."""
+    gc = synthetic.gelu_case(rows * cols, seed=rows ^ cols)
+    x = gc.x.reshape(rows, cols).copy()
+    caps = np.random.default_rng(cols).choice([127, 127, 127, 126, 100, 40, 1, 0, -5, -128], size=rows)
+    x = np.minimum(x, caps[:, None].astype(np.int8))
+    I0 = oracle.recip_i0(gc.S_h)
+    out = oracle.dyadic(gc.out_ratio)
+    y, untouched = guarded((rows, cols))
+    ivit.ivit_shiftgelu_rowmax(dev(x, torch.int8), I0, 30, 8, out, y)
+    np.testing.assert_array_equal(host(y), oracle.shiftgelu_rowmax(x, I0, 30, 8, out))
+    assert untouched()
+
+
 @pytest.mark.parametrize("I0,M,k_out", [(1, 30, 8), (2, 30, 8), (13, 20, 6), (4096, 30, 8)])
 def test_shiftgelu_rowmax_parameters(I0, M, k_out):
     """Every int8 value in every row, at I0 = 2 (both exponentials underflow
