@@ -396,7 +396,8 @@ constexpr int kRowSplit = 2;     // warps (per lane quarter) that split a query 
 constexpr int kSoftWarps = 4 * kRowSplit;  // per softmax group
 constexpr int kSoftGroups = 2;   // groups take alternate items, one TMEM buffer each
 constexpr int kLoadStages = 3;
-constexpr int kPersistThreads = 96 + 32 * kSoftWarps * kSoftGroups;
+constexpr int kReadWarps = 4;    // output readout, one per TMEM lane quarter
+constexpr int kPersistThreads = 96 + 32 * kSoftWarps * kSoftGroups + 32 * kReadWarps;
 
 struct PersistLayout {
   int n64, n32, n16, kblocks;
@@ -568,11 +569,11 @@ __global__ void __launch_bounds__(kPersistThreads, 1)
   uint64_t* s_full = bars + 6;        // [2] S in TMEM buffer g
   uint64_t* p_full = bars + 8;        // [2] P of group g in shared memory (one arrival per warp)
   uint64_t* o_full = bars + 10;       // [2] P V of group g's item in TMEM
-  uint64_t* tmem_empty = bars + 12;   // [2] S buffer g reusable (one arrival per warp)
+  uint64_t* tmem_empty = bars + 12;   // [2] S buffer g reusable
   uint64_t* drain = bars + 14;        // all MMAs of the CTA complete (one commit per issuer)
   uint32_t* tslot = reinterpret_cast<uint32_t*>(bars + 15);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 16);
-  uint64_t* o_empty = bars + 17;      // separate P V region read out (one arrival per warp)
+  uint64_t* o_empty = bars + 17;      // separate P V region read out (one arrival per readout warp)
   const bool sep_o = L.o_col >= 0;
 
   const int tid = threadIdx.x;
@@ -592,10 +593,12 @@ __global__ void __launch_bounds__(kPersistThreads, 1)
       mbar_init(&s_full[g], 1);
       mbar_init(&p_full[g], kSoftWarps);
       mbar_init(&o_full[g], 1);
-      mbar_init(&tmem_empty[g], kSoftWarps);
+      // freed by the softmax warps once P is written (separate P V region),
+      // else by the readout warps once the output in it is read
+      mbar_init(&tmem_empty[g], sep_o ? kSoftWarps : kReadWarps);
     }
     mbar_init(drain, 2);
-    mbar_init(o_empty, kSoftWarps);
+    mbar_init(o_empty, kReadWarps);
     *abort_flag = 0;
     fence_barrier_init();
     prefetch_tensormap(&tm);
@@ -689,7 +692,7 @@ __global__ void __launch_bounds__(kPersistThreads, 1)
       }
       umma_commit(drain);
     }
-  } else {
+  } else if (warp < 3 + kSoftWarps * kSoftGroups) {
     // ------------------------------------------------------------ softmax warps
     const int sw = warp - 3;
     const int group = sw / kSoftWarps;   // handles local items j with j % 2 == group
@@ -707,7 +710,6 @@ __global__ void __launch_bounds__(kPersistThreads, 1)
     const int rlo = row & 7;
     uint8_t* prow = smem + L.p_off + group * L.p_bytes + (row >> 3) * 1024 + rlo * 128;
     const uint32_t t_row = tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(group * L.sbuf);
-    const uint32_t t_out = sep_o ? tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)L.o_col : t_row;
     const int pshift = a.M - (a.k_out - 1);
     bool ok = true;
     int j = group;
@@ -766,10 +768,14 @@ __global__ void __launch_bounds__(kPersistThreads, 1)
       if (sum == 0) sum = 1;  // rows that skipped the passes
       const uint32_t dv = (1u << a.M) / sum;
 
-      // ---- pass 3: P = (Dv e) >> (M - k_out + 1) into the group's swizzled operand
-      // (the previous P of this group was consumed by a P V that completed
-      // before the o_full wait of the previous item)
-      if (work) {
+      // ---- pass 3: P = (Dv e) >> (M - k_out + 1) into the group's swizzled operand,
+      // once the P V of the group's previous item (which read the previous P)
+      // has completed
+      if (j >= 2) {
+        if (ok) ok = wait_or_abort(&o_full[group], (uint32_t)(((j >> 1) - 1) & 1), a.status, abort_flag);
+        ok = __all_sync(0xffffffffu, ok);
+      }
+      if (work && ok) {
         // (Dv e) >> pshift is one mul.hi by Dv 2^(32 - pshift) when Dv < 2^pshift
         const bool hip = pshift >= 1 && __all_sync(0xffffffffu, (uint64_t)dv < ((uint64_t)1 << pshift));
         const uint32_t dvh = hip ? dv << (32 - pshift) : 0u;
@@ -805,40 +811,6 @@ __global__ void __launch_bounds__(kPersistThreads, 1)
         if (sep_o) mbar_arrive(&tmem_empty[group]);  // S is consumed: the next S may land
       }
 
-      // ---- ctx = sat_8((b_o O) >> c_o); slices 0 and 1 write columns [32 h, 32 h + 32)
-      if (ok) ok = wait_or_abort(&o_full[group], ph, a.status, abort_flag);
-      ok = __all_sync(0xffffffffu, ok);
-      tc_fence_after();
-      if (ok && work && half < 2) {  // the output's 64 columns: two slices of 32
-        uint32_t r[32];
-        tmem_ld32(t_out + (uint32_t)(half * 32), r);
-        tmem_ld_wait();
-        const int q = q0 + row;
-        if (q < N) {
-          int8_t* dst = a.ctx + (int64_t)(img * N + q) * D + h * kHeadDim + half * 32;
-          uint32_t packed[8];
-#pragma unroll
-          for (int wd = 0; wd < 8; ++wd) {
-            int32_t y[4];
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              if (a.out_fast) {
-                y[e] = __mulhi(a.out_bq, (int32_t)r[wd * 4 + e]);  // floor(b_o acc / 2^c_o), exact
-              } else {
-                const int32_t acc = min(max((int32_t)r[wd * 4 + e], a.o_lo), a.o_hi);
-                const int64_t v = (int64_t)a.out_b * acc;  // |v >> c| < 2^31 after the clamp
-                y[e] = (int32_t)__funnelshift_r((uint32_t)v, (uint32_t)(v >> 32), (uint32_t)a.out_c);
-              }
-            }
-            packed[wd] = pack_sat4_attn(y[0], y[1], y[2], y[3]);
-          }
-          reinterpret_cast<int4*>(dst)[0] = make_int4(packed[0], packed[1], packed[2], packed[3]);
-          reinterpret_cast<int4*>(dst)[1] = make_int4(packed[4], packed[5], packed[6], packed[7]);
-        }
-      }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(sep_o ? o_empty : &tmem_empty[group]);
       qt += st_q;
       if (qt >= qtiles) {
         qt -= qtiles;
@@ -850,6 +822,60 @@ __global__ void __launch_bounds__(kPersistThreads, 1)
         ++img;
       }
       img += st_i;
+    }
+  } else {
+    // ------------------------------------------------------------ readout warps
+    // ctx = sat_8((b_o O) >> c_o) of every local item in order, while the
+    // softmax groups go on with their next items; each warp reads the 64
+    // output columns of its lane quarter's 32 query rows
+    const int quarter = warp & 3;
+    const int row = quarter * 32 + lane;
+    const int n_local = n_items > (int)blockIdx.x ? (n_items - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
+    bool ok = true;
+    for (int j = 0; j < n_local; ++j) {
+      const int g = j & 1;
+      const int item = (int)blockIdx.x + j * (int)gridDim.x;
+      const int qt = item % qtiles, h = (item / qtiles) % a.H, img = item / (qtiles * a.H);
+      if (ok) ok = wait_or_abort(&o_full[g], (uint32_t)((j >> 1) & 1), a.status, abort_flag);
+      ok = __all_sync(0xffffffffu, ok);
+      tc_fence_after();
+      const int q = qt * kQTile + row;
+      if (ok && qt * kQTile + quarter * 32 < N) {  // the quarter holds at least one real row
+        const uint32_t t_out =
+            tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(sep_o ? L.o_col : g * L.sbuf);
+#pragma unroll
+        for (int part = 0; part < 2; ++part) {
+          uint32_t ra[16], rb[16];
+          tmem_ld16(t_out + (uint32_t)(32 * part), ra);
+          tmem_ld16(t_out + (uint32_t)(32 * part + 16), rb);
+          tmem_ld_wait_regs2(ra, rb);
+          if (q < N) {
+            uint32_t packed[8];
+#pragma unroll
+            for (int wd = 0; wd < 8; ++wd) {
+              int32_t y[4];
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                const int32_t acc = (int32_t)(wd < 4 ? ra[wd * 4 + e] : rb[(wd - 4) * 4 + e]);
+                if (a.out_fast) {
+                  y[e] = __mulhi(a.out_bq, acc);  // floor(b_o acc / 2^c_o), exact
+                } else {
+                  const int32_t ac = min(max(acc, a.o_lo), a.o_hi);
+                  const int64_t v = (int64_t)a.out_b * ac;  // |v >> c| < 2^31 after the clamp
+                  y[e] = (int32_t)__funnelshift_r((uint32_t)v, (uint32_t)(v >> 32), (uint32_t)a.out_c);
+                }
+              }
+              packed[wd] = pack_sat4_attn(y[0], y[1], y[2], y[3]);
+            }
+            int8_t* dst = a.ctx + (int64_t)(img * N + q) * D + h * kHeadDim + part * 32;
+            reinterpret_cast<int4*>(dst)[0] = make_int4(packed[0], packed[1], packed[2], packed[3]);
+            reinterpret_cast<int4*>(dst)[1] = make_int4(packed[4], packed[5], packed[6], packed[7]);
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(sep_o ? o_empty : &tmem_empty[g]);
     }
   }
 
