@@ -107,9 +107,9 @@ __global__ void __launch_bounds__(kAttnThreads)
   int32_t* tab = reinterpret_cast<int32_t*>(smem + L.tab_off);
   uint64_t* bar_qk = reinterpret_cast<uint64_t*>(smem + L.bar_off);
   uint64_t* bar_v = bar_qk + 1;
-  uint64_t* bar_s = bar_qk + 2;
-  uint64_t* bar_o = bar_qk + 3;
-  uint32_t* tslot = reinterpret_cast<uint32_t*>(bar_qk + 4);
+  uint64_t* bar_s = bar_qk + 2;  // [2]: S chunk in TMEM buffer b
+  uint64_t* bar_o = bar_qk + 4;
+  uint32_t* tslot = reinterpret_cast<uint32_t*>(bar_qk + 5);
 
   const int tid = threadIdx.x;
   const int warp = tid >> 5;
@@ -119,11 +119,18 @@ __global__ void __launch_bounds__(kAttnThreads)
   const int D = a.H * kHeadDim;
   const int row0 = img * N;  // first token row of this image in qkv / ctx
   const int nload = L.n64 / 64;
+  // S is computed in chunks of up to 256 keys; with more than one chunk, two
+  // TMEM buffers let the next chunk's MMA run while this one is requantised
+  // (the launcher then keeps one CTA per SM, so the 512 columns are free)
+  const int nchunks = (L.n32 + 255) / 256;
+  const bool dbuf = nchunks >= 2;
+  const uint32_t tcols = dbuf ? 2u * kTmemCols : (uint32_t)kTmemCols;
 
   if (tid == 0) {
     mbar_init(bar_qk, 1);
     mbar_init(bar_v, 1);
-    mbar_init(bar_s, 1);
+    mbar_init(&bar_s[0], 1);
+    mbar_init(&bar_s[1], 1);
     mbar_init(bar_o, 1);
     fence_barrier_init();
     prefetch_tensormap(&tm);
@@ -132,7 +139,7 @@ __global__ void __launch_bounds__(kAttnThreads)
   for (int t = tid; t < (1 << a.k_s); t += kAttnThreads) tab[t] = shift_exp(-t, a.I0);
   if (warp == 0) {
     __syncwarp();
-    tmem_alloc(tslot, kTmemCols);
+    tmem_alloc(tslot, tcols);
     tmem_relinquish();
   }
   tc_fence_before();
@@ -163,31 +170,38 @@ __global__ void __launch_bounds__(kAttnThreads)
   uint32_t* part_sum = reinterpret_cast<uint32_t*>(part_max + kAttnSplit * kQTile);
 
   // ---- S = Q K^T in chunks of up to 256 keys, requantised to k_s-bit logits;
-  // the chunk's 32-column groups go round-robin to the four slices
-  const int nchunks = (L.n32 + 255) / 256;
-  for (int c = 0; c < nchunks; ++c) {
-    const int w = (L.n32 - c * 256) < 256 ? (L.n32 - c * 256) : 256;
-    if (tid == 0 && ok) {
-      if (c == 0 && !mbar_wait(bar_qk, 0, a.status)) ok = false;
-      if (ok) {
-        tc_fence_after();
-        const uint32_t idesc = idesc_i8(kQTile, w, true, true, false);
-        const uint32_t qa = smem_u32(sQ);
-        const uint32_t kb = smem_u32(sK + c * 256 * kHeadDim);
+  // the chunk's 32-column groups go round-robin to the four slices.  Chunk c
+  // lands in buffer c & 1 (dbuf) and completes phase (c >> 1) & 1 of
+  // bar_s[c & 1]: one commit in flight per barrier.
+  auto chunk_width = [&](int c) { return (L.n32 - c * 256) < 256 ? (L.n32 - c * 256) : 256; };
+  auto issue_s = [&](int c) {  // tid 0 only
+    tc_fence_after();
+    const uint32_t idesc = idesc_i8(kQTile, chunk_width(c), true, true, false);
+    const uint32_t qa = smem_u32(sQ);
+    const uint32_t kb = smem_u32(sK + c * 256 * kHeadDim);
+    const uint32_t dst = tmem + (dbuf ? (uint32_t)((c & 1) * kTmemCols) : 0u);
 #pragma unroll
-        for (int k = 0; k < kHeadDim / 32; ++k)
-          umma_i8(tmem, smem_desc(qa + k * 32, 16, 512, kSwizzle64B), smem_desc(kb + k * 32, 16, 512, kSwizzle64B),
-                  idesc, k != 0);
-        umma_commit(bar_s);
-      }
-    }
-    if (!mbar_wait(bar_s, (uint32_t)(c & 1), a.status)) ok = false;
+    for (int k = 0; k < kHeadDim / 32; ++k)
+      umma_i8(dst, smem_desc(qa + k * 32, 16, 512, kSwizzle64B), smem_desc(kb + k * 32, 16, 512, kSwizzle64B), idesc,
+              k != 0);
+    umma_commit(&bar_s[c & 1]);
+  };
+  if (tid == 0) {
+    if (!mbar_wait(bar_qk, 0, a.status)) ok = false;
+    if (ok) issue_s(0);
+  }
+  for (int c = 0; c < nchunks; ++c) {
+    const int w = chunk_width(c);
+    // the other buffer's previous chunk was read before the last __syncthreads
+    if (tid == 0 && ok && dbuf && c + 1 < nchunks) issue_s(c + 1);
+    if (!mbar_wait(&bar_s[c & 1], (uint32_t)((c >> 1) & 1), a.status)) ok = false;
     ok = __all_sync(0xffffffffu, ok);  // warp-uniform: guards a warp-collective TMEM load
     tc_fence_after();
     if (ok) {
+      const uint32_t t_buf = t_lane + (dbuf ? (uint32_t)((c & 1) * kTmemCols) : 0u);
       for (int cc = slice; cc < w / 32; cc += kAttnSplit) {
         uint32_t r[32];
-        tmem_ld32(t_lane + (uint32_t)(cc * 32), r);
+        tmem_ld32(t_buf + (uint32_t)(cc * 32), r);
         tmem_ld_wait();
         const int j0 = c * 256 + cc * 32;
         uint32_t packed[8];
@@ -349,7 +363,7 @@ __global__ void __launch_bounds__(kAttnThreads)
   if (warp == 0) {
     __syncwarp();
     tc_fence_after();
-    tmem_dealloc(tmem, kTmemCols);
+    tmem_dealloc(tmem, tcols);
   }
 }
 
@@ -975,9 +989,11 @@ ivit_status launch_attention(const DeviceCtx& dc, const int8_t* qkv, int32_t B, 
     return e == cudaSuccess ? IVIT_OK : IVIT_ERR_CUDA;
   }
   const AttnLayout L = attn_layout(N);
-  // at most two CTAs per SM, so that their TMEM (256 columns each) always fits
+  // at most two CTAs per SM, so that their TMEM (256 columns each) always
+  // fits; one CTA per SM when S takes two 256-column buffers (N > 256)
   int smem = L.total + 1024;
   if (smem < 80 * 1024) smem = 80 * 1024;
+  if (L.n32 > 256 && smem < 116 * 1024) smem = 116 * 1024;
   static int attr_bytes = 0;
   if (smem > attr_bytes) {
     if (cudaFuncSetAttribute(attention_shiftmax_kernel<true, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
