@@ -380,7 +380,10 @@ __global__ void __launch_bounds__(kAttnThreads)
 //   warp 2      P V issuer: P V of item j once its P is in shared memory.
 //               Two issuing threads, each blocked on its own next event, so
 //               neither softmax group waits behind the other;
-//   warps 3-18  two softmax groups of eight warps.
+//   warps 3-18  two softmax groups of eight warps;
+//   warps 19-22 output readout, one per TMEM lane quarter: each item's
+//               ctx = sat_8((b_o O) >> c_o), in item order, while the
+//               softmax groups go on with their next items.
 // S = Q K^T is N = round16(N) columns wide.
 // Within an item the score row never leaves TMEM: pass 1 takes the row
 // maximum of the raw int32 scores (the logit requant is monotone, so
@@ -392,7 +395,9 @@ __global__ void __launch_bounds__(kAttnThreads)
 // 128B-swizzled K-major P operand.  Warps w and w + 4 of a group share TMEM
 // lanes (query rows) and split the key columns; their partial maxima and sums
 // meet in shared memory behind a named barrier of the group's 256 threads.
-// P V lands in the first 64 columns of the item's S buffer, dead by then.
+// P V lands in a 64-column region of its own when two S buffers and it fit
+// the 512 TMEM columns (N <= 224), else in the first 64 columns of the
+// item's S buffer, dead by then.
 // ---------------------------------------------------------------------------
 constexpr int kShortMaxKeys = 256;
 constexpr int kTableMaxBits = 8;  // ShiftExp by table up to 8-bit logits, computed beyond
@@ -483,8 +488,8 @@ IVIT_DEV bool wait_or_abort(uint64_t* bar, uint32_t parity, int* status, volatil
 IVIT_DEV void softmax_bar(int group) { asm volatile("bar.sync %0, %1;" ::"r"(1 + group), "n"(32 * kSoftWarps) : "memory"); }
 
 // Streams n 16-column chunks of this warp's TMEM lanes starting at taddr,
-// body(r, k) on chunk k.  Single-buffered: with eighteen warps a thread has
-// at most 96 registers, and the other softmax warps cover the load latency.
+// body(r, k) on chunk k.  Single-buffered: with 23 warps a thread has at
+// most 80 registers, and the other softmax warps cover the load latency.
 template <typename F>
 IVIT_DEV void tmem_stream16(uint32_t taddr, int n, F&& body) {
   uint32_t r[16];

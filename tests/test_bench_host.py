@@ -66,3 +66,20 @@ def test_traffic_entries_follow_their_kernels_sources():
         else:
             assert got is None, key
     assert bench.load_traffic("attention", "no_such_workload") is None
+
+
+def test_gpu_local_cpus_is_a_subset_of_the_allowed_cpus_or_none():
+    # on a host without a GPU (or without NVML) the end-to-end buffers keep
+    # the process's own affinity
+    cpus = bench.gpu_local_cpus(0)
+    assert cpus is None or (cpus and cpus <= os.sched_getaffinity(0))
+
+
+def test_profile_op_flag_parses():
+    old = sys.argv
+    try:
+        sys.argv = ["bench.py", "--profile-op", "gemm_o_residual", "--kernel-reps", "2"]
+        args = bench.parse_args()
+    finally:
+        sys.argv = old
+    assert args.profile_op == "gemm_o_residual" and args.kernel_reps == 2
