@@ -524,10 +524,23 @@ def other_workload(ivit, ivit_params, name, args, dev, peaks, num_sms):
     t0 = time.perf_counter()
     wl = synthetic.workload(name, seed=args.seed)
     gen_s = time.perf_counter() - t0
+    import torch
     runner = BlockRunner(ivit, ivit_params, wl, dev, use_graph=not args.no_graph)
     steps = max(10, min(args.steps, 50))
     ms, _ = runner.timed(max(3, args.warmup), steps)
     ms_step = ms / steps
+    # the same steps launched one by one from the host, without a CUDA graph:
+    # the latency a caller sees without capturing (launch overhead included)
+    for i in range(3):
+        runner.step(i % runner.R)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for i in range(steps):
+        runner.step(i % runner.R)
+    e1.record()
+    torch.cuda.synchronize()
+    eager_ms_step = e0.elapsed_time(e1) / steps
     nb = len(wl.blocks)
     ops = wl.B * nb * ops_per_image_block(wl.N, wl.D)
     eff = ops / (ms_step / 1e3) / 1e12
@@ -535,6 +548,7 @@ def other_workload(ivit, ivit_params, name, args, dev, peaks, num_sms):
     alu_peak, _, _ = peak_for("alu", peaks, num_sms)
     attn_ops = SHIFTMAX_OPS_PER_SCORE * wl.B * wl.H * wl.N * wl.N
     out = {"images_per_s": wl.B / (ms_step / 1e3), "ms_per_step": ms_step, "steps": steps,
+           "ms_per_step_without_graph": eager_ms_step,
            "effective_tops": eff, "frac_int8_peak": eff / (peaks["bf16_tflops"] * INT8_PER_BF16),
            "attention_ms": attn_ms, "attention_roofline_frac": attn_ops / (attn_ms / 1e3) / 1e12 / alu_peak,
            "gpu_launches_per_step": int(runner.launches_per_step), "config": workload_config(wl, args),
